@@ -1,0 +1,126 @@
+"""Decode-loop schedule and the whole-path oracle run (test infrastructure only).
+
+Written from the TokenButler summaries, independently of the library's own
+schedule code:
+
+* [ja] 技術概要：TokenButler, コアアーキテクチャ: queries are predicted at fixed
+  depth-stride producer layers and consumed by the layers that follow; each
+  producer call emits G slot-specific queries per head (reading: G = stride,
+  slot j serves layer p + j).
+* [ja] 最適化, バッチ処理: keys are projected in batches of N tokens, not at every
+  step (reading: N is the window size, so every candidate [S, T-N) has a
+  projected key).
+* [ja] 最適化, 予測間隔と近隣取得: the predictor (and therefore the selection)
+  runs once per prediction interval P; the index set is reused in between.
+* [ja] 推論戦略: sink and window are recomputed from the current length at every
+  step; the importance set is the one from the last prediction.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from . import attention, attention_set, predict_queries, project_keys, scores, select
+
+
+def is_prediction_step(step: int, interval: int) -> bool:
+    return step % interval == 0
+
+
+def last_prediction_step(step: int, interval: int) -> int:
+    return step - step % interval
+
+
+def producer_of(layer: int, stride: int) -> int:
+    return layer - layer % stride
+
+
+def slot_of(layer: int, stride: int) -> int:
+    return layer % stride
+
+
+def projection_events(ctx0: int, window: int, steps: int):
+    """(step, begin) pairs at which a batch of `window` new keys is projected.
+    The prefill projects [0, floor(ctx0/N)*N); afterwards a batch is projected
+    at step i when the current length T = ctx0 + i + 1 has run N tokens past
+    the projected prefix."""
+    proj = (ctx0 // window) * window
+    events = []
+    for i in range(steps):
+        T = ctx0 + i + 1
+        if T - proj >= window:
+            events.append((i, proj))
+            proj += window
+    return (ctx0 // window) * window, events
+
+
+def run(w, data, layers, steps, want_attention=True, heads=None):
+    """Run the oracle over decode steps [0, steps) for the given layers.
+
+    `data` provides host arrays (numpy; bf16 as uint16):
+      data.kv(layer) -> (K, V) each [batch][Hkv][ctx_cap][d]
+      data.wk(layer) -> [Hkv][d'][d]
+      data.mlp(producer) -> (W1, W2)            (predictor workloads)
+      data.h(pred_index, producer) -> [batch][hidden]
+      data.qp_direct(pred_index, layer) -> [batch][Hq][d'] float32
+      data.q(step, layer) -> [batch][Hq][d]
+    Returns {(step, layer): {"idx": [[I_bh]], "out": [batch][Hq][d] or None}}.
+    """
+    B, Hq, grp = w.batch, w.n_q_heads, w.group
+    heads = list(range(Hq)) if heads is None else list(heads)
+    ctx0 = w.ctx0_per_seq()
+    scale = 1.0 / math.sqrt(w.head_dim)
+    res = {}
+    cur_idx = {}
+    kp_cache = {}
+    qp_cache = {}
+    for layer in layers:
+        K, V = data.kv(layer)
+        Wk = data.wk(layer)
+        for i in range(steps):
+            if is_prediction_step(i, w.interval):
+                k = i // w.interval
+                if w.hidden > 0:
+                    p = producer_of(layer, w.producer_stride)
+                    if (k, p) not in qp_cache:
+                        W1, W2 = data.mlp(p)
+                        qp_cache[(k, p)] = predict_queries(data.h(k, p), W1, W2).reshape(
+                            B, w.slots, Hq, w.d_proj)
+                    qp = qp_cache[(k, p)][:, slot_of(layer, w.producer_stride)]
+                else:
+                    qp = data.qp_direct(k, layer)
+                sets = []
+                for b in range(B):
+                    T = ctx0[b] + i + 1
+                    hi = T - w.window
+                    per_head = []
+                    for h in range(Hq):
+                        if h not in heads:
+                            per_head.append(None)
+                            continue
+                        g = h // grp
+                        if hi > w.sink:
+                            key = (layer, b, g)
+                            have = kp_cache.get(key)
+                            if have is None or have.shape[0] < hi:
+                                kp_cache[key] = project_keys(K[b, g, :hi], Wk[g])
+                            s = scores(qp[b, h], kp_cache[key], w.sink, hi)
+                        else:
+                            s = np.zeros(0, np.float32)
+                        per_head.append(select(s, T, w.sink, w.window, w.budget, w.nbr))
+                    sets.append(per_head)
+                cur_idx[layer] = sets
+            out = None
+            if want_attention:
+                Q = data.q(i, layer)
+                out = np.zeros((B, Hq, w.head_dim), np.float32)
+                for b in range(B):
+                    T = ctx0[b] + i + 1
+                    for h in heads:
+                        g = h // grp
+                        A = attention_set(T, w.sink, w.window, cur_idx[layer][b][h])
+                        out[b, h] = attention(Q[b, h], K[b, g], V[b, g], A, scale)
+            res[(i, layer)] = {"idx": cur_idx[layer], "out": out}
+        kp_cache.clear()
+    return res

@@ -1,0 +1,319 @@
+"""Checks that pin the oracle to something other than itself.
+
+Each ``pin_*`` function takes a loaded oracle library and raises AssertionError
+on a mismatch.  They are run against the real oracle by test_oracle_pins.py and
+against deliberately broken copies of it by test_oracle_mutants.py, which checks
+that every planted mistake is caught by at least one pin.
+
+What pins what:
+  bf16 rounding      torch's float32 -> bf16 conversion (a library routine) on
+                     random, midpoint and subnormal values, plus closed-form
+                     cases where rounding through float32 first would differ
+  key projection     exact integer matrix products (numpy int64) rounded by torch
+  predictor MLP      torch float64 matmul + SiLU as an independent witness
+  scores             exact integer dot products (numpy int64)
+  selection          hand-worked golden cases, and brute force by rank counting
+                     on tiny inputs with many ties
+  attention set      sink/window/importance invariants
+  attention          closed forms (two-logit softmax, equal logits, constant V),
+                     torch float64 softmax as a witness, sparse == dense when the
+                     budget covers every candidate
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def _bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+
+
+def _round_f64_via_torch(x: np.ndarray) -> np.ndarray:
+    """Round exactly-representable-in-float32 doubles to bf16 with torch."""
+    f = np.asarray(x, np.float64).astype(np.float32)
+    assert np.all(f.astype(np.float64) == x), "witness needs float32-exact inputs"
+    return _bf16_bits(torch.from_numpy(f))
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding
+# ---------------------------------------------------------------------------
+
+def pin_bf16_rounding(lib):
+    rng = np.random.default_rng(1)
+    vals = [rng.standard_normal(4000).astype(np.float32),
+            (rng.standard_normal(2000) * 1e-39).astype(np.float32),   # subnormal range
+            (rng.standard_normal(2000) * 1e30).astype(np.float32)]
+    # exact midpoints between adjacent bf16 values (ties go to the even code)
+    base = rng.integers(0x0080, 0x7f00, 2000).astype(np.uint32)
+    mids = ((base << 16) | 0x8000).view(np.float32)
+    vals.append(mids)
+    vals.append(-mids)
+    x = np.concatenate(vals).astype(np.float64)
+    got = np.array([lib.orc_double_to_bf16(float(v)) for v in x], np.uint16)
+    want = _round_f64_via_torch(x)
+    assert np.array_equal(got, want), "bf16 rounding disagrees with torch"
+    # a double just above a bf16 midpoint must round up; rounding to float32 first
+    # would land on the midpoint and then round to even (down)
+    one_up = lib.orc_double_to_bf16(1.0 + 2.0 ** -8 + 2.0 ** -40)
+    assert one_up == 0x3F81, hex(one_up)
+    assert lib.orc_double_to_bf16(1.0 + 2.0 ** -8) == 0x3F80          # tie -> even
+    assert lib.orc_double_to_bf16(1.0 + 3 * 2.0 ** -8) == 0x3F82      # tie -> even (up)
+    assert lib.orc_double_to_bf16(-2.5) == 0xC020
+    assert lib.orc_double_to_bf16(1e39) == 0x7F80                     # overflow -> inf
+
+
+def pin_bf16_widening(lib):
+    bits = np.arange(0, 1 << 16, 7, dtype=np.uint32).astype(np.uint16)
+    finite = (bits & 0x7F80) != 0x7F80
+    bits = bits[finite]
+    got = np.array([lib.orc_bf16_to_double(int(b)) for b in bits])
+    want = _bits_to_f64(bits)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# key projection
+# ---------------------------------------------------------------------------
+
+def pin_project_keys_integer(lib):
+    rng = np.random.default_rng(2)
+    for (rows, d, dp) in [(37, 64, 16), (5, 128, 32), (1, 8, 16)]:
+        K = rng.integers(-4, 5, (rows, d))
+        W = rng.integers(-4, 5, (dp, d))
+        exact = K.astype(np.int64) @ W.astype(np.int64).T          # [rows][dp]
+        want = _round_f64_via_torch(exact.astype(np.float64))
+        got = oracle.project_keys(_bf16_bits(torch.tensor(K, dtype=torch.float32)),
+                                  _bf16_bits(torch.tensor(W, dtype=torch.float32)), lib=lib)
+        assert np.array_equal(got, want), (rows, d, dp)
+
+
+def pin_project_keys_random(lib):
+    g = torch.Generator().manual_seed(3)
+    K = torch.randn(64, 128, generator=g).bfloat16()
+    W = (torch.randn(32, 128, generator=g) * 0.02).bfloat16()
+    got = _bits_to_f64(oracle.project_keys(_bf16_bits(K), _bf16_bits(W), lib=lib))
+    ref = (K.double() @ W.double().T).numpy()
+    # one bf16 rounding (8 significant bits) of the exact product: relative
+    # error at most the unit roundoff 2^-8
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 * (1 + 1e-12) + 1e-300)
+    # and the nearest code: the adjacent bf16 codes are not closer
+    bits = oracle.project_keys(_bf16_bits(K), _bf16_bits(W), lib=lib).astype(np.int32)
+    for step in (-1, 1):
+        nb = _bits_to_f64((bits + step).astype(np.uint16))
+        assert np.all(np.abs(nb - ref) >= np.abs(got - ref))
+    assert np.mean(got == ref) < 0.5, "inputs are not trivially exact"
+
+
+# ---------------------------------------------------------------------------
+# predictor MLP
+# ---------------------------------------------------------------------------
+
+def pin_predict_queries(lib):
+    g = torch.Generator().manual_seed(4)
+    B, hidden, inter, n_out = 3, 256, 96, 40
+    h = torch.randn(B, hidden, generator=g).bfloat16()
+    W1 = (torch.randn(inter, hidden, generator=g) * 0.1).bfloat16()
+    W2 = (torch.randn(n_out, inter, generator=g) * 0.1).bfloat16()
+    got = oracle.predict_queries(_bf16_bits(h), _bf16_bits(W1), _bf16_bits(W2), lib=lib)
+    a = h.double() @ W1.double().T
+    act = torch.nn.functional.silu(a).bfloat16().double()
+    want = (act @ W2.double().T).numpy()
+    # the witness rounds the activation through float32; rare double-rounding
+    # cases move one activation by one bf16 step, far inside this bound
+    err = np.abs(got.astype(np.float64) - want)
+    assert np.all(err <= 1e-3 * np.abs(want).max() + 1e-6), err.max()
+    # h = 0 gives SiLU(0) = 0 and q' = 0 exactly
+    z = oracle.predict_queries(_bf16_bits(torch.zeros(1, hidden)), _bf16_bits(W1),
+                               _bf16_bits(W2), lib=lib)
+    assert np.all(z == 0.0)
+
+
+def pin_predict_queries_silu_closed_form(lib):
+    # hidden 1, W1 = identity row, W2 = identity: q' = bf16(SiLU(h))
+    hvals = torch.tensor([[-2.0], [0.5], [3.0]])
+    W1 = torch.ones(1, 1)
+    W2 = torch.ones(1, 1)
+    got = oracle.predict_queries(_bf16_bits(hvals), _bf16_bits(W1), _bf16_bits(W2), lib=lib)
+    for k, x in enumerate([-2.0, 0.5, 3.0]):
+        silu = x / (1.0 + math.exp(-x))
+        assert abs(float(got[k, 0]) - silu) <= abs(silu) * 2.0 ** -8, (x, got[k, 0], silu)
+
+
+# ---------------------------------------------------------------------------
+# scores
+# ---------------------------------------------------------------------------
+
+def pin_scores_integer(lib):
+    rng = np.random.default_rng(5)
+    for dp in (16, 32):
+        Kp = rng.integers(-300, 301, (50, dp))
+        q = rng.integers(-4, 5, dp)
+        Kp_bits = _bf16_bits(torch.tensor(Kp, dtype=torch.float32))
+        Kp_val = _bits_to_f64(Kp_bits).astype(np.int64)               # bf16 codes of Kp
+        want = (Kp_val @ q.astype(np.int64)).astype(np.float64)
+        got = oracle.scores(q.astype(np.float32), Kp_bits, 7, 50, lib=lib)
+        assert np.array_equal(got.astype(np.float64), want[7:50])
+
+
+# ---------------------------------------------------------------------------
+# selection
+# ---------------------------------------------------------------------------
+
+def pin_select_golden(lib):
+    with open(os.path.join(GOLDEN, "select_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        got = oracle.select(np.array(c["scores"], np.float32), c["T"], c["S"], c["N"], c["B"],
+                            c["r"], lib=lib)
+        assert got.tolist() == c["expect"], (c["name"], got.tolist())
+
+
+def _brute_select(s, T, S, N, B, r):
+    lo, hi = S, T - N
+    C = list(range(lo, hi))
+    top = []
+    for t in C:
+        rank = sum(1 for u in C if s[u - lo] > s[t - lo] or (s[u - lo] == s[t - lo] and u < t))
+        if rank < B:
+            top.append(t)
+    keep = set()
+    for t in top:
+        for u in range(t - r, t + r + 1):
+            if lo <= u < hi:
+                keep.add(u)
+    return sorted(keep)
+
+
+def pin_select_brute_force(lib):
+    rng = np.random.default_rng(6)
+    for trial in range(300):
+        S = int(rng.integers(0, 5))
+        N = int(rng.integers(1, 6))
+        T = int(rng.integers(1, 40))
+        B = int(rng.integers(1, 12))
+        r = int(rng.integers(0, 3))
+        nC = max(0, T - N - S)
+        s = rng.integers(-3, 4, nC).astype(np.float32)        # many ties
+        if trial % 3 == 0:
+            s = rng.standard_normal(nC).astype(np.float32)
+        got = oracle.select(s, T, S, N, B, r, lib=lib).tolist()
+        want = _brute_select(s, T, S, N, B, r)
+        assert got == want, (S, N, T, B, r, s.tolist(), got, want)
+
+
+# ---------------------------------------------------------------------------
+# attention set and attention
+# ---------------------------------------------------------------------------
+
+def pin_attention_set(lib):
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        S = int(rng.integers(0, 6))
+        N = int(rng.integers(1, 8))
+        T = int(rng.integers(1, 60))
+        lo, hi = S, T - N
+        I = np.array(sorted(x for x in range(lo, hi) if rng.random() < 0.3), np.int32)
+        A = oracle.attention_set(T, S, N, I, lib=lib).tolist()
+        sink = set(range(0, min(S, T)))
+        window = set(range(max(S, T - N), T))
+        assert A == sorted(set(A)), "sorted and unique"
+        assert set(A) == sink | window | set(I.tolist())
+        if T <= S + N:
+            assert A == list(range(T)), "short context is dense"
+
+
+def pin_attention_golden(lib):
+    with open(os.path.join(GOLDEN, "attention_cases.json")) as f:
+        cases = {c["name"]: c for c in json.load(f)["cases"]}
+
+    def run(c):
+        q = _bf16_bits(torch.tensor(c["q"], dtype=torch.float32))
+        K = _bf16_bits(torch.tensor(c["K"], dtype=torch.float32))
+        V = _bf16_bits(torch.tensor(c["V"], dtype=torch.float32))
+        return oracle.attention(q, K, V, np.array(c["rows"], np.int32), c["scale"], lib=lib)
+
+    e2 = math.exp(2.0)
+    o = run(cases["two_rows"])
+    assert np.allclose(o, [1 / (1 + e2), e2 / (1 + e2)], rtol=1e-7, atol=0)
+    o = run(cases["two_rows_scaled"])
+    assert np.allclose(o, [(4 * e2) / (1 + e2), (-2 * e2 + 2) / (1 + e2)], rtol=1e-7, atol=0)
+    o = run(cases["row_subset"])
+    assert np.allclose(o, [2.0, 3.0], rtol=1e-7, atol=0)
+
+
+def pin_attention_constant_v(lib):
+    g = torch.Generator().manual_seed(8)
+    d, rows = 64, 40
+    q = _bf16_bits(torch.randn(d, generator=g))
+    K = _bf16_bits(torch.randn(rows, d, generator=g) * 3)
+    v = torch.randn(d, generator=g).bfloat16()
+    V = _bf16_bits(v.float().expand(rows, d).contiguous())
+    A = np.array([0, 3, 5, 17, 39], np.int32)
+    o = oracle.attention(q, K, V, A, 0.125, lib=lib)
+    assert np.allclose(o, v.float().numpy(), rtol=1e-6, atol=0)
+
+
+def pin_attention_torch_witness(lib):
+    g = torch.Generator().manual_seed(9)
+    d, rows = 128, 300
+    q = torch.randn(d, generator=g).bfloat16()
+    K = torch.randn(rows, d, generator=g).bfloat16()
+    V = torch.randn(rows, d, generator=g).bfloat16()
+    A = np.array(sorted(set(np.random.default_rng(9).integers(0, rows, 120).tolist())), np.int32)
+    scale = 1 / math.sqrt(d)
+    got = oracle.attention(_bf16_bits(q), _bf16_bits(K), _bf16_bits(V), A, scale, lib=lib)
+    Ks, Vs = K.double()[torch.from_numpy(A).long()], V.double()[torch.from_numpy(A).long()]
+    p = torch.softmax((Ks @ q.double()) * scale, dim=0)
+    want = (p @ Vs).numpy()
+    assert np.allclose(got, want, rtol=1e-6, atol=1e-7)
+
+
+def pin_sparse_equals_dense_when_budget_covers(lib):
+    g = torch.Generator().manual_seed(10)
+    T, S, N, d, dp = 90, 4, 8, 64, 16
+    K = torch.randn(T, d, generator=g).bfloat16()
+    V = torch.randn(T, d, generator=g).bfloat16()
+    W = (torch.randn(dp, d, generator=g) * 0.1).bfloat16()
+    q = torch.randn(d, generator=g).bfloat16()
+    qp = torch.randn(dp, generator=g).numpy().astype(np.float32)
+    Kp = oracle.project_keys(_bf16_bits(K), _bf16_bits(W), lib=lib)
+    s = oracle.scores(qp, Kp, S, T - N, lib=lib)
+    I = oracle.select(s, T, S, N, T, 1, lib=lib)                    # budget >= |C|
+    A = oracle.attention_set(T, S, N, I, lib=lib)
+    assert A.tolist() == list(range(T))
+    sparse = oracle.attention(_bf16_bits(q), _bf16_bits(K), _bf16_bits(V), A, 0.125, lib=lib)
+    p = torch.softmax((K.double() @ q.double()) * 0.125, dim=0)
+    dense = (p @ V.double()).numpy()
+    assert np.allclose(sparse, dense, rtol=1e-6, atol=1e-7)
+
+
+ALL_PINS = [
+    pin_bf16_rounding,
+    pin_bf16_widening,
+    pin_project_keys_integer,
+    pin_project_keys_random,
+    pin_predict_queries,
+    pin_predict_queries_silu_closed_form,
+    pin_scores_integer,
+    pin_select_golden,
+    pin_select_brute_force,
+    pin_attention_set,
+    pin_attention_golden,
+    pin_attention_constant_v,
+    pin_attention_torch_witness,
+    pin_sparse_equals_dense_when_budget_covers,
+]

@@ -1,0 +1,64 @@
+"""Plant plausible mistakes in copies of the C oracle and check that the pins
+catch every one of them (CPU only; the real oracle is never modified).
+
+Each mutant is a textual edit of tb_oracle.c compiled into a temporary shared
+library: a transposed operand, a dropped term, a flipped sign, an off-by-one
+range, a reversed tie-break, a skipped rounding step.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "tb_oracle.c")
+
+MUTANTS = [
+    ("wk_transposed", "Wk[(int64_t)j * d + i]", "Wk[(int64_t)i * dp + j]"),
+    ("bf16_truncates", "double r = nearbyint(scaled);", "double r = floor(scaled);"),
+    ("bf16_ties_away", "double r = nearbyint(scaled);", "double r = round(scaled);"),
+    ("bf16_quantum_off", "int qexp = e - 8;", "int qexp = e - 9;"),
+    ("silu_dropped", "double silu = a / (1.0 + exp(-a));", "double silu = a;"),
+    ("silu_sign", "double silu = a / (1.0 + exp(-a));", "double silu = a / (1.0 + exp(a));"),
+    ("w1_transposed", "W1[(int64_t)i * hidden + k]", "W1[(int64_t)k * inter + i]"),
+    ("score_sign", "acc += (double)qp[j] * orc_bf16_to_double(Kp[t * dp + j]);",
+     "acc -= (double)qp[j] * orc_bf16_to_double(Kp[t * dp + j]);"),
+    ("score_drops_last_dim", "for (int j = 0; j < dp; ++j)\n            acc += (double)qp[j]",
+     "for (int j = 0; j < dp - 1; ++j)\n            acc += (double)qp[j]"),
+    ("tie_break_reversed", "return (x->t < y->t) ? -1 : (x->t > y->t) ? 1 : 0;",
+     "return (x->t > y->t) ? -1 : (x->t < y->t) ? 1 : 0;"),
+    ("ascending_scores", "if (x->s > y->s) return -1;\n    if (x->s < y->s) return 1;",
+     "if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;"),
+    ("neighbour_right_dropped", "for (int64_t u = t - r; u <= t + r; ++u)",
+     "for (int64_t u = t - r; u < t + r; ++u)"),
+    ("candidates_into_window", "int64_t c_lo = S, c_hi = T - N;", "int64_t c_lo = S, c_hi = T - N + 1;"),
+    ("candidates_into_sink", "int64_t c_lo = S, c_hi = T - N;", "int64_t c_lo = S - 1, c_hi = T - N;"),
+    ("budget_off_by_one", "int64_t take = B < nC ? B : nC;", "int64_t take = B - 1 < nC ? B - 1 : nC;"),
+    ("window_short", "int64_t win_begin = T - N > S ? T - N : S;",
+     "int64_t win_begin = T - N + 1 > S ? T - N + 1 : S;"),
+    ("sink_dropped", "for (int64_t t = 0; t < sink_end; ++t) A[n++] = (int32_t)t;", ""),
+    ("scale_dropped", "z[k] = acc * scale;", "z[k] = acc;"),
+    ("softmax_unnormalised", "out[j] = (float)(o / l);", "out[j] = (float)o;"),
+    ("v_row_misindexed", "V[(int64_t)A[k] * d + j]", "V[(int64_t)k * d + j]"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(name, old, new, tmp_path):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique/found"
+    mut_src = tmp_path / "tb_oracle_mut.c"
+    mut_src.write_text(src.replace(old, new))
+    so = oracle.build(force=True, src=str(mut_src), out=str(tmp_path / "libmut.so"))
+    lib = oracle.load(so)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+            break
+    assert caught, f"no pin caught mutant {name}"
+    shutil.rmtree(tmp_path, ignore_errors=True)

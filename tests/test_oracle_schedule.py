@@ -1,0 +1,122 @@
+"""The oracle's decode-loop schedule and whole-path run (CPU only).
+
+Invariants fixed by the TokenButler summaries ([ja] 推論戦略 and 最適化):
+sink and window always attended, projection in batches of N that always cover
+the candidates, the selection reused unchanged for a whole prediction interval,
+and sparse attention equal to dense attention when the budget covers every
+candidate.
+"""
+import math
+
+import numpy as np
+import torch
+
+import oracle
+import tb_inputs
+from oracle import schedule
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+class HostData:
+    """Host-side (numpy) view of a workload, generated on the CPU."""
+
+    def __init__(self, w):
+        self.w = w
+
+    def kv(self, layer):
+        K, V = tb_inputs.kv_layer(self.w, layer)
+        return _bits(K), _bits(V)
+
+    def wk(self, layer):
+        return _bits(tb_inputs.wk_layer(self.w, layer))
+
+    def mlp(self, p):
+        W1, W2 = tb_inputs.mlp_weights(self.w, p)
+        return _bits(W1), _bits(W2)
+
+    def h(self, k, p):
+        return _bits(tb_inputs.hidden_state(self.w, k, p))
+
+    def qp_direct(self, k, layer):
+        return tb_inputs.direct_qp(self.w, k, layer).numpy()
+
+    def q(self, i, layer):
+        return _bits(tb_inputs.query(self.w, i, layer))
+
+
+def test_projection_events_cover_candidates():
+    for ctx0 in (1, 63, 64, 65, 299, 8192, 1000):
+        for N in (1, 16, 64):
+            proj, events = schedule.projection_events(ctx0, N, 200)
+            assert proj % N == 0 and proj <= ctx0 < proj + N
+            it = iter(events)
+            nxt = next(it, None)
+            for i in range(200):
+                if nxt is not None and nxt[0] == i:
+                    assert nxt[1] == proj
+                    proj += N
+                    nxt = next(it, None)
+                T = ctx0 + i + 1
+                assert T - N <= proj, "every candidate [S, T-N) has a projected key"
+                assert proj <= T, "only existing tokens are projected"
+
+
+def test_prediction_schedule():
+    assert [i for i in range(40) if schedule.is_prediction_step(i, 16)] == [0, 16, 32]
+    assert schedule.last_prediction_step(37, 16) == 32
+    assert [schedule.producer_of(l, 4) for l in range(9)] == [0, 0, 0, 0, 4, 4, 4, 4, 8]
+    assert [schedule.slot_of(l, 4) for l in range(6)] == [0, 1, 2, 3, 0, 1]
+
+
+def _small_llama(**kw):
+    base = tb_inputs.WORKLOADS["llama8k"].scaled(
+        name="llama_small", n_layers=2, n_q_heads=8, n_kv_heads=2, hidden=256, inter=64,
+        producer_stride=2, ctx0=700, ctx0_lo=700, ctx0_hi=700, sink=4, window=16,
+        budget=40, interval=4, steps=9)
+    return base.scaled(**kw)
+
+
+def test_run_tiny300_invariants():
+    w = tb_inputs.WORKLOADS["tiny300"]
+    res = schedule.run(w, HostData(w), layers=[0], steps=1)
+    r = res[(0, 0)]
+    T = w.ctx0 + 1
+    assert T == 300
+    for h in range(w.n_q_heads):
+        I = r["idx"][0][h]
+        nC = T - w.window - w.sink
+        assert min(w.budget, nC) <= len(I) <= min(3 * w.budget, nC)
+        assert np.all(I >= w.sink) and np.all(I < T - w.window)
+        assert np.all(np.diff(I) > 0)
+    assert np.all(np.isfinite(r["out"]))
+
+
+def test_run_reuses_selection_over_interval():
+    w = _small_llama()
+    res = schedule.run(w, HostData(w), layers=[0, 1], steps=w.steps)
+    for layer in (0, 1):
+        for i in range(w.steps):
+            p = schedule.last_prediction_step(i, w.interval)
+            for h in range(w.n_q_heads):
+                assert np.array_equal(res[(i, layer)]["idx"][0][h], res[(p, layer)]["idx"][0][h])
+        # a new prediction (later, longer context) produces a different set somewhere
+        assert any(not np.array_equal(res[(4, layer)]["idx"][0][h], res[(0, layer)]["idx"][0][h])
+                   for h in range(w.n_q_heads))
+
+
+def test_run_budget_covering_context_equals_dense():
+    w = _small_llama(budget=10_000, steps=2, interval=1)
+    data = HostData(w)
+    res = schedule.run(w, data, layers=[1], steps=2)
+    K, V = data.kv(1)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    for i in range(2):
+        Q = data.q(i, 1)
+        T = w.ctx0 + i + 1
+        for h in range(w.n_q_heads):
+            g = h // w.group
+            dense = oracle.attention(Q[0, h], K[0, g], V[0, g], np.arange(T, dtype=np.int32), scale)
+            assert np.allclose(res[(i, 1)]["out"][0, h], dense, rtol=1e-6, atol=1e-7)
