@@ -1,0 +1,206 @@
+/*
+ * tb.h — C ABI of the TokenButler decode-time selection and sparse-attention
+ * library (libtb.so, CUDA kernels for sm_100a).
+ *
+ * The path (TokenButler technical summary, gist.science, sections
+ * "Core architecture" (コアアーキテクチャ), "Inference strategy" (推論戦略) and
+ * "Optimisations" (最適化)):
+ *
+ *   1. tb_project_keys       K' = K · W_kᵀ into d' dims, in batches of N tokens
+ *   2. tb_predict_queries    producer-layer MLP: q' = SiLU(h·W1ᵀ)·W2ᵀ, G slots
+ *   3+4. tb_score_select     s = q'·K'ᵀ over the candidates, top-B with
+ *                            neighbour fetch outside the sink and window
+ *   5. tb_sparse_decode_attn attention over sink ∪ window ∪ selected rows
+ *   –  tb_decode_attn        dense decode attention (the comparator)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers are DEVICE pointers unless a comment says "host".  Every device
+ *    pointer must be 16-byte aligned.  Nothing here allocates, frees or keeps
+ *    device memory; the caller owns every buffer, including workspaces.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous: it validates its arguments on the host, launches, and
+ *    returns; it never synchronises the device.
+ *  - bf16 values are passed as raw 16-bit patterns (`tb_bf16`).
+ *  - Caches use the layout [batch][n_kv_heads][ctx_cap][dim], row-contiguous
+ *    per (sequence, KV head).  Query-head h belongs to KV head h / (Hq/Hkv).
+ *  - Host-side argument errors return TB_ERR_INVALID_ARG or TB_ERR_UNSUPPORTED
+ *    BEFORE any launch; the message is available from tb_last_error() on the
+ *    calling thread.  A launch failure returns TB_ERR_CUDA.
+ *  - Conditions only the device can see (a per-sequence context length outside
+ *    [1, ctx_cap], a wait that timed out) never trap: the kernel clamps or
+ *    skips, sets a bit in the workspace's flag word, and the caller reads it
+ *    with tb_workspace_check().
+ *  - Workspaces must be zeroed once before first use (tb_workspace_init); every
+ *    call leaves its counters and histograms zeroed again.  Two calls that use
+ *    the same workspace must not overlap on the device.
+ */
+#ifndef TB_H
+#define TB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TB_ABI_VERSION 1
+
+typedef uint16_t tb_bf16;
+
+typedef enum {
+    TB_OK = 0,
+    TB_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad shape */
+    TB_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim, d', group size */
+    TB_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+    TB_ERR_WORKSPACE = 4,     /* workspace too small */
+    TB_ERR_DEVICE_FLAG = 5    /* tb_workspace_check found device-side flags */
+} tb_status;
+
+/* Device-side flag bits reported by tb_workspace_check(). */
+#define TB_FLAG_CTX_RANGE   0x1u  /* some ctx_len[b] outside [1, ctx_cap]: clamped */
+#define TB_FLAG_TIMEOUT     0x2u  /* a bounded wait gave up; the output is invalid */
+#define TB_FLAG_IDX_OVERFLOW 0x4u /* selected set larger than idx_cap: truncated */
+
+/* Shapes shared by the cache-facing calls. */
+typedef struct {
+    int32_t batch;       /* sequences */
+    int32_t n_q_heads;   /* Hq  */
+    int32_t n_kv_heads;  /* Hkv; Hq / Hkv must be 4 */
+    int32_t head_dim;    /* d:  64 or 128 */
+    int32_t d_proj;      /* d': 16 or 32 */
+    int32_t ctx_cap;     /* rows per (sequence, KV head) in K, V and K' */
+} tb_dims;
+
+int32_t     tb_abi_version(void);
+const char *tb_status_str(tb_status s);
+/* Message of the last non-OK status returned on this thread ("" if none). */
+const char *tb_last_error(void);
+
+/* ---- workspaces --------------------------------------------------------- */
+
+/* Bytes of workspace each call needs (>= 256: the first 256 bytes hold the
+ * device flag word).  0 is returned for invalid dims. */
+size_t tb_score_select_workspace_bytes(const tb_dims *dims);
+size_t tb_attn_workspace_bytes(const tb_dims *dims);           /* sparse and dense */
+size_t tb_predict_queries_workspace_bytes(int32_t batch, int32_t hidden, int32_t inter,
+                                          int32_t n_out);
+size_t tb_project_keys_workspace_bytes(void);
+
+/* Zero a workspace (cudaMemsetAsync).  Call once on a new workspace. */
+tb_status tb_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, copy the workspace's device flag word into *flags
+ * (host), clear it, and return TB_ERR_DEVICE_FLAG if any bit was set. */
+tb_status tb_workspace_check(void *ws, size_t ws_bytes, uint32_t *flags, void *stream);
+
+/* ---- 1. key-cache projection -------------------------------------------- */
+/* Each consumer layer projects its keys with a learned matrix into the d'
+ * space of the predicted queries (summary, "Core architecture: key-cache
+ * projection"); the projection runs once per batch of N new tokens rather than
+ * at every step (summary, "Optimisations: batching").
+ *
+ *   Kp[b][g][t][:] = bf16_rne( sum_i K[b][g][t][i] * Wk[g][:][i] )   (fp32 accumulate)
+ *
+ * for t in [tok_begin[b], tok_begin[b] + tok_count[b]) ∩ [0, ctx_cap).
+ *   K          [batch][Hkv][ctx_cap][d]   bf16
+ *   Wk         [Hkv][d'][d]               bf16 (output-major: row j is output dim j)
+ *   Kp         [batch][Hkv][ctx_cap][d']  bf16, only the rows above are written
+ *   tok_begin  [batch] int32; a negative entry skips that sequence
+ *   tok_count  [batch] int32
+ *   max_tok    host: an upper bound on every tok_count[b] (sizes the grid)
+ * Tensor cores (tcgen05) with TMA-loaded operands. */
+tb_status tb_project_keys(const tb_dims *dims, const tb_bf16 *K, const tb_bf16 *Wk,
+                          tb_bf16 *Kp, const int32_t *tok_begin, const int32_t *tok_count,
+                          int32_t max_tok, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- 2. query prediction ------------------------------------------------- */
+/* A light MLP takes the producer layer's hidden state and emits G
+ * slot-specific low-dimensional queries per attention head (summary, "Core
+ * architecture: query prediction").  Bias-free, SiLU between the products, the
+ * activation rounded to bf16 before the second product:
+ *
+ *   a  = bf16_rne( SiLU( h · W1ᵀ ) )          fp32 accumulate
+ *   qp = a · W2ᵀ                               fp32 accumulate and output
+ *
+ *   h   [batch][hidden] bf16;  W1 [inter][hidden] bf16;  W2 [n_out][inter] bf16
+ *   qp  [batch][n_out] fp32, n_out = G * Hq * d', read as [batch][G][Hq][d']
+ * batch <= 16; hidden, inter multiples of 256; n_out a multiple of 128.
+ * Tensor cores (tcgen05), split-K over CTAs, deterministic reduction. */
+tb_status tb_predict_queries(const tb_bf16 *h, const tb_bf16 *W1, const tb_bf16 *W2,
+                             float *qp, int32_t batch, int32_t hidden, int32_t inter,
+                             int32_t n_out, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- 3+4. scoring and budgeted selection ---------------------------------- */
+/* Dot products of the predicted queries with the projected keys give cheap
+ * importance scores for a dynamic per-token selection under a fixed budget
+ * (summary, "Core architecture: scoring"); the first S tokens (sink) and the
+ * last N (local window) are always kept and the importance buffer is filled
+ * from the scores (summary, "Inference strategy"); the selected tokens are
+ * expanded by their spatial neighbours (summary, "Optimisations: prediction
+ * interval and neighbour fetch").  For each sequence b and query head h, with
+ * T = ctx_len[b] and candidates C = [sink, T - window):
+ *
+ *   s[t]  = fp32( sum_j qp[b][h][j] * Kp[b][h/4][t][j] ),  t in C
+ *   Top   = the `budget` members of C first in the order (s desc, t asc)
+ *   I     = ( ∪_{t in Top} [t - nbr, t + nbr] ) ∩ C
+ *
+ *   qp         float [batch][..][Hq][d'] at qp + b*qp_batch_stride + h*d'
+ *              (point at one slot of a [batch][G][Hq][d'] array; stride G*Hq*d')
+ *   Kp         [batch][Hkv][ctx_cap][d'] bf16; rows of C must be projected
+ *   ctx_len    [batch] int32 (device)
+ *   idx        [batch][Hq][idx_cap] int32 out: I sorted ascending
+ *   count      [batch][Hq] int32 out: |I|
+ *   sel_bits   [batch][Hq][ceil(ctx_cap/32)] uint32 out: bit t%32 of word t/32
+ *              is 1 iff t in I (all other bits 0); this is what
+ *              tb_sparse_decode_attn consumes
+ *   idx_cap    >= min((2*nbr+1)*budget, ctx_cap)
+ * Limits: budget >= 1, sink >= 0, window >= 1, 0 <= nbr <= 16, ctx_cap <= 524288.
+ * The result is exact for the fp32 scores the kernel computes (radix select on
+ * the order-preserving integer image of the scores, ties by position). */
+tb_status tb_score_select(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
+                          const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink,
+                          int32_t window, int32_t budget, int32_t nbr, int32_t *idx,
+                          int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
+                          size_t ws_bytes, void *stream);
+
+/* Build the sel_bits bitmap from index lists that came from elsewhere (e.g. a
+ * host-side selection): bit t of row (b,h) is set iff t is among
+ * idx[b][h][0 .. count[b][h]).  Entries outside [0, ctx_cap) are ignored. */
+tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,
+                                  const int32_t *count, uint32_t *sel_bits, void *stream);
+
+/* ---- 5. sparse GQA decode attention --------------------------------------- */
+/* The full KV cache stays resident and only the selected tokens are read
+ * (summary, "Significance"); the kept rows are sink ∪ local window ∪
+ * importance buffer (summary, "Inference strategy").  For each sequence b and
+ * query head h, with T = ctx_len[b]:
+ *
+ *   A   = [0, min(sink,T)) ∪ [max(sink, T-window), T) ∪ { t in [sink, T-window) :
+ *         bit t of sel_bits[b][h] }
+ *   out[b][h] = sum_{t in A} softmax_t( scale * Q[b][h]·K[b][g][t] ) * V[b][g][t]
+ *
+ * fp32 logits, fp32 online softmax, fp32 accumulation; every (b, KV head, t)
+ * row is read once for the whole GQA group of 4 query heads.
+ *   Q    [batch][Hq][d] bf16;  K, V [batch][Hkv][ctx_cap][d] bf16
+ *   out  [batch][Hq][d] fp32
+ * Split over the context across CTAs; the last CTA of each (b, KV head) merges
+ * the partial softmax states (no inter-CTA waiting). */
+tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
+                                const tb_bf16 *V, const int32_t *ctx_len, int32_t sink,
+                                int32_t window, const uint32_t *sel_bits, float scale,
+                                float *out, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- dense decode attention (comparator) ---------------------------------- */
+/* The same computation over A = [0, T): the dense attention baseline the
+ * summaries' on-GPU speedup is measured against ("Contributions 4"). */
+tb_status tb_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
+                         const tb_bf16 *V, const int32_t *ctx_len, float scale, float *out,
+                         void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TB_H */

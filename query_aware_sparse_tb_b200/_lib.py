@@ -1,0 +1,186 @@
+"""ctypes binding of libtb.so (argument marshalling only).
+
+Every function here converts torch tensors into device pointers and sizes and
+calls the C entry point of the same name; all computation happens in the CUDA
+kernels behind it.  There is no fallback: if the library is missing or a call
+fails, a TbError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtb.so")
+
+TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
+TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW = 0x1, 0x2, 0x4
+
+EXPORTS = [
+    "tb_abi_version", "tb_status_str", "tb_last_error",
+    "tb_score_select_workspace_bytes", "tb_attn_workspace_bytes",
+    "tb_predict_queries_workspace_bytes", "tb_project_keys_workspace_bytes",
+    "tb_workspace_init", "tb_workspace_check",
+    "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_select_bits_from_idx",
+    "tb_sparse_decode_attn", "tb_decode_attn",
+]
+
+
+class TbError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+class TbDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("d_proj", ctypes.c_int32), ("ctx_cap", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libtb.so (it must have been built; nothing is compiled here)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise TbError(-1, f"{path} is missing: build it with `python -m query_aware_sparse_tb_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, i32, i64, sz, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    D = ctypes.POINTER(TbDims)
+    sig = {
+        "tb_abi_version": ([], i32),
+        "tb_status_str": ([ctypes.c_int], ctypes.c_char_p),
+        "tb_last_error": ([], ctypes.c_char_p),
+        "tb_score_select_workspace_bytes": ([D], sz),
+        "tb_attn_workspace_bytes": ([D], sz),
+        "tb_predict_queries_workspace_bytes": ([i32, i32, i32, i32], sz),
+        "tb_project_keys_workspace_bytes": ([], sz),
+        "tb_workspace_init": ([P, sz, P], ctypes.c_int),
+        "tb_workspace_check": ([P, sz, ctypes.POINTER(ctypes.c_uint32), P], ctypes.c_int),
+        "tb_project_keys": ([D, P, P, P, P, P, i32, P, sz, P], ctypes.c_int),
+        "tb_predict_queries": ([P, P, P, P, i32, i32, i32, i32, P, sz, P], ctypes.c_int),
+        "tb_score_select": ([D, P, i64, P, P, i32, i32, i32, i32, P, i32, P, P, P, sz, P], ctypes.c_int),
+        "tb_select_bits_from_idx": ([D, P, i32, P, P, P], ctypes.c_int),
+        "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
+        "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != TB_OK:
+        raise TbError(status, load().tb_last_error().decode())
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise TbError(TB_ERR_INVALID_ARG, "libtb takes device tensors")
+    if not t.is_contiguous():
+        raise TbError(TB_ERR_INVALID_ARG, "libtb takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def dims(batch, n_q_heads, n_kv_heads, head_dim, d_proj, ctx_cap) -> TbDims:
+    return TbDims(batch, n_q_heads, n_kv_heads, head_dim, d_proj, ctx_cap)
+
+
+def _bytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+# ------------------------------------------------------------------ workspaces
+
+def score_select_workspace_bytes(d: TbDims) -> int:
+    return load().tb_score_select_workspace_bytes(ctypes.byref(d))
+
+
+def attn_workspace_bytes(d: TbDims) -> int:
+    return load().tb_attn_workspace_bytes(ctypes.byref(d))
+
+
+def predict_queries_workspace_bytes(batch, hidden, inter, n_out) -> int:
+    return load().tb_predict_queries_workspace_bytes(batch, hidden, inter, n_out)
+
+
+def project_keys_workspace_bytes() -> int:
+    return load().tb_project_keys_workspace_bytes()
+
+
+def workspace(nbytes: int, device="cuda", stream=None) -> torch.Tensor:
+    """A zero-initialised workspace tensor of at least `nbytes` bytes."""
+    if nbytes <= 0:
+        raise TbError(TB_ERR_INVALID_ARG, "workspace size must be positive (invalid dims?)")
+    ws = torch.empty((nbytes + 255) // 256 * 256, dtype=torch.uint8, device=device)
+    _check(load().tb_workspace_init(_ptr(ws), _bytes(ws), _stream(stream)))
+    return ws
+
+
+def workspace_check(ws: torch.Tensor, stream=None) -> int:
+    """Return the device flag word (and clear it); 0 means no condition was seen."""
+    flags = ctypes.c_uint32(0)
+    st = load().tb_workspace_check(_ptr(ws), _bytes(ws), ctypes.byref(flags), _stream(stream))
+    if st not in (TB_OK, TB_ERR_DEVICE_FLAG):
+        _check(st)
+    return flags.value
+
+
+# ------------------------------------------------------------------ entry points
+
+def project_keys(d: TbDims, K, Wk, Kp, tok_begin, tok_count, max_tok: int, ws, stream=None):
+    _check(load().tb_project_keys(ctypes.byref(d), _ptr(K), _ptr(Wk), _ptr(Kp), _ptr(tok_begin),
+                                  _ptr(tok_count), int(max_tok), _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def predict_queries(h, W1, W2, qp, ws, stream=None):
+    batch, hidden = h.shape
+    inter = W1.shape[0]
+    n_out = W2.shape[0]
+    _check(load().tb_predict_queries(_ptr(h), _ptr(W1), _ptr(W2), _ptr(qp), batch, hidden, inter, n_out,
+                                     _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def score_select(d: TbDims, qp, qp_batch_stride: int, Kp, ctx_len, sink: int, window: int, budget: int,
+                 nbr: int, idx, count, sel_bits, ws, stream=None):
+    idx_cap = idx.shape[-1]
+    _check(load().tb_score_select(ctypes.byref(d), _ptr(qp), int(qp_batch_stride), _ptr(Kp), _ptr(ctx_len),
+                                  sink, window, budget, nbr, _ptr(idx), idx_cap, _ptr(count), _ptr(sel_bits),
+                                  _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def select_bits_from_idx(d: TbDims, idx, count, sel_bits, stream=None):
+    _check(load().tb_select_bits_from_idx(ctypes.byref(d), _ptr(idx), idx.shape[-1], _ptr(count),
+                                          _ptr(sel_bits), _stream(stream)))
+
+
+def sparse_decode_attn(d: TbDims, Q, K, V, ctx_len, sink: int, window: int, sel_bits, scale: float, out, ws,
+                       stream=None):
+    _check(load().tb_sparse_decode_attn(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), sink,
+                                        window, _ptr(sel_bits), float(scale), _ptr(out), _ptr(ws), _bytes(ws),
+                                        _stream(stream)))
+
+
+def decode_attn(d: TbDims, Q, K, V, ctx_len, scale: float, out, ws, stream=None):
+    _check(load().tb_decode_attn(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), float(scale),
+                                 _ptr(out), _ptr(ws), _bytes(ws), _stream(stream)))

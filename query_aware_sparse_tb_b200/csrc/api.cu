@@ -1,0 +1,244 @@
+// libtb C ABI: host-side validation and dispatch.  Every entry point checks its
+// arguments before any CUDA call, so an invalid call returns an error without
+// touching the device.  See include/tb.h for the contract of each call.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace tb {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+}
+
+namespace {
+
+constexpr int kMaxCtxSelect = 1 << 19;
+constexpr int kMaxCtxAttn = 1 << 22;
+
+tb_status fail(tb_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define TB_CHECK_PTR(p)                                                                      \
+    do {                                                                                     \
+        if (!aligned16(p))                                                                   \
+            return fail(TB_ERR_INVALID_ARG, "%s: pointer '%s' is null or not 16-byte aligned", \
+                        __func__, #p);                                                       \
+    } while (0)
+
+tb_status check_dims(const tb_dims *d, bool need_dproj, const char *fn) {
+    if (!d) return fail(TB_ERR_INVALID_ARG, "%s: dims is null", fn);
+    if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->ctx_cap < 1)
+        return fail(TB_ERR_INVALID_ARG, "%s: batch, head counts and ctx_cap must be >= 1", fn);
+    if (d->n_q_heads % d->n_kv_heads != 0)
+        return fail(TB_ERR_INVALID_ARG, "%s: n_q_heads (%d) not a multiple of n_kv_heads (%d)", fn,
+                    d->n_q_heads, d->n_kv_heads);
+    if (d->n_q_heads / d->n_kv_heads != 4)
+        return fail(TB_ERR_UNSUPPORTED, "%s: only GQA groups of 4 query heads are built (got %d)", fn,
+                    d->n_q_heads / d->n_kv_heads);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(TB_ERR_UNSUPPORTED, "%s: head_dim %d not built (64, 128)", fn, d->head_dim);
+    if (need_dproj && d->d_proj != 16 && d->d_proj != 32)
+        return fail(TB_ERR_UNSUPPORTED, "%s: d_proj %d not built (16, 32)", fn, d->d_proj);
+    return TB_OK;
+}
+
+tb_status check_ws(void *ws, size_t have, size_t need, const char *fn) {
+    if (!aligned16(ws)) return fail(TB_ERR_INVALID_ARG, "%s: workspace is null or not 16-byte aligned", fn);
+    if (have < need)
+        return fail(TB_ERR_WORKSPACE, "%s: workspace has %zu bytes, needs %zu", fn, have, need);
+    return TB_OK;
+}
+
+tb_status cuda_status(cudaError_t e, const char *fn) {
+    if (e == cudaSuccess) return TB_OK;
+    return fail(TB_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+}
+
+}  // namespace
+}  // namespace tb
+
+using namespace tb;
+
+extern "C" {
+
+int32_t tb_abi_version(void) { return TB_ABI_VERSION; }
+
+const char *tb_status_str(tb_status s) {
+    switch (s) {
+        case TB_OK: return "TB_OK";
+        case TB_ERR_INVALID_ARG: return "TB_ERR_INVALID_ARG";
+        case TB_ERR_UNSUPPORTED: return "TB_ERR_UNSUPPORTED";
+        case TB_ERR_CUDA: return "TB_ERR_CUDA";
+        case TB_ERR_WORKSPACE: return "TB_ERR_WORKSPACE";
+        case TB_ERR_DEVICE_FLAG: return "TB_ERR_DEVICE_FLAG";
+    }
+    return "TB_ERR_UNKNOWN";
+}
+
+const char *tb_last_error(void) { return g_err; }
+
+size_t tb_score_select_workspace_bytes(const tb_dims *dims) {
+    if (check_dims(dims, true, __func__) != TB_OK || dims->ctx_cap > kMaxCtxSelect) return 0;
+    return select_ws_bytes(*dims);
+}
+
+size_t tb_attn_workspace_bytes(const tb_dims *dims) {
+    if (check_dims(dims, false, __func__) != TB_OK || dims->ctx_cap > kMaxCtxAttn) return 0;
+    return attn_ws_bytes(*dims);
+}
+
+size_t tb_predict_queries_workspace_bytes(int32_t batch, int32_t hidden, int32_t inter, int32_t n_out) {
+    if (batch < 1 || batch > 16 || hidden < 256 || hidden % 256 || inter < 256 || inter % 256 ||
+        n_out < 128 || n_out % 128)
+        return 0;
+    return predict_ws_bytes(batch, hidden, inter, n_out);
+}
+
+size_t tb_project_keys_workspace_bytes(void) { return kWsHeaderBytes; }
+
+tb_status tb_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!aligned16(ws) || ws_bytes < (size_t)kWsHeaderBytes)
+        return fail(TB_ERR_INVALID_ARG, "tb_workspace_init: bad workspace");
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream), __func__);
+}
+
+tb_status tb_workspace_check(void *ws, size_t ws_bytes, uint32_t *flags, void *stream) {
+    if (!aligned16(ws) || ws_bytes < (size_t)kWsHeaderBytes || !flags)
+        return fail(TB_ERR_INVALID_ARG, "tb_workspace_check: bad arguments");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    tb_status s;
+    if ((s = cuda_status(cudaStreamSynchronize(st), __func__)) != TB_OK) return s;
+    if ((s = cuda_status(cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost), __func__)) != TB_OK) return s;
+    if ((s = cuda_status(cudaMemset(ws, 0, 4), __func__)) != TB_OK) return s;
+    *flags = v;
+    return v ? fail(TB_ERR_DEVICE_FLAG, "device flags 0x%x", v) : TB_OK;
+}
+
+tb_status tb_project_keys(const tb_dims *dims, const tb_bf16 *K, const tb_bf16 *Wk, tb_bf16 *Kp,
+                          const int32_t *tok_begin, const int32_t *tok_count, int32_t max_tok,
+                          void *ws, size_t ws_bytes, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
+    TB_CHECK_PTR(K); TB_CHECK_PTR(Wk); TB_CHECK_PTR(Kp); TB_CHECK_PTR(tok_begin); TB_CHECK_PTR(tok_count);
+    if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
+    if (max_tok < 0) return fail(TB_ERR_INVALID_ARG, "tb_project_keys: max_tok < 0");
+    if ((long long)dims->batch * dims->n_kv_heads * dims->ctx_cap > 0x7fffffffLL)
+        return fail(TB_ERR_UNSUPPORTED, "tb_project_keys: more than 2^31 cache rows");
+    if (max_tok == 0) return TB_OK;
+    return cuda_status(launch_project_keys(*dims, K, Wk, Kp, tok_begin, tok_count, max_tok, ws,
+                                           (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_predict_queries(const tb_bf16 *h, const tb_bf16 *W1, const tb_bf16 *W2, float *qp,
+                             int32_t batch, int32_t hidden, int32_t inter, int32_t n_out, void *ws,
+                             size_t ws_bytes, void *stream) {
+    TB_CHECK_PTR(h); TB_CHECK_PTR(W1); TB_CHECK_PTR(W2); TB_CHECK_PTR(qp);
+    if (batch < 1 || batch > 16)
+        return fail(TB_ERR_UNSUPPORTED, "tb_predict_queries: batch %d outside [1, 16]", batch);
+    if (hidden < 256 || hidden % 256 || inter < 256 || inter % 256)
+        return fail(TB_ERR_UNSUPPORTED, "tb_predict_queries: hidden and inter must be multiples of 256");
+    if (n_out < 128 || n_out % 128)
+        return fail(TB_ERR_UNSUPPORTED, "tb_predict_queries: n_out must be a multiple of 128");
+    tb_status s;
+    if ((s = check_ws(ws, ws_bytes, predict_ws_bytes(batch, hidden, inter, n_out), __func__)) != TB_OK)
+        return s;
+    return cuda_status(launch_predict_queries(h, W1, W2, qp, batch, hidden, inter, n_out, ws,
+                                              (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_score_select(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
+                          const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
+                          int32_t budget, int32_t nbr, int32_t *idx, int32_t idx_cap, int32_t *count,
+                          uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
+    TB_CHECK_PTR(qp); TB_CHECK_PTR(Kp); TB_CHECK_PTR(ctx_len); TB_CHECK_PTR(idx); TB_CHECK_PTR(count);
+    TB_CHECK_PTR(sel_bits);
+    if (dims->ctx_cap > kMaxCtxSelect)
+        return fail(TB_ERR_UNSUPPORTED, "tb_score_select: ctx_cap %d above %d", dims->ctx_cap, kMaxCtxSelect);
+    if (qp_batch_stride < (int64_t)dims->n_q_heads * dims->d_proj || (qp_batch_stride & 3))
+        return fail(TB_ERR_INVALID_ARG, "tb_score_select: qp_batch_stride %lld too small or not a multiple of 4",
+                    (long long)qp_batch_stride);
+    if (sink < 0 || window < 1 || budget < 1)
+        return fail(TB_ERR_INVALID_ARG, "tb_score_select: need sink >= 0, window >= 1, budget >= 1");
+    if (nbr < 0 || nbr > 16) return fail(TB_ERR_INVALID_ARG, "tb_score_select: nbr %d outside [0, 16]", nbr);
+    const long long need_cap = (long long)(2 * nbr + 1) * budget;
+    const long long min_cap = need_cap < dims->ctx_cap ? need_cap : dims->ctx_cap;
+    if (idx_cap < min_cap)
+        return fail(TB_ERR_INVALID_ARG, "tb_score_select: idx_cap %d < min((2*nbr+1)*budget, ctx_cap) = %lld",
+                    idx_cap, min_cap);
+    if ((s = check_ws(ws, ws_bytes, select_ws_bytes(*dims), __func__)) != TB_OK) return s;
+    return cuda_status(launch_score_select(*dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget,
+                                           nbr, idx, idx_cap, count, sel_bits, ws, (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,
+                                  const int32_t *count, uint32_t *sel_bits, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, false, __func__)) != TB_OK) return s;
+    TB_CHECK_PTR(idx); TB_CHECK_PTR(count); TB_CHECK_PTR(sel_bits);
+    if (idx_cap < 1) return fail(TB_ERR_INVALID_ARG, "tb_select_bits_from_idx: idx_cap < 1");
+    if (dims->ctx_cap > kMaxCtxSelect)
+        return fail(TB_ERR_UNSUPPORTED, "tb_select_bits_from_idx: ctx_cap above %d", kMaxCtxSelect);
+    return cuda_status(launch_select_bits(*dims, idx, idx_cap, count, sel_bits, (cudaStream_t)stream), __func__);
+}
+
+static tb_status attn_common(const char *fn, const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
+                             const tb_bf16 *V, const int32_t *ctx_len, float scale, float *out, void *ws,
+                             size_t ws_bytes) {
+    tb_status s;
+    if ((s = check_dims(dims, false, fn)) != TB_OK) return s;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(ctx_len) || !aligned16(out))
+        return fail(TB_ERR_INVALID_ARG, "%s: Q, K, V, ctx_len and out must be non-null and 16-byte aligned", fn);
+    if (dims->ctx_cap > kMaxCtxAttn)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", fn, dims->ctx_cap, kMaxCtxAttn);
+    if (!isfinite(scale)) return fail(TB_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+    return check_ws(ws, ws_bytes, attn_ws_bytes(*dims), fn);
+}
+
+tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
+                                const int32_t *ctx_len, int32_t sink, int32_t window,
+                                const uint32_t *sel_bits, float scale, float *out, void *ws,
+                                size_t ws_bytes, void *stream) {
+    tb_status s = attn_common(__func__, dims, Q, K, V, ctx_len, scale, out, ws, ws_bytes);
+    if (s != TB_OK) return s;
+    TB_CHECK_PTR(sel_bits);
+    if (sink < 0 || window < 1)
+        return fail(TB_ERR_INVALID_ARG, "tb_sparse_decode_attn: need sink >= 0 and window >= 1");
+    return cuda_status(launch_attn(*dims, Q, K, V, ctx_len, sink, window, sel_bits, true, scale, out, ws,
+                                   (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
+                         const int32_t *ctx_len, float scale, float *out, void *ws, size_t ws_bytes,
+                         void *stream) {
+    tb_status s = attn_common(__func__, dims, Q, K, V, ctx_len, scale, out, ws, ws_bytes);
+    if (s != TB_OK) return s;
+    return cuda_status(launch_attn(*dims, Q, K, V, ctx_len, 0, 1, nullptr, false, scale, out, ws,
+                                   (cudaStream_t)stream),
+                       __func__);
+}
+
+}  // extern "C"

@@ -1,0 +1,490 @@
+// Decode attention over the kept rows of a GQA group: sparse (sink ∪ window ∪
+// selected) and dense (all rows) share one kernel template.
+//
+// TokenButler technical summary (gist.science), "Inference strategy": the
+// cache is split into a sink (first S tokens, always kept), a local window
+// (last N tokens, always kept) and an importance buffer filled from the
+// predicted scores; "Significance": the full cache stays resident and only the
+// selected tokens are read, which is what relieves the memory-bandwidth
+// bottleneck.  The attention itself is standard scaled dot-product attention
+// restricted to those rows (fp32 logits, fp32 online softmax, fp32 sums).
+//
+// Work split: one CTA per (sequence b, KV head g, context chunk).  The CTA
+// builds the chunk's row list (sparse: union over the 4 query heads of the
+// group of their selected bits, plus sink and window rows, each row tagged
+// with a 4-bit head mask), then streams the K and V rows of that list through
+// a 3-stage cp.async pipeline in shared memory, so every (b, g, t) row crosses
+// HBM once for the whole group.  Each warp takes 8 rows of a 64-row tile; a
+// half-warp owns 4 rows and each lane 1/16 of head_dim, so every K/V element
+// a lane loads is used by all 4 query heads.  Partial dot products are summed
+// across the 16 lanes of a row by a transposing butterfly (15 shuffles for 16
+// sums), the online-softmax state is per warp, and the last CTA of each
+// (b, g) — found with an atomic ticket, never a wait — merges the chunks'
+// partial states into the fp32 output.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace tb {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kTile = 64;       // rows per pipeline stage
+constexpr int kStages = 3;
+constexpr int kGroup = 4;       // query heads per KV head
+constexpr int kMaxChunk = 2048; // context positions per CTA (upper bound)
+constexpr int kMinChunk = 256;
+constexpr int kMaxSplits = 2048;
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+struct Smem {
+    static constexpr int kStageBytes = 2 * kTile * D * 2;  // K tile + V tile, bf16
+    static constexpr int kPipe = kStages * kStageBytes;
+    static constexpr int kList = kMaxChunk * 4;
+    static constexpr int kP = kWarps * 32 * 4;
+    static constexpr int kWords = (kMaxChunk / 32) * 4;
+    static constexpr int kTotal = kPipe + kList + kP + kWords;
+    // the pipeline region is reused for the end-of-CTA combine and the merge
+    static_assert(kWarps * kGroup * (D + 2) * 4 <= kPipe, "combine scratch");
+    static_assert(kMaxSplits * kGroup * 4 <= kPipe, "merge scratch");
+};
+
+__device__ __forceinline__ float pick4(const float (&v)[4], int i) {
+    return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
+}
+__device__ __forceinline__ float comp4(const float4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// Load DPL bf16 values of one row chunk from shared memory as fp32.
+template <int DPL>
+__device__ __forceinline__ void load_chunk(const uint16_t *p, float (&f)[DPL]) {
+    if constexpr (DPL == 8) {
+        uint4 u = *reinterpret_cast<const uint4 *>(p);
+        f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+        f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+    } else {
+        uint2 u = *reinterpret_cast<const uint2 *>(p);
+        f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+    }
+}
+
+template <int D, bool SPARSE>
+__global__ void __launch_bounds__(kThreads, 2)
+attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
+            const uint16_t *__restrict__ V, const int32_t *__restrict__ ctx_len,
+            const uint32_t *__restrict__ sel_bits, int Hq, int Hkv, int Tcap, int W, int sink,
+            int window, float qscale, int chunk, int nsplit, float *__restrict__ part,
+            uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags) {
+    constexpr int DPL = D / 16;  // head_dim elements per lane
+    constexpr int CPR = D / 8;   // 16-byte chunks per row
+    constexpr int kCopies = kTile * CPR / kThreads;
+    constexpr int kPartStride = kGroup * (D + 2);
+    using S = Smem<D>;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint16_t *pipe = reinterpret_cast<uint16_t *>(smem);
+    int32_t *list = reinterpret_cast<int32_t *>(smem + S::kPipe);
+    float *pbuf = reinterpret_cast<float *>(smem + S::kPipe + S::kList);
+    int32_t *wcnt = reinterpret_cast<int32_t *>(smem + S::kPipe + S::kList + S::kP);
+    __shared__ int s_nrows, s_last;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = lane >> 4, c = lane & 15;
+    const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
+    const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
+    const int p0 = split * chunk;
+    const int p1 = min(p0 + chunk, T);
+    const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
+    const uint16_t *Kb = K + slab * D;
+    const uint16_t *Vb = V + slab * D;
+    float *part_bg = part + (size_t)(b * Hkv + g) * nsplit * kPartStride;
+
+    if (p0 < T) {
+        // ------------------------------------------------ row list (sparse)
+        int n_rows = p1 - p0;
+        if constexpr (SPARSE) {
+            const int hi_c = T - window;  // candidates are [sink, hi_c)
+            const int nwords = (p1 - p0 + 31) >> 5;
+            const int w0 = p0 >> 5;
+            const uint32_t *sb = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W + w0;
+            auto word_mask = [&](int wi, int &p, int &m) -> uint32_t {
+                uint32_t hb = lane < kGroup ? __ldg(sb + (size_t)lane * W + wi) : 0u;
+                uint32_t b0 = __shfl_sync(kFull, hb, 0), b1 = __shfl_sync(kFull, hb, 1);
+                uint32_t b2 = __shfl_sync(kFull, hb, 2), b3 = __shfl_sync(kFull, hb, 3);
+                p = p0 + (wi << 5) + lane;
+                m = 0;
+                if (p < p1) {
+                    if (p < sink || p >= hi_c) {
+                        m = 0xF;
+                    } else {
+                        m = ((b0 >> lane) & 1u) | (((b1 >> lane) & 1u) << 1) |
+                            (((b2 >> lane) & 1u) << 2) | (((b3 >> lane) & 1u) << 3);
+                    }
+                }
+                return __ballot_sync(kFull, m != 0);
+            };
+            for (int wi = warp; wi < nwords; wi += kWarps) {
+                int p, m;
+                uint32_t bal = word_mask(wi, p, m);
+                if (lane == 0) wcnt[wi] = __popc(bal);
+            }
+            __syncthreads();
+            if (warp == 0) {  // exclusive scan of <= 64 word counts
+                int a0 = (2 * lane < nwords) ? wcnt[2 * lane] : 0;
+                int a1 = (2 * lane + 1 < nwords) ? wcnt[2 * lane + 1] : 0;
+                int sum = a0 + a1, incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    int v = __shfl_up_sync(kFull, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                int excl = incl - sum;
+                if (2 * lane < nwords) wcnt[2 * lane] = excl;
+                if (2 * lane + 1 < nwords) wcnt[2 * lane + 1] = excl + a0;
+                if (lane == 31) s_nrows = incl;
+            }
+            __syncthreads();
+            for (int wi = warp; wi < nwords; wi += kWarps) {
+                int p, m;
+                uint32_t bal = word_mask(wi, p, m);
+                if (m) list[wcnt[wi] + __popc(bal & ((1u << lane) - 1u))] = (p << 4) | m;
+            }
+            __syncthreads();
+            n_rows = s_nrows;
+        }
+
+        // ------------------------------------------------ per-lane query slice
+        float q[kGroup][DPL];
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            const uint16_t *qp = Q + ((size_t)b * Hq + g * kGroup + h) * D + c * DPL;
+            if constexpr (DPL == 8) {
+                uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp));
+                q[h][0] = bf16_lo(u.x); q[h][1] = bf16_hi(u.x); q[h][2] = bf16_lo(u.y);
+                q[h][3] = bf16_hi(u.y); q[h][4] = bf16_lo(u.z); q[h][5] = bf16_hi(u.z);
+                q[h][6] = bf16_lo(u.w); q[h][7] = bf16_hi(u.w);
+            } else {
+                uint2 u = __ldg(reinterpret_cast<const uint2 *>(qp));
+                q[h][0] = bf16_lo(u.x); q[h][1] = bf16_hi(u.x); q[h][2] = bf16_lo(u.y);
+                q[h][3] = bf16_hi(u.y);
+            }
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) q[h][e] *= qscale;
+        }
+
+        float m_run[kGroup], l[kGroup], acc[kGroup][DPL];
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            m_run[h] = -INFINITY;
+            l[h] = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+        }
+
+        const int n_tiles = (n_rows + kTile - 1) / kTile;
+        const uint32_t pipe_s = smem_addr(pipe);
+
+        auto issue = [&](int t) {
+            const uint32_t kbase = pipe_s + (t % kStages) * S::kStageBytes;
+            const uint32_t vbase = kbase + kTile * D * 2;
+#pragma unroll
+            for (int k = 0; k < kCopies; ++k) {
+                const int e = tid + k * kThreads;
+                const int r = e / CPR, ch = e % CPR;
+                const int gr = t * kTile + r;
+                const bool valid = gr < n_rows;
+                int pos = p0;
+                if (valid) pos = SPARSE ? (list[gr] >> 4) : (p0 + gr);
+                const size_t off = (size_t)pos * D + ch * 8;
+                const uint32_t so = (uint32_t)(r * D + ch * 8) * 2u;
+                cp_async16(kbase + so, Kb + off, valid);
+                cp_async16(vbase + so, Vb + off, valid);
+            }
+        };
+
+#pragma unroll
+        for (int s = 0; s < kStages - 1; ++s) {
+            if (s < n_tiles) issue(s);
+            cp_async_commit();
+        }
+
+        const int rb = warp * 8 + half * 4;  // this half-warp's first row in a tile
+        for (int t = 0; t < n_tiles; ++t) {
+            cp_async_wait<kStages - 2>();
+            __syncthreads();
+            if (t + kStages - 1 < n_tiles) issue(t + kStages - 1);
+            cp_async_commit();
+
+            const uint16_t *Ks = pipe + (t % kStages) * (S::kStageBytes / 2);
+            const uint16_t *Vs = Ks + kTile * D;
+
+            // partial q.k over this lane's slice: 4 rows x 4 heads
+            float s[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float kf[DPL];
+                load_chunk<DPL>(Ks + (rb + j) * D + c * DPL, kf);
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) a = fmaf(q[h][e], kf[e], a);
+                    s[j * 4 + h] = a;
+                }
+            }
+            // transposing butterfly over the 16 lanes of a row group: lane c
+            // ends with the full sum of value c = (row c>>2, head c&3)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const bool up = c & 8;
+                float send = up ? s[k] : s[k + 8], keep = up ? s[k + 8] : s[k];
+                s[k] = keep + __shfl_xor_sync(kFull, send, 8);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const bool up = c & 4;
+                float send = up ? s[k] : s[k + 4], keep = up ? s[k + 4] : s[k];
+                s[k] = keep + __shfl_xor_sync(kFull, send, 4);
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const bool up = c & 2;
+                float send = up ? s[k] : s[k + 2], keep = up ? s[k + 2] : s[k];
+                s[k] = keep + __shfl_xor_sync(kFull, send, 2);
+            }
+            {
+                const bool up = c & 1;
+                float send = up ? s[0] : s[1], keep = up ? s[1] : s[0];
+                s[0] = keep + __shfl_xor_sync(kFull, send, 1);
+            }
+            float x = s[0];
+            const int hh = c & 3;
+            {
+                const int gr = t * kTile + rb + (c >> 2);
+                uint32_t mk = 0;
+                if (gr < n_rows) mk = SPARSE ? (uint32_t)(list[gr] & 0xF) : 0xFu;
+                if (!((mk >> hh) & 1u)) x = -INFINITY;
+            }
+            // tile max per head over the warp's 8 rows
+            float mx = x;
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+            float alpha[kGroup];
+            bool changed = false;
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                const float mt = __shfl_sync(kFull, mx, h);
+                const float mn = fmaxf(m_run[h], mt);
+                alpha[h] = (mn == m_run[h]) ? 1.f : exp2f(m_run[h] - mn);
+                changed |= (mn != m_run[h]);
+                m_run[h] = mn;
+            }
+            const float p = (x == -INFINITY) ? 0.f : exp2f(x - pick4(m_run, hh));
+            __syncwarp();
+            pbuf[warp * 32 + lane] = p;
+            __syncwarp();
+            float4 pr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                pr[j] = *reinterpret_cast<const float4 *>(pbuf + warp * 32 + half * 16 + j * 4);
+
+            if (changed) {
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    l[h] *= alpha[h];
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) acc[h][e] *= alpha[h];
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h)
+                l[h] += comp4(pr[0], h) + comp4(pr[1], h) + comp4(pr[2], h) + comp4(pr[3], h);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float vf[DPL];
+                load_chunk<DPL>(Vs + (rb + j) * D + c * DPL, vf);
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    const float ph = comp4(pr[j], h);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(ph, vf[e], acc[h][e]);
+                }
+            }
+        }
+        cp_async_wait<0>();
+        __syncthreads();
+
+        // ------------------------------------------------ combine halves, warps
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            l[h] += __shfl_xor_sync(kFull, l[h], 16);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] += __shfl_xor_sync(kFull, acc[h][e], 16);
+        }
+        float *cacc = reinterpret_cast<float *>(smem);           // [warp][head][D]
+        float *cml = cacc + kWarps * kGroup * D;                 // [warp][head][m, l]
+        if (half == 0) {
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h)
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) cacc[(warp * kGroup + h) * D + c * DPL + e] = acc[h][e];
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                cml[(warp * kGroup + h) * 2] = m_run[h];
+                cml[(warp * kGroup + h) * 2 + 1] = l[h];
+            }
+        }
+        __syncthreads();
+        float *pp = part_bg + (size_t)split * kPartStride;
+        for (int it = tid; it < kGroup * D; it += kThreads) {
+            const int h = it / D, dim = it % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cml[(w * kGroup + h) * 2]);
+            float O = 0.f, L = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    const float mw = cml[(w * kGroup + h) * 2];
+                    if (mw != -INFINITY) {
+                        const float f = exp2f(mw - M);
+                        O = fmaf(cacc[(w * kGroup + h) * D + dim], f, O);
+                        L = fmaf(cml[(w * kGroup + h) * 2 + 1], f, L);
+                    }
+                }
+            }
+            pp[h * (D + 2) + dim] = O;
+            if (dim == 0) {
+                pp[h * (D + 2) + D] = M;
+                pp[h * (D + 2) + D + 1] = L;
+            }
+        }
+    }
+
+    // ---------------------------------------------------- last CTA merges
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned prev = atomicAdd(&counters[b * Hkv + g], 1u);
+        s_last = (prev == (unsigned)nsplit - 1u);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    const int ns = (T + chunk - 1) / chunk;  // chunks that hold rows
+    float *wsm = reinterpret_cast<float *>(smem);  // [ns][head] merge weights
+    if (warp < kGroup) {
+        const int h = warp;
+        float M = -INFINITY;
+        for (int s = lane; s < ns; s += 32)
+            M = fmaxf(M, __ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + D));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+        float L = 0.f;
+        for (int s = lane; s < ns; s += 32) {
+            const float ms = __ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + D);
+            const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+            wsm[s * kGroup + h] = f;
+            L = fmaf(f, __ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + D + 1), L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        for (int s = lane; s < ns; s += 32) wsm[s * kGroup + h] *= inv;
+    }
+    __syncthreads();
+    for (int it = tid; it < kGroup * D; it += kThreads) {
+        const int h = it / D, dim = it % D;
+        float O = 0.f;
+        for (int s = 0; s < ns; ++s)
+            O = fmaf(__ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + dim), wsm[s * kGroup + h], O);
+        out[((size_t)b * Hq + g * kGroup + h) * D + dim] = O;
+    }
+    if (tid == 0) counters[b * Hkv + g] = 0u;  // leave the ticket zeroed for the next call
+}
+
+int g_num_sms = 0;
+
+int num_sms() {
+    if (g_num_sms == 0) {
+        int dev = 0, n = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            g_num_sms = n;
+        else
+            g_num_sms = 148;
+    }
+    return g_num_sms;
+}
+
+template <int D, bool SPARSE>
+cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                     const int32_t *ctx_len, int32_t sink, int32_t window, const uint32_t *sel_bits,
+                     float scale, float *out, void *ws, cudaStream_t st) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, SPARSE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Smem<D>::kTotal);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int chunk = attn_chunk(d);
+    const int nsplit = (d.ctx_cap + chunk - 1) / chunk;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    uint32_t *flags = reinterpret_cast<uint32_t *>(w);
+    uint32_t *counters = reinterpret_cast<uint32_t *>(w + kWsHeaderBytes);
+    float *part = reinterpret_cast<float *>(
+        w + kWsHeaderBytes + align_up((size_t)d.batch * d.n_kv_heads * 4, 256));
+    const int W = (d.ctx_cap + 31) / 32;
+    const float qscale = scale * 1.4426950408889634f;  // logits in log2 units for exp2
+    dim3 grid(nsplit, d.n_kv_heads, d.batch);
+    attn_kernel<D, SPARSE><<<grid, kThreads, Smem<D>::kTotal, st>>>(
+        Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, qscale,
+        chunk, nsplit, part, counters, out, flags);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Context positions per CTA: the largest power of two in [256, 2048] that
+// still gives at least three waves of two CTAs per SM.
+int attn_chunk(const tb_dims &d) {
+    const long long slots = 2LL * num_sms();
+    int chunk = kMaxChunk;
+    while (chunk > kMinChunk) {
+        const long long ctas = (long long)d.batch * d.n_kv_heads * ((d.ctx_cap + chunk - 1) / chunk);
+        if (ctas >= 3 * slots) break;
+        chunk >>= 1;
+    }
+    while ((d.ctx_cap + chunk - 1) / chunk > kMaxSplits && chunk < kMaxChunk) chunk <<= 1;
+    return chunk;
+}
+
+size_t attn_ws_bytes(const tb_dims &d) {
+    const size_t max_splits = (size_t)(d.ctx_cap + kMinChunk - 1) / kMinChunk;
+    return kWsHeaderBytes + align_up((size_t)d.batch * d.n_kv_heads * 4, 256) +
+           (size_t)d.batch * d.n_kv_heads * max_splits * kGroup * (d.head_dim + 2) * 4;
+}
+
+cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                        const int32_t *ctx_len, int32_t sink, int32_t window,
+                        const uint32_t *sel_bits, bool sparse, float scale, float *out, void *ws,
+                        cudaStream_t st) {
+    if (d.head_dim == 128) {
+        return sparse ? launch_t<128, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st)
+                      : launch_t<128, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st);
+    }
+    return sparse ? launch_t<64, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st)
+                  : launch_t<64, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st);
+}
+
+}  // namespace tb

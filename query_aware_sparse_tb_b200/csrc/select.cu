@@ -1,0 +1,475 @@
+// Importance scoring and budgeted top-B selection with neighbour fetch.
+//
+// TokenButler technical summary (gist.science), "Core architecture: scoring":
+// the predicted queries are dot-multiplied with the projected keys to give
+// cheap per-token importance scores, which drive a dynamic token selection
+// under a fixed budget.  "Inference strategy": the first S tokens (sink) and
+// the last N tokens (local window) are always kept, so the candidates are
+// C = [S, T-N).  "Optimisations: prediction interval and neighbour fetch": the
+// selected tokens are expanded by their spatial neighbours.
+//
+// Exact top-B on the fp32 scores, ties broken by the lower position:
+//   1. score_hist   one CTA per (b, KV head, 1024 positions): reads each K'
+//                   row once for the 4 query heads of the group, writes the
+//                   order-preserving uint32 image of every score, and builds
+//                   a histogram of its top 11 bits per query head.  The last
+//                   CTA of each (b, KV head) (atomic ticket, no waiting) finds
+//                   the bin that holds the B-th largest key.
+//   2. mark_collect same grid: keys above that bin become bits of the Top
+//                   bitmap; keys inside it go to a per-head candidate list.
+//   3. finalize     one CTA per (b, query head): two more 11/10-bit radix
+//                   passes over the candidate list fix the B-th key exactly,
+//                   ties on it are taken in position order, and the Top bitmap
+//                   is dilated by +-nbr, clipped to C, and written out both as
+//                   the bitmap and as the sorted index list.
+#include "common.cuh"
+#include "internal.h"
+
+namespace tb {
+namespace {
+
+constexpr int kGroup = 4;
+constexpr int kChunk = 1024;          // positions per CTA in the streaming kernels
+constexpr int kThreads = 256;
+constexpr int kBins1 = 2048;          // key bits 31..21
+constexpr int kBins2 = 2048;          // key bits 20..10
+constexpr int kBins3 = 1024;          // key bits 9..0
+constexpr int kFinThreads = 1024;
+constexpr unsigned kFull = 0xffffffffu;
+
+enum : uint32_t { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
+
+struct HeadState {   // 8 words per (b, query head)
+    uint32_t mode, b1, k_rem, cand_count, n_in_bin, pad[3];
+};
+
+struct SelWs {
+    uint32_t *flags, *keys, *hist, *counters;
+    HeadState *state;
+    unsigned long long *cand;
+    uint32_t *top;
+};
+
+SelWs carve(const tb_dims &d, void *ws) {
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    const size_t rows = (size_t)d.batch * d.n_q_heads;
+    SelWs s;
+    size_t off = 0;
+    s.flags = reinterpret_cast<uint32_t *>(p);
+    off += kWsHeaderBytes;
+    s.keys = reinterpret_cast<uint32_t *>(p + off);
+    off += align_up(rows * d.ctx_cap * 4, 256);
+    s.hist = reinterpret_cast<uint32_t *>(p + off);
+    off += align_up(rows * kBins1 * 4, 256);
+    s.state = reinterpret_cast<HeadState *>(p + off);
+    off += align_up(rows * sizeof(HeadState), 256);
+    s.counters = reinterpret_cast<uint32_t *>(p + off);
+    off += align_up((size_t)d.batch * d.n_kv_heads * 4, 256);
+    s.cand = reinterpret_cast<unsigned long long *>(p + off);
+    off += align_up(rows * d.ctx_cap * 8, 256);
+    s.top = reinterpret_cast<uint32_t *>(p + off);
+    return s;
+}
+
+size_t carve_bytes(const tb_dims &d) {
+    const size_t rows = (size_t)d.batch * d.n_q_heads;
+    const size_t W = (d.ctx_cap + 31) / 32;
+    return kWsHeaderBytes + align_up(rows * d.ctx_cap * 4, 256) + align_up(rows * kBins1 * 4, 256) +
+           align_up(rows * sizeof(HeadState), 256) + align_up((size_t)d.batch * d.n_kv_heads * 4, 256) +
+           align_up(rows * d.ctx_cap * 8, 256) + align_up(rows * W * 4, 256);
+}
+
+// Walk `nbins` histogram bins from the highest down (one warp) and find the bin
+// in which the running count reaches `need`.  Returns the bin; *rem receives
+// how many keys of that bin are still needed.
+__device__ int find_bin_desc(const uint32_t *hist, int nbins, uint32_t need, uint32_t *rem,
+                             bool cg) {
+    const int lane = threadIdx.x & 31;
+    for (int base = nbins - 1; base >= 0; base -= 32) {
+        const int bin = base - lane;
+        const uint32_t v = bin >= 0 ? (cg ? __ldcg(hist + bin) : hist[bin]) : 0u;
+        uint32_t incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const uint32_t total = __shfl_sync(kFull, incl, 31);
+        if (need <= total) {
+            const uint32_t hit = __ballot_sync(kFull, incl >= need);
+            const int L = __ffs(hit) - 1;
+            const uint32_t vL = __shfl_sync(kFull, v, L);
+            const uint32_t iL = __shfl_sync(kFull, incl, L);
+            *rem = need - (iL - vL);
+            return base - L;
+        }
+        need -= total;
+    }
+    *rem = 0;
+    return 0;
+}
+
+// ------------------------------------------------------------------ kernel 1
+
+template <int DP>
+__global__ void __launch_bounds__(kThreads)
+score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
+                  const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
+                  int window, int budget, SelWs ws) {
+    __shared__ float qs[kGroup][DP];
+    __shared__ uint32_t hist[kGroup][kBins1];
+    __shared__ int s_last;
+    const int tid = threadIdx.x;
+    const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
+    const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
+    const int lo = sink, hi = T - window;
+    const int p0 = ch * kChunk;
+
+    for (int i = tid; i < kGroup * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
+    if (tid < kGroup * DP) (&qs[0][0])[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
+    __syncthreads();
+
+    const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
+#pragma unroll
+    for (int k = 0; k < kChunk / kThreads; ++k) {
+        const int p = p0 + k * kThreads + tid;
+        if (p >= lo && p < hi) {
+            const uint4 *row = reinterpret_cast<const uint4 *>(Kp + (slab + p) * DP);
+            float kf[DP];
+#pragma unroll
+            for (int v = 0; v < DP / 8; ++v) {
+                const uint4 u = __ldg(row + v);
+                kf[8 * v + 0] = bf16_lo(u.x); kf[8 * v + 1] = bf16_hi(u.x);
+                kf[8 * v + 2] = bf16_lo(u.y); kf[8 * v + 3] = bf16_hi(u.y);
+                kf[8 * v + 4] = bf16_lo(u.z); kf[8 * v + 5] = bf16_hi(u.z);
+                kf[8 * v + 6] = bf16_lo(u.w); kf[8 * v + 7] = bf16_hi(u.w);
+            }
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < DP; ++j) s = fmaf(qs[h][j], kf[j], s);
+                const uint32_t key = score_key(s);
+                ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
+                atomicAdd(&hist[h][key >> 21], 1u);
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < kGroup * kBins1; i += kThreads) {
+        const uint32_t v = (&hist[0][0])[i];
+        if (v) atomicAdd(ws.hist + ((size_t)b * Hq + g * kGroup + i / kBins1) * kBins1 + (i % kBins1), v);
+    }
+
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(ws.counters + b * Hkv + g, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < kGroup) {
+        const size_t row = (size_t)b * Hq + g * kGroup + warp;
+        uint32_t *gh = ws.hist + row * kBins1;
+        const int nC = hi > lo ? hi - lo : 0;
+        HeadState st = {};
+        if (nC == 0) {
+            st.mode = kModeEmpty;
+        } else if (nC <= budget) {
+            st.mode = kModeAll;
+        } else {
+            uint32_t rem;
+            const int bin = find_bin_desc(gh, kBins1, (uint32_t)budget, &rem, true);
+            st.mode = kModeSelect;
+            st.b1 = (uint32_t)bin;
+            st.k_rem = rem;
+            st.n_in_bin = __ldcg(gh + bin);
+        }
+        __syncwarp();
+        for (int i = lane; i < kBins1; i += 32) gh[i] = 0u;  // leave zeroed for the next call
+        if (lane == 0) ws.state[row] = st;
+    }
+    if (tid == 0) ws.counters[b * Hkv + g] = 0u;
+}
+
+// ------------------------------------------------------------------ kernel 2
+
+__global__ void __launch_bounds__(kThreads)
+mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int W,
+                    int sink, int window, SelWs ws) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
+    const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, false);
+    const int lo = sink, hi = T - window;
+    const int w0 = ch * (kChunk / 32);
+
+    uint32_t mode[kGroup], b1[kGroup];
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) {
+        const HeadState &st = ws.state[(size_t)b * Hq + g * kGroup + h];
+        mode[h] = st.mode;
+        b1[h] = st.b1;
+    }
+    for (int wi = warp; wi < kChunk / 32; wi += kThreads / 32) {
+        const int w = w0 + wi;
+        if (w >= W) break;
+        const int p = (w << 5) + lane;
+        const bool in_c = p >= lo && p < hi;
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            const size_t row = (size_t)b * Hq + g * kGroup + h;
+            uint32_t key = 0;
+            if (in_c && mode[h] == kModeSelect) key = ws.keys[row * Tcap + p];
+            const uint32_t d1 = key >> 21;
+            const bool top = in_c && (mode[h] == kModeAll || (mode[h] == kModeSelect && d1 > b1[h]));
+            const bool cand = in_c && mode[h] == kModeSelect && d1 == b1[h];
+            const uint32_t tb = __ballot_sync(kFull, top);
+            if (lane == 0) ws.top[row * W + w] = tb;
+            const uint32_t cb = __ballot_sync(kFull, cand);
+            if (cb) {
+                const int leader = __ffs(cb) - 1;
+                uint32_t base = 0;
+                if (lane == leader) base = atomicAdd(&ws.state[row].cand_count, (uint32_t)__popc(cb));
+                base = __shfl_sync(kFull, base, leader);
+                if (cand)
+                    ws.cand[row * Tcap + base + __popc(cb & ((1u << lane) - 1u))] =
+                        ((unsigned long long)key << 32) | (uint32_t)p;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ kernel 3
+
+// Exclusive prefix sum over the block (1024 threads); *total gets the sum.
+__device__ int block_excl_scan(int v, int *scratch, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = scratch[lane];
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(kFull, wi, o);
+            if (lane >= o) wi += t;
+        }
+        scratch[lane] = wi - w;
+        if (lane == 31) scratch[32] = wi;
+    }
+    __syncthreads();
+    const int res = scratch[warp] + incl - v;
+    *total = scratch[32];
+    __syncthreads();
+    return res;
+}
+
+__device__ __forceinline__ uint32_t range_mask(int w, int lo, int hi) {
+    if (hi <= lo) return 0u;
+    const int start = max(lo - (w << 5), 0), end = min(hi - (w << 5), 32);
+    if (end <= start) return 0u;
+    const uint32_t upto = end == 32 ? 0xffffffffu : ((1u << end) - 1u);
+    return upto & ~((1u << start) - 1u);
+}
+
+__global__ void __launch_bounds__(kFinThreads)
+finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int sink, int window,
+                int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
+                uint32_t *__restrict__ sel_bits, SelWs ws) {
+    extern __shared__ uint32_t fsm[];
+    uint32_t *top_s = fsm;       // [W]
+    uint32_t *tie_s = fsm + W;   // [W]
+    __shared__ uint32_t hist[kBins2];
+    __shared__ int scratch[33];
+    __shared__ uint32_t s_bin, s_rem;
+
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t row = (size_t)b * Hq + h;
+    const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, false);
+    const int lo = sink, hi = T - window;
+    const HeadState st = ws.state[row];
+
+    for (int w = tid; w < W; w += kFinThreads) {
+        top_s[w] = ws.top[row * W + w];
+        tie_s[w] = 0u;
+    }
+    if (st.mode == kModeSelect) {
+        const unsigned long long *cand = ws.cand + row * Tcap;
+        const int n = (int)st.cand_count;
+        // digit 2: key bits 20..10 inside bin b1
+        for (int i = tid; i < kBins2; i += kFinThreads) hist[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < n; i += kFinThreads) {
+            const uint32_t key = (uint32_t)(cand[i] >> 32);
+            atomicAdd(&hist[(key >> 10) & 0x7FFu], 1u);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            uint32_t rem;
+            const int bin = find_bin_desc(hist, kBins2, st.k_rem, &rem, false);
+            if (tid == 0) { s_bin = bin; s_rem = rem; }
+        }
+        __syncthreads();
+        const uint32_t b2 = s_bin, k2 = s_rem;
+        // digit 3: key bits 9..0 inside (b1, b2)
+        for (int i = tid; i < kBins3; i += kFinThreads) hist[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < n; i += kFinThreads) {
+            const uint32_t key = (uint32_t)(cand[i] >> 32);
+            if (((key >> 10) & 0x7FFu) == b2) atomicAdd(&hist[key & 0x3FFu], 1u);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            uint32_t rem;
+            const int bin = find_bin_desc(hist, kBins3, k2, &rem, false);
+            if (tid == 0) { s_bin = bin; s_rem = rem; }
+        }
+        __syncthreads();
+        const uint32_t tau = (st.b1 << 21) | (b2 << 10) | s_bin;
+        const uint32_t k3 = s_rem;  // keys equal to tau still to take, lowest positions first
+        for (int i = tid; i < n; i += kFinThreads) {
+            const unsigned long long e = cand[i];
+            const uint32_t key = (uint32_t)(e >> 32), p = (uint32_t)e;
+            if (key > tau) atomicOr(&top_s[p >> 5], 1u << (p & 31));
+            else if (key == tau) atomicOr(&tie_s[p >> 5], 1u << (p & 31));
+        }
+        __syncthreads();
+        // ties in position order: each thread owns a contiguous run of words
+        const int wpt = (W + kFinThreads - 1) / kFinThreads;
+        const int wb = tid * wpt, we = min(wb + wpt, W);
+        int mine = 0;
+        for (int w = wb; w < we; ++w) mine += __popc(tie_s[w]);
+        int tot;
+        int before = block_excl_scan(mine, scratch, &tot);
+        for (int w = wb; w < we; ++w) {
+            uint32_t t = tie_s[w];
+            const int pc = __popc(t);
+            uint32_t keep = 0u;
+            if (before + pc <= (int)k3) {
+                keep = t;
+            } else if (before < (int)k3) {
+                for (int k = 0; k < (int)k3 - before; ++k) {
+                    const uint32_t low = t & (0u - t);
+                    keep |= low;
+                    t ^= low;
+                }
+            }
+            top_s[w] |= keep;
+            before += pc;
+        }
+    }
+    __syncthreads();
+
+    // neighbour fetch, clip to C, emit bitmap and sorted index list
+    const int wpt = (W + kFinThreads - 1) / kFinThreads;
+    const int wb = tid * wpt, we = min(wb + wpt, W);
+    int mine = 0;
+    for (int w = wb; w < we; ++w) {
+        const uint32_t t = top_s[w];
+        const uint32_t pv = w > 0 ? top_s[w - 1] : 0u, nx = w + 1 < W ? top_s[w + 1] : 0u;
+        uint32_t e = t;
+        for (int k = 1; k <= nbr; ++k) e |= (t << k) | (pv >> (32 - k)) | (t >> k) | (nx << (32 - k));
+        e &= range_mask(w, lo, hi);
+        tie_s[w] = e;  // reuse as the output bitmap
+        mine += __popc(e);
+    }
+    int total;
+    int base = block_excl_scan(mine, scratch, &total);
+    int32_t *out = idx + row * (size_t)idx_cap;
+    for (int w = wb; w < we; ++w) {
+        uint32_t e = tie_s[w];
+        sel_bits[row * W + w] = e;
+        while (e) {
+            const int bit = __ffs(e) - 1;
+            e &= e - 1u;
+            if (base < idx_cap) out[base] = (w << 5) + bit;
+            ++base;
+        }
+    }
+    if (tid == 0) {
+        if (total > idx_cap) raise_flag(ws.flags, TB_FLAG_IDX_OVERFLOW);
+        count[row] = total < idx_cap ? total : idx_cap;
+    }
+}
+
+// ------------------------------------------------------ bitmap from indices
+
+__global__ void __launch_bounds__(kFinThreads)
+bits_from_idx_kernel(const int32_t *__restrict__ idx, int idx_cap, const int32_t *__restrict__ count,
+                     int Hq, int Tcap, int W, uint32_t *__restrict__ sel_bits) {
+    extern __shared__ uint32_t bsm[];
+    const int tid = threadIdx.x;
+    const size_t row = (size_t)blockIdx.y * Hq + blockIdx.x;
+    for (int w = tid; w < W; w += kFinThreads) bsm[w] = 0u;
+    __syncthreads();
+    int n = count[row];
+    n = n < 0 ? 0 : (n > idx_cap ? idx_cap : n);
+    for (int i = tid; i < n; i += kFinThreads) {
+        const int t = idx[row * idx_cap + i];
+        if (t >= 0 && t < Tcap) atomicOr(&bsm[t >> 5], 1u << (t & 31));
+    }
+    __syncthreads();
+    for (int w = tid; w < W; w += kFinThreads) sel_bits[row * W + w] = bsm[w];
+}
+
+}  // namespace
+
+size_t select_ws_bytes(const tb_dims &d) { return carve_bytes(d); }
+
+cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_stride,
+                                const uint16_t *Kp, const int32_t *ctx_len, int32_t sink,
+                                int32_t window, int32_t budget, int32_t nbr, int32_t *idx,
+                                int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
+                                cudaStream_t st) {
+    const SelWs s = carve(d, ws);
+    const int W = (d.ctx_cap + 31) / 32;
+    const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
+    dim3 grid(nch, d.n_kv_heads, d.batch);
+    if (d.d_proj == 32)
+        score_hist_kernel<32><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
+                                                         d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    else
+        score_hist_kernel<16><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
+                                                         d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mark_collect_kernel<<<grid, kThreads, 0, st>>>(ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W,
+                                                   sink, window, s);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t fsm = (size_t)2 * W * 4;
+    static size_t configured = 0;
+    if (fsm > 48 * 1024 && fsm > configured) {
+        e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
+        if (e != cudaSuccess) return e;
+        configured = fsm;
+    }
+    finalize_kernel<<<dim3(d.n_q_heads, d.batch), kFinThreads, fsm, st>>>(
+        ctx_len, d.n_q_heads, d.ctx_cap, W, sink, window, nbr, idx, idx_cap, count, sel_bits, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx_cap,
+                               const int32_t *count, uint32_t *sel_bits, cudaStream_t st) {
+    const int W = (d.ctx_cap + 31) / 32;
+    const size_t sm = (size_t)W * 4;
+    static size_t configured = 0;
+    if (sm > 48 * 1024 && sm > configured) {
+        cudaError_t e = cudaFuncSetAttribute(bits_from_idx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        configured = sm;
+    }
+    bits_from_idx_kernel<<<dim3(d.n_q_heads, d.batch), kFinThreads, sm, st>>>(
+        idx, idx_cap, count, d.n_q_heads, d.ctx_cap, W, sel_bits);
+    return cudaGetLastError();
+}
+
+}  // namespace tb

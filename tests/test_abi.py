@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/tb.h declares, sizes workspaces, and rejects bad arguments on the host
+before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch  # noqa: F401  (loads the CUDA runtime libtb links against)
+
+from query_aware_sparse_tb_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tb.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tb_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_match_header(lib):
+    declared = _declared()
+    assert declared, "no declarations found"
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in tb.h but not exported"
+    assert sorted(_lib.EXPORTS) == declared
+
+
+def test_version_and_strings(lib):
+    assert lib.tb_abi_version() == 1
+    assert lib.tb_status_str(0) == b"TB_OK"
+    assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
+
+
+def _d(**kw):
+    base = dict(batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128, d_proj=32, ctx_cap=65792)
+    base.update(kw)
+    return _lib.TbDims(*[base[k] for k in ("batch", "n_q_heads", "n_kv_heads", "head_dim", "d_proj", "ctx_cap")])
+
+
+def test_workspace_sizes(lib):
+    d = _d()
+    a = lib.tb_attn_workspace_bytes(ctypes.byref(d))
+    s = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
+    assert a > 256 and s > 256
+    # selection workspace holds at least keys (4 B) + candidates (8 B) per (head, position)
+    assert s >= 32 * 65792 * 12
+    assert lib.tb_attn_workspace_bytes(ctypes.byref(_d(head_dim=96))) == 0
+    assert lib.tb_score_select_workspace_bytes(ctypes.byref(_d(d_proj=24))) == 0
+    assert lib.tb_score_select_workspace_bytes(ctypes.byref(_d(ctx_cap=(1 << 19) + 1))) == 0
+    assert lib.tb_predict_queries_workspace_bytes(1, 4096, 1024, 4096) > 0
+    assert lib.tb_predict_queries_workspace_bytes(17, 4096, 1024, 4096) == 0
+    assert lib.tb_project_keys_workspace_bytes() == 256
+
+
+FAKE = 1 << 20          # 16-byte aligned, never dereferenced: validation fails first
+MIS = FAKE + 8          # misaligned
+
+
+def test_attention_rejects_bad_arguments(lib):
+    d = _d()
+    ws_bytes = lib.tb_attn_workspace_bytes(ctypes.byref(d))
+    ok_args = dict(Q=FAKE, K=FAKE, V=FAKE, ctx=FAKE, out=FAKE, ws=FAKE)
+
+    def call(dims, **kw):
+        a = dict(ok_args, **kw)
+        return lib.tb_decode_attn(ctypes.byref(dims), a["Q"], a["K"], a["V"], a["ctx"], 0.088, a["out"],
+                                  a["ws"], kw.get("ws_bytes", ws_bytes), None)
+
+    assert call(_d(head_dim=96)) == _lib.TB_ERR_UNSUPPORTED
+    assert b"head_dim" in lib.tb_last_error()
+    assert call(_d(n_q_heads=24)) == _lib.TB_ERR_UNSUPPORTED           # group of 3
+    assert call(_d(n_q_heads=30)) == _lib.TB_ERR_INVALID_ARG           # not a multiple
+    assert call(d, Q=0) == _lib.TB_ERR_INVALID_ARG
+    assert call(d, K=MIS) == _lib.TB_ERR_INVALID_ARG
+    assert call(d, ws_bytes=ws_bytes - 1) == _lib.TB_ERR_WORKSPACE
+    assert call(_d(batch=0)) == _lib.TB_ERR_INVALID_ARG
+    st = lib.tb_sparse_decode_attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16, 0, FAKE, 0.088, FAKE, FAKE,
+                                   ws_bytes, None)
+    assert st == _lib.TB_ERR_INVALID_ARG and b"window" in lib.tb_last_error()
+    st = lib.tb_sparse_decode_attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16, 64, 0, 0.088, FAKE, FAKE,
+                                   ws_bytes, None)
+    assert st == _lib.TB_ERR_INVALID_ARG
+
+
+def test_select_rejects_bad_arguments(lib):
+    d = _d()
+    wsb = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
+
+    def call(dims=d, stride=32 * 32, sink=16, window=64, budget=8192, nbr=1, idx_cap=3 * 8192, ws_bytes=wsb):
+        return lib.tb_score_select(ctypes.byref(dims), FAKE, stride, FAKE, FAKE, sink, window, budget, nbr, FAKE,
+                                   idx_cap, FAKE, FAKE, FAKE, ws_bytes, None)
+
+    assert call(idx_cap=3 * 8192 - 1) == _lib.TB_ERR_INVALID_ARG
+    assert b"idx_cap" in lib.tb_last_error()
+    assert call(nbr=17) == _lib.TB_ERR_INVALID_ARG
+    assert call(budget=0) == _lib.TB_ERR_INVALID_ARG
+    assert call(sink=-1) == _lib.TB_ERR_INVALID_ARG
+    assert call(stride=31 * 32) == _lib.TB_ERR_INVALID_ARG
+    assert call(dims=_d(d_proj=8)) == _lib.TB_ERR_UNSUPPORTED
+    assert call(ws_bytes=wsb // 2) == _lib.TB_ERR_WORKSPACE
+    # small contexts: idx_cap may be ctx_cap when that is below (2*nbr+1)*budget
+    small = _d(ctx_cap=300)
+    w2 = lib.tb_score_select_workspace_bytes(ctypes.byref(small))
+    st = lib.tb_score_select(ctypes.byref(small), FAKE, 32 * 32, FAKE, FAKE, 4, 16, 8192, 1, FAKE, 299,
+                             FAKE, FAKE, FAKE, w2, None)
+    assert st == _lib.TB_ERR_INVALID_ARG
+
+
+def test_predict_and_project_reject_bad_arguments(lib):
+    wsb = lib.tb_predict_queries_workspace_bytes(1, 4096, 1024, 4096)
+    assert lib.tb_predict_queries(FAKE, FAKE, FAKE, FAKE, 17, 4096, 1024, 4096, FAKE, wsb, None) == \
+        _lib.TB_ERR_UNSUPPORTED
+    assert lib.tb_predict_queries(FAKE, FAKE, FAKE, FAKE, 1, 4000, 1024, 4096, FAKE, wsb, None) == \
+        _lib.TB_ERR_UNSUPPORTED
+    assert lib.tb_predict_queries(FAKE, MIS, FAKE, FAKE, 1, 4096, 1024, 4096, FAKE, wsb, None) == \
+        _lib.TB_ERR_INVALID_ARG
+    assert lib.tb_predict_queries(FAKE, FAKE, FAKE, FAKE, 1, 4096, 1024, 4096, FAKE, wsb - 1, None) == \
+        _lib.TB_ERR_WORKSPACE
+    d = _d()
+    assert lib.tb_project_keys(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, -1, FAKE, 256, None) == \
+        _lib.TB_ERR_INVALID_ARG
+    assert lib.tb_project_keys(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, 256, None) == _lib.TB_OK
+    assert lib.tb_project_keys(ctypes.byref(_d(d_proj=64)), FAKE, FAKE, FAKE, FAKE, FAKE, 64, FAKE, 256, None) \
+        == _lib.TB_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_host_tensors(lib):
+    d = _d(ctx_cap=128)
+    t = torch.zeros(16, dtype=torch.bfloat16)
+    with pytest.raises(_lib.TbError):
+        _lib.decode_attn(d, t, t, t, torch.zeros(1, dtype=torch.int32), 0.1, torch.zeros(4), t)
