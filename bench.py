@@ -1,0 +1,588 @@
+#!/usr/bin/env python
+"""Benchmark of the TokenButler sparse decode path on B200.
+
+One bench step = one full decode run of the workload (llama64k: 32 layers,
+64K context, 256 decode steps with a prediction every 16 steps, producer every
+4 layers, key projection every 64 tokens), replayed as one CUDA graph on
+inputs already resident in HBM.  The same run is timed for the dense decode
+kernel (the comparator) and end to end (per-step host->device copies of the
+step's queries, new K/V rows and producer hidden states, and a device->host
+copy of the step's outputs, all inside the graph).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference      # the CPU oracle on a bounded sample
+
+Under torchrun every rank decodes its own independent replica (its own seeded
+sequences): weak scaling, no collective on the data path; the barrier and the
+max-over-ranks reduction of the device time use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import tb_inputs  # noqa: E402
+from query_aware_sparse_tb_b200 import _lib as L  # noqa: E402
+from query_aware_sparse_tb_b200.decode import (DecodeShape, SparseDecoder, is_prediction_step,  # noqa: E402
+                                              memcpy2d_async, record_event)
+
+HBM_NOMINAL_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+ROW_BYTES_PER_DIM = 2 * 2      # K and V, bf16
+
+
+# ----------------------------------------------------------------------------
+# workload on the device
+# ----------------------------------------------------------------------------
+
+class Run:
+    """All device buffers of one workload replica plus its decoder."""
+
+    def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None):
+        self.w = w
+        self.device = device
+        self.steps = steps or w.steps
+        self.ctx0 = w.ctx0_per_seq()
+        nL = w.n_layers
+        self.K, self.V, self.Wk = [], [], []
+        for l in range(nL):
+            K, V = tb_inputs.kv_layer(w, l, device)
+            self.K.append(K)
+            self.V.append(V)
+            self.Wk.append(tb_inputs.wk_layer(w, l, device))
+        stride = w.producer_stride if w.hidden > 0 else 1
+        self.producers = [l for l in range(nL) if l % stride == 0]
+        self.mlp = {p: tb_inputs.mlp_weights(w, p, device) for p in self.producers} if w.hidden > 0 else {}
+        self.Q = torch.stack([torch.stack([tb_inputs.query(w, i, l, device) for l in range(nL)])
+                              for i in range(self.steps)])                       # [steps][L][B][Hq][d]
+        self.n_pred = (self.steps + w.interval - 1) // w.interval
+        if w.hidden > 0:
+            self.h = torch.stack([torch.stack([tb_inputs.hidden_state(w, k, p, device) for p in self.producers])
+                                  for k in range(self.n_pred)])                   # [npred][nprod][B][hidden]
+            self.qp_direct = None
+        else:
+            self.h = None
+            self.qp_direct = torch.stack([torch.stack([tb_inputs.direct_qp(w, k, l, device) for l in range(nL)])
+                                          for k in range(self.n_pred)])          # [npred][L][B][Hq][d']
+        self.shape = DecodeShape(batch=w.batch, n_layers=nL, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                                 head_dim=w.head_dim, d_proj=w.d_proj, hidden=w.hidden, inter=w.inter,
+                                 stride=stride, sink=w.sink, window=w.window, budget=w.budget, nbr=w.nbr,
+                                 interval=w.interval, ctx_cap=w.ctx_cap)
+        self.dec = SparseDecoder(self.shape, self.K, self.V, self.Wk, self.mlp, self.ctx0, self.steps, device)
+        self.out = torch.zeros(nL, w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=device)
+
+    def step_inputs(self, i):
+        k = i // self.w.interval
+        h = self.h[k] if self.h is not None else None
+        qd = self.qp_direct[k] if self.qp_direct is not None else None
+        return self.Q[i], h, qd
+
+    def run_sparse(self, stream=None, marks=None):
+        for i in range(self.steps):
+            Q, h, qd = self.step_inputs(i)
+            self.dec.step(i, Q, self.out, h=h, qp_direct=qd, stream=stream,
+                          marks=(lambda name, i=i: marks(name, i)) if marks else None)
+
+    def run_dense(self, stream=None, marks=None):
+        for i in range(self.steps):
+            self.dec.dense_step(i, self.Q[i], self.out, stream=stream,
+                                marks=(lambda name, i=i: marks(name, i)) if marks else None)
+
+    # ------------------------------------------------------------ accounting
+    def launches(self):
+        """(sparse kernel launches, dense kernel launches) of one run."""
+        nL = self.w.n_layers
+        n_proj = len(self.dec.proj_steps)
+        sel = 3 * nL * self.n_pred
+        pred = 4 * len(self.producers) * self.n_pred if self.w.hidden > 0 else 0
+        return self.steps * nL + sel + pred + n_proj * nL, self.steps * nL
+
+    def union_rows(self):
+        """Kept (b, kv-head, t) rows of every sparse attention launch of one run,
+        counting a row once for the 4 query heads of its group: sink + window +
+        |OR of the group's selected bits|.  Runs the schedule once, eagerly."""
+        w, dec = self.w, self.dec
+        lut = torch.tensor([bin(x).count("1") for x in range(256)], dtype=torch.int64, device=self.device)
+        rows = torch.zeros(self.steps, w.n_layers, dtype=torch.int64)
+        sel_sizes = torch.zeros(self.steps, w.n_layers, dtype=torch.int64)
+        cand = torch.zeros(self.steps, dtype=torch.int64)
+        union = None
+        isets = None
+        for i in range(self.steps):
+            Q, h, qd = self.step_inputs(i)
+            dec.step(i, Q, self.out, h=h, qp_direct=qd)
+            if is_prediction_step(i, w.interval):
+                u = []
+                s_ = []
+                for l in range(w.n_layers):
+                    b = dec.bits[l].view(w.batch, w.n_kv_heads, w.group, -1)
+                    orb = b[:, :, 0] | b[:, :, 1] | b[:, :, 2] | b[:, :, 3]
+                    u.append(lut[orb.contiguous().view(torch.uint8).long()].sum())
+                    s_.append(dec.cnt[l].sum())
+                union = torch.stack(u).cpu()
+                isets = torch.stack(s_).cpu()
+            T = [t + i + 1 for t in self.ctx0]
+            keep = sum(min(w.sink, t) + (t - max(w.sink, t - w.window)) for t in T) * w.n_kv_heads
+            rows[i] = union + keep
+            sel_sizes[i] = isets
+            cand[i] = sum(max(0, t - w.window - w.sink) for t in T)
+        torch.cuda.synchronize()
+        return rows, sel_sizes, cand
+
+    def bytes_model(self):
+        """Algorithmic HBM bytes of one run (the sum over decode steps of the
+        per-step formula): sparse path, its attention part, dense path."""
+        w = self.w
+        d, dp = w.head_dim, w.d_proj
+        rows, sel_sizes, cand = self.union_rows()
+        attn_rows = rows.sum().item()
+        row_b = d * ROW_BYTES_PER_DIM
+        qo = self.steps * w.n_layers * w.batch * w.n_q_heads * d * (2 + 4)
+        attn_bytes = attn_rows * row_b
+        sel_bytes = 0
+        for i in range(self.steps):
+            if is_prediction_step(i, w.interval):
+                sel_bytes += w.n_layers * (w.n_kv_heads * cand[i].item() * dp * 2)
+                sel_bytes += 4 * sel_sizes[i].sum().item()
+        mlp_bytes = 0
+        if w.hidden > 0:
+            mlp_bytes = self.n_pred * len(self.producers) * (w.inter * w.hidden + w.n_out * w.inter) * 2
+        proj_bytes = len(self.dec.proj_steps) * w.n_layers * w.batch * w.window * w.n_kv_heads * (d + dp) * 2
+        sparse_total = attn_bytes + qo + sel_bytes + mlp_bytes + proj_bytes
+        dense_rows = sum(sum(t + i + 1 for t in self.ctx0) for i in range(self.steps)) * w.n_kv_heads * w.n_layers
+        dense_total = dense_rows * row_b + qo
+        return dict(attn_bytes=attn_bytes, attn_rows=attn_rows, sparse_total=sparse_total, dense_total=dense_total,
+                    dense_rows=dense_rows, sel_bytes=sel_bytes, mlp_bytes=mlp_bytes, proj_bytes=proj_bytes,
+                    sum_head_rows=int(sel_sizes.sum().item()))
+
+
+# ----------------------------------------------------------------------------
+# graphs and timing
+# ----------------------------------------------------------------------------
+
+class Marks:
+    """External event records at the attention-block boundaries of each
+    decode step (inside a capture they are graph nodes)."""
+
+    def __init__(self, steps):
+        self.ev = {(n, i): torch.cuda.Event(enable_timing=True) for i in range(steps)
+                   for n in ("attn_begin", "attn_end")}
+        for ev in self.ev.values():     # torch creates the CUDA event on first record
+            ev.record()
+        torch.cuda.synchronize()
+        self.stream = None
+
+    def __call__(self, name, i):
+        record_event(self.ev[(name, i)], self.stream)
+
+    def attn_ms(self, steps):
+        return [self.ev[("attn_begin", i)].elapsed_time(self.ev[("attn_end", i)]) for i in range(steps)]
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(stream)
+    return g
+
+
+class E2E:
+    """Per-step host<->device traffic of the public-API loop: the step's queries,
+    the new token's K and V rows of every layer and (prediction steps) the
+    producer hidden states go host->device from pinned memory; the step's
+    attention outputs come back device->host."""
+
+    def __init__(self, run: Run):
+        self.run = run
+        w = run.w
+        self.q_host = run.Q.cpu().pin_memory()
+        self.q_dev = torch.empty_like(run.Q[0])
+        nL = w.n_layers
+        pos = [[t + i for t in run.ctx0] for i in range(run.steps)]     # new token position T-1
+        self.pos = pos
+        kv = torch.empty(run.steps, nL, 2, w.batch, w.n_kv_heads, w.head_dim, dtype=torch.bfloat16)
+        for i in range(run.steps):
+            for l in range(nL):
+                for b in range(w.batch):
+                    kv[i, l, 0, b] = run.K[l][b, :, pos[i][b]].cpu()
+                    kv[i, l, 1, b] = run.V[l][b, :, pos[i][b]].cpu()
+        self.kv_host = kv.pin_memory()
+        self.h_host = run.h.cpu().pin_memory() if run.h is not None else None
+        self.h_dev = torch.empty_like(run.h[0]) if run.h is not None else None
+        self.out_host = torch.empty(run.steps, *run.out.shape, dtype=torch.float32).pin_memory()
+        row = w.head_dim * 2
+        self.h2d = run.Q[0].numel() * 2 + nL * 2 * w.batch * w.n_kv_heads * row
+        self.h2d_pred = self.h_host[0].numel() * 2 if self.h_host is not None else 0
+        self.d2h = run.out.numel() * 4
+
+    def bytes_per_run(self):
+        r = self.run
+        return self.h2d * r.steps + self.h2d_pred * r.n_pred, self.d2h * r.steps
+
+    def body(self, stream):
+        r, w = self.run, self.run.w
+        row = w.head_dim * 2
+        cap = w.ctx_cap
+        for i in range(r.steps):
+            self.q_dev.copy_(self.q_host[i], non_blocking=True)
+            for l in range(w.n_layers):
+                for kind, cache in ((0, r.K[l]), (1, r.V[l])):
+                    src = self.kv_host[i, l, kind]
+                    if len(set(self.pos[i])) == 1:
+                        dst = cache.data_ptr() + self.pos[i][0] * row
+                        memcpy2d_async(dst, cap * row, src.data_ptr(), row, row, w.batch * w.n_kv_heads, 1, stream)
+                    else:
+                        for b in range(w.batch):
+                            dst = cache[b].data_ptr() + self.pos[i][b] * row
+                            memcpy2d_async(dst, cap * row, src[b].data_ptr(), row, row, w.n_kv_heads, 1, stream)
+            h = None
+            if is_prediction_step(i, w.interval) and self.h_host is not None:
+                self.h_dev.copy_(self.h_host[i // w.interval], non_blocking=True)
+                h = self.h_dev
+            qd = r.qp_direct[i // w.interval] if r.qp_direct is not None else None
+            r.dec.step(i, self.q_dev, r.out, h=h, qp_direct=qd, stream=stream)
+            self.out_host[i].copy_(r.out, non_blocking=True)
+
+
+def time_graph(g, warmup, steps, dist_on, device):
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if dist_on:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+        ms = t.item()
+    return ms
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ----------------------------------------------------------------------------
+
+class OracleSample:
+    """The oracle on one layer of the workload: the key projection of the
+    prefilled context (setup), then decode steps of that layer in schedule
+    order; a prediction step runs the predictor MLP, scoring and selection for
+    every query head, every step runs attention for every query head.  The
+    per-layer times are scaled to a whole decode step (x n_layers)."""
+
+    def __init__(self, w: tb_inputs.Workload, layer: int = 0):
+        import numpy as np
+
+        import oracle
+        self.np, self.o = np, oracle
+        self.w = w
+        self.layer = layer
+        K, V = tb_inputs.kv_layer(w, layer, "cpu")
+        self.K = K.view(torch.int16).numpy().view(np.uint16)
+        self.V = V.view(torch.int16).numpy().view(np.uint16)
+        self.Wk = tb_inputs.wk_layer(w, layer, "cpu").view(torch.int16).numpy().view(np.uint16)
+        self.ctx0 = w.ctx0_per_seq()
+        self.scale = 1.0 / math.sqrt(w.head_dim)
+        self.Kp = {}
+        t0 = time.perf_counter()
+        for b in range(w.batch):
+            for g in range(w.n_kv_heads):
+                n = (self.ctx0[b] // w.window) * w.window
+                self.Kp[(b, g)] = self.o.project_keys(self.K[b, g, :n + w.window], self.Wk[g])
+        self.proj_s = time.perf_counter() - t0
+        self.rows_projected = sum((t // w.window) * w.window + w.window for t in self.ctx0) * w.n_kv_heads
+        if w.hidden > 0:
+            W1, W2 = tb_inputs.mlp_weights(w, 0, "cpu")
+            self.W1 = W1.view(torch.int16).numpy().view(np.uint16)
+            self.W2 = W2.view(torch.int16).numpy().view(np.uint16)
+        self.I = None
+
+    def step(self, i):
+        np, o, w = self.np, self.o, self.w
+        ctx = [t + i + 1 for t in self.ctx0]
+        if is_prediction_step(i, w.interval):
+            if w.hidden > 0:
+                h = tb_inputs.hidden_state(w, i // w.interval, 0, "cpu").view(torch.int16).numpy().view(np.uint16)
+                qp = o.predict_queries(h, self.W1, self.W2).reshape(w.batch, w.slots, w.n_q_heads, w.d_proj)[:, 0]
+            else:
+                qp = tb_inputs.direct_qp(w, i // w.interval, self.layer, "cpu").numpy()
+            self.I = []
+            for b in range(w.batch):
+                T = ctx[b]
+                hi = max(w.sink, T - w.window)
+                per = []
+                for h_ in range(w.n_q_heads):
+                    s = o.scores(qp[b, h_], self.Kp[(b, h_ // w.group)], w.sink, hi)
+                    per.append(o.select(s, T, w.sink, w.window, w.budget, w.nbr))
+                self.I.append(per)
+        Q = tb_inputs.query(w, i, self.layer, "cpu").view(torch.int16).numpy().view(np.uint16)
+        for b in range(w.batch):
+            for h_ in range(w.n_q_heads):
+                A = o.attention_set(ctx[b], w.sink, w.window, self.I[b][h_])
+                o.attention(Q[b, h_], self.K[b, h_ // w.group], self.V[b, h_ // w.group], A, self.scale)
+
+    def per_decode_step_s(self, t_pred, t_reuse):
+        """Whole-model seconds per decode step from per-layer step times: every
+        layer pays attention each step and selection once per interval; the
+        predictor is paid by 1/stride of the layers (it was timed on every
+        prediction step of the sampled producer layer, so this over-counts
+        it); key projection is paid once per token."""
+        w = self.w
+        per_layer = (t_pred + (w.interval - 1) * t_reuse) / w.interval
+        rows_per_step = w.batch * w.n_kv_heads                 # one new row per (b, kv head) per step
+        proj = self.proj_s / self.rows_projected * rows_per_step
+        return w.n_layers * (per_layer + proj)
+
+
+def cpu_baseline(w, budget_s=25.0):
+    smp = OracleSample(w)
+    t_pred, t_reuse = [], []
+    t_start = time.perf_counter()
+    i = 0
+    while True:
+        t0 = time.perf_counter()
+        smp.step(i)
+        dt = time.perf_counter() - t0
+        (t_pred if is_prediction_step(i, w.interval) else t_reuse).append(dt)
+        i += 1
+        if t_reuse and time.perf_counter() - t_start > budget_s:
+            break
+        if i >= w.steps:
+            break
+    s_per_step = smp.per_decode_step_s(statistics.mean(t_pred), statistics.mean(t_reuse))
+    return {"value": w.batch / s_per_step, "unit": "decode steps/s", "cores": 1, "kind": "oracle",
+            "sample": (f"layer 0 of {w.name}: key projection of the prefilled context ({smp.proj_s:.1f} s), "
+                       f"{len(t_pred)} prediction + {len(t_reuse)} reuse decode steps of all {w.n_q_heads} query "
+                       f"heads; scaled x{w.n_layers} layers, selection amortised over the interval, projection "
+                       f"per token"),
+            "sample_seconds": round(time.perf_counter() - t_start + smp.proj_s, 1)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = tb_inputs.WORKLOADS[args.workload]
+    smp = OracleSample(w)
+    t_pred, t_reuse = [], []
+    for i in range(args.warmup):
+        smp.step(1 + i if w.interval > 1 else 0)
+    order = list(range(args.steps))
+    t_all0 = time.perf_counter()
+    for i in order:
+        t0 = time.perf_counter()
+        smp.step(i)
+        (t_pred if is_prediction_step(i, w.interval) else t_reuse).append(time.perf_counter() - t0)
+    wall = time.perf_counter() - t_all0
+    if not t_reuse:
+        t_reuse = t_pred
+    s_per_step = smp.per_decode_step_s(statistics.mean(t_pred), statistics.mean(t_reuse))
+    value = w.batch / s_per_step
+    sample = (f"each step: one decode step of layer 0 of {w.name} (all {w.n_q_heads} query heads; the first step "
+              f"also predicts and selects), scaled x{w.n_layers} layers with selection amortised over the "
+              f"{w.interval}-step interval")
+    line = {"impl": "reference", "metric": "sparse decode steps/s", "value": round(value, 4),
+            "unit": "decode steps/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000 * wall / max(1, len(order)), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx0, "layers": w.n_layers},
+            "cpu_baseline": {"value": round(value, 4), "unit": "decode steps/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "decode steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# main
+# ----------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama64k", choices=sorted(tb_inputs.WORKLOADS))
+    ap.add_argument("--impl", default="tb", choices=["tb", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=None, help="decode steps per run (default: workload's)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device(device))
+    L.load()
+    base = tb_inputs.WORKLOADS[args.workload]
+    w = base.scaled(seed=base.seed + rank)           # an independent replica per rank
+    run = Run(w, device, steps=args.decode_steps)
+    run.dec.prefill()
+    torch.cuda.synchronize()
+
+    acct = run.bytes_model()       # eager pass: warms every kernel and counts the kept rows
+    stream = torch.cuda.Stream(device=device)
+    marks_s = Marks(run.steps)
+    marks_s.stream = stream
+    g_sparse = capture(lambda st: run.run_sparse(st, marks_s), stream)
+    marks_d = Marks(run.steps)
+    marks_d.stream = stream
+    g_dense = capture(lambda st: run.run_dense(st, marks_d), stream)
+    e2e = None
+    if not args.no_e2e:
+        e2e = E2E(run)
+        g_e2e = capture(e2e.body, stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    ms_sparse = time_graph(g_sparse, args.warmup, args.steps, dist_on, device)
+    attn_ms = marks_s.attn_ms(run.steps)
+    ms_dense = time_graph(g_dense, args.warmup, args.steps, dist_on, device)
+    dense_attn_ms = marks_d.attn_ms(run.steps)
+    clk = clocks.stop()
+    ms_e2e = time_graph(g_e2e, args.warmup, args.steps, dist_on, device) if e2e else None
+
+    flags = L.workspace_check(run.dec.ws_attn) | L.workspace_check(run.dec.ws_sel) | \
+        L.workspace_check(run.dec.ws_proj) | (L.workspace_check(run.dec.ws_pred) if run.dec.ws_pred is not None else 0)
+
+    tokens_per_run = run.steps * w.batch
+    per_step_sparse = ms_sparse / args.steps
+    per_step_dense = ms_dense / args.steps
+    value = world * tokens_per_run / (per_step_sparse / 1000.0)
+    dense_value = world * tokens_per_run / (per_step_dense / 1000.0)
+    peak, peak_kind = measured_peaks()
+    n_attn = run.steps * w.n_layers
+    attn_launch_ms = sum(attn_ms) / n_attn
+    attn_bytes_per_launch = acct["attn_bytes"] / n_attn
+    achieved = attn_bytes_per_launch / (attn_launch_ms / 1000.0) / 1e9
+    dense_launch_ms = sum(dense_attn_ms) / n_attn
+    dense_achieved = (acct["dense_total"] / n_attn) / (dense_launch_ms / 1000.0) / 1e9
+    path_gbs = acct["sparse_total"] / (per_step_sparse / 1000.0) / 1e9
+    dense_path_gbs = acct["dense_total"] / (per_step_dense / 1000.0) / 1e9
+    sparse_launches, dense_launches = run.launches()
+
+    if rank != 0:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return 0
+    line = {
+        "metric": "sparse decode steps/s", "value": round(value, 3), "unit": "decode steps/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_sparse, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; Llama-3.1-8B attention shapes, random weights)",
+        "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
+                   "layers": w.n_layers, "decode_steps_per_bench_step": run.steps, "budget": w.budget,
+                   "interval": w.interval, "sink": w.sink, "window": w.window, "d_proj": w.d_proj,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (KV %.1f GB)" % (2 * sum(k.numel() for k in run.K) * 2 / 1e9),
+                   "graph": "one CUDA graph per bench step"},
+        "speedup_vs_dense": round(value / dense_value, 4),
+        "dense": {"value": round(dense_value, 3), "unit": "decode steps/s", "ms_per_step": round(per_step_dense, 4),
+                  "path_gbs": round(dense_path_gbs, 1), "attn_launch_us": round(1000 * dense_launch_ms, 3),
+                  "attn_achieved_gbs": round(dense_achieved, 1)},
+        "hbm": {"path_gbs": round(path_gbs, 1), "path_frac_of_8tbs": round(path_gbs / HBM_NOMINAL_GBS, 4),
+                "path_frac_of_measured": round(path_gbs / peak, 4), "bytes_per_bench_step": acct["sparse_total"],
+                "attn_rows_union": acct["attn_rows"], "attn_rows_per_head_sum": acct["sum_head_rows"],
+                "dense_bytes_per_bench_step": acct["dense_total"]},
+        "roofline": {"kernel": "attn_kernel<128,true> (sparse GQA decode attention)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "bytes_per_launch": round(attn_bytes_per_launch), "launch_us": round(1000 * attn_launch_ms, 3)},
+        "gpu_launches": (sparse_launches) * args.steps,
+        "clocks": clk,
+        "device_flags": flags,
+    }
+    if e2e is not None:
+        h2d, d2h = e2e.bytes_per_run()
+        line["e2e"] = {"value": round(world * tokens_per_run / (ms_e2e / args.steps / 1000.0), 3),
+                       "unit": "decode steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(ms_e2e / args.steps, 4)}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line))
+    if dist_on:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

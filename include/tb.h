@@ -15,9 +15,11 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Pointers are DEVICE pointers unless a comment says "host".  Every device
- *    pointer must be 16-byte aligned.  Nothing here allocates, frees or keeps
- *    device memory; the caller owns every buffer, including workspaces.
+ *  - Pointers are DEVICE pointers unless a comment says "host".  bf16 arrays
+ *    (K, V, K', Q, W_k, W1, W2, h) and workspaces must be 16-byte aligned;
+ *    int32, uint32 and float arrays 4-byte aligned.  Nothing here allocates,
+ *    frees or keeps device memory; the caller owns every buffer, including
+ *    workspaces.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  *    asynchronous: it validates its arguments on the host, launches, and
  *    returns; it never synchronises the device.

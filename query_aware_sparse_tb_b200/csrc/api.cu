@@ -34,11 +34,20 @@ tb_status fail(tb_status s, const char *fmt, ...) {
 }
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// bf16 tensors are read with 16-byte vector loads, cp.async and TMA
 #define TB_CHECK_PTR(p)                                                                      \
     do {                                                                                     \
         if (!aligned16(p))                                                                   \
             return fail(TB_ERR_INVALID_ARG, "%s: pointer '%s' is null or not 16-byte aligned", \
+                        __func__, #p);                                                       \
+    } while (0)
+// int32 / float / uint32 arrays are accessed a word at a time
+#define TB_CHECK_PTR4(p)                                                                     \
+    do {                                                                                     \
+        if (!aligned4(p))                                                                    \
+            return fail(TB_ERR_INVALID_ARG, "%s: pointer '%s' is null or not 4-byte aligned",  \
                         __func__, #p);                                                       \
     } while (0)
 
@@ -137,7 +146,7 @@ tb_status tb_project_keys(const tb_dims *dims, const tb_bf16 *K, const tb_bf16 *
                           void *ws, size_t ws_bytes, void *stream) {
     tb_status s;
     if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
-    TB_CHECK_PTR(K); TB_CHECK_PTR(Wk); TB_CHECK_PTR(Kp); TB_CHECK_PTR(tok_begin); TB_CHECK_PTR(tok_count);
+    TB_CHECK_PTR(K); TB_CHECK_PTR(Wk); TB_CHECK_PTR(Kp); TB_CHECK_PTR4(tok_begin); TB_CHECK_PTR4(tok_count);
     if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
     if (max_tok < 0) return fail(TB_ERR_INVALID_ARG, "tb_project_keys: max_tok < 0");
     if ((long long)dims->batch * dims->n_kv_heads * dims->ctx_cap > 0x7fffffffLL)
@@ -151,7 +160,7 @@ tb_status tb_project_keys(const tb_dims *dims, const tb_bf16 *K, const tb_bf16 *
 tb_status tb_predict_queries(const tb_bf16 *h, const tb_bf16 *W1, const tb_bf16 *W2, float *qp,
                              int32_t batch, int32_t hidden, int32_t inter, int32_t n_out, void *ws,
                              size_t ws_bytes, void *stream) {
-    TB_CHECK_PTR(h); TB_CHECK_PTR(W1); TB_CHECK_PTR(W2); TB_CHECK_PTR(qp);
+    TB_CHECK_PTR(h); TB_CHECK_PTR(W1); TB_CHECK_PTR(W2); TB_CHECK_PTR4(qp);
     if (batch < 1 || batch > 16)
         return fail(TB_ERR_UNSUPPORTED, "tb_predict_queries: batch %d outside [1, 16]", batch);
     if (hidden < 256 || hidden % 256 || inter < 256 || inter % 256)
@@ -172,12 +181,12 @@ tb_status tb_score_select(const tb_dims *dims, const float *qp, int64_t qp_batch
                           uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream) {
     tb_status s;
     if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
-    TB_CHECK_PTR(qp); TB_CHECK_PTR(Kp); TB_CHECK_PTR(ctx_len); TB_CHECK_PTR(idx); TB_CHECK_PTR(count);
-    TB_CHECK_PTR(sel_bits);
+    TB_CHECK_PTR4(qp); TB_CHECK_PTR(Kp); TB_CHECK_PTR4(ctx_len); TB_CHECK_PTR4(idx); TB_CHECK_PTR4(count);
+    TB_CHECK_PTR4(sel_bits);
     if (dims->ctx_cap > kMaxCtxSelect)
         return fail(TB_ERR_UNSUPPORTED, "tb_score_select: ctx_cap %d above %d", dims->ctx_cap, kMaxCtxSelect);
-    if (qp_batch_stride < (int64_t)dims->n_q_heads * dims->d_proj || (qp_batch_stride & 3))
-        return fail(TB_ERR_INVALID_ARG, "tb_score_select: qp_batch_stride %lld too small or not a multiple of 4",
+    if (qp_batch_stride < (int64_t)dims->n_q_heads * dims->d_proj)
+        return fail(TB_ERR_INVALID_ARG, "tb_score_select: qp_batch_stride %lld smaller than Hq*d'",
                     (long long)qp_batch_stride);
     if (sink < 0 || window < 1 || budget < 1)
         return fail(TB_ERR_INVALID_ARG, "tb_score_select: need sink >= 0, window >= 1, budget >= 1");
@@ -197,7 +206,7 @@ tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32
                                   const int32_t *count, uint32_t *sel_bits, void *stream) {
     tb_status s;
     if ((s = check_dims(dims, false, __func__)) != TB_OK) return s;
-    TB_CHECK_PTR(idx); TB_CHECK_PTR(count); TB_CHECK_PTR(sel_bits);
+    TB_CHECK_PTR4(idx); TB_CHECK_PTR4(count); TB_CHECK_PTR4(sel_bits);
     if (idx_cap < 1) return fail(TB_ERR_INVALID_ARG, "tb_select_bits_from_idx: idx_cap < 1");
     if (dims->ctx_cap > kMaxCtxSelect)
         return fail(TB_ERR_UNSUPPORTED, "tb_select_bits_from_idx: ctx_cap above %d", kMaxCtxSelect);
@@ -209,8 +218,10 @@ static tb_status attn_common(const char *fn, const tb_dims *dims, const tb_bf16 
                              size_t ws_bytes) {
     tb_status s;
     if ((s = check_dims(dims, false, fn)) != TB_OK) return s;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(ctx_len) || !aligned16(out))
-        return fail(TB_ERR_INVALID_ARG, "%s: Q, K, V, ctx_len and out must be non-null and 16-byte aligned", fn);
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V))
+        return fail(TB_ERR_INVALID_ARG, "%s: Q, K and V must be non-null and 16-byte aligned", fn);
+    if (!aligned4(ctx_len) || !aligned4(out))
+        return fail(TB_ERR_INVALID_ARG, "%s: ctx_len and out must be non-null and 4-byte aligned", fn);
     if (dims->ctx_cap > kMaxCtxAttn)
         return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", fn, dims->ctx_cap, kMaxCtxAttn);
     if (!isfinite(scale)) return fail(TB_ERR_INVALID_ARG, "%s: scale is not finite", fn);
@@ -223,7 +234,7 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
                                 size_t ws_bytes, void *stream) {
     tb_status s = attn_common(__func__, dims, Q, K, V, ctx_len, scale, out, ws, ws_bytes);
     if (s != TB_OK) return s;
-    TB_CHECK_PTR(sel_bits);
+    TB_CHECK_PTR4(sel_bits);
     if (sink < 0 || window < 1)
         return fail(TB_ERR_INVALID_ARG, "tb_sparse_decode_attn: need sink >= 0 and window >= 1");
     return cuda_status(launch_attn(*dims, Q, K, V, ctx_len, sink, window, sel_bits, true, scale, out, ws,

@@ -23,6 +23,8 @@
 // partial states into the fp32 output.
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -34,9 +36,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kTile = 64;       // rows per pipeline stage
 constexpr int kStages = 3;
 constexpr int kGroup = 4;       // query heads per KV head
-constexpr int kMaxChunk = 2048; // context positions per CTA (upper bound)
-constexpr int kMinChunk = 256;
-constexpr int kMaxSplits = 2048;
+constexpr int kMaxChunk = 2048; // positions per row list (a CTA walks its range in sub-chunks)
+constexpr int kMaxSplits = 64;   // partial states merged per (sequence, KV head)
 constexpr unsigned kFull = 0xffffffffu;
 
 template <int D>
@@ -77,12 +78,15 @@ __global__ void __launch_bounds__(kThreads, 2)
 attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             const uint16_t *__restrict__ V, const int32_t *__restrict__ ctx_len,
             const uint32_t *__restrict__ sel_bits, int Hq, int Hkv, int Tcap, int W, int sink,
-            int window, float qscale, int chunk, int nsplit, float *__restrict__ part,
+            int window, float qscale, int splits, float *__restrict__ part,
             uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags) {
     constexpr int DPL = D / 16;  // head_dim elements per lane
     constexpr int CPR = D / 8;   // 16-byte chunks per row
     constexpr int kCopies = kTile * CPR / kThreads;
-    constexpr int kPartStride = kGroup * (D + 2);
+    // one partial state per head: O[D], M, L, 2 pad floats, so every head's
+    // record starts 16-byte aligned for the float4 loads of the merge
+    constexpr int kHS = D + 4;
+    constexpr int kPartStride = kGroup * kHS;
     using S = Smem<D>;
 
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -91,72 +95,23 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     float *pbuf = reinterpret_cast<float *>(smem + S::kPipe + S::kList);
     int32_t *wcnt = reinterpret_cast<int32_t *>(smem + S::kPipe + S::kList + S::kP);
     __shared__ int s_nrows, s_last;
+    __shared__ float s_red[kWarps][kGroup];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int half = lane >> 4, c = lane & 15;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
-    const int p0 = split * chunk;
-    const int p1 = min(p0 + chunk, T);
+    // this sequence's length split evenly over the CTAs of (b, g), in 64-row units
+    const int chunk = ((T + splits - 1) / splits + kTile - 1) / kTile * kTile;
+    const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
+    const int p_begin = split * chunk;
+    const int p_end = min(p_begin + chunk, T);
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     const uint16_t *Kb = K + slab * D;
     const uint16_t *Vb = V + slab * D;
-    float *part_bg = part + (size_t)(b * Hkv + g) * nsplit * kPartStride;
+    float *part_bg = part + (size_t)(b * Hkv + g) * splits * kPartStride;
 
-    if (p0 < T) {
-        // ------------------------------------------------ row list (sparse)
-        int n_rows = p1 - p0;
-        if constexpr (SPARSE) {
-            const int hi_c = T - window;  // candidates are [sink, hi_c)
-            const int nwords = (p1 - p0 + 31) >> 5;
-            const int w0 = p0 >> 5;
-            const uint32_t *sb = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W + w0;
-            auto word_mask = [&](int wi, int &p, int &m) -> uint32_t {
-                uint32_t hb = lane < kGroup ? __ldg(sb + (size_t)lane * W + wi) : 0u;
-                uint32_t b0 = __shfl_sync(kFull, hb, 0), b1 = __shfl_sync(kFull, hb, 1);
-                uint32_t b2 = __shfl_sync(kFull, hb, 2), b3 = __shfl_sync(kFull, hb, 3);
-                p = p0 + (wi << 5) + lane;
-                m = 0;
-                if (p < p1) {
-                    if (p < sink || p >= hi_c) {
-                        m = 0xF;
-                    } else {
-                        m = ((b0 >> lane) & 1u) | (((b1 >> lane) & 1u) << 1) |
-                            (((b2 >> lane) & 1u) << 2) | (((b3 >> lane) & 1u) << 3);
-                    }
-                }
-                return __ballot_sync(kFull, m != 0);
-            };
-            for (int wi = warp; wi < nwords; wi += kWarps) {
-                int p, m;
-                uint32_t bal = word_mask(wi, p, m);
-                if (lane == 0) wcnt[wi] = __popc(bal);
-            }
-            __syncthreads();
-            if (warp == 0) {  // exclusive scan of <= 64 word counts
-                int a0 = (2 * lane < nwords) ? wcnt[2 * lane] : 0;
-                int a1 = (2 * lane + 1 < nwords) ? wcnt[2 * lane + 1] : 0;
-                int sum = a0 + a1, incl = sum;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    int v = __shfl_up_sync(kFull, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                int excl = incl - sum;
-                if (2 * lane < nwords) wcnt[2 * lane] = excl;
-                if (2 * lane + 1 < nwords) wcnt[2 * lane + 1] = excl + a0;
-                if (lane == 31) s_nrows = incl;
-            }
-            __syncthreads();
-            for (int wi = warp; wi < nwords; wi += kWarps) {
-                int p, m;
-                uint32_t bal = word_mask(wi, p, m);
-                if (m) list[wcnt[wi] + __popc(bal & ((1u << lane) - 1u))] = (p << 4) | m;
-            }
-            __syncthreads();
-            n_rows = s_nrows;
-        }
-
+    if (p_begin < T) {
         // ------------------------------------------------ per-lane query slice
         float q[kGroup][DPL];
 #pragma unroll
@@ -184,140 +139,196 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
 #pragma unroll
             for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
         }
-
-        const int n_tiles = (n_rows + kTile - 1) / kTile;
         const uint32_t pipe_s = smem_addr(pipe);
-
-        auto issue = [&](int t) {
-            const uint32_t kbase = pipe_s + (t % kStages) * S::kStageBytes;
-            const uint32_t vbase = kbase + kTile * D * 2;
-#pragma unroll
-            for (int k = 0; k < kCopies; ++k) {
-                const int e = tid + k * kThreads;
-                const int r = e / CPR, ch = e % CPR;
-                const int gr = t * kTile + r;
-                const bool valid = gr < n_rows;
-                int pos = p0;
-                if (valid) pos = SPARSE ? (list[gr] >> 4) : (p0 + gr);
-                const size_t off = (size_t)pos * D + ch * 8;
-                const uint32_t so = (uint32_t)(r * D + ch * 8) * 2u;
-                cp_async16(kbase + so, Kb + off, valid);
-                cp_async16(vbase + so, Vb + off, valid);
-            }
-        };
-
-#pragma unroll
-        for (int s = 0; s < kStages - 1; ++s) {
-            if (s < n_tiles) issue(s);
-            cp_async_commit();
-        }
-
         const int rb = warp * 8 + half * 4;  // this half-warp's first row in a tile
-        for (int t = 0; t < n_tiles; ++t) {
-            cp_async_wait<kStages - 2>();
-            __syncthreads();
-            if (t + kStages - 1 < n_tiles) issue(t + kStages - 1);
-            cp_async_commit();
 
-            const uint16_t *Ks = pipe + (t % kStages) * (S::kStageBytes / 2);
-            const uint16_t *Vs = Ks + kTile * D;
-
-            // partial q.k over this lane's slice: 4 rows x 4 heads
-            float s[16];
+        // the CTA's range in sub-chunks of at most kMaxChunk positions
+        for (int p0 = p_begin; p0 < p_end; p0 += kMaxChunk) {
+            const int p1 = min(p0 + kMaxChunk, p_end);
+            // -------------------------------------------- row list (sparse)
+            int n_rows = p1 - p0;
+            if constexpr (SPARSE) {
+                const int hi_c = T - window;  // candidates are [sink, hi_c)
+                const int nwords = (p1 - p0 + 31) >> 5;
+                const int w0 = p0 >> 5;
+                const uint32_t *sb = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W + w0;
+                auto word_mask = [&](int wi, int &p, int &m) -> uint32_t {
+                    uint32_t hb = lane < kGroup ? __ldg(sb + (size_t)lane * W + wi) : 0u;
+                    uint32_t b0 = __shfl_sync(kFull, hb, 0), b1 = __shfl_sync(kFull, hb, 1);
+                    uint32_t b2 = __shfl_sync(kFull, hb, 2), b3 = __shfl_sync(kFull, hb, 3);
+                    p = p0 + (wi << 5) + lane;
+                    m = 0;
+                    if (p < p1) {
+                        if (p < sink || p >= hi_c) {
+                            m = 0xF;
+                        } else {
+                            m = ((b0 >> lane) & 1u) | (((b1 >> lane) & 1u) << 1) |
+                                (((b2 >> lane) & 1u) << 2) | (((b3 >> lane) & 1u) << 3);
+                        }
+                    }
+                    return __ballot_sync(kFull, m != 0);
+                };
+                for (int wi = warp; wi < nwords; wi += kWarps) {
+                    int p, m;
+                    uint32_t bal = word_mask(wi, p, m);
+                    if (lane == 0) wcnt[wi] = __popc(bal);
+                }
+                __syncthreads();
+                if (warp == 0) {  // exclusive scan of <= 64 word counts
+                    int a0 = (2 * lane < nwords) ? wcnt[2 * lane] : 0;
+                    int a1 = (2 * lane + 1 < nwords) ? wcnt[2 * lane + 1] : 0;
+                    int sum = a0 + a1, incl = sum;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float kf[DPL];
-                load_chunk<DPL>(Ks + (rb + j) * D + c * DPL, kf);
+                    for (int o = 1; o < 32; o <<= 1) {
+                        int v = __shfl_up_sync(kFull, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    int excl = incl - sum;
+                    if (2 * lane < nwords) wcnt[2 * lane] = excl;
+                    if (2 * lane + 1 < nwords) wcnt[2 * lane + 1] = excl + a0;
+                    if (lane == 31) s_nrows = incl;
+                }
+                __syncthreads();
+                for (int wi = warp; wi < nwords; wi += kWarps) {
+                    int p, m;
+                    uint32_t bal = word_mask(wi, p, m);
+                    if (m) list[wcnt[wi] + __popc(bal & ((1u << lane) - 1u))] = (p << 4) | m;
+                }
+                __syncthreads();
+                n_rows = s_nrows;
+            }
+
+            const int n_tiles = (n_rows + kTile - 1) / kTile;
+            auto issue = [&](int t) {
+                const uint32_t kbase = pipe_s + (t % kStages) * S::kStageBytes;
+                const uint32_t vbase = kbase + kTile * D * 2;
+#pragma unroll
+                for (int k = 0; k < kCopies; ++k) {
+                    const int e = tid + k * kThreads;
+                    const int r = e / CPR, ch = e % CPR;
+                    const int gr = t * kTile + r;
+                    const bool valid = gr < n_rows;
+                    int pos = p0;
+                    if (valid) pos = SPARSE ? (list[gr] >> 4) : (p0 + gr);
+                    const size_t off = (size_t)pos * D + ch * 8;
+                    const uint32_t so = (uint32_t)(r * D + ch * 8) * 2u;
+                    cp_async16(kbase + so, Kb + off, valid);
+                    cp_async16(vbase + so, Vb + off, valid);
+                }
+            };
+
+#pragma unroll
+            for (int s = 0; s < kStages - 1; ++s) {
+                if (s < n_tiles) issue(s);
+                cp_async_commit();
+            }
+
+            for (int t = 0; t < n_tiles; ++t) {
+                cp_async_wait<kStages - 2>();
+                __syncthreads();
+                if (t + kStages - 1 < n_tiles) issue(t + kStages - 1);
+                cp_async_commit();
+
+                const uint16_t *Ks = pipe + (t % kStages) * (S::kStageBytes / 2);
+                const uint16_t *Vs = Ks + kTile * D;
+
+                // partial q.k over this lane's slice: 4 rows x 4 heads
+                float s[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float kf[DPL];
+                    load_chunk<DPL>(Ks + (rb + j) * D + c * DPL, kf);
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) a = fmaf(q[h][e], kf[e], a);
+                        s[j * 4 + h] = a;
+                    }
+                }
+                // transposing butterfly over the 16 lanes of a row group: lane c
+                // ends with the full sum of value c = (row c>>2, head c&3)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const bool up = c & 8;
+                    float send = up ? s[k] : s[k + 8], keep = up ? s[k + 8] : s[k];
+                    s[k] = keep + __shfl_xor_sync(kFull, send, 8);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const bool up = c & 4;
+                    float send = up ? s[k] : s[k + 4], keep = up ? s[k + 4] : s[k];
+                    s[k] = keep + __shfl_xor_sync(kFull, send, 4);
+                }
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const bool up = c & 2;
+                    float send = up ? s[k] : s[k + 2], keep = up ? s[k + 2] : s[k];
+                    s[k] = keep + __shfl_xor_sync(kFull, send, 2);
+                }
+                {
+                    const bool up = c & 1;
+                    float send = up ? s[0] : s[1], keep = up ? s[1] : s[0];
+                    s[0] = keep + __shfl_xor_sync(kFull, send, 1);
+                }
+                float x = s[0];
+                const int hh = c & 3;
+                {
+                    const int gr = t * kTile + rb + (c >> 2);
+                    uint32_t mk = 0;
+                    if (gr < n_rows) mk = SPARSE ? (uint32_t)(list[gr] & 0xF) : 0xFu;
+                    if (!((mk >> hh) & 1u)) x = -INFINITY;
+                }
+                // tile max per head over the warp's 8 rows
+                float mx = x;
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+                float alpha[kGroup];
+                bool changed = false;
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) {
-                    float a = 0.f;
-#pragma unroll
-                    for (int e = 0; e < DPL; ++e) a = fmaf(q[h][e], kf[e], a);
-                    s[j * 4 + h] = a;
+                    const float mt = __shfl_sync(kFull, mx, h);
+                    const float mn = fmaxf(m_run[h], mt);
+                    alpha[h] = (mn == m_run[h]) ? 1.f : exp2f(m_run[h] - mn);
+                    changed |= (mn != m_run[h]);
+                    m_run[h] = mn;
                 }
-            }
-            // transposing butterfly over the 16 lanes of a row group: lane c
-            // ends with the full sum of value c = (row c>>2, head c&3)
+                const float p = (x == -INFINITY) ? 0.f : exp2f(x - pick4(m_run, hh));
+                __syncwarp();
+                pbuf[warp * 32 + lane] = p;
+                __syncwarp();
+                float4 pr[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const bool up = c & 8;
-                float send = up ? s[k] : s[k + 8], keep = up ? s[k + 8] : s[k];
-                s[k] = keep + __shfl_xor_sync(kFull, send, 8);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const bool up = c & 4;
-                float send = up ? s[k] : s[k + 4], keep = up ? s[k + 4] : s[k];
-                s[k] = keep + __shfl_xor_sync(kFull, send, 4);
-            }
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const bool up = c & 2;
-                float send = up ? s[k] : s[k + 2], keep = up ? s[k + 2] : s[k];
-                s[k] = keep + __shfl_xor_sync(kFull, send, 2);
-            }
-            {
-                const bool up = c & 1;
-                float send = up ? s[0] : s[1], keep = up ? s[1] : s[0];
-                s[0] = keep + __shfl_xor_sync(kFull, send, 1);
-            }
-            float x = s[0];
-            const int hh = c & 3;
-            {
-                const int gr = t * kTile + rb + (c >> 2);
-                uint32_t mk = 0;
-                if (gr < n_rows) mk = SPARSE ? (uint32_t)(list[gr] & 0xF) : 0xFu;
-                if (!((mk >> hh) & 1u)) x = -INFINITY;
-            }
-            // tile max per head over the warp's 8 rows
-            float mx = x;
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-            float alpha[kGroup];
-            bool changed = false;
-#pragma unroll
-            for (int h = 0; h < kGroup; ++h) {
-                const float mt = __shfl_sync(kFull, mx, h);
-                const float mn = fmaxf(m_run[h], mt);
-                alpha[h] = (mn == m_run[h]) ? 1.f : exp2f(m_run[h] - mn);
-                changed |= (mn != m_run[h]);
-                m_run[h] = mn;
-            }
-            const float p = (x == -INFINITY) ? 0.f : exp2f(x - pick4(m_run, hh));
-            __syncwarp();
-            pbuf[warp * 32 + lane] = p;
-            __syncwarp();
-            float4 pr[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                pr[j] = *reinterpret_cast<const float4 *>(pbuf + warp * 32 + half * 16 + j * 4);
+                for (int j = 0; j < 4; ++j)
+                    pr[j] = *reinterpret_cast<const float4 *>(pbuf + warp * 32 + half * 16 + j * 4);
 
-            if (changed) {
+                if (changed) {
 #pragma unroll
-                for (int h = 0; h < kGroup; ++h) {
-                    l[h] *= alpha[h];
+                    for (int h = 0; h < kGroup; ++h) {
+                        l[h] *= alpha[h];
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) acc[h][e] *= alpha[h];
+                        for (int e = 0; e < DPL; ++e) acc[h][e] *= alpha[h];
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h)
+                    l[h] += comp4(pr[0], h) + comp4(pr[1], h) + comp4(pr[2], h) + comp4(pr[3], h);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float vf[DPL];
+                    load_chunk<DPL>(Vs + (rb + j) * D + c * DPL, vf);
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) {
+                        const float ph = comp4(pr[j], h);
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(ph, vf[e], acc[h][e]);
+                    }
                 }
             }
-#pragma unroll
-            for (int h = 0; h < kGroup; ++h)
-                l[h] += comp4(pr[0], h) + comp4(pr[1], h) + comp4(pr[2], h) + comp4(pr[3], h);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float vf[DPL];
-                load_chunk<DPL>(Vs + (rb + j) * D + c * DPL, vf);
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) {
-                    const float ph = comp4(pr[j], h);
-#pragma unroll
-                    for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(ph, vf[e], acc[h][e]);
-                }
-            }
+            cp_async_wait<0>();
+            __syncthreads();  // pipeline and list free for the next sub-chunk
         }
-        cp_async_wait<0>();
-        __syncthreads();
 
         // ------------------------------------------------ combine halves, warps
 #pragma unroll
@@ -360,10 +371,10 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                     }
                 }
             }
-            pp[h * (D + 2) + dim] = O;
+            pp[h * kHS + dim] = O;
             if (dim == 0) {
-                pp[h * (D + 2) + D] = M;
-                pp[h * (D + 2) + D + 1] = L;
+                pp[h * kHS + D] = M;
+                pp[h * kHS + D + 1] = L;
             }
         }
     }
@@ -373,40 +384,79 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     __syncthreads();
     if (tid == 0) {
         const unsigned prev = atomicAdd(&counters[b * Hkv + g], 1u);
-        s_last = (prev == (unsigned)nsplit - 1u);
+        s_last = (prev == (unsigned)splits - 1u);
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
 
-    const int ns = (T + chunk - 1) / chunk;  // chunks that hold rows
-    float *wsm = reinterpret_cast<float *>(smem);  // [ns][head] merge weights
-    if (warp < kGroup) {
-        const int h = warp;
-        float M = -INFINITY;
-        for (int s = lane; s < ns; s += 32)
-            M = fmaxf(M, __ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + D));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-        float L = 0.f;
-        for (int s = lane; s < ns; s += 32) {
-            const float ms = __ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + D);
-            const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-            wsm[s * kGroup + h] = f;
-            L = fmaf(f, __ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + D + 1), L);
+    // weights w[s][h] = exp2(M_sh - M*_h) / L*_h over the ns <= 64 partials:
+    // one (split, head) pair per thread, head = tid & 3
+    float *wsm = reinterpret_cast<float *>(smem);  // [ns][head]
+    {
+        const int h = tid & 3, s = tid >> 2;
+        float m = -INFINITY, lw = 0.f;
+        if (s < ns) {
+            m = __ldcg(part_bg + (size_t)s * kPartStride + h * kHS + D);
+            lw = __ldcg(part_bg + (size_t)s * kPartStride + h * kHS + D + 1);
         }
+        float mx = m;
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+        if (lane < kGroup) s_red[warp][lane] = mx;
+        __syncthreads();
+        float Mh = -INFINITY;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        for (int s = lane; s < ns; s += 32) wsm[s * kGroup + h] *= inv;
+        for (int w = 0; w < kWarps; ++w) Mh = fmaxf(Mh, s_red[w][h]);
+        const float f = (m == -INFINITY) ? 0.f : exp2f(m - Mh);
+        float lsum = f * lw;
+        lsum += __shfl_xor_sync(kFull, lsum, 4);
+        lsum += __shfl_xor_sync(kFull, lsum, 8);
+        lsum += __shfl_xor_sync(kFull, lsum, 16);
+        __syncthreads();
+        if (lane < kGroup) s_red[warp][lane] = lsum;
+        __syncthreads();
+        float Lh = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) Lh += s_red[w][h];
+        if (s < ns) wsm[s * kGroup + h] = Lh > 0.f ? f / Lh : 0.f;
     }
     __syncthreads();
-    for (int it = tid; it < kGroup * D; it += kThreads) {
-        const int h = it / D, dim = it % D;
-        float O = 0.f;
-        for (int s = 0; s < ns; ++s)
-            O = fmaf(__ldcg(part_bg + (size_t)s * kPartStride + h * (D + 2) + dim), wsm[s * kGroup + h], O);
-        out[((size_t)b * Hq + g * kGroup + h) * D + dim] = O;
+    // outputs as float4 groups (head, 4 dims); TPG threads per group split the
+    // partials and combine with shuffles; loads are issued 8 at a time
+    constexpr int kGroups4 = kGroup * D / 4;
+    constexpr int TPG = kThreads / kGroups4;
+    {
+        const int grp = tid / TPG, j = tid % TPG;
+        const int h = grp / (D / 4), d4 = grp % (D / 4);
+        const float *src = part_bg + h * kHS + d4 * 4;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = j; s0 < ns; s0 += 8 * TPG) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = s0 + u * TPG;
+                v[u] = s < ns ? __ldcg(reinterpret_cast<const float4 *>(src + (size_t)s * kPartStride))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = s0 + u * TPG;
+                const float wgt = s < ns ? wsm[s * kGroup + h] : 0.f;
+                o.x = fmaf(v[u].x, wgt, o.x); o.y = fmaf(v[u].y, wgt, o.y);
+                o.z = fmaf(v[u].z, wgt, o.z); o.w = fmaf(v[u].w, wgt, o.w);
+            }
+        }
+#pragma unroll
+        for (int off = 1; off < TPG; off <<= 1) {
+            o.x += __shfl_xor_sync(kFull, o.x, off); o.y += __shfl_xor_sync(kFull, o.y, off);
+            o.z += __shfl_xor_sync(kFull, o.z, off); o.w += __shfl_xor_sync(kFull, o.w, off);
+        }
+        if (j == 0) {  // scalar stores: `out` is only required to be 4-byte aligned
+            float *dst = out + ((size_t)b * Hq + g * kGroup + h) * D + d4 * 4;
+            dst[0] = o.x; dst[1] = o.y; dst[2] = o.z; dst[3] = o.w;
+        }
     }
     if (tid == 0) counters[b * Hkv + g] = 0u;  // leave the ticket zeroed for the next call
 }
@@ -437,8 +487,7 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const int chunk = attn_chunk(d);
-    const int nsplit = (d.ctx_cap + chunk - 1) / chunk;
+    const int splits = attn_splits(d);
     uint8_t *w = static_cast<uint8_t *>(ws);
     uint32_t *flags = reinterpret_cast<uint32_t *>(w);
     uint32_t *counters = reinterpret_cast<uint32_t *>(w + kWsHeaderBytes);
@@ -446,33 +495,41 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
         w + kWsHeaderBytes + align_up((size_t)d.batch * d.n_kv_heads * 4, 256));
     const int W = (d.ctx_cap + 31) / 32;
     const float qscale = scale * 1.4426950408889634f;  // logits in log2 units for exp2
-    dim3 grid(nsplit, d.n_kv_heads, d.batch);
+    dim3 grid(splits, d.n_kv_heads, d.batch);
     attn_kernel<D, SPARSE><<<grid, kThreads, Smem<D>::kTotal, st>>>(
         Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, qscale,
-        chunk, nsplit, part, counters, out, flags);
+        splits, part, counters, out, flags);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-// Context positions per CTA: the largest power of two in [256, 2048] that
-// still gives at least three waves of two CTAs per SM.
-int attn_chunk(const tb_dims &d) {
+// CTAs per (sequence, KV head): enough for one wave of two CTAs per SM over
+// all (sequence, KV head) pairs, at most kMaxSplits, each with at least one
+// 64-row tile of the longest sequence; among the candidates up to twice that,
+// the count with the best wave quantisation.
+int attn_splits(const tb_dims &d) {
     const long long slots = 2LL * num_sms();
-    int chunk = kMaxChunk;
-    while (chunk > kMinChunk) {
-        const long long ctas = (long long)d.batch * d.n_kv_heads * ((d.ctx_cap + chunk - 1) / chunk);
-        if (ctas >= 3 * slots) break;
-        chunk >>= 1;
+    const long long pairs = (long long)d.batch * d.n_kv_heads;
+    const int max_useful = (d.ctx_cap + kTile - 1) / kTile;
+    int lo = (int)((slots + pairs - 1) / pairs);
+    lo = std::max(1, std::min({lo, kMaxSplits, max_useful}));
+    int best = lo;
+    double best_eff = 0.0;
+    for (int s = lo; s <= std::min({2 * lo, kMaxSplits, max_useful}); ++s) {
+        const long long ctas = pairs * s;
+        const double eff = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = s;
+        }
     }
-    while ((d.ctx_cap + chunk - 1) / chunk > kMaxSplits && chunk < kMaxChunk) chunk <<= 1;
-    return chunk;
+    return best;
 }
 
 size_t attn_ws_bytes(const tb_dims &d) {
-    const size_t max_splits = (size_t)(d.ctx_cap + kMinChunk - 1) / kMinChunk;
     return kWsHeaderBytes + align_up((size_t)d.batch * d.n_kv_heads * 4, 256) +
-           (size_t)d.batch * d.n_kv_heads * max_splits * kGroup * (d.head_dim + 2) * 4;
+           (size_t)d.batch * d.n_kv_heads * kMaxSplits * kGroup * (d.head_dim + 4) * 4;
 }
 
 cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,

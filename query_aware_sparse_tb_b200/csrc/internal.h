@@ -11,7 +11,7 @@ namespace tb {
 
 // ---- attention (attn.cu) ----
 size_t attn_ws_bytes(const tb_dims &d);
-int attn_chunk(const tb_dims &d);
+int attn_splits(const tb_dims &d);
 cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *ctx_len, int32_t sink, int32_t window,
                         const uint32_t *sel_bits, bool sparse, float scale, float *out, void *ws,

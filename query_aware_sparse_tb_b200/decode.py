@@ -1,0 +1,243 @@
+"""Decode-loop driver for the TokenButler path on device-resident buffers.
+
+The schedule (TokenButler technical summary, gist.science):
+  * "Core architecture": queries are predicted at producer layers placed at a
+    fixed depth stride and consumed by the following layers; each producer
+    call emits G slot-specific queries per head (here G = stride and slot j
+    serves layer p + j).
+  * "Optimisations: batching": keys are projected in batches of N tokens, not
+    at every step (N = the local window, so every candidate [S, T-N) always
+    has a projected key).
+  * "Optimisations: prediction interval and neighbour fetch": the predictor,
+    and with it scoring and selection, runs once every P steps; the selection
+    is reused unchanged in between, while sink and window follow the current
+    length.
+
+Every step of the path runs in libtb's CUDA kernels; this module only decides
+which entry point runs when, on which buffers, and can record a whole run into
+one CUDA graph.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib as L
+
+
+def is_prediction_step(step: int, interval: int) -> bool:
+    return step % interval == 0
+
+
+def producer_layer(layer: int, stride: int) -> int:
+    return layer - layer % stride
+
+
+def query_slot(layer: int, stride: int) -> int:
+    return layer % stride
+
+
+def projection_schedule(ctx0: list[int], window: int, steps: int):
+    """Prefill lengths and per-step projection batches.
+
+    Returns (prefill, events) where prefill[b] = floor(ctx0[b]/N)*N rows are
+    projected before decoding, and events maps a step index to a list of
+    per-sequence batch starts (-1 = this sequence projects nothing at that
+    step).  A sequence projects its next N rows at the first step whose length
+    T = ctx0 + step + 1 is N past its projected prefix."""
+    prefill = [(t // window) * window for t in ctx0]
+    proj = list(prefill)
+    events: dict[int, list[int]] = {}
+    for i in range(steps):
+        begins = [-1] * len(ctx0)
+        for b, t0 in enumerate(ctx0):
+            if t0 + i + 1 - proj[b] >= window:
+                begins[b] = proj[b]
+                proj[b] += window
+        if any(x >= 0 for x in begins):
+            events[i] = begins
+    return prefill, events
+
+
+@dataclass(frozen=True)
+class DecodeShape:
+    batch: int
+    n_layers: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    d_proj: int
+    hidden: int            # 0: q' is supplied directly (no predictor MLP)
+    inter: int
+    stride: int            # producer depth stride = slots per producer call
+    sink: int
+    window: int
+    budget: int
+    nbr: int
+    interval: int
+    ctx_cap: int
+
+    @property
+    def n_out(self) -> int:
+        return self.stride * self.n_q_heads * self.d_proj
+
+    @property
+    def idx_cap(self) -> int:
+        return min((2 * self.nbr + 1) * self.budget, self.ctx_cap)
+
+    @property
+    def words(self) -> int:
+        return (self.ctx_cap + 31) // 32
+
+
+class SparseDecoder:
+    """Owns the per-layer state of the sparse path (projected keys, predicted
+    queries, selections) and the workspaces, and issues the schedule.
+
+    K[l], V[l]: [batch][Hkv][ctx_cap][d] bf16 caches (rows of future decode
+    tokens may already be present; only rows < T are ever read).
+    Wk[l]: [Hkv][d'][d] bf16.  mlp[p] = (W1, W2) for each producer layer p."""
+
+    def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda"):
+        s = self.shape = shape
+        self.K, self.V, self.Wk, self.mlp = K, V, Wk, mlp
+        self.ctx0 = list(ctx0)
+        self.steps = steps
+        self.device = device
+        self.dims = L.dims(s.batch, s.n_q_heads, s.n_kv_heads, s.head_dim, s.d_proj, s.ctx_cap)
+        self.scale = 1.0 / math.sqrt(s.head_dim)
+        B, Hq, Hkv = s.batch, s.n_q_heads, s.n_kv_heads
+        self.Kp = [torch.zeros(B, Hkv, s.ctx_cap, s.d_proj, dtype=torch.bfloat16, device=device)
+                   for _ in range(s.n_layers)]
+        self.producers = [l for l in range(s.n_layers) if l % s.stride == 0]
+        self.qp = {p: torch.zeros(B, s.stride, Hq, s.d_proj, dtype=torch.float32, device=device)
+                   for p in self.producers}
+        self.idx = [torch.zeros(B, Hq, s.idx_cap, dtype=torch.int32, device=device) for _ in range(s.n_layers)]
+        self.cnt = [torch.zeros(B, Hq, dtype=torch.int32, device=device) for _ in range(s.n_layers)]
+        self.bits = [torch.zeros(B, Hq, s.words, dtype=torch.int32, device=device) for _ in range(s.n_layers)]
+        self.ws_sel = L.workspace(L.score_select_workspace_bytes(self.dims), device)
+        self.ws_attn = L.workspace(L.attn_workspace_bytes(self.dims), device)
+        self.ws_proj = L.workspace(L.project_keys_workspace_bytes(), device)
+        self.ws_pred = (L.workspace(L.predict_queries_workspace_bytes(B, s.hidden, s.inter, s.n_out), device)
+                        if s.hidden > 0 else None)
+        self.ctx = torch.tensor([[t + i + 1 for t in ctx0] for i in range(steps)], dtype=torch.int32,
+                                device=device)
+        prefill, events = projection_schedule(self.ctx0, s.window, steps)
+        self.prefill_len = prefill
+        self.proj_steps = sorted(events)
+        self.proj_begin = {i: torch.tensor(events[i], dtype=torch.int32, device=device) for i in events}
+        self.proj_count = {i: torch.tensor([s.window if x >= 0 else 0 for x in events[i]], dtype=torch.int32,
+                                           device=device) for i in events}
+        self._zero_begin = torch.zeros(B, dtype=torch.int32, device=device)
+        self._prefill_t = torch.tensor(prefill, dtype=torch.int32, device=device)
+
+    # -------------------------------------------------------------- pieces
+    def prefill(self, stream=None):
+        """Project the prefilled prefix [0, floor(T0/N)*N) of every layer."""
+        mx = max(self.prefill_len)
+        for l in range(self.shape.n_layers):
+            L.project_keys(self.dims, self.K[l], self.Wk[l], self.Kp[l], self._zero_begin, self._prefill_t, mx,
+                           self.ws_proj, stream)
+
+    def project(self, step: int, layer: int, stream=None):
+        if step in self.proj_begin:
+            L.project_keys(self.dims, self.K[layer], self.Wk[layer], self.Kp[layer], self.proj_begin[step],
+                           self.proj_count[step], self.shape.window, self.ws_proj, stream)
+
+    def predict(self, producer: int, h, stream=None):
+        W1, W2 = self.mlp[producer]
+        L.predict_queries(h, W1, W2, self.qp[producer], self.ws_pred, stream)
+
+    def select(self, step: int, layer: int, qp_direct=None, stream=None):
+        s = self.shape
+        if qp_direct is not None:
+            qp, stride = qp_direct, s.n_q_heads * s.d_proj
+        else:
+            # slot j of the producer's [batch][G][Hq][d'] buffer: base + j*Hq*d',
+            # batch stride G*Hq*d' (floats)
+            buf = self.qp[producer_layer(layer, s.stride)]
+            qp = buf.data_ptr() + query_slot(layer, s.stride) * s.n_q_heads * s.d_proj * 4
+            stride = s.stride * s.n_q_heads * s.d_proj
+        L.score_select(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window, s.budget, s.nbr,
+                       self.idx[layer], self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+
+    def attend(self, step: int, layer: int, Q, out, stream=None):
+        s = self.shape
+        L.sparse_decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], s.sink, s.window,
+                             self.bits[layer], self.scale, out, self.ws_attn, stream)
+
+    def attend_dense(self, step: int, layer: int, Q, out, stream=None):
+        L.decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], self.scale, out, self.ws_attn,
+                      stream)
+
+    # -------------------------------------------------------------- one step
+    def step(self, step: int, Q, out, h=None, qp_direct=None, stream=None, marks=None):
+        """One decode step over all layers.
+
+        Q: [n_layers][batch][Hq][d] bf16; out: [n_layers][batch][Hq][d] fp32;
+        h: [n_producers][batch][hidden] bf16 (prediction steps, MLP shapes);
+        qp_direct: [n_layers][batch][Hq][d'] fp32 (shapes without an MLP).
+        The selection work of a prediction step is issued before the step's
+        attention launches; `marks(name)` is called between the two groups so
+        a caller can bracket them with events."""
+        s = self.shape
+        if step in self.proj_begin:
+            for l in range(s.n_layers):
+                self.project(step, l, stream)
+        if is_prediction_step(step, s.interval):
+            for l in range(s.n_layers):
+                if s.hidden > 0 and l in self.qp:
+                    self.predict(l, h[self.producers.index(l)], stream)
+                self.select(step, l, None if qp_direct is None else qp_direct[l], stream)
+        if marks:
+            marks("attn_begin")
+        for l in range(s.n_layers):
+            self.attend(step, l, Q[l], out[l], stream)
+        if marks:
+            marks("attn_end")
+
+    def dense_step(self, step: int, Q, out, stream=None, marks=None):
+        if marks:
+            marks("attn_begin")
+        for l in range(self.shape.n_layers):
+            self.attend_dense(step, l, Q[l], out[l], stream)
+        if marks:
+            marks("attn_end")
+
+
+# ------------------------------------------------------------------ events
+
+_cudart = None
+
+
+def _rt():
+    """The CUDA runtime torch already loaded (for external event records)."""
+    global _cudart
+    if _cudart is None:
+        _cudart = ctypes.CDLL("libcudart.so.12")
+        _cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        _cudart.cudaEventRecordWithFlags.restype = ctypes.c_int
+        _cudart.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t,
+                                              ctypes.c_size_t, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+        _cudart.cudaMemcpy2DAsync.restype = ctypes.c_int
+    return _cudart
+
+
+def record_event(ev: torch.cuda.Event, stream: torch.cuda.Stream):
+    """Record `ev` on `stream`; inside a stream capture this becomes an event
+    record node of the graph (cudaEventRecordExternal), so its timestamp is
+    taken on every replay."""
+    err = _rt().cudaEventRecordWithFlags(ctypes.c_void_p(ev.cuda_event), ctypes.c_void_p(stream.cuda_stream), 1)
+    if err != 0:
+        raise RuntimeError(f"cudaEventRecordWithFlags failed ({err})")
+
+
+def memcpy2d_async(dst: int, dpitch: int, src: int, spitch: int, width: int, height: int, kind: int,
+                   stream: torch.cuda.Stream):
+    err = _rt().cudaMemcpy2DAsync(ctypes.c_void_p(dst), dpitch, ctypes.c_void_p(src), spitch, width, height, kind,
+                                  ctypes.c_void_p(stream.cuda_stream))
+    if err != 0:
+        raise RuntimeError(f"cudaMemcpy2DAsync failed ({err})")
