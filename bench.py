@@ -475,6 +475,7 @@ def main():
     ap.add_argument("--workload", default="llama64k", choices=sorted(tb_inputs.WORKLOADS))
     ap.add_argument("--impl", default="tb", choices=["tb", "reference"])
     ap.add_argument("--decode-steps", type=int, default=None, help="decode steps per run (default: workload's)")
+    ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -495,6 +496,8 @@ def main():
     L.load()
     base = tb_inputs.WORKLOADS[args.workload]
     w = base.scaled(seed=base.seed + rank)           # an independent replica per rank
+    if args.layers:
+        w = w.scaled(n_layers=args.layers)
     run = Run(w, device, steps=args.decode_steps)
     run.dec.prefill()
     torch.cuda.synchronize()

@@ -47,7 +47,11 @@ struct Smem {
     static constexpr int kList = kMaxChunk * 4;
     static constexpr int kP = kWarps * 32 * 4;
     static constexpr int kWords = (kMaxChunk / 32) * 4;
-    static constexpr int kTotal = kPipe + kList + kP + kWords;
+    // per-warp transpose buffer (16 values x 32 lanes): at D = 128 it overlays
+    // the warp's own 8 K rows of the current stage (2 KB), at D = 64 it has its
+    // own space
+    static constexpr int kRed = D == 128 ? 0 : kWarps * 16 * 32 * 4;
+    static constexpr int kTotal = kPipe + kList + kP + kWords + kRed;
     // the pipeline region is reused for the end-of-CTA combine and the merge
     static_assert(kWarps * kGroup * (D + 2) * 4 <= kPipe, "combine scratch");
     static_assert(kMaxSplits * kGroup * 4 <= kPipe, "merge scratch");
@@ -60,16 +64,24 @@ __device__ __forceinline__ float comp4(const float4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// Load DPL bf16 values of one row chunk from shared memory as fp32.
+// Raw DPL bf16 values of one row chunk (8 -> uint4, 4 -> uint2 in .x/.y).
 template <int DPL>
-__device__ __forceinline__ void load_chunk(const uint16_t *p, float (&f)[DPL]) {
+__device__ __forceinline__ uint4 load_raw(const uint16_t *p) {
     if constexpr (DPL == 8) {
-        uint4 u = *reinterpret_cast<const uint4 *>(p);
-        f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
-        f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+        return *reinterpret_cast<const uint4 *>(p);
     } else {
-        uint2 u = *reinterpret_cast<const uint2 *>(p);
-        f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        return make_uint4(u.x, u.y, 0u, 0u);
+    }
+}
+// bf16 pairs -> fp32 pairs (element 2e in .x, 2e+1 in .y).
+template <int DPL>
+__device__ __forceinline__ void unpack2(const uint4 &u, float2 (&f)[DPL / 2]) {
+    f[0] = make_float2(bf16_lo(u.x), bf16_hi(u.x));
+    f[1] = make_float2(bf16_lo(u.y), bf16_hi(u.y));
+    if constexpr (DPL == 8) {
+        f[2] = make_float2(bf16_lo(u.z), bf16_hi(u.z));
+        f[3] = make_float2(bf16_lo(u.w), bf16_hi(u.w));
     }
 }
 
@@ -113,32 +125,39 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
 
     if (p_begin < T) {
         // ------------------------------------------------ per-lane query slice
-        float q[kGroup][DPL];
+        // (pairs of dims, pre-scaled into log2 units)
+        constexpr int DP2 = DPL / 2;
+        float2 q2[kGroup][DP2];
 #pragma unroll
         for (int h = 0; h < kGroup; ++h) {
             const uint16_t *qp = Q + ((size_t)b * Hq + g * kGroup + h) * D + c * DPL;
+            uint4 u;
             if constexpr (DPL == 8) {
-                uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp));
-                q[h][0] = bf16_lo(u.x); q[h][1] = bf16_hi(u.x); q[h][2] = bf16_lo(u.y);
-                q[h][3] = bf16_hi(u.y); q[h][4] = bf16_lo(u.z); q[h][5] = bf16_hi(u.z);
-                q[h][6] = bf16_lo(u.w); q[h][7] = bf16_hi(u.w);
+                u = __ldg(reinterpret_cast<const uint4 *>(qp));
             } else {
-                uint2 u = __ldg(reinterpret_cast<const uint2 *>(qp));
-                q[h][0] = bf16_lo(u.x); q[h][1] = bf16_hi(u.x); q[h][2] = bf16_lo(u.y);
-                q[h][3] = bf16_hi(u.y);
+                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(qp));
+                u = make_uint4(v.x, v.y, 0u, 0u);
             }
+            unpack2<DPL>(u, q2[h]);
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) q[h][e] *= qscale;
+            for (int e = 0; e < DP2; ++e) q2[h][e] = __fmul2_rn(q2[h][e], make_float2(qscale, qscale));
         }
 
-        float m_run[kGroup], l[kGroup], acc[kGroup][DPL];
+        // online-softmax state: m_run is a shared reference per head, raised
+        // only when a logit exceeds it by more than kLazy (log2 units), so every
+        // weight exp2(x - m_run) stays <= 2^kLazy; the result is the same
+        // softmax, m_run just need not be the running maximum
+        constexpr float kLazy = 8.0f;
+        float m_run[kGroup];
+        float2 l2[2];
+        float2 acc2[kGroup][DP2];
 #pragma unroll
         for (int h = 0; h < kGroup; ++h) {
             m_run[h] = -INFINITY;
-            l[h] = 0.f;
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+            for (int e = 0; e < DP2; ++e) acc2[h][e] = make_float2(0.f, 0.f);
         }
+        l2[0] = l2[1] = make_float2(0.f, 0.f);
         const uint32_t pipe_s = smem_addr(pipe);
         const int rb = warp * 8 + half * 4;  // this half-warp's first row in a tile
 
@@ -233,45 +252,52 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                 const uint16_t *Vs = Ks + kTile * D;
 
                 // partial q.k over this lane's slice: 4 rows x 4 heads
+                uint4 kr[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) kr[j] = load_raw<DPL>(Ks + (rb + j) * D + c * DPL);
                 float s[16];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    float kf[DPL];
-                    load_chunk<DPL>(Ks + (rb + j) * D + c * DPL, kf);
+                    float2 k2[DP2];
+                    unpack2<DPL>(kr[j], k2);
 #pragma unroll
                     for (int h = 0; h < kGroup; ++h) {
-                        float a = 0.f;
+                        float2 a = __fmul2_rn(q2[h][0], k2[0]);
 #pragma unroll
-                        for (int e = 0; e < DPL; ++e) a = fmaf(q[h][e], kf[e], a);
-                        s[j * 4 + h] = a;
+                        for (int e = 1; e < DP2; ++e) a = __ffma2_rn(q2[h][e], k2[e], a);
+                        s[j * 4 + h] = a.x + a.y;
                     }
                 }
-                // transposing butterfly over the 16 lanes of a row group: lane c
-                // ends with the full sum of value c = (row c>>2, head c&3)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const bool up = c & 8;
-                    float send = up ? s[k] : s[k + 8], keep = up ? s[k + 8] : s[k];
-                    s[k] = keep + __shfl_xor_sync(kFull, send, 8);
+                // transpose through shared memory: value v = (row v>>2, head
+                // v&3) of lane l goes to red[v][l ^ swz(v)]; lane c of each
+                // half then sums the 16 values (row c>>2, head c&3) of its
+                // half.  The XOR swizzle keeps both sides bank-conflict free.
+                float *red;
+                if constexpr (D == 128) {
+                    red = reinterpret_cast<float *>(const_cast<uint16_t *>(Ks) + warp * 8 * D);
+                } else {
+                    red = reinterpret_cast<float *>(smem + S::kPipe + S::kList + S::kP + S::kWords) +
+                          warp * 16 * 32;
                 }
+                __syncwarp();  // every lane holds its K chunks before the rows are overwritten
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const bool up = c & 4;
-                    float send = up ? s[k] : s[k + 4], keep = up ? s[k + 4] : s[k];
-                    s[k] = keep + __shfl_xor_sync(kFull, send, 4);
-                }
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const bool up = c & 2;
-                    float send = up ? s[k] : s[k + 2], keep = up ? s[k + 2] : s[k];
-                    s[k] = keep + __shfl_xor_sync(kFull, send, 2);
-                }
+                for (int v = 0; v < 16; ++v) red[v * 32 + (lane ^ ((v & 7) << 2))] = s[v];
+                __syncwarp();
+                float x;
                 {
-                    const bool up = c & 1;
-                    float send = up ? s[0] : s[1], keep = up ? s[1] : s[0];
-                    s[0] = keep + __shfl_xor_sync(kFull, send, 1);
+                    const float *rp = red + c * 32;
+                    const int sw = (c & 7) << 2;
+                    const float4 r0 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 0) ^ sw));
+                    const float4 r1 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 4) ^ sw));
+                    const float4 r2 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 8) ^ sw));
+                    const float4 r3 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 12) ^ sw));
+                    float2 a0 = __fadd2_rn(make_float2(r0.x, r0.y), make_float2(r0.z, r0.w));
+                    float2 a1 = __fadd2_rn(make_float2(r1.x, r1.y), make_float2(r1.z, r1.w));
+                    float2 a2 = __fadd2_rn(make_float2(r2.x, r2.y), make_float2(r2.z, r2.w));
+                    float2 a3 = __fadd2_rn(make_float2(r3.x, r3.y), make_float2(r3.z, r3.w));
+                    a0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+                    x = a0.x + a0.y;
                 }
-                float x = s[0];
                 const int hh = c & 3;
                 {
                     const int gr = t * kTile + rb + (c >> 2);
@@ -279,50 +305,51 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                     if (gr < n_rows) mk = SPARSE ? (uint32_t)(list[gr] & 0xF) : 0xFu;
                     if (!((mk >> hh) & 1u)) x = -INFINITY;
                 }
-                // tile max per head over the warp's 8 rows
-                float mx = x;
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                float alpha[kGroup];
-                bool changed = false;
+                // raise the per-head references only when some logit of the
+                // warp's 8 rows exceeds its reference by more than kLazy
+                if (__any_sync(kFull, x > pick4(m_run, hh) + kLazy)) {
+                    float mx = x;
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
 #pragma unroll
-                for (int h = 0; h < kGroup; ++h) {
-                    const float mt = __shfl_sync(kFull, mx, h);
-                    const float mn = fmaxf(m_run[h], mt);
-                    alpha[h] = (mn == m_run[h]) ? 1.f : exp2f(m_run[h] - mn);
-                    changed |= (mn != m_run[h]);
-                    m_run[h] = mn;
+                    for (int h = 0; h < kGroup; ++h) {
+                        const float mn = fmaxf(m_run[h], __shfl_sync(kFull, mx, h));
+                        if (mn > m_run[h]) {
+                            const float alpha = exp2f(m_run[h] - mn);  // 0 while m_run is -inf
+                            const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+                            for (int e = 0; e < DP2; ++e) acc2[h][e] = __fmul2_rn(acc2[h][e], a2);
+                            if (h == 0) l2[0].x *= alpha;
+                            if (h == 1) l2[0].y *= alpha;
+                            if (h == 2) l2[1].x *= alpha;
+                            if (h == 3) l2[1].y *= alpha;
+                            m_run[h] = mn;
+                        }
+                    }
                 }
                 const float p = (x == -INFINITY) ? 0.f : exp2f(x - pick4(m_run, hh));
-                __syncwarp();
-                pbuf[warp * 32 + lane] = p;
+                __syncwarp();  // transpose values read before the slot is reused
+                red[lane] = p;
                 __syncwarp();
                 float4 pr[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    pr[j] = *reinterpret_cast<const float4 *>(pbuf + warp * 32 + half * 16 + j * 4);
-
-                if (changed) {
-#pragma unroll
-                    for (int h = 0; h < kGroup; ++h) {
-                        l[h] *= alpha[h];
-#pragma unroll
-                        for (int e = 0; e < DPL; ++e) acc[h][e] *= alpha[h];
-                    }
-                }
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h)
-                    l[h] += comp4(pr[0], h) + comp4(pr[1], h) + comp4(pr[2], h) + comp4(pr[3], h);
+                for (int j = 0; j < 4; ++j) pr[j] = *reinterpret_cast<const float4 *>(red + half * 16 + j * 4);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    float vf[DPL];
-                    load_chunk<DPL>(Vs + (rb + j) * D + c * DPL, vf);
+                    l2[0] = __fadd2_rn(l2[0], make_float2(pr[j].x, pr[j].y));
+                    l2[1] = __fadd2_rn(l2[1], make_float2(pr[j].z, pr[j].w));
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float2 v2[DP2];
+                    unpack2<DPL>(load_raw<DPL>(Vs + (rb + j) * D + c * DPL), v2);
 #pragma unroll
                     for (int h = 0; h < kGroup; ++h) {
                         const float ph = comp4(pr[j], h);
+                        const float2 pp = make_float2(ph, ph);
 #pragma unroll
-                        for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(ph, vf[e], acc[h][e]);
+                        for (int e = 0; e < DP2; ++e) acc2[h][e] = __ffma2_rn(pp, v2[e], acc2[h][e]);
                     }
                 }
             }
@@ -331,11 +358,16 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
         }
 
         // ------------------------------------------------ combine halves, warps
+        float l[kGroup] = {l2[0].x, l2[0].y, l2[1].x, l2[1].y};
+        float acc[kGroup][DPL];
 #pragma unroll
         for (int h = 0; h < kGroup; ++h) {
             l[h] += __shfl_xor_sync(kFull, l[h], 16);
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[h][e] += __shfl_xor_sync(kFull, acc[h][e], 16);
+            for (int e = 0; e < DP2; ++e) {
+                acc[h][2 * e] = acc2[h][e].x + __shfl_xor_sync(kFull, acc2[h][e].x, 16);
+                acc[h][2 * e + 1] = acc2[h][e].y + __shfl_xor_sync(kFull, acc2[h][e].y, 16);
+            }
         }
         float *cacc = reinterpret_cast<float *>(smem);           // [warp][head][D]
         float *cml = cacc + kWarps * kGroup * D;                 // [warp][head][m, l]
