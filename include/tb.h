@@ -201,6 +201,29 @@ tb_status tb_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K
                          const tb_bf16 *V, const int32_t *ctx_len, float scale, float *out,
                          void *ws, size_t ws_bytes, void *stream);
 
+/* ---- sparse decode attention without a workspace ------------------------- */
+/* No counterpart in the paper: an integration convenience of this library.
+ * For callers that cannot allocate device memory for the call — a plugin or
+ * custom-operator boundary that is handed only its inputs and outputs, or a
+ * decode loop that must not call cudaMalloc on the hot path because it can
+ * synchronise the whole device.  Same arguments and result as
+ * tb_sparse_decode_attn, minus the workspace: the scratch is one fixed,
+ * file-scope device array of TB_NOALLOC_SCRATCH_BYTES that every GPU loading
+ * the library keeps until the process exits.
+ *  - Limit: dims whose tb_attn_workspace_bytes() exceeds
+ *    TB_NOALLOC_SCRATCH_BYTES are rejected with TB_ERR_WORKSPACE (at
+ *    head_dim 128 that is at most 31 (sequence, KV head) pairs).
+ *  - The first call on a device sets the scratch up (address lookup and a
+ *    synchronous clear); make that first call before any stream capture.
+ *  - All calls on a device share the scratch: calls that overlap on the GPU
+ *    race and give wrong outputs.  Device-side flags are not reported.
+ *  - Nothing is allocated or freed. */
+#define TB_NOALLOC_SCRATCH_BYTES (4u << 20)
+tb_status tb_sparse_decode_attn_noalloc(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
+                                        const tb_bf16 *V, const int32_t *ctx_len, int32_t sink,
+                                        int32_t window, const uint32_t *sel_bits, float scale,
+                                        float *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,7 @@ EXPORTS = [
     "tb_predict_queries_workspace_bytes", "tb_project_keys_workspace_bytes",
     "tb_workspace_init", "tb_workspace_check",
     "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_select_bits_from_idx",
-    "tb_sparse_decode_attn", "tb_decode_attn",
+    "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc",
 ]
 
 
@@ -69,6 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_select_bits_from_idx": ([D, P, i32, P, P, P], ctypes.c_int),
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
+        "tb_sparse_decode_attn_noalloc": ([D, P, P, P, P, i32, i32, P, f32, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -179,6 +180,14 @@ def sparse_decode_attn(d: TbDims, Q, K, V, ctx_len, sink: int, window: int, sel_
     _check(load().tb_sparse_decode_attn(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), sink,
                                         window, _ptr(sel_bits), float(scale), _ptr(out), _ptr(ws), _bytes(ws),
                                         _stream(stream)))
+
+
+def sparse_decode_attn_noalloc(d: TbDims, Q, K, V, ctx_len, sink: int, window: int, sel_bits, scale: float,
+                               out, stream=None):
+    """tb_sparse_decode_attn with the library's fixed scratch instead of a
+    workspace (for callers that cannot allocate; see include/tb.h)."""
+    _check(load().tb_sparse_decode_attn_noalloc(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), sink,
+                                                window, _ptr(sel_bits), float(scale), _ptr(out), _stream(stream)))
 
 
 def decode_attn(d: TbDims, Q, K, V, ctx_len, scale: float, out, ws, stream=None):
