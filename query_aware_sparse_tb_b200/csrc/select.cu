@@ -35,6 +35,7 @@ constexpr int kBins1 = 2048;          // key bits 31..21
 constexpr int kBins2 = 2048;          // key bits 20..10
 constexpr int kBins3 = 1024;          // key bits 9..0
 constexpr int kFinThreads = 1024;
+constexpr int kCandCache = 8192;      // candidates staged in shared memory by finalize
 constexpr unsigned kFull = 0xffffffffu;
 
 enum : uint32_t { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
@@ -79,47 +80,86 @@ size_t carve_bytes(const tb_dims &d) {
            align_up(rows * d.ctx_cap * 8, 256) + align_up(rows * W * 4, 256);
 }
 
-// Walk `nbins` histogram bins from the highest down (one warp) and find the bin
-// in which the running count reaches `need`.  Returns the bin; *rem receives
-// how many keys of that bin are still needed.
-__device__ int find_bin_desc(const uint32_t *hist, int nbins, uint32_t need, uint32_t *rem,
-                             bool cg) {
-    const int lane = threadIdx.x & 31;
-    for (int base = nbins - 1; base >= 0; base -= 32) {
-        const int bin = base - lane;
-        const uint32_t v = bin >= 0 ? (cg ? __ldcg(hist + bin) : hist[bin]) : 0u;
-        uint32_t incl = v;
+// Exclusive prefix sum over the block (NT threads, in thread order); *total
+// gets the sum.  `scratch` holds NT/32 + 1 ints.  All threads must call.
+template <int NT>
+__device__ int block_excl_scan(int v, int *scratch, int *total) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < NW ? scratch[lane] : 0;
+        int wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += t;
+            const int t = __shfl_up_sync(kFull, wi, o);
+            if (lane >= o) wi += t;
         }
-        const uint32_t total = __shfl_sync(kFull, incl, 31);
-        if (need <= total) {
-            const uint32_t hit = __ballot_sync(kFull, incl >= need);
-            const int L = __ffs(hit) - 1;
-            const uint32_t vL = __shfl_sync(kFull, v, L);
-            const uint32_t iL = __shfl_sync(kFull, incl, L);
-            *rem = need - (iL - vL);
-            return base - L;
-        }
-        need -= total;
+        if (lane < NW) scratch[lane] = wi - w;
+        if (lane == NW - 1) scratch[NW] = wi;
     }
-    *rem = 0;
-    return 0;
+    __syncthreads();
+    const int res = scratch[warp] + incl - v;
+    *total = scratch[NW];
+    __syncthreads();
+    return res;
+}
+
+// The bin that holds the `need`-th largest key of a histogram (bins in key
+// order), searched from the top by the whole block: thread t owns the t-th
+// group of bins counted from the top, a block scan gives every thread the
+// count above its group, and the one thread whose group crosses `need` walks
+// it.  Returns the bin; *rem = how many keys of that bin are still needed.
+// `hist` may be global (read through L2) or shared; `scratch` holds NT/32 + 3
+// ints.  All threads must call; nbins is a multiple of NT.
+template <int NT>
+__device__ int block_find_bin_desc(const uint32_t *hist, int nbins, uint32_t need, uint32_t *rem,
+                                   int *scratch, bool from_global) {
+    const int per = nbins / NT;
+    const int hi = nbins - threadIdx.x * per;  // this thread's bins are [hi - per, hi)
+    int mine = 0;
+    for (int j = 1; j <= per; ++j) mine += (int)(from_global ? __ldcg(hist + hi - j) : hist[hi - j]);
+    int total;
+    const int above = block_excl_scan<NT>(mine, scratch, &total);
+    if ((uint32_t)above < need && need <= (uint32_t)(above + mine)) {
+        uint32_t acc = (uint32_t)above;
+        for (int j = 1; j <= per; ++j) {
+            const uint32_t v = from_global ? __ldcg(hist + hi - j) : hist[hi - j];
+            if (acc + v >= need) {
+                scratch[NT / 32 + 1] = hi - j;
+                scratch[NT / 32 + 2] = (int)(need - acc);
+                break;
+            }
+            acc += v;
+        }
+    }
+    __syncthreads();
+    const int bin = scratch[NT / 32 + 1];
+    *rem = (uint32_t)scratch[NT / 32 + 2];
+    __syncthreads();
+    return bin;
 }
 
 // ------------------------------------------------------------------ kernel 1
 
 template <int DP>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
+    constexpr int PER = kChunk / kThreads;  // positions per thread
     __shared__ float qs[kGroup][DP];
     __shared__ uint32_t hist[kGroup][kBins1];
     __shared__ int s_last;
-    const int tid = threadIdx.x;
+    __shared__ int scratch[kThreads / 32 + 3];
+    const int tid = threadIdx.x, lane = tid & 31;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
     const int lo = sink, hi = T - window;
@@ -130,28 +170,57 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     __syncthreads();
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
+    if (hi > lo && p0 < hi && p0 + kChunk > lo) {
+        // two rows per batch: both rows' loads (clamped into C) first, then
+        // the arithmetic straight from the packed bf16 pairs
 #pragma unroll
-    for (int k = 0; k < kChunk / kThreads; ++k) {
-        const int p = p0 + k * kThreads + tid;
-        if (p >= lo && p < hi) {
-            const uint4 *row = reinterpret_cast<const uint4 *>(Kp + (slab + p) * DP);
-            float kf[DP];
+        for (int k0 = 0; k0 < PER; k0 += 2) {
+            uint4 raw[2][DP / 8];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int p = min(max(p0 + (k0 + k) * kThreads + tid, lo), hi - 1);
+                const uint4 *row = reinterpret_cast<const uint4 *>(Kp + (slab + p) * DP);
+#pragma unroll
+                for (int v = 0; v < DP / 8; ++v) raw[k][v] = __ldg(row + v);
+            }
+            float sc[2][kGroup];
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) sc[k][h] = 0.f;
 #pragma unroll
             for (int v = 0; v < DP / 8; ++v) {
-                const uint4 u = __ldg(row + v);
-                kf[8 * v + 0] = bf16_lo(u.x); kf[8 * v + 1] = bf16_hi(u.x);
-                kf[8 * v + 2] = bf16_lo(u.y); kf[8 * v + 3] = bf16_hi(u.y);
-                kf[8 * v + 4] = bf16_lo(u.z); kf[8 * v + 5] = bf16_hi(u.z);
-                kf[8 * v + 6] = bf16_lo(u.w); kf[8 * v + 7] = bf16_hi(u.w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 8 * v + 2 * e;  // dims j, j+1 of both rows
+                    float kl[2], kh[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const uint32_t wd = e == 0 ? raw[k][v].x : e == 1 ? raw[k][v].y : e == 2 ? raw[k][v].z : raw[k][v].w;
+                        kl[k] = bf16_lo(wd);
+                        kh[k] = bf16_hi(wd);
+                    }
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) {
+                        const float qa = qs[h][j], qb = qs[h][j + 1];
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) sc[k][h] = fmaf(qb, kh[k], fmaf(qa, kl[k], sc[k][h]));
+                    }
+                }
             }
 #pragma unroll
-            for (int h = 0; h < kGroup; ++h) {
-                float s = 0.f;
+            for (int k = 0; k < 2; ++k) {
+                const int p = p0 + (k0 + k) * kThreads + tid;
+                const bool valid = p >= lo && p < hi;
 #pragma unroll
-                for (int j = 0; j < DP; ++j) s = fmaf(qs[h][j], kf[j], s);
-                const uint32_t key = score_key(s);
-                ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
-                atomicAdd(&hist[h][key >> 21], 1u);
+                for (int h = 0; h < kGroup; ++h) {
+                    const uint32_t key = score_key(sc[k][h]);
+                    if (valid) ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
+                    // lanes of the warp that fall in the same bin add once
+                    const uint32_t bin = valid ? (key >> 21) : 0xFFFFFFFFu;
+                    const uint32_t peers = __match_any_sync(kFull, bin);
+                    if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[h][bin], (uint32_t)__popc(peers));
+                }
             }
         }
     }
@@ -168,28 +237,49 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     if (!s_last) return;
     __threadfence();
 
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < kGroup) {
-        const size_t row = (size_t)b * Hq + g * kGroup + warp;
-        uint32_t *gh = ws.hist + row * kBins1;
-        const int nC = hi > lo ? hi - lo : 0;
-        HeadState st = {};
-        if (nC == 0) {
-            st.mode = kModeEmpty;
-        } else if (nC <= budget) {
-            st.mode = kModeAll;
-        } else {
-            uint32_t rem;
-            const int bin = find_bin_desc(gh, kBins1, (uint32_t)budget, &rem, true);
-            st.mode = kModeSelect;
-            st.b1 = (uint32_t)bin;
-            st.k_rem = rem;
-            st.n_in_bin = __ldcg(gh + bin);
+    const int nC = hi > lo ? hi - lo : 0;
+    const uint32_t *gh0 = ws.hist + ((size_t)b * Hq + g * kGroup) * kBins1;
+    if (nC > budget) {
+        // thread t owns bins [hi_t - PERB, hi_t) of each head's histogram,
+        // counted from the top; all loads first, then one scan per head
+        constexpr int PERB = kBins1 / kThreads;
+        const int hb = kBins1 - tid * PERB;
+        uint32_t v[kGroup][PERB];
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h)
+#pragma unroll
+            for (int j = 0; j < PERB; ++j) v[h][j] = __ldcg(gh0 + (size_t)h * kBins1 + hb - 1 - j);
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            int mine = 0;
+#pragma unroll
+            for (int j = 0; j < PERB; ++j) mine += (int)v[h][j];
+            int total;
+            const int above = block_excl_scan<kThreads>(mine, scratch, &total);
+            if ((uint32_t)above < (uint32_t)budget && (uint32_t)budget <= (uint32_t)(above + mine)) {
+                uint32_t acc = (uint32_t)above;
+#pragma unroll
+                for (int j = 0; j < PERB; ++j) {
+                    if (acc + v[h][j] >= (uint32_t)budget) {
+                        HeadState st = {};
+                        st.mode = kModeSelect;
+                        st.b1 = (uint32_t)(hb - 1 - j);
+                        st.k_rem = (uint32_t)budget - acc;
+                        st.n_in_bin = v[h][j];
+                        ws.state[(size_t)b * Hq + g * kGroup + h] = st;
+                        break;
+                    }
+                    acc += v[h][j];
+                }
+            }
         }
-        __syncwarp();
-        for (int i = lane; i < kBins1; i += 32) gh[i] = 0u;  // leave zeroed for the next call
-        if (lane == 0) ws.state[row] = st;
+    } else if (tid < kGroup) {
+        HeadState st = {};
+        st.mode = nC == 0 ? kModeEmpty : kModeAll;
+        ws.state[(size_t)b * Hq + g * kGroup + tid] = st;
     }
+    __syncthreads();
+    for (int i = tid; i < kGroup * kBins1; i += kThreads) ws.hist[((size_t)b * Hq + g * kGroup) * kBins1 + i] = 0u;
     if (tid == 0) ws.counters[b * Hkv + g] = 0u;
 }
 
@@ -198,11 +288,14 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
 __global__ void __launch_bounds__(kThreads)
 mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int W,
                     int sink, int window, SelWs ws) {
+    constexpr int kWordsPerWarp = kChunk / 32 / (kThreads / 32);  // 4
+    __shared__ uint32_t s_cnt[kGroup], s_base[kGroup];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, false);
     const int lo = sink, hi = T - window;
     const int w0 = ch * (kChunk / 32);
+    if (tid < kGroup) s_cnt[tid] = 0u;
 
     uint32_t mode[kGroup], b1[kGroup];
 #pragma unroll
@@ -211,65 +304,61 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
         mode[h] = st.mode;
         b1[h] = st.b1;
     }
-    for (int wi = warp; wi < kChunk / 32; wi += kThreads / 32) {
-        const int w = w0 + wi;
-        if (w >= W) break;
+    __syncthreads();
+    // pass 1: Top bits, candidate ballots and this warp's offsets inside the CTA
+    // (every key load issued before the first ballot)
+    uint32_t key[kWordsPerWarp][kGroup], cb[kWordsPerWarp][kGroup], off[kWordsPerWarp][kGroup];
+#pragma unroll
+    for (int i = 0; i < kWordsPerWarp; ++i) {
+        const int w = w0 + warp + i * (kThreads / 32);
         const int p = (w << 5) + lane;
-        const bool in_c = p >= lo && p < hi;
+        const bool in_c = w < W && p >= lo && p < hi;
 #pragma unroll
         for (int h = 0; h < kGroup; ++h) {
             const size_t row = (size_t)b * Hq + g * kGroup + h;
-            uint32_t key = 0;
-            if (in_c && mode[h] == kModeSelect) key = ws.keys[row * Tcap + p];
-            const uint32_t d1 = key >> 21;
+            key[i][h] = (in_c && mode[h] == kModeSelect) ? __ldcg(ws.keys + row * Tcap + p) : 0u;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kWordsPerWarp; ++i) {
+        const int w = w0 + warp + i * (kThreads / 32);
+        const int p = (w << 5) + lane;
+        const bool in_c = w < W && p >= lo && p < hi;
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            const size_t row = (size_t)b * Hq + g * kGroup + h;
+            const uint32_t k = key[i][h];
+            const uint32_t d1 = k >> 21;
             const bool top = in_c && (mode[h] == kModeAll || (mode[h] == kModeSelect && d1 > b1[h]));
             const bool cand = in_c && mode[h] == kModeSelect && d1 == b1[h];
             const uint32_t tb = __ballot_sync(kFull, top);
-            if (lane == 0) ws.top[row * W + w] = tb;
-            const uint32_t cb = __ballot_sync(kFull, cand);
-            if (cb) {
-                const int leader = __ffs(cb) - 1;
-                uint32_t base = 0;
-                if (lane == leader) base = atomicAdd(&ws.state[row].cand_count, (uint32_t)__popc(cb));
-                base = __shfl_sync(kFull, base, leader);
-                if (cand)
-                    ws.cand[row * Tcap + base + __popc(cb & ((1u << lane) - 1u))] =
-                        ((unsigned long long)key << 32) | (uint32_t)p;
+            if (lane == 0 && w < W) ws.top[row * W + w] = tb;
+            cb[i][h] = __ballot_sync(kFull, cand);
+            uint32_t o = 0;
+            if (lane == 0 && cb[i][h]) o = atomicAdd(&s_cnt[h], (uint32_t)__popc(cb[i][h]));
+            off[i][h] = __shfl_sync(kFull, o, 0);
+        }
+    }
+    __syncthreads();
+    if (tid < kGroup && s_cnt[tid])
+        s_base[tid] = atomicAdd(&ws.state[(size_t)b * Hq + g * kGroup + tid].cand_count, s_cnt[tid]);
+    __syncthreads();
+    // pass 2: the candidates, (key, position) pairs, in the reserved range
+#pragma unroll
+    for (int i = 0; i < kWordsPerWarp; ++i) {
+        const int p = ((w0 + warp + i * (kThreads / 32)) << 5) + lane;
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            if ((cb[i][h] >> lane) & 1u) {
+                const size_t row = (size_t)b * Hq + g * kGroup + h;
+                ws.cand[row * Tcap + s_base[h] + off[i][h] + __popc(cb[i][h] & ((1u << lane) - 1u))] =
+                    ((unsigned long long)key[i][h] << 32) | (uint32_t)p;
             }
         }
     }
 }
 
 // ------------------------------------------------------------------ kernel 3
-
-// Exclusive prefix sum over the block (1024 threads); *total gets the sum.
-__device__ int block_excl_scan(int v, int *scratch, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = scratch[lane];
-        int wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(kFull, wi, o);
-            if (lane >= o) wi += t;
-        }
-        scratch[lane] = wi - w;
-        if (lane == 31) scratch[32] = wi;
-    }
-    __syncthreads();
-    const int res = scratch[warp] + incl - v;
-    *total = scratch[32];
-    __syncthreads();
-    return res;
-}
 
 __device__ __forceinline__ uint32_t range_mask(int w, int lo, int hi) {
     if (hi <= lo) return 0u;
@@ -283,12 +372,12 @@ __global__ void __launch_bounds__(kFinThreads)
 finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int sink, int window,
                 int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
                 uint32_t *__restrict__ sel_bits, SelWs ws) {
-    extern __shared__ uint32_t fsm[];
-    uint32_t *top_s = fsm;       // [W]
-    uint32_t *tie_s = fsm + W;   // [W]
+    extern __shared__ unsigned long long fsm8[];
+    unsigned long long *cand_s = fsm8;                                  // [kCandCache]
+    uint32_t *top_s = reinterpret_cast<uint32_t *>(fsm8 + kCandCache);  // [W]
+    uint32_t *tie_s = top_s + W;                                        // [W]
     __shared__ uint32_t hist[kBins2];
-    __shared__ int scratch[33];
-    __shared__ uint32_t s_bin, s_rem;
+    __shared__ int scratch[kFinThreads / 32 + 3];
 
     const int tid = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
@@ -302,8 +391,14 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         tie_s[w] = 0u;
     }
     if (st.mode == kModeSelect) {
-        const unsigned long long *cand = ws.cand + row * Tcap;
         const int n = (int)st.cand_count;
+        // the candidate list is read three times: stage it in shared memory
+        // when it fits
+        const unsigned long long *cand = ws.cand + row * Tcap;
+        if (n <= kCandCache) {
+            for (int i = tid; i < n; i += kFinThreads) cand_s[i] = cand[i];
+            cand = cand_s;
+        }
         // digit 2: key bits 20..10 inside bin b1
         for (int i = tid; i < kBins2; i += kFinThreads) hist[i] = 0u;
         __syncthreads();
@@ -312,13 +407,8 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
             atomicAdd(&hist[(key >> 10) & 0x7FFu], 1u);
         }
         __syncthreads();
-        if (tid < 32) {
-            uint32_t rem;
-            const int bin = find_bin_desc(hist, kBins2, st.k_rem, &rem, false);
-            if (tid == 0) { s_bin = bin; s_rem = rem; }
-        }
-        __syncthreads();
-        const uint32_t b2 = s_bin, k2 = s_rem;
+        uint32_t k2;
+        const uint32_t b2 = (uint32_t)block_find_bin_desc<kFinThreads>(hist, kBins2, st.k_rem, &k2, scratch, false);
         // digit 3: key bits 9..0 inside (b1, b2)
         for (int i = tid; i < kBins3; i += kFinThreads) hist[i] = 0u;
         __syncthreads();
@@ -327,14 +417,9 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
             if (((key >> 10) & 0x7FFu) == b2) atomicAdd(&hist[key & 0x3FFu], 1u);
         }
         __syncthreads();
-        if (tid < 32) {
-            uint32_t rem;
-            const int bin = find_bin_desc(hist, kBins3, k2, &rem, false);
-            if (tid == 0) { s_bin = bin; s_rem = rem; }
-        }
-        __syncthreads();
-        const uint32_t tau = (st.b1 << 21) | (b2 << 10) | s_bin;
-        const uint32_t k3 = s_rem;  // keys equal to tau still to take, lowest positions first
+        uint32_t k3;  // keys equal to tau still to take, lowest positions first
+        const uint32_t b3 = (uint32_t)block_find_bin_desc<kFinThreads>(hist, kBins3, k2, &k3, scratch, false);
+        const uint32_t tau = (st.b1 << 21) | (b2 << 10) | b3;
         for (int i = tid; i < n; i += kFinThreads) {
             const unsigned long long e = cand[i];
             const uint32_t key = (uint32_t)(e >> 32), p = (uint32_t)e;
@@ -348,7 +433,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         int mine = 0;
         for (int w = wb; w < we; ++w) mine += __popc(tie_s[w]);
         int tot;
-        int before = block_excl_scan(mine, scratch, &tot);
+        int before = block_excl_scan<kFinThreads>(mine, scratch, &tot);
         for (int w = wb; w < we; ++w) {
             uint32_t t = tie_s[w];
             const int pc = __popc(t);
@@ -382,7 +467,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         mine += __popc(e);
     }
     int total;
-    int base = block_excl_scan(mine, scratch, &total);
+    int base = block_excl_scan<kFinThreads>(mine, scratch, &total);
     int32_t *out = idx + row * (size_t)idx_cap;
     for (int w = wb; w < we; ++w) {
         uint32_t e = tie_s[w];
@@ -445,7 +530,7 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                                    sink, window, s);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t fsm = (size_t)2 * W * 4;
+    const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4;
     static size_t configured = 0;
     if (fsm > 48 * 1024 && fsm > configured) {
         e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
