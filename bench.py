@@ -256,6 +256,26 @@ class E2E:
             self.out_host[i].copy_(r.out, non_blocking=True)
 
 
+def replica(base: tb_inputs.Workload, rank: int) -> tb_inputs.Workload:
+    """Rank `rank`'s independent replica: same shapes, its own seeded data."""
+    return base.scaled(seed=base.seed + rank)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (the job is as slow as its slowest
+    rank); identity outside torch.distributed."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def aggregate_rate(world: int, units_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return world * units_per_rank_step / (ms_per_step / 1000.0)
+
+
 def time_graph(g, warmup, steps, dist_on, device):
     for _ in range(warmup):
         g.replay()
@@ -269,12 +289,9 @@ def time_graph(g, warmup, steps, dist_on, device):
         g.replay()
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), device)
     if dist_on:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-        ms = t.item()
     return ms
 
 
@@ -316,6 +333,21 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu capture of `kernel`, or
+    None when that kernel's source has changed since the capture."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+                return None
+        return rec["dram_read_bytes"] + rec["dram_write_bytes"]
+    except Exception:
+        return None
 
 
 def measured_peaks():
@@ -427,6 +459,14 @@ def cpu_baseline(w, budget_s=25.0):
             "sample_seconds": round(time.perf_counter() - t_start + smp.proj_s, 1)}
 
 
+def config_of(w: tb_inputs.Workload, decode_steps: int, world: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": w.name, "batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
+            "layers": w.n_layers, "decode_steps_per_bench_step": decode_steps, "budget": w.budget,
+            "interval": w.interval, "sink": w.sink, "window": w.window, "d_proj": w.d_proj,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -434,8 +474,8 @@ def run_reference(args):
     w = tb_inputs.WORKLOADS[args.workload]
     smp = OracleSample(w)
     t_pred, t_reuse = [], []
-    for i in range(args.warmup):
-        smp.step(1 + i if w.interval > 1 else 0)
+    for i in range(args.warmup):        # step 0 predicts, so reuse steps have a selection
+        smp.step(i)
     order = list(range(args.steps))
     t_all0 = time.perf_counter()
     for i in order:
@@ -454,7 +494,7 @@ def run_reference(args):
             "unit": "decode steps/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1000 * wall / max(1, len(order)), 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx0, "layers": w.n_layers},
+            "config": config_of(w, args.decode_steps or w.steps, args.gpus),
             "cpu_baseline": {"value": round(value, 4), "unit": "decode steps/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "decode steps/s", "h2d_bytes_per_step": 0,
@@ -495,7 +535,7 @@ def main():
                                              device_id=torch.device(device))
     L.load()
     base = tb_inputs.WORKLOADS[args.workload]
-    w = base.scaled(seed=base.seed + rank)           # an independent replica per rank
+    w = replica(base, rank)                          # an independent replica per rank
     if args.layers:
         w = w.scaled(n_layers=args.layers)
     run = Run(w, device, steps=args.decode_steps)
@@ -530,8 +570,8 @@ def main():
     tokens_per_run = run.steps * w.batch
     per_step_sparse = ms_sparse / args.steps
     per_step_dense = ms_dense / args.steps
-    value = world * tokens_per_run / (per_step_sparse / 1000.0)
-    dense_value = world * tokens_per_run / (per_step_dense / 1000.0)
+    value = aggregate_rate(world, tokens_per_run, per_step_sparse)
+    dense_value = aggregate_rate(world, tokens_per_run, per_step_dense)
     peak, peak_kind = measured_peaks()
     n_attn = run.steps * w.n_layers
     attn_launch_ms = sum(attn_ms) / n_attn
@@ -552,12 +592,9 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_sparse, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; Llama-3.1-8B attention shapes, random weights)",
-        "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
-                   "layers": w.n_layers, "decode_steps_per_bench_step": run.steps, "budget": w.budget,
-                   "interval": w.interval, "sink": w.sink, "window": w.window, "d_proj": w.d_proj,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (KV %.1f GB)" % (2 * sum(k.numel() for k in run.K) * 2 / 1e9),
-                   "graph": "one CUDA graph per bench step"},
+        "config": dict(config_of(w, run.steps, world),
+                       l2="inputs larger than L2 (KV %.1f GB)" % (2 * sum(k.numel() for k in run.K) * 2 / 1e9),
+                       graph="one CUDA graph per bench step"),
         "speedup_vs_dense": round(value / dense_value, 4),
         "dense": {"value": round(dense_value, 3), "unit": "decode steps/s", "ms_per_step": round(per_step_dense, 4),
                   "path_gbs": round(dense_path_gbs, 1), "attn_launch_us": round(1000 * dense_launch_ms, 3),
@@ -568,7 +605,7 @@ def main():
                 "dense_bytes_per_bench_step": acct["dense_total"]},
         "roofline": {"kernel": "attn_kernel<128,true> (sparse GQA decode attention)", "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("attn_kernel<128,true>"),
                      "bytes_per_launch": round(attn_bytes_per_launch), "launch_us": round(1000 * attn_launch_ms, 3)},
         "gpu_launches": (sparse_launches) * args.steps,
         "clocks": clk,
@@ -576,7 +613,7 @@ def main():
     }
     if e2e is not None:
         h2d, d2h = e2e.bytes_per_run()
-        line["e2e"] = {"value": round(world * tokens_per_run / (ms_e2e / args.steps / 1000.0), 3),
+        line["e2e"] = {"value": round(aggregate_rate(world, tokens_per_run, ms_e2e / args.steps), 3),
                        "unit": "decode steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": round(ms_e2e / args.steps, 4)}
     if world == 1 and not args.no_cpu_baseline:
