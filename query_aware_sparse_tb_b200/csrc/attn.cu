@@ -9,18 +9,30 @@
 // bottleneck.  The attention itself is standard scaled dot-product attention
 // restricted to those rows (fp32 logits, fp32 online softmax, fp32 sums).
 //
-// Work split: one CTA per (sequence b, KV head g, context chunk).  The CTA
-// builds the chunk's row list (sparse: union over the 4 query heads of the
-// group of their selected bits, plus sink and window rows, each row tagged
-// with a 4-bit head mask), then streams the K and V rows of that list through
-// a 3-stage cp.async pipeline in shared memory, so every (b, g, t) row crosses
-// HBM once for the whole group.  Each warp takes 8 rows of a 64-row tile; a
-// half-warp owns 4 rows and each lane 1/16 of head_dim, so every K/V element
-// a lane loads is used by all 4 query heads.  Partial dot products are summed
-// across the 16 lanes of a row by a transposing butterfly (15 shuffles for 16
-// sums), the online-softmax state is per warp, and the last CTA of each
-// (b, g) — found with an atomic ticket, never a wait — merges the chunks'
+// Work split: one CTA per (sequence b, KV head g, context slice), one CTA per
+// SM.  Every kept (b, g, t) row crosses HBM once for the whole group of 4
+// query heads.  Warp roles:
+//   * 4 load warps build the slice's row list (sparse: union over the group's
+//     heads of their selected bits, plus sink and window rows, each row
+//     tagged with a 4-bit head mask) and stream 128-row K and V tiles into a
+//     3-stage shared-memory ring with cp.async, in the 128-byte-swizzled
+//     layout the tensor cores read;
+//   * 1 MMA warp issues, per tile, S^T = K Q^T (M = 128 rows, N = 16 with the
+//     4 heads in columns 0..3) and O^T = V^T P^T (M = 128 head dims, N = 16:
+//     columns 0..3 take the bf16 high parts of the softmax weights, 4..7 the
+//     bf16 remainders, so the weights keep ~16 significant bits), both bf16
+//     tcgen05.mma into fp32 TMEM accumulators;
+//   * 4 softmax warps (thread = tile row, then thread = head dim) read the
+//     logits from TMEM, keep the online-softmax state, write P to shared
+//     memory and fold each tile's O^T into fp32 registers.
+// The S product of tile i+1 overlaps the softmax of tile i, and the PV
+// product of tile i overlaps the softmax of tile i+1.  The last CTA of each
+// (b, g), found with an atomic ticket, never a wait, merges the slices'
 // partial states into the fp32 output.
+//
+// Every mbarrier wait is bounded; a wait that runs out flags TB_FLAG_TIMEOUT,
+// tells the other roles through shared memory, and every role leaves its loop
+// (the roles agree before each named barrier, so none is left waiting there).
 #include <math.h>
 
 #include <algorithm>
@@ -31,90 +43,114 @@
 namespace tb {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kTile = 64;       // rows per pipeline stage
+constexpr int kGroup = 4;          // query heads per KV head
+constexpr int kRows = 128;         // KV rows per tile (M of the S^T product)
 constexpr int kStages = 3;
-constexpr int kGroup = 4;       // query heads per KV head
-constexpr int kMaxChunk = 2048; // positions per row list (a CTA walks its range in sub-chunks)
-constexpr int kMaxSplits = 64;   // partial states merged per (sequence, KV head)
+constexpr int kSub = 4096;         // positions per row list (sparse)
+constexpr int kMaxSplits = 64;     // partial states merged per (sequence, KV head)
+constexpr int kN = 16;             // N of both products (padded)
+constexpr int kRoleThreads = 128;  // threads of the softmax role and of the load role
+constexpr int kThreads = 2 * kRoleThreads + 32;
+constexpr int kMergeThreads = 256;
+constexpr uint32_t kTmemCols = 64;  // S^T x2 buffers, O^T x2 buffers, 16 columns each
 constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLazy = 8.0f;
+// named barrier ids (0 is __syncthreads)
+constexpr uint32_t kBarLoad = 1, kBarMath = 2, kBarMath2 = 3;
 
-template <int D>
+// Shared memory map, offsets from the 1024-byte aligned base.
 struct Smem {
-    static constexpr int kStageBytes = 2 * kTile * D * 2;  // K tile + V tile, bf16
-    static constexpr int kPipe = kStages * kStageBytes;
-    static constexpr int kList = kMaxChunk * 4;
-    static constexpr int kP = kWarps * 32 * 4;
-    static constexpr int kWords = (kMaxChunk / 32) * 4;
-    // per-warp transpose buffer (16 values x 32 lanes): at D = 128 it overlays
-    // the warp's own 8 K rows of the current stage (2 KB), at D = 64 it has its
-    // own space
-    static constexpr int kRed = D == 128 ? 0 : kWarps * 16 * 32 * 4;
-    static constexpr int kTotal = kPipe + kList + kP + kWords + kRed;
-    // the pipeline region is reused for the end-of-CTA combine and the merge
-    static_assert(kWarps * kGroup * (D + 2) * 4 <= kPipe, "combine scratch");
-    static_assert(kMaxSplits * kGroup * 4 <= kPipe, "merge scratch");
+    static constexpr int kHalf = kRows * 128;         // [128 rows][64 dims] bf16, swizzled
+    static constexpr int kSlot = 2 * kHalf;           // one tensor tile, head dims 0..63 | 64..127
+    static constexpr int kStage = 2 * kSlot;          // K tile, V tile
+    static constexpr int kQ = kStages * kStage;       // Q operand: 2 dim halves x 16 rows x 128 B
+    static constexpr int kP = kQ + 4096;              // P operands: 2 buffers x (2 row halves x 16 x 128 B)
+    static constexpr int kMask = kP + 2 * 4096;       // head masks [kStages][kRows]
+    static constexpr int kList = kMask + kStages * kRows;  // row list: (offset << 4) | mask, uint16
+    static constexpr int kWsum = kList + kSub * 2;         // per-warp row counts of the list build
+    static constexpr int kBar = kWsum + 64;
+    static constexpr int kNumBars = 2 * kStages + 10;
+    static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort, n_rows, meta, reductions
+    static constexpr int kEnd = kMisc + 256;
+    static constexpr int kBytes = kEnd + 1024;  // + alignment slack
+    static_assert(kQ % 1024 == 0 && kP % 1024 == 0, "operand alignment");
+    static_assert(kBar % 8 == 0, "mbarrier alignment");
 };
+static_assert(Smem::kBytes <= 227 * 1024, "shared memory");
 
-__device__ __forceinline__ float pick4(const float (&v)[4], int i) {
-    return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
-}
-__device__ __forceinline__ float comp4(const float4 &v, int i) {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
+// Misc area layout (int/float words)
+constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscMeta = 4, kMiscRed = 8;  // red: 2 x 16 floats
 
-// Raw DPL bf16 values of one row chunk (8 -> uint4, 4 -> uint2 in .x/.y).
-template <int DPL>
-__device__ __forceinline__ uint4 load_raw(const uint16_t *p) {
-    if constexpr (DPL == 8) {
-        return *reinterpret_cast<const uint4 *>(p);
-    } else {
-        const uint2 u = *reinterpret_cast<const uint2 *>(p);
-        return make_uint4(u.x, u.y, 0u, 0u);
+// A bounded mbarrier wait that also gives up as soon as another role of the
+// CTA has given up.
+__device__ __forceinline__ bool wait_role(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t *flags) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitBudgetCycles) {
+            raise_flag(flags, TB_FLAG_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
     }
 }
-// bf16 pairs -> fp32 pairs (element 2e in .x, 2e+1 in .y).
-template <int DPL>
-__device__ __forceinline__ void unpack2(const uint4 &u, float2 (&f)[DPL / 2]) {
-    f[0] = make_float2(bf16_lo(u.x), bf16_hi(u.x));
-    f[1] = make_float2(bf16_lo(u.y), bf16_hi(u.y));
-    if constexpr (DPL == 8) {
-        f[2] = make_float2(bf16_lo(u.z), bf16_hi(u.z));
-        f[3] = make_float2(bf16_lo(u.w), bf16_hi(u.w));
-    }
+
+// bits 0 .. n-1 set (n clamped to [0, 32])
+__device__ __forceinline__ uint32_t bits_below(int n) {
+    return n <= 0 ? 0u : n >= 32 ? 0xffffffffu : (1u << n) - 1u;
+}
+
+// byte offset of element (row r, 16-byte chunk c) in a [rows][64] bf16 half
+// written with the 128-byte swizzle (1024-byte atoms of 8 rows)
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+    return (uint32_t)(r * 128 + (((c ^ r) & 7) << 4));
 }
 
 template <int D, bool SPARSE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             const uint16_t *__restrict__ V, const int32_t *__restrict__ ctx_len,
             const uint32_t *__restrict__ sel_bits, int Hq, int Hkv, int Tcap, int W, int sink,
             int window, float qscale, int splits, float *__restrict__ part,
             uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags) {
-    constexpr int DPL = D / 16;  // head_dim elements per lane
-    constexpr int CPR = D / 8;   // 16-byte chunks per row
-    constexpr int kCopies = kTile * CPR / kThreads;
-    // one partial state per head: O[D], M, L, 2 pad floats, so every head's
-    // record starts 16-byte aligned for the float4 loads of the merge
+    constexpr int CPR = D / 8;      // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;   // rows per warp-wide copy instruction
+    constexpr int kKSteps = D / 16; // MMA K steps of S^T
+    // one partial state per head: O[D], M, L, 2 pad floats (16-byte aligned records)
     constexpr int kHS = D + 4;
     constexpr int kPartStride = kGroup * kHS;
-    using S = Smem<D>;
 
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint16_t *pipe = reinterpret_cast<uint16_t *>(smem);
-    int32_t *list = reinterpret_cast<int32_t *>(smem + S::kPipe);
-    float *pbuf = reinterpret_cast<float *>(smem + S::kPipe + S::kList);
-    int32_t *wcnt = reinterpret_cast<int32_t *>(smem + S::kPipe + S::kList + S::kP);
-    __shared__ int s_nrows, s_last;
-    __shared__ float s_red[kWarps][kGroup];
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_addr(sm);
+    uint8_t *masks = sm + Smem::kMask;
+    uint16_t *list = reinterpret_cast<uint16_t *>(sm + Smem::kList);
+    volatile int *wsum = reinterpret_cast<volatile int *>(sm + Smem::kWsum);
+    volatile int *misc = reinterpret_cast<volatile int *>(sm + Smem::kMisc);
+    volatile int *abort_flag = misc + kMiscAbort;
+    volatile int *meta = misc + kMiscMeta;
+    float *red = reinterpret_cast<float *>(sm + Smem::kMisc) + kMiscRed;
+    const uint32_t qbase = sb + Smem::kQ, pbase = sb + Smem::kP;
+    auto bar = [&](int i) -> uint32_t { return sb + Smem::kBar + 8u * (uint32_t)i; };
+    auto full = [&](int s) { return bar(s); };
+    auto empty = [&](int s) { return bar(kStages + s); };
+    auto s_done = [&](int q) { return bar(2 * kStages + q); };
+    auto p_ready = [&](int q) { return bar(2 * kStages + 2 + q); };
+    auto o_done = [&](int q) { return bar(2 * kStages + 4 + q); };
+    auto o_free = [&](int q) { return bar(2 * kStages + 6 + q); };
+    const uint32_t drain = bar(2 * kStages + 8);
+    const uint32_t q_ready = bar(2 * kStages + 9);
+    __shared__ int s_last;
+    __shared__ float s_red[kMergeThreads / 32][kGroup];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int half = lane >> 4, c = lane & 15;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
-    // this sequence's length split evenly over the CTAs of (b, g), in 64-row units
-    const int chunk = ((T + splits - 1) / splits + kTile - 1) / kTile * kTile;
+    // this sequence's length split evenly over the CTAs of (b, g), in 128-row units
+    const int chunk = ((T + splits - 1) / splits + kRows - 1) / kRows * kRows;
     const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
     const int p_begin = split * chunk;
     const int p_end = min(p_begin + chunk, T);
@@ -123,297 +159,358 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     const uint16_t *Vb = V + slab * D;
     float *part_bg = part + (size_t)(b * Hkv + g) * splits * kPartStride;
 
-    if (p_begin < T) {
-        // ------------------------------------------------ per-lane query slice
-        // (pairs of dims, pre-scaled into log2 units)
-        constexpr int DP2 = DPL / 2;
-        float2 q2[kGroup][DP2];
+    // ------------------------------------------------------------ set-up
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full(s), kRoleThreads);
+            mbar_init(empty(s), 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(s_done(q), 1);
+            mbar_init(p_ready(q), kRoleThreads);
+            mbar_init(o_done(q), 1);
+            mbar_init(o_free(q), kRoleThreads);
+        }
+        mbar_init(drain, 1);
+        mbar_init(q_ready, kRoleThreads);
+        misc[kMiscAbort] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(sb + Smem::kMisc + 4 * kMiscTmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[kMiscTmem];
+
+    float m_ref[kGroup], o_acc[kGroup], L[kGroup];
+    bool math_fail = false;
+
+    if (warp >= 4 && warp < 8) {
+        // ============================================================ loads
+        const int pt = tid - kRoleThreads, pw = warp - 4;
+        int it = 0;
+        bool fail = false;
+        const int step = SPARSE ? kSub : max(p_end - p_begin, 1);
+        // sparse: thread pt owns word pt (32 positions) of a sub-chunk; the
+        // group's 4 selection words of the next sub-chunk are loaded ahead
+        const int hi_c = T - window;  // candidates are [sink, hi_c)
+        const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
+        uint32_t hw[kGroup] = {0u, 0u, 0u, 0u};
+        auto fetch_words = [&](int q0) {
+            const int q1 = min(q0 + kSub, p_end);
+            if (q0 < p_end && q0 + 32 * pt < q1) {
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
-            const uint16_t *qp = Q + ((size_t)b * Hq + g * kGroup + h) * D + c * DPL;
-            uint4 u;
-            if constexpr (DPL == 8) {
-                u = __ldg(reinterpret_cast<const uint4 *>(qp));
-            } else {
-                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(qp));
-                u = make_uint4(v.x, v.y, 0u, 0u);
+                for (int h = 0; h < kGroup; ++h) hw[h] = __ldg(sbits + (size_t)h * W + (q0 >> 5) + pt);
             }
-            unpack2<DPL>(u, q2[h]);
-#pragma unroll
-            for (int e = 0; e < DP2; ++e) q2[h][e] = __fmul2_rn(q2[h][e], make_float2(qscale, qscale));
-        }
-
-        // online-softmax state: m_run is a shared reference per head, raised
-        // only when a logit exceeds it by more than kLazy (log2 units), so every
-        // weight exp2(x - m_run) stays <= 2^kLazy; the result is the same
-        // softmax, m_run just need not be the running maximum
-        constexpr float kLazy = 8.0f;
-        float m_run[kGroup];
-        float2 l2[2];
-        float2 acc2[kGroup][DP2];
-#pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
-            m_run[h] = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < DP2; ++e) acc2[h][e] = make_float2(0.f, 0.f);
-        }
-        l2[0] = l2[1] = make_float2(0.f, 0.f);
-        const uint32_t pipe_s = smem_addr(pipe);
-        const int rb = warp * 8 + half * 4;  // this half-warp's first row in a tile
-
-        // the CTA's range in sub-chunks of at most kMaxChunk positions
-        for (int p0 = p_begin; p0 < p_end; p0 += kMaxChunk) {
-            const int p1 = min(p0 + kMaxChunk, p_end);
-            // -------------------------------------------- row list (sparse)
+        };
+        if constexpr (SPARSE) fetch_words(p_begin);
+        for (int p0 = p_begin; p0 < p_end && !fail; p0 += step) {
+            const int p1 = min(p0 + step, p_end);
             int n_rows = p1 - p0;
             if constexpr (SPARSE) {
-                const int hi_c = T - window;  // candidates are [sink, hi_c)
-                const int nwords = (p1 - p0 + 31) >> 5;
-                const int w0 = p0 >> 5;
-                const uint32_t *sb = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W + w0;
-                auto word_mask = [&](int wi, int &p, int &m) -> uint32_t {
-                    uint32_t hb = lane < kGroup ? __ldg(sb + (size_t)lane * W + wi) : 0u;
-                    uint32_t b0 = __shfl_sync(kFull, hb, 0), b1 = __shfl_sync(kFull, hb, 1);
-                    uint32_t b2 = __shfl_sync(kFull, hb, 2), b3 = __shfl_sync(kFull, hb, 3);
-                    p = p0 + (wi << 5) + lane;
-                    m = 0;
-                    if (p < p1) {
-                        if (p < sink || p >= hi_c) {
-                            m = 0xF;
-                        } else {
-                            m = ((b0 >> lane) & 1u) | (((b1 >> lane) & 1u) << 1) |
-                                (((b2 >> lane) & 1u) << 2) | (((b3 >> lane) & 1u) << 3);
-                        }
-                    }
-                    return __ballot_sync(kFull, m != 0);
-                };
-                for (int wi = warp; wi < nwords; wi += kWarps) {
-                    int p, m;
-                    uint32_t bal = word_mask(wi, p, m);
-                    if (lane == 0) wcnt[wi] = __popc(bal);
-                }
-                __syncthreads();
-                if (warp == 0) {  // exclusive scan of <= 64 word counts
-                    int a0 = (2 * lane < nwords) ? wcnt[2 * lane] : 0;
-                    int a1 = (2 * lane + 1 < nwords) ? wcnt[2 * lane + 1] : 0;
-                    int sum = a0 + a1, incl = sum;
+                // union over the group of the kept positions of this word,
+                // each tagged with its head mask (sink and window: all heads)
+                const int p = p0 + 32 * pt;
+                const uint32_t vmask = bits_below(p1 - p);
+                const uint32_t forced = (bits_below(sink - p) | ~bits_below(hi_c - p)) & vmask;
+                uint32_t sel[kGroup], U = forced;
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        int v = __shfl_up_sync(kFull, incl, o);
-                        if (lane >= o) incl += v;
-                    }
-                    int excl = incl - sum;
-                    if (2 * lane < nwords) wcnt[2 * lane] = excl;
-                    if (2 * lane + 1 < nwords) wcnt[2 * lane + 1] = excl + a0;
-                    if (lane == 31) s_nrows = incl;
+                for (int h = 0; h < kGroup; ++h) {
+                    sel[h] = hw[h] & vmask & ~forced;
+                    U |= sel[h];
                 }
-                __syncthreads();
-                for (int wi = warp; wi < nwords; wi += kWarps) {
-                    int p, m;
-                    uint32_t bal = word_mask(wi, p, m);
-                    if (m) list[wcnt[wi] + __popc(bal & ((1u << lane) - 1u))] = (p << 4) | m;
+                const int cnt = __popc(U);
+                int incl = cnt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(kFull, incl, o);
+                    if (lane >= o) incl += v;
                 }
-                __syncthreads();
-                n_rows = s_nrows;
+                if (lane == 31) wsum[pw] = incl;
+                bar_named(kBarLoad, kRoleThreads);
+                int off = incl - cnt;
+                for (int w = 0; w < pw; ++w) off += wsum[w];
+                n_rows = wsum[0] + wsum[1] + wsum[2] + wsum[3];
+                for (uint32_t u = U; u; u &= u - 1u) {
+                    const int j = __ffs(u) - 1;
+                    const uint32_t mk = ((forced >> j) & 1u)
+                                            ? 0xFu
+                                            : ((sel[0] >> j) & 1u) | (((sel[1] >> j) & 1u) << 1) |
+                                                  (((sel[2] >> j) & 1u) << 2) | (((sel[3] >> j) & 1u) << 3);
+                    list[off++] = (uint16_t)(((32 * pt + j) << 4) | mk);
+                }
+                fetch_words(p0 + step);
+                bar_named(kBarLoad, kRoleThreads);
             }
-
-            const int n_tiles = (n_rows + kTile - 1) / kTile;
-            auto issue = [&](int t) {
-                const uint32_t kbase = pipe_s + (t % kStages) * S::kStageBytes;
-                const uint32_t vbase = kbase + kTile * D * 2;
+            const int n_tiles = (n_rows + kRows - 1) / kRows;
+            for (int t = 0; t < n_tiles; ++t, ++it) {
+                const int s = it % kStages;
+                bool ok = true;
+                if (it >= kStages) ok = wait_role(empty(s), ((it / kStages) + 1) & 1, abort_flag, flags);
+                if (bar_any(kBarLoad, kRoleThreads, !ok)) {
+                    fail = true;
+                    break;
+                }
+                const uint32_t kslot = sb + s * Smem::kStage, vslot = kslot + Smem::kSlot;
 #pragma unroll
-                for (int k = 0; k < kCopies; ++k) {
-                    const int e = tid + k * kThreads;
-                    const int r = e / CPR, ch = e % CPR;
-                    const int gr = t * kTile + r;
+                for (int i = 0; i < CPR; ++i) {
+                    const int r = pw * 32 + i * RPI + lane / CPR, c = lane % CPR;
+                    const int gr = t * kRows + r;
                     const bool valid = gr < n_rows;
-                    int pos = p0;
-                    if (valid) pos = SPARSE ? (list[gr] >> 4) : (p0 + gr);
-                    const size_t off = (size_t)pos * D + ch * 8;
-                    const uint32_t so = (uint32_t)(r * D + ch * 8) * 2u;
-                    cp_async16(kbase + so, Kb + off, valid);
-                    cp_async16(vbase + so, Vb + off, valid);
-                }
-            };
-
-#pragma unroll
-            for (int s = 0; s < kStages - 1; ++s) {
-                if (s < n_tiles) issue(s);
-                cp_async_commit();
-            }
-
-            for (int t = 0; t < n_tiles; ++t) {
-                cp_async_wait<kStages - 2>();
-                __syncthreads();
-                if (t + kStages - 1 < n_tiles) issue(t + kStages - 1);
-                cp_async_commit();
-
-                const uint16_t *Ks = pipe + (t % kStages) * (S::kStageBytes / 2);
-                const uint16_t *Vs = Ks + kTile * D;
-
-                // partial q.k over this lane's slice: 4 rows x 4 heads
-                uint4 kr[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) kr[j] = load_raw<DPL>(Ks + (rb + j) * D + c * DPL);
-                float s[16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float2 k2[DP2];
-                    unpack2<DPL>(kr[j], k2);
-#pragma unroll
-                    for (int h = 0; h < kGroup; ++h) {
-                        float2 a = __fmul2_rn(q2[h][0], k2[0]);
-#pragma unroll
-                        for (int e = 1; e < DP2; ++e) a = __ffma2_rn(q2[h][e], k2[e], a);
-                        s[j * 4 + h] = a.x + a.y;
-                    }
-                }
-                // transpose through shared memory: value v = (row v>>2, head
-                // v&3) of lane l goes to red[v][l ^ swz(v)]; lane c of each
-                // half then sums the 16 values (row c>>2, head c&3) of its
-                // half.  The XOR swizzle keeps both sides bank-conflict free.
-                float *red;
-                if constexpr (D == 128) {
-                    red = reinterpret_cast<float *>(const_cast<uint16_t *>(Ks) + warp * 8 * D);
-                } else {
-                    red = reinterpret_cast<float *>(smem + S::kPipe + S::kList + S::kP + S::kWords) +
-                          warp * 16 * 32;
-                }
-                __syncwarp();  // every lane holds its K chunks before the rows are overwritten
-#pragma unroll
-                for (int v = 0; v < 16; ++v) red[v * 32 + (lane ^ ((v & 7) << 2))] = s[v];
-                __syncwarp();
-                float x;
-                {
-                    const float *rp = red + c * 32;
-                    const int sw = (c & 7) << 2;
-                    const float4 r0 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 0) ^ sw));
-                    const float4 r1 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 4) ^ sw));
-                    const float4 r2 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 8) ^ sw));
-                    const float4 r3 = *reinterpret_cast<const float4 *>(rp + ((half * 16 + 12) ^ sw));
-                    float2 a0 = __fadd2_rn(make_float2(r0.x, r0.y), make_float2(r0.z, r0.w));
-                    float2 a1 = __fadd2_rn(make_float2(r1.x, r1.y), make_float2(r1.z, r1.w));
-                    float2 a2 = __fadd2_rn(make_float2(r2.x, r2.y), make_float2(r2.z, r2.w));
-                    float2 a3 = __fadd2_rn(make_float2(r3.x, r3.y), make_float2(r3.z, r3.w));
-                    a0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
-                    x = a0.x + a0.y;
-                }
-                const int hh = c & 3;
-                {
-                    const int gr = t * kTile + rb + (c >> 2);
-                    uint32_t mk = 0;
-                    if (gr < n_rows) mk = SPARSE ? (uint32_t)(list[gr] & 0xF) : 0xFu;
-                    if (!((mk >> hh) & 1u)) x = -INFINITY;
-                }
-                // raise the per-head references only when some logit of the
-                // warp's 8 rows exceeds its reference by more than kLazy
-                if (__any_sync(kFull, x > pick4(m_run, hh) + kLazy)) {
-                    float mx = x;
-                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-#pragma unroll
-                    for (int h = 0; h < kGroup; ++h) {
-                        const float mn = fmaxf(m_run[h], __shfl_sync(kFull, mx, h));
-                        if (mn > m_run[h]) {
-                            const float alpha = exp2f(m_run[h] - mn);  // 0 while m_run is -inf
-                            const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-                            for (int e = 0; e < DP2; ++e) acc2[h][e] = __fmul2_rn(acc2[h][e], a2);
-                            if (h == 0) l2[0].x *= alpha;
-                            if (h == 1) l2[0].y *= alpha;
-                            if (h == 2) l2[1].x *= alpha;
-                            if (h == 3) l2[1].y *= alpha;
-                            m_run[h] = mn;
+                    int pos = p0, mk = 0;
+                    if (valid) {
+                        if constexpr (SPARSE) {
+                            const int e = list[gr];
+                            pos = p0 + (e >> 4);
+                            mk = e & 0xF;
+                        } else {
+                            pos = p0 + gr;
+                            mk = 0xF;
                         }
                     }
+                    const size_t off = (size_t)pos * D + c * 8;
+                    const uint32_t so = (uint32_t)((c >> 3) * Smem::kHalf) + sw128_off(r, c);
+                    cp_async16(kslot + so, Kb + off, valid);
+                    cp_async16(vslot + so, Vb + off, valid);
+                    if (c == 0) masks[s * kRows + r] = (uint8_t)mk;
                 }
-                const float p = (x == -INFINITY) ? 0.f : exp2f(x - pick4(m_run, hh));
-                __syncwarp();  // transpose values read before the slot is reused
-                red[lane] = p;
-                __syncwarp();
-                float4 pr[4];
+                if (pt == 0) meta[s] = 1;
+                cp_async_mbar_arrive(full(s));
+                mbar_arrive(full(s));
+            }
+            if constexpr (SPARSE) bar_named(kBarLoad, kRoleThreads);  // list and counts read before rebuilding
+        }
+        if (!fail) {  // end marker: a stage with no rows
+            const int s = it % kStages;
+            bool ok = true;
+            if (it >= kStages) ok = wait_role(empty(s), ((it / kStages) + 1) & 1, abort_flag, flags);
+            if (!bar_any(kBarLoad, kRoleThreads, !ok)) {
+                if (pt == 0) meta[s] = 0;
+                mbar_arrive(full(s));
+            }
+        }
+        cp_async_wait_all();
+    } else if (warp == 8) {
+        // ============================================================ MMA issue
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16_f32(kRows, kN);
+            const uint32_t id_o = idesc_bf16_f32(128, kN) | (1u << 15);  // A (V^T) MN-major
+            auto issue_s = [&](int i) {
+                const uint32_t kslot = sb + (i % kStages) * Smem::kStage;
+                const uint32_t d = tmem + (uint32_t)((i & 1) * kN);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) pr[j] = *reinterpret_cast<const float4 *>(red + half * 16 + j * 4);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    l2[0] = __fadd2_rn(l2[0], make_float2(pr[j].x, pr[j].y));
-                    l2[1] = __fadd2_rn(l2[1], make_float2(pr[j].z, pr[j].w));
+                for (int k = 0; k < kKSteps; ++k) {
+                    const uint32_t ko = (uint32_t)((k >> 2) * Smem::kHalf + (k & 3) * 32);
+                    const uint32_t qo = (uint32_t)((k >> 2) * 2048 + (k & 3) * 32);
+                    umma_bf16(d, sw128_kmajor_desc(kslot + ko), sw128_kmajor_desc(qbase + qo), id_s, k > 0);
                 }
+                umma_commit(s_done(i & 1));
+            };
+            auto issue_pv = [&](int i) {
+                const int s = i % kStages;
+                const uint32_t vslot = sb + s * Smem::kStage + Smem::kSlot;
+                const uint32_t pb = pbase + (uint32_t)((i & 1) * 4096);
+                const uint32_t d = tmem + (uint32_t)(2 * kN + (i & 1) * kN);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float2 v2[DP2];
-                    unpack2<DPL>(load_raw<DPL>(Vs + (rb + j) * D + c * DPL), v2);
-#pragma unroll
-                    for (int h = 0; h < kGroup; ++h) {
-                        const float ph = comp4(pr[j], h);
-                        const float2 pp = make_float2(ph, ph);
-#pragma unroll
-                        for (int e = 0; e < DP2; ++e) acc2[h][e] = __ffma2_rn(pp, v2[e], acc2[h][e]);
+                for (int k = 0; k < kRows / 16; ++k) {
+                    const uint32_t po = (uint32_t)((k >> 2) * 2048 + (k & 3) * 32);
+                    umma_bf16(d, sw128_mnmajor_desc(vslot + k * 2048, Smem::kHalf), sw128_kmajor_desc(pb + po),
+                              id_o, k > 0);
+                }
+                umma_commit(o_done(i & 1));
+                umma_commit(empty(s));
+            };
+            bool ok = wait_role(q_ready, 0, abort_flag, flags);
+            if (ok) ok = wait_role(full(0), 0, abort_flag, flags);
+            if (ok && meta[0] != 0) {
+                fence_proxy_async_smem();
+                tc_fence_after();
+                issue_s(0);
+                for (int i = 0;; ++i) {
+                    const int nx = i + 1, sn = nx % kStages;
+                    ok = wait_role(full(sn), (nx / kStages) & 1, abort_flag, flags);
+                    if (!ok) break;
+                    const bool has_next = meta[sn] != 0;
+                    if (has_next) {
+                        fence_proxy_async_smem();
+                        tc_fence_after();
+                        issue_s(nx);
                     }
+                    ok = wait_role(p_ready(i & 1), (i >> 1) & 1, abort_flag, flags);
+                    if (ok && i >= 2) ok = wait_role(o_free(i & 1), ((i >> 1) + 1) & 1, abort_flag, flags);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(i);
+                    if (!has_next) break;
                 }
             }
-            cp_async_wait<0>();
-            __syncthreads();  // pipeline and list free for the next sub-chunk
+            // every MMA of this thread has finished before TMEM is released
+            umma_commit(drain);
+            mbar_wait_bounded(drain, 0, flags);
         }
-
-        // ------------------------------------------------ combine halves, warps
-        float l[kGroup] = {l2[0].x, l2[0].y, l2[1].x, l2[1].y};
-        float acc[kGroup][DPL];
+        __syncwarp();
+    } else {
+        // ============================================================ softmax
+        const int mt = tid;  // tile row, then head dim
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        {
+            // Q operand (K-major, 16 rows: the group's 4 query heads, then
+            // zeros); P operands: rows 8..15 stay zero
+            const uint16_t *Qg = Q + ((size_t)b * Hq + (size_t)g * kGroup) * D;
+            for (int e = mt; e < 2 * kN * 64; e += kRoleThreads) {
+                const int hf = e >> 10, n = (e >> 6) & 15, dd = e & 63, d = hf * 64 + dd;
+                uint16_t v = 0;
+                if (n < kGroup && d < D) v = Qg[(size_t)n * D + d];
+                *reinterpret_cast<uint16_t *>(sm + Smem::kQ + hf * 2048 + (n >> 3) * 1024 +
+                                              sw128_off(n & 7, dd >> 3) + (dd & 7) * 2) = v;
+            }
+            uint4 *pz = reinterpret_cast<uint4 *>(sm + Smem::kP);
+            for (int e = mt; e < 2 * 4096 / 16; e += kRoleThreads) pz[e] = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();
+            mbar_arrive(q_ready);
+        }
+        float l_part[kGroup], mt0[kGroup], mt1[kGroup];
 #pragma unroll
         for (int h = 0; h < kGroup; ++h) {
-            l[h] += __shfl_xor_sync(kFull, l[h], 16);
-#pragma unroll
-            for (int e = 0; e < DP2; ++e) {
-                acc[h][2 * e] = acc2[h][e].x + __shfl_xor_sync(kFull, acc2[h][e].x, 16);
-                acc[h][2 * e + 1] = acc2[h][e].y + __shfl_xor_sync(kFull, acc2[h][e].y, 16);
-            }
+            m_ref[h] = -INFINITY;
+            l_part[h] = 0.f;
+            o_acc[h] = 0.f;
+            mt0[h] = mt1[h] = -INFINITY;
         }
-        float *cacc = reinterpret_cast<float *>(smem);           // [warp][head][D]
-        float *cml = cacc + kWarps * kGroup * D;                 // [warp][head][m, l]
-        if (half == 0) {
-#pragma unroll
-            for (int h = 0; h < kGroup; ++h)
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) cacc[(warp * kGroup + h) * D + c * DPL + e] = acc[h][e];
-        }
-        if (lane == 0) {
+        // fold tile j's O^T (relative to that tile's references) into o_acc
+        auto epilogue = [&](int j) -> bool {
+            const bool ok = wait_role(o_done(j & 1), (j >> 1) & 1, abort_flag, flags);
+            if (bar_any(kBarMath, kRoleThreads, !ok)) return false;
+            tc_fence_after();
+            float ov[8];
+            tmem_ld8(tmem + lane_off + (uint32_t)(2 * kN + (j & 1) * kN), ov);
 #pragma unroll
             for (int h = 0; h < kGroup; ++h) {
-                cml[(warp * kGroup + h) * 2] = m_run[h];
-                cml[(warp * kGroup + h) * 2 + 1] = l[h];
+                const float mj = (j & 1) ? mt1[h] : mt0[h];
+                const float f = (mj == m_ref[h]) ? 1.f : exp2f(mj - m_ref[h]);
+                o_acc[h] = fmaf(ov[h] + ov[kGroup + h], f, o_acc[h]);
             }
-        }
-        __syncthreads();
-        float *pp = part_bg + (size_t)split * kPartStride;
-        for (int it = tid; it < kGroup * D; it += kThreads) {
-            const int h = it / D, dim = it % D;
-            float M = -INFINITY;
+            tc_fence_before();
+            mbar_arrive(o_free(j & 1));
+            return true;
+        };
+        int i = 0;
+        for (;; ++i) {
+            const int s = i % kStages;
+            bool ok = wait_role(full(s), (i / kStages) & 1, abort_flag, flags);
+            if (bar_any(kBarMath, kRoleThreads, !ok)) {
+                math_fail = true;
+                break;
+            }
+            if (meta[s] == 0) break;
+            ok = wait_role(s_done(i & 1), (i >> 1) & 1, abort_flag, flags);
+            if (bar_any(kBarMath, kRoleThreads, !ok)) {
+                math_fail = true;
+                break;
+            }
+            tc_fence_after();
+            float sv[4];
+            tmem_ld4(tmem + lane_off + (uint32_t)((i & 1) * kN), sv);
+            const uint32_t mk = masks[s * kRows + mt];
+            float t[kGroup];
+            bool need = false;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cml[(w * kGroup + h) * 2]);
-            float O = 0.f, L = 0.f;
-            if (M != -INFINITY) {
+            for (int h = 0; h < kGroup; ++h) {
+                t[h] = ((mk >> h) & 1u) ? sv[h] * qscale : -INFINITY;
+                need |= t[h] > m_ref[h] + kLazy;
+            }
+            // raise the per-head references (to the tile maximum) only when a
+            // logit exceeds its reference by more than kLazy, so every weight
+            // exp2(t - m_ref) stays <= 2^kLazy; the softmax is unchanged
+            if (bar_any(kBarMath, kRoleThreads, need)) {
+                float mx[kGroup];
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    const float mw = cml[(w * kGroup + h) * 2];
-                    if (mw != -INFINITY) {
-                        const float f = exp2f(mw - M);
-                        O = fmaf(cacc[(w * kGroup + h) * D + dim], f, O);
-                        L = fmaf(cml[(w * kGroup + h) * 2 + 1], f, L);
+                for (int h = 0; h < kGroup; ++h) {
+                    mx[h] = t[h];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], o));
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) red[warp * kGroup + h] = mx[h];
+                }
+                bar_named(kBarMath2, kRoleThreads);
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    float mn = m_ref[h];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) mn = fmaxf(mn, red[w * kGroup + h]);
+                    if (mn > m_ref[h]) {
+                        const float alpha = exp2f(m_ref[h] - mn);  // 0 while m_ref is -inf
+                        l_part[h] *= alpha;
+                        o_acc[h] *= alpha;
+                        m_ref[h] = mn;
                     }
                 }
+                bar_named(kBarMath2, kRoleThreads);  // red read by all before reuse
             }
-            pp[h * kHS + dim] = O;
-            if (dim == 0) {
-                pp[h * kHS + D] = M;
-                pp[h * kHS + D + 1] = L;
+            // weights as bf16 high part (N rows 0..3) + bf16 remainder (rows 4..7)
+            uint8_t *pb = sm + Smem::kP + (i & 1) * 4096 + (mt >> 6) * 2048 + (mt & 7) * 2;
+            const int rc = (mt & 63) >> 3;
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                const float p = (t[h] == -INFINITY) ? 0.f : exp2f(t[h] - m_ref[h]);
+                l_part[h] += p;
+                const uint16_t hi = f32_to_bf16_rne(p);
+                const uint16_t lo = f32_to_bf16_rne(p - __uint_as_float((uint32_t)hi << 16));
+                *reinterpret_cast<uint16_t *>(pb + sw128_off(h, rc)) = hi;
+                *reinterpret_cast<uint16_t *>(pb + sw128_off(kGroup + h, rc)) = lo;
+                if (i & 1) mt1[h] = m_ref[h]; else mt0[h] = m_ref[h];
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_ready(i & 1));
+            if (i >= 1 && !epilogue(i - 1)) {
+                math_fail = true;
+                break;
+            }
+        }
+        if (!math_fail && i >= 1 && !epilogue(i - 1)) math_fail = true;
+
+        // softmax sums over the 128 rows of the role
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+            float v = l_part[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+            if (lane == 0) red[16 + warp * kGroup + h] = v;
+        }
+        bar_named(kBarMath2, kRoleThreads);
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h)
+            L[h] = red[16 + h] + red[16 + kGroup + h] + red[16 + 2 * kGroup + h] + red[16 + 3 * kGroup + h];
+        if (p_begin < T) {
+            float *pp = part_bg + (size_t)split * kPartStride;
+            if (mt < D) {
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) pp[h * kHS + mt] = o_acc[h];
+            }
+            if (mt == 0) {
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    pp[h * kHS + D] = m_ref[h];
+                    pp[h * kHS + D + 1] = L[h];
+                }
             }
         }
     }
 
-    // ---------------------------------------------------- last CTA merges
+    // ---------------------------------------------------- release, ticket
     __threadfence();
+    tc_fence_before();
     __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
     if (tid == 0) {
         const unsigned prev = atomicAdd(&counters[b * Hkv + g], 1u);
         s_last = (prev == (unsigned)splits - 1u);
@@ -422,44 +519,53 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     if (!s_last) return;
     __threadfence();
 
+    // ---------------------------------------------------- last CTA merges
     // weights w[s][h] = exp2(M_sh - M*_h) / L*_h over the ns <= 64 partials:
     // one (split, head) pair per thread, head = tid & 3
-    float *wsm = reinterpret_cast<float *>(smem);  // [ns][head]
-    {
-        const int h = tid & 3, s = tid >> 2;
-        float m = -INFINITY, lw = 0.f;
-        if (s < ns) {
-            m = __ldcg(part_bg + (size_t)s * kPartStride + h * kHS + D);
-            lw = __ldcg(part_bg + (size_t)s * kPartStride + h * kHS + D + 1);
+    float *wsm = reinterpret_cast<float *>(sm);  // [ns][head]
+    const bool mthr = tid < kMergeThreads;
+    const int mw = tid >> 5;
+    float m = -INFINITY, lw = 0.f, f = 0.f;
+    const int hm = tid & 3, sm_i = tid >> 2;
+    if (mthr) {
+        if (sm_i < ns) {
+            m = __ldcg(part_bg + (size_t)sm_i * kPartStride + hm * kHS + D);
+            lw = __ldcg(part_bg + (size_t)sm_i * kPartStride + hm * kHS + D + 1);
         }
         float mx = m;
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-        if (lane < kGroup) s_red[warp][lane] = mx;
-        __syncthreads();
+        if (lane < kGroup) s_red[mw][lane] = mx;
+    }
+    __syncthreads();
+    if (mthr) {
         float Mh = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) Mh = fmaxf(Mh, s_red[w][h]);
-        const float f = (m == -INFINITY) ? 0.f : exp2f(m - Mh);
+        for (int w = 0; w < kMergeThreads / 32; ++w) Mh = fmaxf(Mh, s_red[w][hm]);
+        f = (m == -INFINITY) ? 0.f : exp2f(m - Mh);
+    }
+    __syncthreads();
+    if (mthr) {
         float lsum = f * lw;
         lsum += __shfl_xor_sync(kFull, lsum, 4);
         lsum += __shfl_xor_sync(kFull, lsum, 8);
         lsum += __shfl_xor_sync(kFull, lsum, 16);
-        __syncthreads();
-        if (lane < kGroup) s_red[warp][lane] = lsum;
-        __syncthreads();
+        if (lane < kGroup) s_red[mw][lane] = lsum;
+    }
+    __syncthreads();
+    if (mthr) {
         float Lh = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) Lh += s_red[w][h];
-        if (s < ns) wsm[s * kGroup + h] = Lh > 0.f ? f / Lh : 0.f;
+        for (int w = 0; w < kMergeThreads / 32; ++w) Lh += s_red[w][hm];
+        if (sm_i < ns) wsm[sm_i * kGroup + hm] = Lh > 0.f ? f / Lh : 0.f;
     }
     __syncthreads();
     // outputs as float4 groups (head, 4 dims); TPG threads per group split the
     // partials and combine with shuffles; loads are issued 8 at a time
     constexpr int kGroups4 = kGroup * D / 4;
-    constexpr int TPG = kThreads / kGroups4;
-    {
+    constexpr int TPG = kMergeThreads / kGroups4;
+    if (mthr) {
         const int grp = tid / TPG, j = tid % TPG;
         const int h = grp / (D / 4), d4 = grp % (D / 4);
         const float *src = part_bg + h * kHS + d4 * 4;
@@ -514,8 +620,7 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, SPARSE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Smem<D>::kTotal);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::kBytes);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -528,7 +633,7 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
     const int W = (d.ctx_cap + 31) / 32;
     const float qscale = scale * 1.4426950408889634f;  // logits in log2 units for exp2
     dim3 grid(splits, d.n_kv_heads, d.batch);
-    attn_kernel<D, SPARSE><<<grid, kThreads, Smem<D>::kTotal, st>>>(
+    attn_kernel<D, SPARSE><<<grid, kThreads, Smem::kBytes, st>>>(
         Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, qscale,
         splits, part, counters, out, flags);
     return cudaGetLastError();
@@ -536,23 +641,21 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
 
 }  // namespace
 
-// CTAs per (sequence, KV head): enough for one wave of two CTAs per SM over
-// all (sequence, KV head) pairs, at most kMaxSplits, each with at least one
-// 64-row tile of the longest sequence; among the candidates up to twice that,
-// the count with the best wave quantisation.
+// CTAs per (sequence, KV head), one CTA per SM: the count s <= kMaxSplits that
+// minimises waves(s) x (tiles per CTA + 2 tiles of pipeline fill), with the
+// context capacity standing in for the (device-side) lengths.
 int attn_splits(const tb_dims &d) {
-    const long long slots = 2LL * num_sms();
+    const long long slots = num_sms();
     const long long pairs = (long long)d.batch * d.n_kv_heads;
-    const int max_useful = (d.ctx_cap + kTile - 1) / kTile;
-    int lo = (int)((slots + pairs - 1) / pairs);
-    lo = std::max(1, std::min({lo, kMaxSplits, max_useful}));
-    int best = lo;
-    double best_eff = 0.0;
-    for (int s = lo; s <= std::min({2 * lo, kMaxSplits, max_useful}); ++s) {
-        const long long ctas = pairs * s;
-        const double eff = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
+    const int max_useful = std::max(1, (d.ctx_cap + kRows - 1) / kRows);
+    int best = 1;
+    long long best_cost = -1;
+    for (int s = 1; s <= std::min(kMaxSplits, max_useful); ++s) {
+        const long long waves = (pairs * s + slots - 1) / slots;
+        const long long tiles = ((long long)d.ctx_cap + (long long)s * kRows - 1) / ((long long)s * kRows);
+        const long long cost = waves * (tiles + 2);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
             best = s;
         }
     }

@@ -187,6 +187,21 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand in the canonical
+// 128-byte-swizzled layout: 64 consecutive MN elements (128 B) per line, 8
+// lines (consecutive K) per 1024-byte atom, K atoms 1024 B apart, MN atoms
+// `mn_stride` bytes apart.  A row-major [K][64] bf16 tile written with the
+// 128-byte swizzle is exactly one column of such atoms.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t mn_stride) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);               // start address
+    d |= (uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16;     // leading byte offset: next MN atom
+    d |= (uint64_t)(1024u >> 4) << 32;                      // stride byte offset: next 8 K lines
+    d |= (uint64_t)1u << 46;                                // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                                // layout: 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                      // D format: fp32
@@ -234,6 +249,65 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
                  : "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i) r[i] = __uint_as_float(v[i]);
+}
+// As tmem_ld16, 4 and 8 columns.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&r)[4]) {
+    uint32_t v[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = __uint_as_float(v[i]);
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8]) {
+    uint32_t v[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = __uint_as_float(v[i]);
+}
+
+// ------------------------------------------------- cp.async -> mbarrier ----
+
+// Arrive on `bar` when every cp.async this thread issued so far has landed
+// (the barrier's pending count is raised now and dropped on completion, so
+// the thread still makes its own regular arrival).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// ------------------------------------------------------ named barriers ----
+
+// Barrier `id` over `n` threads (whole warps) that also returns whether any of
+// them passed `v`.
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t n, bool v) {
+    __syncwarp();  // the barrier is warp-aligned: reconverge after per-lane polling
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void bar_named(uint32_t id, uint32_t n) {
+    __syncwarp();
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
 
 }  // namespace tb
