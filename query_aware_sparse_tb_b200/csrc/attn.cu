@@ -50,7 +50,7 @@ constexpr int kSub = 4096;         // positions per row list (sparse)
 constexpr int kMaxSplits = 64;     // partial states merged per (sequence, KV head)
 constexpr int kN = 16;             // N of both products (padded)
 constexpr int kRoleThreads = 128;  // threads of the softmax role and of the load role
-constexpr int kThreads = 2 * kRoleThreads + 32;
+constexpr int kThreads = 2 * kRoleThreads + 64;  // + an S-issue warp and a PV-issue warp
 constexpr int kMergeThreads = 256;
 constexpr uint32_t kTmemCols = 64;  // S^T x2 buffers, O^T x2 buffers, 16 columns each
 constexpr unsigned kFull = 0xffffffffu;
@@ -82,13 +82,13 @@ static_assert(Smem::kBytes <= 227 * 1024, "shared memory");
 constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscMeta = 4, kMiscRed = 8;  // red: 2 x 16 floats
 
 // A bounded mbarrier wait that also gives up as soon as another role of the
-// CTA has given up.
+// CTA has given up.  The thread sleeps in the barrier between checks.
 __device__ __forceinline__ bool wait_role(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           uint32_t *flags) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitBudgetCycles) {
             raise_flag(flags, TB_FLAG_TIMEOUT);
@@ -96,6 +96,16 @@ __device__ __forceinline__ bool wait_role(uint32_t bar, uint32_t parity, volatil
             return false;
         }
     }
+}
+
+// Shared-memory store of 16 bits when `pred` is non-zero (predicated, no branch).
+__device__ __forceinline__ void st_shared_u16_if(uint32_t addr, uint16_t v, uint32_t pred) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %2, 0;\n\t"
+        "@p st.shared.u16 [%0], %1;\n\t}\n" ::"r"(addr),
+        "h"(v), "r"(pred)
+        : "memory");
 }
 
 // bits 0 .. n-1 set (n clamped to [0, 32])
@@ -127,7 +137,8 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_addr(sm);
     uint8_t *masks = sm + Smem::kMask;
-    uint16_t *list = reinterpret_cast<uint16_t *>(sm + Smem::kList);
+    const uint16_t *list = reinterpret_cast<const uint16_t *>(sm + Smem::kList);
+    const uint32_t list_s = sb + Smem::kList;
     volatile int *wsum = reinterpret_cast<volatile int *>(sm + Smem::kWsum);
     volatile int *misc = reinterpret_cast<volatile int *>(sm + Smem::kMisc);
     volatile int *abort_flag = misc + kMiscAbort;
@@ -144,20 +155,39 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     const uint32_t drain = bar(2 * kStages + 8);
     const uint32_t q_ready = bar(2 * kStages + 9);
     __shared__ int s_last;
-    __shared__ float s_red[kMergeThreads / 32][kGroup];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
-    const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
-    // this sequence's length split evenly over the CTAs of (b, g), in 128-row units
-    const int chunk = ((T + splits - 1) / splits + kRows - 1) / kRows * kRows;
-    const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
+    // the capacity split evenly over the CTAs of (b, g), in 128-row units, so
+    // that a CTA's first positions are known before the length arrives
+    const int chunk = ((Tcap + splits - 1) / splits + kRows - 1) / kRows * kRows;
     const int p_begin = split * chunk;
+    const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
+    const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
     const int p_end = min(p_begin + chunk, T);
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     const uint16_t *Kb = K + slab * D;
     const uint16_t *Vb = V + slab * D;
     float *part_bg = part + (size_t)(b * Hkv + g) * splits * kPartStride;
+
+    // sparse: load warp thread pt owns word pt (32 positions) of a sub-chunk;
+    // the group's 4 selection words of the first sub-chunk are requested
+    // before the set-up, those of the next one while the current is streamed
+    const int pt = tid - kRoleThreads, pw = warp - 4;
+    const bool loader = warp >= 4 && warp < 8;
+    const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
+    uint32_t hw[kGroup] = {0u, 0u, 0u, 0u};
+    // (bounded by the slice and the capacity only: words past the length are
+    // masked when the list is built)
+    const int p_cap_end = min(p_begin + chunk, Tcap);
+    auto fetch_words = [&](int q0) {
+        const int q1 = min(q0 + kSub, p_cap_end);
+        if (q0 + 32 * pt < q1) {
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) hw[h] = __ldg(sbits + (size_t)h * W + (q0 >> 5) + pt);
+        }
+    };
+    if (SPARSE && loader) fetch_words(p_begin);
 
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
@@ -171,12 +201,12 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             mbar_init(o_done(q), 1);
             mbar_init(o_free(q), kRoleThreads);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);
         mbar_init(q_ready, kRoleThreads);
         misc[kMiscAbort] = 0;
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == 8) {  // the S-issue warp owns the TMEM allocation
         tmem_alloc(sb + Smem::kMisc + 4 * kMiscTmem, kTmemCols);
         tmem_relinquish();
     }
@@ -188,25 +218,12 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     float m_ref[kGroup], o_acc[kGroup], L[kGroup];
     bool math_fail = false;
 
-    if (warp >= 4 && warp < 8) {
+    if (loader) {
         // ============================================================ loads
-        const int pt = tid - kRoleThreads, pw = warp - 4;
         int it = 0;
         bool fail = false;
         const int step = SPARSE ? kSub : max(p_end - p_begin, 1);
-        // sparse: thread pt owns word pt (32 positions) of a sub-chunk; the
-        // group's 4 selection words of the next sub-chunk are loaded ahead
         const int hi_c = T - window;  // candidates are [sink, hi_c)
-        const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
-        uint32_t hw[kGroup] = {0u, 0u, 0u, 0u};
-        auto fetch_words = [&](int q0) {
-            const int q1 = min(q0 + kSub, p_end);
-            if (q0 < p_end && q0 + 32 * pt < q1) {
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) hw[h] = __ldg(sbits + (size_t)h * W + (q0 >> 5) + pt);
-            }
-        };
-        if constexpr (SPARSE) fetch_words(p_begin);
         for (int p0 = p_begin; p0 < p_end && !fail; p0 += step) {
             const int p1 = min(p0 + step, p_end);
             int n_rows = p1 - p0;
@@ -216,11 +233,11 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                 const int p = p0 + 32 * pt;
                 const uint32_t vmask = bits_below(p1 - p);
                 const uint32_t forced = (bits_below(sink - p) | ~bits_below(hi_c - p)) & vmask;
-                uint32_t sel[kGroup], U = forced;
+                uint32_t keep[kGroup], U = 0u;  // keep[h]: positions head h attends to
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) {
-                    sel[h] = hw[h] & vmask & ~forced;
-                    U |= sel[h];
+                    keep[h] = (hw[h] & vmask) | forced;
+                    U |= keep[h];
                 }
                 const int cnt = __popc(U);
                 int incl = cnt;
@@ -234,13 +251,20 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                 int off = incl - cnt;
                 for (int w = 0; w < pw; ++w) off += wsum[w];
                 n_rows = wsum[0] + wsum[1] + wsum[2] + wsum[3];
-                for (uint32_t u = U; u; u &= u - 1u) {
-                    const int j = __ffs(u) - 1;
-                    const uint32_t mk = ((forced >> j) & 1u)
-                                            ? 0xFu
-                                            : ((sel[0] >> j) & 1u) | (((sel[1] >> j) & 1u) << 1) |
-                                                  (((sel[2] >> j) & 1u) << 2) | (((sel[3] >> j) & 1u) << 3);
-                    list[off++] = (uint16_t)(((32 * pt + j) << 4) | mk);
+                // the warp writes its 32 words one at a time, lane = bit
+                // (unrolled: the words are independent, so their shuffle ->
+                // count -> store chains overlap)
+                const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 8
+                for (int k = 0; k < 32; ++k) {
+                    const uint32_t k0 = __shfl_sync(kFull, keep[0], k), k1 = __shfl_sync(kFull, keep[1], k);
+                    const uint32_t k2 = __shfl_sync(kFull, keep[2], k), k3 = __shfl_sync(kFull, keep[3], k);
+                    const uint32_t Uk = k0 | k1 | k2 | k3;
+                    const int ok_ = __shfl_sync(kFull, off, k);
+                    const uint32_t mk = ((k0 >> lane) & 1u) | (((k1 >> lane) & 1u) << 1) |
+                                        (((k2 >> lane) & 1u) << 2) | (((k3 >> lane) & 1u) << 3);
+                    st_shared_u16_if(list_s + 2u * (uint32_t)(ok_ + __popc(Uk & lt)),
+                                     (uint16_t)((((pw * 32 + k) * 32 + lane) << 4) | mk), (Uk >> lane) & 1u);
                 }
                 fetch_words(p0 + step);
                 bar_named(kBarLoad, kRoleThreads);
@@ -293,61 +317,55 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             }
         }
         cp_async_wait_all();
-    } else if (warp == 8) {
+    } else if (warp >= 8) {
         // ============================================================ MMA issue
+        // warp 8 issues the S^T products, warp 9 the O^T products; each waits
+        // on one barrier at a time.  S(i) needs tile i's rows and S buffer i&1
+        // read by the softmax of tile i-2; PV(i) needs the softmax of tile i
+        // and O buffer i&1 folded by the epilogue of tile i-2.  A tile's stage
+        // is released by the commit after its PV product (the S product of
+        // the tile has completed before its softmax could start).
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16_f32(kRows, kN);
             const uint32_t id_o = idesc_bf16_f32(128, kN) | (1u << 15);  // A (V^T) MN-major
-            auto issue_s = [&](int i) {
-                const uint32_t kslot = sb + (i % kStages) * Smem::kStage;
-                const uint32_t d = tmem + (uint32_t)((i & 1) * kN);
-#pragma unroll
-                for (int k = 0; k < kKSteps; ++k) {
-                    const uint32_t ko = (uint32_t)((k >> 2) * Smem::kHalf + (k & 3) * 32);
-                    const uint32_t qo = (uint32_t)((k >> 2) * 2048 + (k & 3) * 32);
-                    umma_bf16(d, sw128_kmajor_desc(kslot + ko), sw128_kmajor_desc(qbase + qo), id_s, k > 0);
-                }
-                umma_commit(s_done(i & 1));
-            };
-            auto issue_pv = [&](int i) {
-                const int s = i % kStages;
-                const uint32_t vslot = sb + s * Smem::kStage + Smem::kSlot;
-                const uint32_t pb = pbase + (uint32_t)((i & 1) * 4096);
-                const uint32_t d = tmem + (uint32_t)(2 * kN + (i & 1) * kN);
-#pragma unroll
-                for (int k = 0; k < kRows / 16; ++k) {
-                    const uint32_t po = (uint32_t)((k >> 2) * 2048 + (k & 3) * 32);
-                    umma_bf16(d, sw128_mnmajor_desc(vslot + k * 2048, Smem::kHalf), sw128_kmajor_desc(pb + po),
-                              id_o, k > 0);
-                }
-                umma_commit(o_done(i & 1));
-                umma_commit(empty(s));
-            };
             bool ok = wait_role(q_ready, 0, abort_flag, flags);
-            if (ok) ok = wait_role(full(0), 0, abort_flag, flags);
-            if (ok && meta[0] != 0) {
-                fence_proxy_async_smem();
-                tc_fence_after();
-                issue_s(0);
-                for (int i = 0;; ++i) {
-                    const int nx = i + 1, sn = nx % kStages;
-                    ok = wait_role(full(sn), (nx / kStages) & 1, abort_flag, flags);
+            for (int i = 0; ok; ++i) {
+                const int s = i % kStages;
+                ok = wait_role(full(s), (i / kStages) & 1, abort_flag, flags);
+                if (!ok || meta[s] == 0) break;
+                if (warp == 8) {
+                    if (i >= 2) ok = wait_role(p_ready(i & 1), ((i >> 1) + 1) & 1, abort_flag, flags);
                     if (!ok) break;
-                    const bool has_next = meta[sn] != 0;
-                    if (has_next) {
-                        fence_proxy_async_smem();
-                        tc_fence_after();
-                        issue_s(nx);
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    const uint32_t kslot = sb + s * Smem::kStage;
+                    const uint32_t d = tmem + (uint32_t)((i & 1) * kN);
+#pragma unroll
+                    for (int k = 0; k < kKSteps; ++k) {
+                        const uint32_t ko = (uint32_t)((k >> 2) * Smem::kHalf + (k & 3) * 32);
+                        const uint32_t qo = (uint32_t)((k >> 2) * 2048 + (k & 3) * 32);
+                        umma_bf16(d, sw128_kmajor_desc(kslot + ko), sw128_kmajor_desc(qbase + qo), id_s, k > 0);
                     }
+                    umma_commit(s_done(i & 1));
+                } else {
                     ok = wait_role(p_ready(i & 1), (i >> 1) & 1, abort_flag, flags);
                     if (ok && i >= 2) ok = wait_role(o_free(i & 1), ((i >> 1) + 1) & 1, abort_flag, flags);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(i);
-                    if (!has_next) break;
+                    const uint32_t vslot = sb + s * Smem::kStage + Smem::kSlot;
+                    const uint32_t pb = pbase + (uint32_t)((i & 1) * 4096);
+                    const uint32_t d = tmem + (uint32_t)(2 * kN + (i & 1) * kN);
+#pragma unroll
+                    for (int k = 0; k < kRows / 16; ++k) {
+                        const uint32_t po = (uint32_t)((k >> 2) * 2048 + (k & 3) * 32);
+                        umma_bf16(d, sw128_mnmajor_desc(vslot + k * 2048, Smem::kHalf), sw128_kmajor_desc(pb + po),
+                                  id_o, k > 0);
+                    }
+                    umma_commit(o_done(i & 1));
+                    umma_commit(empty(s));
                 }
             }
-            // every MMA of this thread has finished before TMEM is released
+            // every MMA of both issuers has finished before TMEM is released
             umma_commit(drain);
             mbar_wait_bounded(drain, 0, flags);
         }
@@ -520,80 +538,56 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     __threadfence();
 
     // ---------------------------------------------------- last CTA merges
-    // weights w[s][h] = exp2(M_sh - M*_h) / L*_h over the ns <= 64 partials:
-    // one (split, head) pair per thread, head = tid & 3
-    float *wsm = reinterpret_cast<float *>(sm);  // [ns][head]
-    const bool mthr = tid < kMergeThreads;
-    const int mw = tid >> 5;
-    float m = -INFINITY, lw = 0.f, f = 0.f;
-    const int hm = tid & 3, sm_i = tid >> 2;
-    if (mthr) {
-        if (sm_i < ns) {
-            m = __ldcg(part_bg + (size_t)sm_i * kPartStride + hm * kHS + D);
-            lw = __ldcg(part_bg + (size_t)sm_i * kPartStride + hm * kHS + D + 1);
-        }
-        float mx = m;
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-        if (lane < kGroup) s_red[mw][lane] = mx;
-    }
-    __syncthreads();
-    if (mthr) {
-        float Mh = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kMergeThreads / 32; ++w) Mh = fmaxf(Mh, s_red[w][hm]);
-        f = (m == -INFINITY) ? 0.f : exp2f(m - Mh);
-    }
-    __syncthreads();
-    if (mthr) {
-        float lsum = f * lw;
-        lsum += __shfl_xor_sync(kFull, lsum, 4);
-        lsum += __shfl_xor_sync(kFull, lsum, 8);
-        lsum += __shfl_xor_sync(kFull, lsum, 16);
-        if (lane < kGroup) s_red[mw][lane] = lsum;
-    }
-    __syncthreads();
-    if (mthr) {
-        float Lh = 0.f;
-#pragma unroll
-        for (int w = 0; w < kMergeThreads / 32; ++w) Lh += s_red[w][hm];
-        if (sm_i < ns) wsm[sm_i * kGroup + hm] = Lh > 0.f ? f / Lh : 0.f;
-    }
-    __syncthreads();
-    // outputs as float4 groups (head, 4 dims); TPG threads per group split the
-    // partials and combine with shuffles; loads are issued 8 at a time
+    // One output group (head, 4 dims) per TPG threads; each thread folds its
+    // share of the ns <= 64 partial states with an online rescale (all loads
+    // of a batch issued first), then the TPG lanes combine with shuffles.
     constexpr int kGroups4 = kGroup * D / 4;
     constexpr int TPG = kMergeThreads / kGroups4;
-    if (mthr) {
+    if (tid < kMergeThreads) {
         const int grp = tid / TPG, j = tid % TPG;
         const int h = grp / (D / 4), d4 = grp % (D / 4);
-        const float *src = part_bg + h * kHS + d4 * 4;
+        const float *src = part_bg + h * kHS;
+        float M = -INFINITY, Ls = 0.f;
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        auto fold = [&](float m2, float l2, float4 o2) {
+            if (m2 == -INFINITY) return;  // a slice with no kept row for this head
+            const float Mn = fmaxf(M, m2);
+            const float a = exp2f(M - Mn), c = exp2f(m2 - Mn);  // a = 0 while M is -inf
+            o.x = fmaf(o.x, a, o2.x * c); o.y = fmaf(o.y, a, o2.y * c);
+            o.z = fmaf(o.z, a, o2.z * c); o.w = fmaf(o.w, a, o2.w * c);
+            Ls = fmaf(Ls, a, l2 * c);
+            M = Mn;
+        };
         for (int s0 = j; s0 < ns; s0 += 8 * TPG) {
+            float2 ml[8];
             float4 v[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int s = s0 + u * TPG;
-                v[u] = s < ns ? __ldcg(reinterpret_cast<const float4 *>(src + (size_t)s * kPartStride))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s < ns) {
+                    const float *rec = src + (size_t)s * kPartStride;
+                    ml[u] = __ldcg(reinterpret_cast<const float2 *>(rec + D));
+                    v[u] = __ldcg(reinterpret_cast<const float4 *>(rec + d4 * 4));
+                } else {
+                    ml[u] = make_float2(-INFINITY, 0.f);
+                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int s = s0 + u * TPG;
-                const float wgt = s < ns ? wsm[s * kGroup + h] : 0.f;
-                o.x = fmaf(v[u].x, wgt, o.x); o.y = fmaf(v[u].y, wgt, o.y);
-                o.z = fmaf(v[u].z, wgt, o.z); o.w = fmaf(v[u].w, wgt, o.w);
-            }
+            for (int u = 0; u < 8; ++u) fold(ml[u].x, ml[u].y, v[u]);
         }
 #pragma unroll
         for (int off = 1; off < TPG; off <<= 1) {
-            o.x += __shfl_xor_sync(kFull, o.x, off); o.y += __shfl_xor_sync(kFull, o.y, off);
-            o.z += __shfl_xor_sync(kFull, o.z, off); o.w += __shfl_xor_sync(kFull, o.w, off);
+            const float m2 = __shfl_xor_sync(kFull, M, off), l2 = __shfl_xor_sync(kFull, Ls, off);
+            float4 o2;
+            o2.x = __shfl_xor_sync(kFull, o.x, off); o2.y = __shfl_xor_sync(kFull, o.y, off);
+            o2.z = __shfl_xor_sync(kFull, o.z, off); o2.w = __shfl_xor_sync(kFull, o.w, off);
+            fold(m2, l2, o2);
         }
         if (j == 0) {  // scalar stores: `out` is only required to be 4-byte aligned
+            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
             float *dst = out + ((size_t)b * Hq + g * kGroup + h) * D + d4 * 4;
-            dst[0] = o.x; dst[1] = o.y; dst[2] = o.z; dst[3] = o.w;
+            dst[0] = o.x * inv; dst[1] = o.y * inv; dst[2] = o.z * inv; dst[3] = o.w * inv;
         }
     }
     if (tid == 0) counters[b * Hkv + g] = 0u;  // leave the ticket zeroed for the next call
