@@ -155,11 +155,11 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
     constexpr int PER = kChunk / kThreads;  // positions per thread
-    __shared__ float qs[kGroup][DP];
+    __shared__ __align__(16) float qs[kGroup][DP];
     __shared__ uint32_t hist[kGroup][kBins1];
     __shared__ int s_last;
     __shared__ int scratch[kThreads / 32 + 3];
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
     const int lo = sink, hi = T - window;
@@ -171,55 +171,62 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     if (hi > lo && p0 < hi && p0 + kChunk > lo) {
-        // two rows per batch: both rows' loads (clamped into C) first, then
-        // the arithmetic straight from the packed bf16 pairs
+        // four rows per batch: all rows' loads (clamped into C) first, then
+        // the arithmetic straight from the packed bf16 pairs, with the 4
+        // heads' q' read from shared memory once per 8 dims
+        constexpr int R = 4;
 #pragma unroll
-        for (int k0 = 0; k0 < PER; k0 += 2) {
-            uint4 raw[2][DP / 8];
+        for (int k0 = 0; k0 < PER; k0 += R) {
+            uint4 raw[R][DP / 8];
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
+            for (int k = 0; k < R; ++k) {
                 const int p = min(max(p0 + (k0 + k) * kThreads + tid, lo), hi - 1);
                 const uint4 *row = reinterpret_cast<const uint4 *>(Kp + (slab + p) * DP);
 #pragma unroll
                 for (int v = 0; v < DP / 8; ++v) raw[k][v] = __ldg(row + v);
             }
-            float sc[2][kGroup];
+            float sc[R][kGroup];
 #pragma unroll
-            for (int k = 0; k < 2; ++k)
+            for (int k = 0; k < R; ++k)
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) sc[k][h] = 0.f;
 #pragma unroll
             for (int v = 0; v < DP / 8; ++v) {
+                float4 qv[kGroup][2];
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    qv[h][0] = *reinterpret_cast<const float4 *>(&qs[h][8 * v]);
+                    qv[h][1] = *reinterpret_cast<const float4 *>(&qs[h][8 * v + 4]);
+                }
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int j = 8 * v + 2 * e;  // dims j, j+1 of both rows
-                    float kl[2], kh[2];
+                    float kl[R], kh[R];
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
+                    for (int k = 0; k < R; ++k) {
                         const uint32_t wd = e == 0 ? raw[k][v].x : e == 1 ? raw[k][v].y : e == 2 ? raw[k][v].z : raw[k][v].w;
                         kl[k] = bf16_lo(wd);
                         kh[k] = bf16_hi(wd);
                     }
 #pragma unroll
                     for (int h = 0; h < kGroup; ++h) {
-                        const float qa = qs[h][j], qb = qs[h][j + 1];
+                        const float4 &q4 = qv[h][e >> 1];
+                        const float qa = (e & 1) ? q4.z : q4.x, qb = (e & 1) ? q4.w : q4.y;
 #pragma unroll
-                        for (int k = 0; k < 2; ++k) sc[k][h] = fmaf(qb, kh[k], fmaf(qa, kl[k], sc[k][h]));
+                        for (int k = 0; k < R; ++k) sc[k][h] = fmaf(qb, kh[k], fmaf(qa, kl[k], sc[k][h]));
                     }
                 }
             }
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
+            for (int k = 0; k < R; ++k) {
                 const int p = p0 + (k0 + k) * kThreads + tid;
                 const bool valid = p >= lo && p < hi;
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) {
                     const uint32_t key = score_key(sc[k][h]);
-                    if (valid) ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
-                    // lanes of the warp that fall in the same bin add once
-                    const uint32_t bin = valid ? (key >> 21) : 0xFFFFFFFFu;
-                    const uint32_t peers = __match_any_sync(kFull, bin);
-                    if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[h][bin], (uint32_t)__popc(peers));
+                    if (valid) {
+                        ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
+                        atomicAdd(&hist[h][key >> 21], 1u);
+                    }
                 }
             }
         }
@@ -467,16 +474,21 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         mine += __popc(e);
     }
     int total;
-    int base = block_excl_scan<kFinThreads>(mine, scratch, &total);
-    int32_t *out = idx + row * (size_t)idx_cap;
-    for (int w = wb; w < we; ++w) {
-        uint32_t e = tie_s[w];
-        sel_bits[row * W + w] = e;
-        while (e) {
-            const int bit = __ffs(e) - 1;
-            e &= e - 1u;
-            if (base < idx_cap) out[base] = (w << 5) + bit;
-            ++base;
+    const int base = block_excl_scan<kFinThreads>(mine, scratch, &total);
+    for (int w = wb; w < we; ++w) sel_bits[row * W + w] = tie_s[w];
+    // the index list, lane-parallel: a warp walks its threads' words in
+    // order (they are contiguous), lane = bit, one predicated store each
+    {
+        const int lane = tid & 31;
+        const uint32_t lt = (1u << lane) - 1u;
+        int32_t *out = idx + row * (size_t)idx_cap;
+        const int w_first = (tid - lane) * wpt, w_last = min(w_first + 32 * wpt, W);
+        int run = __shfl_sync(kFull, base, 0);
+        for (int w = w_first; w < w_last; ++w) {
+            const uint32_t e = tie_s[w];
+            const int slot = run + __popc(e & lt);
+            if (((e >> lane) & 1u) && slot < idx_cap) out[slot] = (w << 5) + lane;
+            run += __popc(e);
         }
     }
     if (tid == 0) {
