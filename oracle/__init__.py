@@ -47,6 +47,8 @@ def _bind(path: str):
     lib.orc_predict_queries.restype = None
     lib.orc_scores.argtypes = [P, P, i32, i64, i64, P]
     lib.orc_scores.restype = None
+    lib.orc_group_scores.argtypes = [P, i32, P, i32, i64, i64, i32, P]
+    lib.orc_group_scores.restype = None
     lib.orc_select.argtypes = [P, i64, i64, i64, i64, i32, P]
     lib.orc_select.restype = i64
     lib.orc_attention_set.argtypes = [i64, i64, i64, P, i64, P]
@@ -139,6 +141,27 @@ def scores(qp: np.ndarray, Kp: np.ndarray, t_begin: int, t_end: int, lib=None) -
     out = np.empty(n, dtype=np.float32)
     if n:
         lib.orc_scores(_ptr(qp), _ptr(Kp), dp, t_begin, t_end, _ptr(out))
+    return out
+
+
+GROUP_REDUCE = {"max": 0, "sum": 1}
+
+
+def group_scores(qp: np.ndarray, Kp: np.ndarray, t_begin: int, t_end: int, reduce: str,
+                 lib=None) -> np.ndarray:
+    """fp32 group scores of positions [t_begin, t_end) for the G heads of one
+    GQA group (qp [G][d']): the largest or the fp32 sum, in head order, of the
+    heads' fp32 scores."""
+    lib = lib or load()
+    qp = np.ascontiguousarray(qp, dtype=np.float32)
+    Kp = _u16(Kp)
+    dp = Kp.shape[1]
+    assert qp.ndim == 2 and qp.shape[1] == dp
+    n = max(0, t_end - t_begin)
+    out = np.empty(n, dtype=np.float32)
+    if n:
+        lib.orc_group_scores(_ptr(qp), qp.shape[0], _ptr(Kp), dp, t_begin, t_end, GROUP_REDUCE[reduce],
+                             _ptr(out))
     return out
 
 

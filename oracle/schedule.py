@@ -21,7 +21,7 @@ import math
 
 import numpy as np
 
-from . import attention, attention_set, predict_queries, project_keys, scores, select
+from . import attention, attention_set, group_scores, predict_queries, project_keys, scores, select
 
 
 def is_prediction_step(step: int, interval: int) -> bool:
@@ -55,7 +55,7 @@ def projection_events(ctx0: int, window: int, steps: int):
     return (ctx0 // window) * window, events
 
 
-def run(w, data, layers, steps, want_attention=True, heads=None):
+def run(w, data, layers, steps, want_attention=True, heads=None, selection="head"):
     """Run the oracle over decode steps [0, steps) for the given layers.
 
     `data` provides host arrays (numpy; bf16 as uint16):
@@ -65,8 +65,13 @@ def run(w, data, layers, steps, want_attention=True, heads=None):
       data.h(pred_index, producer) -> [batch][hidden]
       data.qp_direct(pred_index, layer) -> [batch][Hq][d'] float32
       data.q(step, layer) -> [batch][Hq][d]
+    `selection` is "head" (one importance set per query head, reading R1) or
+    "group_max" / "group_sum" (one set per KV head from the largest or the
+    fp32 sum of the group's head scores, the group-shared variant; every head
+    of the group then attends to that set).
     Returns {(step, layer): {"idx": [[I_bh]], "out": [batch][Hq][d] or None}}.
     """
+    assert selection in ("head", "group_max", "group_sum")
     B, Hq, grp = w.batch, w.n_q_heads, w.group
     heads = list(range(Hq)) if heads is None else list(heads)
     ctx0 = w.ctx0_per_seq()
@@ -95,20 +100,31 @@ def run(w, data, layers, steps, want_attention=True, heads=None):
                     T = ctx0[b] + i + 1
                     hi = T - w.window
                     per_head = []
+                    group_sets = {}
                     for h in range(Hq):
                         if h not in heads:
                             per_head.append(None)
                             continue
                         g = h // grp
+                        if selection != "head" and g in group_sets:
+                            per_head.append(group_sets[g])
+                            continue
                         if hi > w.sink:
                             key = (layer, b, g)
                             have = kp_cache.get(key)
                             if have is None or have.shape[0] < hi:
                                 kp_cache[key] = project_keys(K[b, g, :hi], Wk[g])
-                            s = scores(qp[b, h], kp_cache[key], w.sink, hi)
+                            if selection == "head":
+                                s = scores(qp[b, h], kp_cache[key], w.sink, hi)
+                            else:
+                                s = group_scores(qp[b, g * grp:(g + 1) * grp], kp_cache[key], w.sink, hi,
+                                                 selection[len("group_"):])
                         else:
                             s = np.zeros(0, np.float32)
-                        per_head.append(select(s, T, w.sink, w.window, w.budget, w.nbr))
+                        I = select(s, T, w.sink, w.window, w.budget, w.nbr)
+                        if selection != "head":
+                            group_sets[g] = I
+                        per_head.append(I)
                     sets.append(per_head)
                 cur_idx[layer] = sets
             out = None

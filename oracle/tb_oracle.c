@@ -166,6 +166,38 @@ void orc_scores(const float *qp, const uint16_t *Kp, int dp,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Step 3, group-shared variant (not on the pages).                          */
+/* An alternative to reading R1 in which the G query heads of a GQA group    */
+/* share one importance set, chosen from one group score per position: the   */
+/* largest (reduce = 0) or the sum (reduce = 1) of the heads' fp32 scores.    */
+/* Each head's score is exactly the fp32 score of orc_scores; the sum is     */
+/* taken in fp32 in head order, ((s0 + s1) + s2) + ..., which is the value a */
+/* device that holds fp32 head scores and adds them in that order computes.  */
+/* qp holds the G heads' projected queries, [G][dp].                          */
+/* ------------------------------------------------------------------------ */
+
+void orc_group_scores(const float *qp, int G, const uint16_t *Kp, int dp,
+                      int64_t t_begin, int64_t t_end, int reduce, float *s)
+{
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        float g = 0.0f;
+        for (int h = 0; h < G; ++h) {
+            double acc = 0.0;
+            for (int j = 0; j < dp; ++j)
+                acc += (double)qp[(int64_t)h * dp + j] * orc_bf16_to_double(Kp[t * dp + j]);
+            const float sh = (float)acc;
+            if (h == 0)
+                g = sh;
+            else if (reduce == 0)
+                g = sh > g ? sh : g;
+            else
+                g = g + sh;
+        }
+        s[t - t_begin] = g;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Step 4: budgeted selection with neighbour fetch                           */
 /* [ja] コアアーキテクチャ, スコアリング: dynamic token selection under a fixed */
 /* budget.  [ja] 推論戦略: the first S tokens (sink) and the last N tokens     */

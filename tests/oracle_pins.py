@@ -12,6 +12,10 @@ What pins what:
   key projection     exact integer matrix products (numpy int64) rounded by torch
   predictor MLP      torch float64 matmul + SiLU as an independent witness
   scores             exact integer dot products (numpy int64)
+  group scores       exact integer closed forms (max over heads, dot product
+                     with the summed queries), a case where fp32 head-order
+                     rounding decides the sum, and the invariant that identical
+                     heads select what one head selects
   selection          hand-worked golden cases, and brute force by rank counting
                      on tiny inputs with many ties
   attention set      sink/window/importance invariants
@@ -169,6 +173,44 @@ def pin_scores_integer(lib):
         assert np.array_equal(got.astype(np.float64), want[7:50])
 
 
+def pin_group_scores_integer(lib):
+    rng = np.random.default_rng(11)
+    for dp in (16, 32):
+        Kp = rng.integers(-300, 301, (60, dp))
+        q = rng.integers(-4, 5, (4, dp))
+        Kp_bits = _bf16_bits(torch.tensor(Kp, dtype=torch.float32))
+        Kp_val = _bits_to_f64(Kp_bits).astype(np.int64)
+        per_head = Kp_val @ q.T.astype(np.int64)                           # [60][4], exact
+        got = oracle.group_scores(q.astype(np.float32), Kp_bits, 5, 60, "max", lib=lib)
+        assert np.array_equal(got.astype(np.float64), per_head.max(axis=1)[5:].astype(np.float64))
+        # |sum| <= 4 * 4 * 300 * 32 < 2^24: every fp32 partial sum is exact
+        got = oracle.group_scores(q.astype(np.float32), Kp_bits, 5, 60, "sum", lib=lib)
+        assert np.array_equal(got.astype(np.float64), (Kp_val @ q.sum(axis=0))[5:].astype(np.float64))
+
+
+def pin_group_sum_fp32_head_order(lib):
+    # head scores 2^24, 1, 1, 0 at one position.  In fp32, in head order, each
+    # "+ 1" is a tie that rounds to the even 2^24, so the group sum is 2^24;
+    # in the reverse order 1 + 1 = 2 first, and 2^24 + 2 is representable.
+    Kp_bits = _bf16_bits(torch.tensor([[1.0] + [0.0] * 15], dtype=torch.float32))
+    q = np.zeros((4, 16), np.float32)
+    q[0, 0], q[1, 0], q[2, 0] = 2.0 ** 24, 1.0, 1.0
+    assert oracle.group_scores(q, Kp_bits, 0, 1, "sum", lib=lib)[0] == np.float32(2.0 ** 24)
+    assert oracle.group_scores(q[::-1].copy(), Kp_bits, 0, 1, "sum", lib=lib)[0] == np.float32(2.0 ** 24 + 2)
+    assert oracle.group_scores(q, Kp_bits, 0, 1, "max", lib=lib)[0] == np.float32(2.0 ** 24)
+
+
+def pin_group_selection_identical_heads(lib):
+    rng = np.random.default_rng(12)
+    T, S, N, B, r = 120, 4, 8, 17, 1
+    Kp_bits = _bf16_bits(torch.randn(T, 16, generator=torch.Generator().manual_seed(12)))
+    q1 = rng.standard_normal(16).astype(np.float32)
+    per_head = oracle.select(oracle.scores(q1, Kp_bits, S, T - N, lib=lib), T, S, N, B, r, lib=lib)
+    for red in ("max", "sum"):
+        s = oracle.group_scores(np.stack([q1] * 4), Kp_bits, S, T - N, red, lib=lib)
+        assert oracle.select(s, T, S, N, B, r, lib=lib).tolist() == per_head.tolist(), red
+
+
 # ---------------------------------------------------------------------------
 # selection
 # ---------------------------------------------------------------------------
@@ -309,6 +351,9 @@ ALL_PINS = [
     pin_predict_queries,
     pin_predict_queries_silu_closed_form,
     pin_scores_integer,
+    pin_group_scores_integer,
+    pin_group_sum_fp32_head_order,
+    pin_group_selection_identical_heads,
     pin_select_golden,
     pin_select_brute_force,
     pin_attention_set,

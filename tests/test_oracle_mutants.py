@@ -42,6 +42,9 @@ MUTANTS = [
     ("scale_dropped", "z[k] = acc * scale;", "z[k] = acc;"),
     ("softmax_unnormalised", "out[j] = (float)(o / l);", "out[j] = (float)o;"),
     ("v_row_misindexed", "V[(int64_t)A[k] * d + j]", "V[(int64_t)k * d + j]"),
+    ("group_max_is_min", "g = sh > g ? sh : g;", "g = sh < g ? sh : g;"),
+    ("group_drops_last_head", "for (int h = 0; h < G; ++h) {", "for (int h = 0; h < G - 1; ++h) {"),
+    ("group_sum_in_double", "        float g = 0.0f;", "        double g = 0.0;"),
 ]
 
 
