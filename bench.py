@@ -50,7 +50,7 @@ ROW_BYTES_PER_DIM = 2 * 2      # K and V, bf16
 class Run:
     """All device buffers of one workload replica plus its decoder."""
 
-    def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None):
+    def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head"):
         self.w = w
         self.device = device
         self.steps = steps or w.steps
@@ -80,7 +80,8 @@ class Run:
                                  head_dim=w.head_dim, d_proj=w.d_proj, hidden=w.hidden, inter=w.inter,
                                  stride=stride, sink=w.sink, window=w.window, budget=w.budget, nbr=w.nbr,
                                  interval=w.interval, ctx_cap=w.ctx_cap)
-        self.dec = SparseDecoder(self.shape, self.K, self.V, self.Wk, self.mlp, self.ctx0, self.steps, device)
+        self.dec = SparseDecoder(self.shape, self.K, self.V, self.Wk, self.mlp, self.ctx0, self.steps, device,
+                                 selection=selection)
         self.out = torch.zeros(nL, w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):
@@ -459,11 +460,12 @@ def cpu_baseline(w, budget_s=25.0):
             "sample_seconds": round(time.perf_counter() - t_start + smp.proj_s, 1)}
 
 
-def config_of(w: tb_inputs.Workload, decode_steps: int, world: int) -> dict:
+def config_of(w: tb_inputs.Workload, decode_steps: int, world: int, selection: str = "head") -> dict:
     """The workload description both arms print."""
     return {"workload": w.name, "batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
             "layers": w.n_layers, "decode_steps_per_bench_step": decode_steps, "budget": w.budget,
             "interval": w.interval, "sink": w.sink, "window": w.window, "d_proj": w.d_proj,
+            "selection": "per query head" if selection == "head" else f"per KV head ({selection})",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -518,6 +520,9 @@ def main():
     ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--selection", default="head", choices=list(SparseDecoder.SELECTIONS),
+                    help="head: one importance set per query head (the default, the pages' reading); "
+                         "group_max / group_sum: one set per KV head (the group-shared variant)")
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -538,7 +543,7 @@ def main():
     w = replica(base, rank)                          # an independent replica per rank
     if args.layers:
         w = w.scaled(n_layers=args.layers)
-    run = Run(w, device, steps=args.decode_steps)
+    run = Run(w, device, steps=args.decode_steps, selection=args.selection)
     run.dec.prefill()
     torch.cuda.synchronize()
 
@@ -592,7 +597,7 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_sparse, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; Llama-3.1-8B attention shapes, random weights)",
-        "config": dict(config_of(w, run.steps, world),
+        "config": dict(config_of(w, run.steps, world, args.selection),
                        l2="inputs larger than L2 (KV %.1f GB)" % (2 * sum(k.numel() for k in run.K) * 2 / 1e9),
                        graph="one CUDA graph per bench step"),
         "speedup_vs_dense": round(value / dense_value, 4),
@@ -605,7 +610,8 @@ def main():
                 "dense_bytes_per_bench_step": acct["dense_total"]},
         "roofline": {"kernel": "attn_kernel<128,true> (sparse GQA decode attention)", "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("attn_kernel<128,true>"),
+                     "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic("attn_kernel<128,true>") if args.selection == "head" else None,
                      "bytes_per_launch": round(attn_bytes_per_launch), "launch_us": round(1000 * attn_launch_ms, 3)},
         "gpu_launches": (sparse_launches) * args.steps,
         "clocks": clk,

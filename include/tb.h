@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 1
+#define TB_ABI_VERSION 2
 
 typedef uint16_t tb_bf16;
 
@@ -166,6 +166,26 @@ tb_status tb_score_select(const tb_dims *dims, const float *qp, int64_t qp_batch
                           int32_t window, int32_t budget, int32_t nbr, int32_t *idx,
                           int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
                           size_t ws_bytes, void *stream);
+
+/* Group-shared variant (no counterpart on the pages; an alternative to their
+ * per-attention-head selection for GQA).  The 4 query heads of a KV head
+ * share one importance set, chosen as above from one group score per position:
+ *
+ *   s_g[t] = max_h s_h[t]                          (reduce = TB_GROUP_MAX)
+ *   s_g[t] = ((s_0[t] + s_1[t]) + s_2[t]) + s_3[t] in fp32 (TB_GROUP_SUM)
+ *
+ * where s_h is the fp32 score of head h defined above.  Arguments, layouts,
+ * limits and the workspace (tb_score_select_workspace_bytes) are those of
+ * tb_score_select; idx, count and sel_bits receive the group's set in each of
+ * its 4 heads' rows, so tb_sparse_decode_attn reads it unchanged.  Any other
+ * reduce value is TB_ERR_INVALID_ARG. */
+#define TB_GROUP_MAX 0
+#define TB_GROUP_SUM 1
+tb_status tb_score_select_group(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
+                                const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
+                                int32_t budget, int32_t nbr, int32_t reduce, int32_t *idx, int32_t idx_cap,
+                                int32_t *count, uint32_t *sel_bits, void *ws, size_t ws_bytes,
+                                void *stream);
 
 /* Build the sel_bits bitmap from index lists that came from elsewhere (e.g. a
  * host-side selection): bit t of row (b,h) is set iff t is among

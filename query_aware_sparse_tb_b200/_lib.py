@@ -17,13 +17,14 @@ LIB_PATH = os.path.join(_PKG, "libtb.so")
 
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
 TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW = 0x1, 0x2, 0x4
+TB_GROUP_REDUCE = {"max": 0, "sum": 1}
 
 EXPORTS = [
     "tb_abi_version", "tb_status_str", "tb_last_error",
     "tb_score_select_workspace_bytes", "tb_attn_workspace_bytes",
     "tb_predict_queries_workspace_bytes", "tb_project_keys_workspace_bytes",
     "tb_workspace_init", "tb_workspace_check",
-    "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_select_bits_from_idx",
+    "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_select_bits_from_idx",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc",
 ]
 
@@ -66,6 +67,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_project_keys": ([D, P, P, P, P, P, i32, P, sz, P], ctypes.c_int),
         "tb_predict_queries": ([P, P, P, P, i32, i32, i32, i32, P, sz, P], ctypes.c_int),
         "tb_score_select": ([D, P, i64, P, P, i32, i32, i32, i32, P, i32, P, P, P, sz, P], ctypes.c_int),
+        "tb_score_select_group": ([D, P, i64, P, P, i32, i32, i32, i32, i32, P, i32, P, P, P, sz, P],
+                                  ctypes.c_int),
         "tb_select_bits_from_idx": ([D, P, i32, P, P, P], ctypes.c_int),
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
@@ -168,6 +171,16 @@ def score_select(d: TbDims, qp, qp_batch_stride: int, Kp, ctx_len, sink: int, wi
     _check(load().tb_score_select(ctypes.byref(d), _ptr(qp), int(qp_batch_stride), _ptr(Kp), _ptr(ctx_len),
                                   sink, window, budget, nbr, _ptr(idx), idx_cap, _ptr(count), _ptr(sel_bits),
                                   _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def score_select_group(d: TbDims, qp, qp_batch_stride: int, Kp, ctx_len, sink: int, window: int, budget: int,
+                       nbr: int, reduce: str, idx, count, sel_bits, ws, stream=None):
+    """tb_score_select_group: one set per KV head from the max or sum of the
+    group's head scores, written to each of the group's 4 head rows."""
+    idx_cap = idx.shape[-1]
+    _check(load().tb_score_select_group(ctypes.byref(d), _ptr(qp), int(qp_batch_stride), _ptr(Kp), _ptr(ctx_len),
+                                        sink, window, budget, nbr, TB_GROUP_REDUCE[reduce], _ptr(idx), idx_cap,
+                                        _ptr(count), _ptr(sel_bits), _ptr(ws), _bytes(ws), _stream(stream)))
 
 
 def select_bits_from_idx(d: TbDims, idx, count, sel_bits, stream=None):

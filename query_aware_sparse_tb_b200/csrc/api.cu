@@ -37,19 +37,21 @@ bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr
 bool aligned4(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // bf16 tensors are read with 16-byte vector loads, cp.async and TMA
-#define TB_CHECK_PTR(p)                                                                      \
+#define TB_CHECK_PTR_IN(p, fn)                                                               \
     do {                                                                                     \
         if (!aligned16(p))                                                                   \
             return fail(TB_ERR_INVALID_ARG, "%s: pointer '%s' is null or not 16-byte aligned", \
-                        __func__, #p);                                                       \
+                        fn, #p);                                                             \
     } while (0)
 // int32 / float / uint32 arrays are accessed a word at a time
-#define TB_CHECK_PTR4(p)                                                                     \
+#define TB_CHECK_PTR4_IN(p, fn)                                                              \
     do {                                                                                     \
         if (!aligned4(p))                                                                    \
             return fail(TB_ERR_INVALID_ARG, "%s: pointer '%s' is null or not 4-byte aligned",  \
-                        __func__, #p);                                                       \
+                        fn, #p);                                                             \
     } while (0)
+#define TB_CHECK_PTR(p) TB_CHECK_PTR_IN(p, __func__)
+#define TB_CHECK_PTR4(p) TB_CHECK_PTR4_IN(p, __func__)
 
 tb_status check_dims(const tb_dims *d, bool need_dproj, const char *fn) {
     if (!d) return fail(TB_ERR_INVALID_ARG, "%s: dims is null", fn);
@@ -175,31 +177,51 @@ tb_status tb_predict_queries(const tb_bf16 *h, const tb_bf16 *W1, const tb_bf16 
                        __func__);
 }
 
+static tb_status score_select_impl(const char *fn, const tb_dims *dims, const float *qp,
+                                   int64_t qp_batch_stride, const tb_bf16 *Kp, const int32_t *ctx_len,
+                                   int32_t sink, int32_t window, int32_t budget, int32_t nbr,
+                                   int32_t group_reduce, int32_t *idx, int32_t idx_cap, int32_t *count,
+                                   uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, true, fn)) != TB_OK) return s;
+    TB_CHECK_PTR4_IN(qp, fn); TB_CHECK_PTR_IN(Kp, fn); TB_CHECK_PTR4_IN(ctx_len, fn); TB_CHECK_PTR4_IN(idx, fn);
+    TB_CHECK_PTR4_IN(count, fn); TB_CHECK_PTR4_IN(sel_bits, fn);
+    if (dims->ctx_cap > kMaxCtxSelect)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", fn, dims->ctx_cap, kMaxCtxSelect);
+    if (qp_batch_stride < (int64_t)dims->n_q_heads * dims->d_proj)
+        return fail(TB_ERR_INVALID_ARG, "%s: qp_batch_stride %lld smaller than Hq*d'", fn,
+                    (long long)qp_batch_stride);
+    if (sink < 0 || window < 1 || budget < 1)
+        return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0, window >= 1, budget >= 1", fn);
+    if (nbr < 0 || nbr > 16) return fail(TB_ERR_INVALID_ARG, "%s: nbr %d outside [0, 16]", fn, nbr);
+    const long long need_cap = (long long)(2 * nbr + 1) * budget;
+    const long long min_cap = need_cap < dims->ctx_cap ? need_cap : dims->ctx_cap;
+    if (idx_cap < min_cap)
+        return fail(TB_ERR_INVALID_ARG, "%s: idx_cap %d < min((2*nbr+1)*budget, ctx_cap) = %lld", fn, idx_cap,
+                    min_cap);
+    if ((s = check_ws(ws, ws_bytes, select_ws_bytes(*dims), fn)) != TB_OK) return s;
+    return cuda_status(launch_score_select(*dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget, nbr,
+                                           group_reduce, idx, idx_cap, count, sel_bits, ws, (cudaStream_t)stream),
+                       fn);
+}
+
 tb_status tb_score_select(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
                           const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
                           int32_t budget, int32_t nbr, int32_t *idx, int32_t idx_cap, int32_t *count,
                           uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream) {
-    tb_status s;
-    if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
-    TB_CHECK_PTR4(qp); TB_CHECK_PTR(Kp); TB_CHECK_PTR4(ctx_len); TB_CHECK_PTR4(idx); TB_CHECK_PTR4(count);
-    TB_CHECK_PTR4(sel_bits);
-    if (dims->ctx_cap > kMaxCtxSelect)
-        return fail(TB_ERR_UNSUPPORTED, "tb_score_select: ctx_cap %d above %d", dims->ctx_cap, kMaxCtxSelect);
-    if (qp_batch_stride < (int64_t)dims->n_q_heads * dims->d_proj)
-        return fail(TB_ERR_INVALID_ARG, "tb_score_select: qp_batch_stride %lld smaller than Hq*d'",
-                    (long long)qp_batch_stride);
-    if (sink < 0 || window < 1 || budget < 1)
-        return fail(TB_ERR_INVALID_ARG, "tb_score_select: need sink >= 0, window >= 1, budget >= 1");
-    if (nbr < 0 || nbr > 16) return fail(TB_ERR_INVALID_ARG, "tb_score_select: nbr %d outside [0, 16]", nbr);
-    const long long need_cap = (long long)(2 * nbr + 1) * budget;
-    const long long min_cap = need_cap < dims->ctx_cap ? need_cap : dims->ctx_cap;
-    if (idx_cap < min_cap)
-        return fail(TB_ERR_INVALID_ARG, "tb_score_select: idx_cap %d < min((2*nbr+1)*budget, ctx_cap) = %lld",
-                    idx_cap, min_cap);
-    if ((s = check_ws(ws, ws_bytes, select_ws_bytes(*dims), __func__)) != TB_OK) return s;
-    return cuda_status(launch_score_select(*dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget,
-                                           nbr, idx, idx_cap, count, sel_bits, ws, (cudaStream_t)stream),
-                       __func__);
+    return score_select_impl(__func__, dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget, nbr, -1,
+                             idx, idx_cap, count, sel_bits, ws, ws_bytes, stream);
+}
+
+tb_status tb_score_select_group(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
+                                const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
+                                int32_t budget, int32_t nbr, int32_t reduce, int32_t *idx, int32_t idx_cap,
+                                int32_t *count, uint32_t *sel_bits, void *ws, size_t ws_bytes,
+                                void *stream) {
+    if (reduce != TB_GROUP_MAX && reduce != TB_GROUP_SUM)
+        return fail(TB_ERR_INVALID_ARG, "%s: reduce %d is neither TB_GROUP_MAX nor TB_GROUP_SUM", __func__, reduce);
+    return score_select_impl(__func__, dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget, nbr, reduce,
+                             idx, idx_cap, count, sel_bits, ws, ws_bytes, stream);
 }
 
 tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,

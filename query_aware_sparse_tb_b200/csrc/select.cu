@@ -40,6 +40,12 @@ constexpr unsigned kFull = 0xffffffffu;
 
 enum : uint32_t { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
 
+// What is selected: one set per query head, or one set per KV head (group)
+// from the largest or the fp32 sum (heads in order) of the group's scores.
+// A group's set is kept in the rows of its first head until finalize copies
+// it to all 4 heads.
+enum : int { kSelHead = 0, kSelGroupMax = 1, kSelGroupSum = 2 };
+
 struct HeadState {   // 8 words per (b, query head)
     uint32_t mode, b1, k_rem, cand_count, n_in_bin, pad[3];
 };
@@ -149,14 +155,15 @@ __device__ int block_find_bin_desc(const uint32_t *hist, int nbins, uint32_t nee
 
 // ------------------------------------------------------------------ kernel 1
 
-template <int DP>
+template <int DP, int SEL>
 __global__ void __launch_bounds__(kThreads, 2)
 score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
     constexpr int PER = kChunk / kThreads;  // positions per thread
+    constexpr int NH = SEL == kSelHead ? kGroup : 1;  // score rows per (b, KV head)
     __shared__ __align__(16) float qs[kGroup][DP];
-    __shared__ uint32_t hist[kGroup][kBins1];
+    __shared__ uint32_t hist[NH][kBins1];
     __shared__ int s_last;
     __shared__ int scratch[kThreads / 32 + 3];
     const int tid = threadIdx.x;
@@ -165,7 +172,7 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     const int lo = sink, hi = T - window;
     const int p0 = ch * kChunk;
 
-    for (int i = tid; i < kGroup * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
+    for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
     if (tid < kGroup * DP) (&qs[0][0])[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
     __syncthreads();
 
@@ -220,19 +227,30 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
             for (int k = 0; k < R; ++k) {
                 const int p = p0 + (k0 + k) * kThreads + tid;
                 const bool valid = p >= lo && p < hi;
+                if constexpr (SEL == kSelHead) {
 #pragma unroll
-                for (int h = 0; h < kGroup; ++h) {
-                    const uint32_t key = score_key(sc[k][h]);
+                    for (int h = 0; h < kGroup; ++h) {
+                        const uint32_t key = score_key(sc[k][h]);
+                        if (valid) {
+                            ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
+                            atomicAdd(&hist[h][key >> 21], 1u);
+                        }
+                    }
+                } else {
+                    float gs = sc[k][0];
+#pragma unroll
+                    for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, sc[k][h]) : gs + sc[k][h];
+                    const uint32_t key = score_key(gs);
                     if (valid) {
-                        ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
-                        atomicAdd(&hist[h][key >> 21], 1u);
+                        ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
+                        atomicAdd(&hist[0][key >> 21], 1u);
                     }
                 }
             }
         }
     }
     __syncthreads();
-    for (int i = tid; i < kGroup * kBins1; i += kThreads) {
+    for (int i = tid; i < NH * kBins1; i += kThreads) {
         const uint32_t v = (&hist[0][0])[i];
         if (v) atomicAdd(ws.hist + ((size_t)b * Hq + g * kGroup + i / kBins1) * kBins1 + (i % kBins1), v);
     }
@@ -251,13 +269,13 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
         // counted from the top; all loads first, then one scan per head
         constexpr int PERB = kBins1 / kThreads;
         const int hb = kBins1 - tid * PERB;
-        uint32_t v[kGroup][PERB];
+        uint32_t v[NH][PERB];
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h)
+        for (int h = 0; h < NH; ++h)
 #pragma unroll
             for (int j = 0; j < PERB; ++j) v[h][j] = __ldcg(gh0 + (size_t)h * kBins1 + hb - 1 - j);
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
+        for (int h = 0; h < NH; ++h) {
             int mine = 0;
 #pragma unroll
             for (int j = 0; j < PERB; ++j) mine += (int)v[h][j];
@@ -280,22 +298,24 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                 }
             }
         }
-    } else if (tid < kGroup) {
+    } else if (tid < NH) {
         HeadState st = {};
         st.mode = nC == 0 ? kModeEmpty : kModeAll;
         ws.state[(size_t)b * Hq + g * kGroup + tid] = st;
     }
     __syncthreads();
-    for (int i = tid; i < kGroup * kBins1; i += kThreads) ws.hist[((size_t)b * Hq + g * kGroup) * kBins1 + i] = 0u;
+    for (int i = tid; i < NH * kBins1; i += kThreads) ws.hist[((size_t)b * Hq + g * kGroup) * kBins1 + i] = 0u;
     if (tid == 0) ws.counters[b * Hkv + g] = 0u;
 }
 
 // ------------------------------------------------------------------ kernel 2
 
+template <int SEL>
 __global__ void __launch_bounds__(kThreads)
 mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int W,
                     int sink, int window, SelWs ws) {
     constexpr int kWordsPerWarp = kChunk / 32 / (kThreads / 32);  // 4
+    constexpr int NH = SEL == kSelHead ? kGroup : 1;
     __shared__ uint32_t s_cnt[kGroup], s_base[kGroup];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
@@ -304,9 +324,9 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
     const int w0 = ch * (kChunk / 32);
     if (tid < kGroup) s_cnt[tid] = 0u;
 
-    uint32_t mode[kGroup], b1[kGroup];
+    uint32_t mode[NH], b1[NH];
 #pragma unroll
-    for (int h = 0; h < kGroup; ++h) {
+    for (int h = 0; h < NH; ++h) {
         const HeadState &st = ws.state[(size_t)b * Hq + g * kGroup + h];
         mode[h] = st.mode;
         b1[h] = st.b1;
@@ -314,14 +334,14 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
     __syncthreads();
     // pass 1: Top bits, candidate ballots and this warp's offsets inside the CTA
     // (every key load issued before the first ballot)
-    uint32_t key[kWordsPerWarp][kGroup], cb[kWordsPerWarp][kGroup], off[kWordsPerWarp][kGroup];
+    uint32_t key[kWordsPerWarp][NH], cb[kWordsPerWarp][NH], off[kWordsPerWarp][NH];
 #pragma unroll
     for (int i = 0; i < kWordsPerWarp; ++i) {
         const int w = w0 + warp + i * (kThreads / 32);
         const int p = (w << 5) + lane;
         const bool in_c = w < W && p >= lo && p < hi;
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
+        for (int h = 0; h < NH; ++h) {
             const size_t row = (size_t)b * Hq + g * kGroup + h;
             key[i][h] = (in_c && mode[h] == kModeSelect) ? __ldcg(ws.keys + row * Tcap + p) : 0u;
         }
@@ -332,7 +352,7 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
         const int p = (w << 5) + lane;
         const bool in_c = w < W && p >= lo && p < hi;
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
+        for (int h = 0; h < NH; ++h) {
             const size_t row = (size_t)b * Hq + g * kGroup + h;
             const uint32_t k = key[i][h];
             const uint32_t d1 = k >> 21;
@@ -347,7 +367,7 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
         }
     }
     __syncthreads();
-    if (tid < kGroup && s_cnt[tid])
+    if (tid < NH && s_cnt[tid])
         s_base[tid] = atomicAdd(&ws.state[(size_t)b * Hq + g * kGroup + tid].cand_count, s_cnt[tid]);
     __syncthreads();
     // pass 2: the candidates, (key, position) pairs, in the reserved range
@@ -355,7 +375,7 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
     for (int i = 0; i < kWordsPerWarp; ++i) {
         const int p = ((w0 + warp + i * (kThreads / 32)) << 5) + lane;
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
+        for (int h = 0; h < NH; ++h) {
             if ((cb[i][h] >> lane) & 1u) {
                 const size_t row = (size_t)b * Hq + g * kGroup + h;
                 ws.cand[row * Tcap + s_base[h] + off[i][h] + __popc(cb[i][h] & ((1u << lane) - 1u))] =
@@ -375,6 +395,7 @@ __device__ __forceinline__ uint32_t range_mask(int w, int lo, int hi) {
     return upto & ~((1u << start) - 1u);
 }
 
+template <int SEL>
 __global__ void __launch_bounds__(kFinThreads)
 finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int sink, int window,
                 int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
@@ -386,8 +407,10 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
     __shared__ uint32_t hist[kBins2];
     __shared__ int scratch[kFinThreads / 32 + 3];
 
+    // a group's set is computed in its first head's rows and written to all 4
+    constexpr int NOUT = SEL == kSelHead ? 1 : kGroup;
     const int tid = threadIdx.x;
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int h = blockIdx.x * NOUT, b = blockIdx.y;
     const size_t row = (size_t)b * Hq + h;
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, false);
     const int lo = sink, hi = T - window;
@@ -475,7 +498,9 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
     }
     int total;
     const int base = block_excl_scan<kFinThreads>(mine, scratch, &total);
-    for (int w = wb; w < we; ++w) sel_bits[row * W + w] = tie_s[w];
+    for (int w = wb; w < we; ++w)
+#pragma unroll
+        for (int o = 0; o < NOUT; ++o) sel_bits[(row + o) * W + w] = tie_s[w];
     // the index list, lane-parallel: a warp walks its threads' words in
     // order (they are contiguous), lane = bit, one predicated store each
     {
@@ -487,13 +512,17 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         for (int w = w_first; w < w_last; ++w) {
             const uint32_t e = tie_s[w];
             const int slot = run + __popc(e & lt);
-            if (((e >> lane) & 1u) && slot < idx_cap) out[slot] = (w << 5) + lane;
+            if (((e >> lane) & 1u) && slot < idx_cap) {
+#pragma unroll
+                for (int o = 0; o < NOUT; ++o) out[(size_t)o * idx_cap + slot] = (w << 5) + lane;
+            }
             run += __popc(e);
         }
     }
     if (tid == 0) {
         if (total > idx_cap) raise_flag(ws.flags, TB_FLAG_IDX_OVERFLOW);
-        count[row] = total < idx_cap ? total : idx_cap;
+#pragma unroll
+        for (int o = 0; o < NOUT; ++o) count[row + o] = total < idx_cap ? total : idx_cap;
     }
 }
 
@@ -517,41 +546,57 @@ bits_from_idx_kernel(const int32_t *__restrict__ idx, int idx_cap, const int32_t
     for (int w = tid; w < W; w += kFinThreads) sel_bits[row * W + w] = bsm[w];
 }
 
+template <int SEL>
+cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
+                       const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, int32_t nbr,
+                       int32_t *idx, int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
+                       cudaStream_t st) {
+    const SelWs s = carve(d, ws);
+    const int W = (d.ctx_cap + 31) / 32;
+    const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
+    dim3 grid(nch, d.n_kv_heads, d.batch);
+    if (d.d_proj == 32)
+        score_hist_kernel<32, SEL><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
+                                                              d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    else
+        score_hist_kernel<16, SEL><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
+                                                              d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mark_collect_kernel<SEL><<<grid, kThreads, 0, st>>>(ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W,
+                                                        sink, window, s);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4;
+    static size_t configured = 0;
+    if (fsm > 48 * 1024 && fsm > configured) {
+        e = cudaFuncSetAttribute(finalize_kernel<SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
+        if (e != cudaSuccess) return e;
+        configured = fsm;
+    }
+    const int rows = SEL == kSelHead ? d.n_q_heads : d.n_q_heads / kGroup;
+    finalize_kernel<SEL><<<dim3(rows, d.batch), kFinThreads, fsm, st>>>(
+        ctx_len, d.n_q_heads, d.ctx_cap, W, sink, window, nbr, idx, idx_cap, count, sel_bits, s);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t select_ws_bytes(const tb_dims &d) { return carve_bytes(d); }
 
 cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_stride,
                                 const uint16_t *Kp, const int32_t *ctx_len, int32_t sink,
-                                int32_t window, int32_t budget, int32_t nbr, int32_t *idx,
-                                int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
+                                int32_t window, int32_t budget, int32_t nbr, int32_t group_reduce,
+                                int32_t *idx, int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
                                 cudaStream_t st) {
-    const SelWs s = carve(d, ws);
-    const int W = (d.ctx_cap + 31) / 32;
-    const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
-    dim3 grid(nch, d.n_kv_heads, d.batch);
-    if (d.d_proj == 32)
-        score_hist_kernel<32><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
-                                                         d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
-    else
-        score_hist_kernel<16><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
-                                                         d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    mark_collect_kernel<<<grid, kThreads, 0, st>>>(ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W,
-                                                   sink, window, s);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4;
-    static size_t configured = 0;
-    if (fsm > 48 * 1024 && fsm > configured) {
-        e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
-        if (e != cudaSuccess) return e;
-        configured = fsm;
-    }
-    finalize_kernel<<<dim3(d.n_q_heads, d.batch), kFinThreads, fsm, st>>>(
-        ctx_len, d.n_q_heads, d.ctx_cap, W, sink, window, nbr, idx, idx_cap, count, sel_bits, s);
-    return cudaGetLastError();
+    if (group_reduce == 0)
+        return launch_sel<kSelGroupMax>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap,
+                                        count, sel_bits, ws, st);
+    if (group_reduce == 1)
+        return launch_sel<kSelGroupSum>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap,
+                                        count, sel_bits, ws, st);
+    return launch_sel<kSelHead>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap, count,
+                                sel_bits, ws, st);
 }
 
 cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx_cap,

@@ -99,9 +99,17 @@ class SparseDecoder:
 
     K[l], V[l]: [batch][Hkv][ctx_cap][d] bf16 caches (rows of future decode
     tokens may already be present; only rows < T are ever read).
-    Wk[l]: [Hkv][d'][d] bf16.  mlp[p] = (W1, W2) for each producer layer p."""
+    Wk[l]: [Hkv][d'][d] bf16.  mlp[p] = (W1, W2) for each producer layer p.
+    selection: "head" (one importance set per query head) or "group_max" /
+    "group_sum" (one set per KV head, tb_score_select_group)."""
 
-    def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda"):
+    SELECTIONS = ("head", "group_max", "group_sum")
+
+    def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda",
+                 selection: str = "head"):
+        if selection not in self.SELECTIONS:
+            raise ValueError(f"selection must be one of {self.SELECTIONS}")
+        self.selection = selection
         s = self.shape = shape
         self.K, self.V, self.Wk, self.mlp = K, V, Wk, mlp
         self.ctx0 = list(ctx0)
@@ -161,8 +169,13 @@ class SparseDecoder:
             buf = self.qp[producer_layer(layer, s.stride)]
             qp = buf.data_ptr() + query_slot(layer, s.stride) * s.n_q_heads * s.d_proj * 4
             stride = s.stride * s.n_q_heads * s.d_proj
-        L.score_select(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window, s.budget, s.nbr,
-                       self.idx[layer], self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+        if self.selection == "head":
+            L.score_select(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window, s.budget,
+                           s.nbr, self.idx[layer], self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+        else:
+            L.score_select_group(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window,
+                                 s.budget, s.nbr, self.selection[len("group_"):], self.idx[layer],
+                                 self.cnt[layer], self.bits[layer], self.ws_sel, stream)
 
     def attend(self, step: int, layer: int, Q, out, stream=None):
         s = self.shape

@@ -34,7 +34,7 @@ def test_exports_match_header(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.tb_abi_version() == 1
+    assert lib.tb_abi_version() == 2
     assert lib.tb_status_str(0) == b"TB_OK"
     assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
 
@@ -112,6 +112,23 @@ def test_select_rejects_bad_arguments(lib):
     st = lib.tb_score_select(ctypes.byref(small), FAKE, 32 * 32, FAKE, FAKE, 4, 16, 8192, 1, FAKE, 299,
                              FAKE, FAKE, FAKE, w2, None)
     assert st == _lib.TB_ERR_INVALID_ARG
+
+
+def test_select_group_rejects_bad_arguments(lib):
+    d = _d()
+    wsb = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
+
+    def call(reduce=0, qp=FAKE, idx_cap=3 * 8192):
+        return lib.tb_score_select_group(ctypes.byref(d), qp, 32 * 32, FAKE, FAKE, 16, 64, 8192, 1, reduce, FAKE,
+                                         idx_cap, FAKE, FAKE, FAKE, wsb, None)
+
+    assert call(reduce=2) == _lib.TB_ERR_INVALID_ARG
+    assert b"reduce" in lib.tb_last_error()
+    assert call(reduce=-1) == _lib.TB_ERR_INVALID_ARG
+    # a valid reduce goes through the same checks as tb_score_select
+    assert call(qp=0) == _lib.TB_ERR_INVALID_ARG
+    assert b"tb_score_select_group" in lib.tb_last_error() and b"qp" in lib.tb_last_error()
+    assert call(reduce=1, idx_cap=3 * 8192 - 1) == _lib.TB_ERR_INVALID_ARG
 
 
 def test_predict_and_project_reject_bad_arguments(lib):

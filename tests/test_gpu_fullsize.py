@@ -44,6 +44,7 @@ def test_full_size_sampled(name):
 
     Kp_in = Kp_gpu.clone()
     refs = {}
+    kp_refs = {}
     for (b, g) in samples:
         T = ctx0[b] + 1
         Kb = parity.bits16(K0[b, g])
@@ -53,6 +54,7 @@ def test_full_size_sampled(name):
         # the oracle's own K' and selection for this (b, g)
         Kp_ref = oracle.project_keys(Kb[:T - w.window], Wk[g])
         Kp_in[b, g, :T - w.window] = parity.from_bits16(Kp_ref)
+        kp_refs[(b, g)] = Kp_ref
         for hh in range(4 * g, 4 * g + 4):
             s = oracle.scores(qp_ref[b, hh], Kp_ref, w.sink, T - w.window)
             refs[(b, hh)] = (s, oracle.select(s, T, w.sink, w.window, w.budget, w.nbr))
@@ -70,6 +72,20 @@ def test_full_size_sampled(name):
     for (b, hh), (s, ref) in refs.items():
         got = idx[b, hh, :cnt[b, hh]].cpu().numpy()
         n_diff += parity.assert_sets_match(got, ref, s, w.sink, w.budget, w.nbr, False, f"{name} b={b} h={hh}")
+
+    # (c') the group-shared variant (one set per KV head, group max) on the same inputs
+    tb.score_select_group(dm, qpt, w.n_q_heads * w.d_proj, Kp_in, dec.ctx[0], w.sink, w.window, w.budget, w.nbr,
+                          "max", idx, cnt, bits, dec.ws_sel)
+    torch.cuda.synchronize()
+    assert tb.workspace_check(dec.ws_sel) == 0
+    for (b, g), Kp_ref in kp_refs.items():
+        T = ctx0[b] + 1
+        s = oracle.group_scores(qp_ref[b, 4 * g:4 * g + 4], Kp_ref, w.sink, T - w.window, "max")
+        ref = oracle.select(s, T, w.sink, w.window, w.budget, w.nbr)
+        got = idx[b, 4 * g, :cnt[b, 4 * g]].cpu().numpy()
+        n_diff += parity.assert_sets_match(got, ref, s, w.sink, w.budget, w.nbr, False, f"{name} group b={b} g={g}")
+        for hh in range(4 * g + 1, 4 * g + 4):
+            assert np.array_equal(idx[b, hh, :cnt[b, hh]].cpu().numpy(), got)
 
     # (d) sparse attention on the oracle's sets, dense attention
     W = dec.shape.words
