@@ -518,6 +518,8 @@ def main():
     ap.add_argument("--impl", default="tb", choices=["tb", "reference"])
     ap.add_argument("--decode-steps", type=int, default=None, help="decode steps per run (default: workload's)")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling runs)")
+    ap.add_argument("--interval", type=int, default=None,
+                    help="override the prediction interval P (1: predict and select at every step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--selection", default="head", choices=list(SparseDecoder.SELECTIONS),
@@ -543,6 +545,8 @@ def main():
     w = replica(base, rank)                          # an independent replica per rank
     if args.layers:
         w = w.scaled(n_layers=args.layers)
+    if args.interval:
+        w = w.scaled(interval=args.interval)
     run = Run(w, device, steps=args.decode_steps, selection=args.selection)
     run.dec.prefill()
     torch.cuda.synchronize()
