@@ -68,7 +68,9 @@ struct Smem {
     static constexpr int kMask = kP + 2 * 4096;       // head masks [kStages][kRows]
     static constexpr int kList = kMask + kStages * kRows;  // row list: (offset << 4) | mask, uint16
     static constexpr int kWsum = kList + kSub * 2;         // per-warp row counts of the list build
-    static constexpr int kBar = kWsum + 64;
+    static constexpr int kWords = kWsum + 64;              // staged words: 4 head masks (uint4) each
+    static constexpr int kWoff = kWords + (kSub / 32) * 16; // staged words: first list slot, + end
+    static constexpr int kBar = kWoff + (kSub / 32 + 4) * 4;
     static constexpr int kNumBars = 2 * kStages + 10;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort, n_rows, meta, reductions
     static constexpr int kEnd = kMisc + 256;
@@ -140,6 +142,8 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     const uint16_t *list = reinterpret_cast<const uint16_t *>(sm + Smem::kList);
     const uint32_t list_s = sb + Smem::kList;
     volatile int *wsum = reinterpret_cast<volatile int *>(sm + Smem::kWsum);
+    uint4 *words_s = reinterpret_cast<uint4 *>(sm + Smem::kWords);
+    int *woff_s = reinterpret_cast<int *>(sm + Smem::kWoff);
     volatile int *misc = reinterpret_cast<volatile int *>(sm + Smem::kMisc);
     volatile int *abort_flag = misc + kMiscAbort;
     volatile int *meta = misc + kMiscMeta;
@@ -251,27 +255,42 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                 int off = incl - cnt;
                 for (int w = 0; w < pw; ++w) off += wsum[w];
                 n_rows = wsum[0] + wsum[1] + wsum[2] + wsum[3];
-                // the warp writes its 32 words one at a time, lane = bit
-                // (unrolled: the words are independent, so their shuffle ->
-                // count -> store chains overlap)
-                const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll 8
-                for (int k = 0; k < 32; ++k) {
-                    const uint32_t k0 = __shfl_sync(kFull, keep[0], k), k1 = __shfl_sync(kFull, keep[1], k);
-                    const uint32_t k2 = __shfl_sync(kFull, keep[2], k), k3 = __shfl_sync(kFull, keep[3], k);
-                    const uint32_t Uk = k0 | k1 | k2 | k3;
-                    const int ok_ = __shfl_sync(kFull, off, k);
-                    const uint32_t mk = ((k0 >> lane) & 1u) | (((k1 >> lane) & 1u) << 1) |
-                                        (((k2 >> lane) & 1u) << 2) | (((k3 >> lane) & 1u) << 3);
-                    st_shared_u16_if(list_s + 2u * (uint32_t)(ok_ + __popc(Uk & lt)),
-                                     (uint16_t)((((pw * 32 + k) * 32 + lane) << 4) | mk), (Uk >> lane) & 1u);
-                }
+                // stage the word; the list itself is written progressively,
+                // just ahead of the tiles that read it (see compact_upto)
+                words_s[pt] = make_uint4(keep[0], keep[1], keep[2], keep[3]);
+                woff_s[pt] = off;
+                if (pt == 0) woff_s[kSub / 32] = n_rows;
                 fetch_words(p0 + step);
                 bar_named(kBarLoad, kRoleThreads);
             }
+            // sparse: list slots [0, woff_s[done]) are written once words
+            // [0, done) are compacted; a round compacts 8 words, 2 per warp,
+            // lane = bit, with predicated stores (no divergence)
+            int done = 0;
+            const int nwords = (p1 - p0 + 31) >> 5;
+            auto compact_upto = [&](int rows_needed) {
+                const uint32_t lt = (1u << lane) - 1u;
+                while (done < nwords && woff_s[done] < rows_needed) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int wq = done + 2 * pw + j;
+                        if (wq < nwords) {
+                            const uint4 kq = words_s[wq];
+                            const int o = woff_s[wq];
+                            const uint32_t Uk = kq.x | kq.y | kq.z | kq.w;
+                            const uint32_t mk = ((kq.x >> lane) & 1u) | (((kq.y >> lane) & 1u) << 1) |
+                                                (((kq.z >> lane) & 1u) << 2) | (((kq.w >> lane) & 1u) << 3);
+                            st_shared_u16_if(list_s + 2u * (uint32_t)(o + __popc(Uk & lt)),
+                                             (uint16_t)(((wq * 32 + lane) << 4) | mk), (Uk >> lane) & 1u);
+                        }
+                    }
+                    done += 8;
+                }
+            };
             const int n_tiles = (n_rows + kRows - 1) / kRows;
             for (int t = 0; t < n_tiles; ++t, ++it) {
                 const int s = it % kStages;
+                if constexpr (SPARSE) compact_upto(min((t + 1) * kRows, n_rows));
                 bool ok = true;
                 if (it >= kStages) ok = wait_role(empty(s), ((it / kStages) + 1) & 1, abort_flag, flags);
                 if (bar_any(kBarLoad, kRoleThreads, !ok)) {
