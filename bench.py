@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 import tb_inputs  # noqa: E402
 from query_aware_sparse_tb_b200 import _lib as L  # noqa: E402
 from query_aware_sparse_tb_b200.decode import (DecodeShape, SparseDecoder, is_prediction_step,  # noqa: E402
-                                              memcpy2d_async, record_event)
+                                              record_event)
 
 HBM_NOMINAL_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -200,31 +200,40 @@ def capture(fn, stream):
 
 
 class E2E:
-    """Per-step host<->device traffic of the public-API loop: the step's queries,
-    the new token's K and V rows of every layer and (prediction steps) the
-    producer hidden states go host->device from pinned memory; the step's
-    attention outputs come back device->host."""
+    """Per-step host<->device traffic of the public-API loop.  Every step, one
+    host->device copy brings the step's inputs from pinned memory (all layers'
+    queries and the new token's K and V rows, packed), tb_kv_append writes the
+    rows into every layer's cache in one launch, prediction steps also copy the
+    producer hidden states, and one device->host copy returns all layers'
+    attention outputs."""
 
     def __init__(self, run: Run):
         self.run = run
         w = run.w
-        self.q_host = run.Q.cpu().pin_memory()
-        self.q_dev = torch.empty_like(run.Q[0])
         nL = w.n_layers
         pos = [[t + i for t in run.ctx0] for i in range(run.steps)]     # new token position T-1
-        self.pos = pos
-        kv = torch.empty(run.steps, nL, 2, w.batch, w.n_kv_heads, w.head_dim, dtype=torch.bfloat16)
+        q_el = run.Q[0].numel()
+        kv_el = nL * 2 * w.batch * w.n_kv_heads * w.head_dim
+        packed = torch.empty(run.steps, q_el + kv_el, dtype=torch.bfloat16)
         for i in range(run.steps):
+            packed[i, :q_el] = run.Q[i].reshape(-1).cpu()
+            kv = torch.empty(nL, 2, w.batch, w.n_kv_heads, w.head_dim, dtype=torch.bfloat16)
             for l in range(nL):
                 for b in range(w.batch):
-                    kv[i, l, 0, b] = run.K[l][b, :, pos[i][b]].cpu()
-                    kv[i, l, 1, b] = run.V[l][b, :, pos[i][b]].cpu()
-        self.kv_host = kv.pin_memory()
+                    kv[l, 0, b] = run.K[l][b, :, pos[i][b]].cpu()
+                    kv[l, 1, b] = run.V[l][b, :, pos[i][b]].cpu()
+            packed[i, q_el:] = kv.reshape(-1)
+        self.host = packed.pin_memory()
+        self.dev = torch.empty(q_el + kv_el, dtype=torch.bfloat16, device=run.device)
+        self.q_dev = self.dev[:q_el].view(run.Q[0].shape)
+        self.kv_dev = self.dev[q_el:]
+        self.caches = torch.tensor([p for l in range(nL) for p in (run.K[l].data_ptr(), run.V[l].data_ptr())],
+                                   dtype=torch.int64, device=run.device)
+        self.ws = L.workspace(256, run.device)
         self.h_host = run.h.cpu().pin_memory() if run.h is not None else None
         self.h_dev = torch.empty_like(run.h[0]) if run.h is not None else None
         self.out_host = torch.empty(run.steps, *run.out.shape, dtype=torch.float32).pin_memory()
-        row = w.head_dim * 2
-        self.h2d = run.Q[0].numel() * 2 + nL * 2 * w.batch * w.n_kv_heads * row
+        self.h2d = (q_el + kv_el) * 2
         self.h2d_pred = self.h_host[0].numel() * 2 if self.h_host is not None else 0
         self.d2h = run.out.numel() * 4
 
@@ -234,20 +243,9 @@ class E2E:
 
     def body(self, stream):
         r, w = self.run, self.run.w
-        row = w.head_dim * 2
-        cap = w.ctx_cap
         for i in range(r.steps):
-            self.q_dev.copy_(self.q_host[i], non_blocking=True)
-            for l in range(w.n_layers):
-                for kind, cache in ((0, r.K[l]), (1, r.V[l])):
-                    src = self.kv_host[i, l, kind]
-                    if len(set(self.pos[i])) == 1:
-                        dst = cache.data_ptr() + self.pos[i][0] * row
-                        memcpy2d_async(dst, cap * row, src.data_ptr(), row, row, w.batch * w.n_kv_heads, 1, stream)
-                    else:
-                        for b in range(w.batch):
-                            dst = cache[b].data_ptr() + self.pos[i][b] * row
-                            memcpy2d_async(dst, cap * row, src[b].data_ptr(), row, row, w.n_kv_heads, 1, stream)
+            self.dev.copy_(self.host[i], non_blocking=True)
+            L.kv_append(r.dec.dims, w.n_layers, self.kv_dev, self.caches, r.dec.ctx[i], self.ws, stream)
             h = None
             if is_prediction_step(i, w.interval) and self.h_host is not None:
                 self.h_dev.copy_(self.h_host[i // w.interval], non_blocking=True)

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 2
+#define TB_ABI_VERSION 3
 
 typedef uint16_t tb_bf16;
 
@@ -64,6 +64,7 @@ typedef enum {
 #define TB_FLAG_CTX_RANGE   0x1u  /* some ctx_len[b] outside [1, ctx_cap]: clamped */
 #define TB_FLAG_TIMEOUT     0x2u  /* a bounded wait gave up; the output is invalid */
 #define TB_FLAG_IDX_OVERFLOW 0x4u /* selected set larger than idx_cap: truncated */
+#define TB_FLAG_BAD_CACHE   0x8u  /* tb_kv_append: a cache address was null or misaligned: skipped */
 
 /* Shapes shared by the cache-facing calls. */
 typedef struct {
@@ -192,6 +193,27 @@ tb_status tb_score_select_group(const tb_dims *dims, const float *qp, int64_t qp
  * idx[b][h][0 .. count[b][h]).  Entries outside [0, ctx_cap) are ignored. */
 tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,
                                   const int32_t *count, uint32_t *sel_bits, void *stream);
+
+/* ---- KV cache append ------------------------------------------------------ */
+/* The full KV cache stays resident and attention reads the kept rows
+ * (summary, "Significance"), so at every decode step the token being decoded
+ * is appended to every layer's cache.  This writes, in one launch, for every
+ * layer l < n_layers, sequence b and KV head g, with pos = ctx_len[b] - 1:
+ *
+ *   K_l[b][g][pos][:] = src[l][0][b][g][:],   V_l[b][g][pos][:] = src[l][1][b][g][:]
+ *
+ *   src      [n_layers][2][batch][Hkv][head_dim] bf16 (device, 16-byte aligned)
+ *   caches   [2 * n_layers] uint64 device array of cache base addresses: K of
+ *            layer l at 2l, V at 2l + 1, each [batch][Hkv][ctx_cap][head_dim]
+ *            bf16, 16-byte aligned
+ *   ctx_len  [batch] int32 (device): T including the token being decoded
+ *   ws       any libtb workspace of at least 256 bytes (its flag word)
+ * Rows whose pos lies outside [0, ctx_cap) are skipped and TB_FLAG_CTX_RANGE
+ * is raised; a null or misaligned cache address is skipped with
+ * TB_FLAG_BAD_CACHE.  No counterpart on the pages: the decode loop's cache
+ * write, gathered into one call. */
+tb_status tb_kv_append(const tb_dims *dims, int32_t n_layers, const tb_bf16 *src, const uint64_t *caches,
+                       const int32_t *ctx_len, void *ws, size_t ws_bytes, void *stream);
 
 /* ---- 5. sparse GQA decode attention --------------------------------------- */
 /* The full KV cache stays resident and only the selected tokens are read

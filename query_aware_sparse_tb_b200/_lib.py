@@ -16,7 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtb.so")
 
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
-TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW = 0x1, 0x2, 0x4
+TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW, TB_FLAG_BAD_CACHE = 0x1, 0x2, 0x4, 0x8
 TB_GROUP_REDUCE = {"max": 0, "sum": 1}
 
 EXPORTS = [
@@ -25,7 +25,7 @@ EXPORTS = [
     "tb_predict_queries_workspace_bytes", "tb_project_keys_workspace_bytes",
     "tb_workspace_init", "tb_workspace_check",
     "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_select_bits_from_idx",
-    "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc",
+    "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
 ]
 
 
@@ -73,6 +73,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_sparse_decode_attn_noalloc": ([D, P, P, P, P, i32, i32, P, f32, P, P], ctypes.c_int),
+        "tb_kv_append": ([D, i32, P, P, P, P, sz, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -206,3 +207,11 @@ def sparse_decode_attn_noalloc(d: TbDims, Q, K, V, ctx_len, sink: int, window: i
 def decode_attn(d: TbDims, Q, K, V, ctx_len, scale: float, out, ws, stream=None):
     _check(load().tb_decode_attn(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), float(scale),
                                  _ptr(out), _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def kv_append(d: TbDims, n_layers: int, src, caches, ctx_len, ws, stream=None):
+    """tb_kv_append: src [n_layers][2][batch][Hkv][d] bf16 rows of the token
+    being decoded; caches an int64 device tensor of the 2*n_layers cache base
+    addresses (K of layer l at 2l, V at 2l+1)."""
+    _check(load().tb_kv_append(ctypes.byref(d), int(n_layers), _ptr(src), _ptr(caches), _ptr(ctx_len), _ptr(ws),
+                               _bytes(ws), _stream(stream)))

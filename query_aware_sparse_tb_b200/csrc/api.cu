@@ -224,6 +224,19 @@ tb_status tb_score_select_group(const tb_dims *dims, const float *qp, int64_t qp
                              idx, idx_cap, count, sel_bits, ws, ws_bytes, stream);
 }
 
+tb_status tb_kv_append(const tb_dims *dims, int32_t n_layers, const tb_bf16 *src, const uint64_t *caches,
+                       const int32_t *ctx_len, void *ws, size_t ws_bytes, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, false, __func__)) != TB_OK) return s;
+    TB_CHECK_PTR(src); TB_CHECK_PTR4(ctx_len);
+    if (!caches || (reinterpret_cast<uintptr_t>(caches) & 7u) != 0)
+        return fail(TB_ERR_INVALID_ARG, "%s: caches is null or not 8-byte aligned", __func__);
+    if (n_layers < 1 || (long long)n_layers * 2 * dims->batch * dims->n_kv_heads > (1LL << 30))
+        return fail(TB_ERR_INVALID_ARG, "%s: n_layers %d out of range", __func__, n_layers);
+    if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
+    return cuda_status(launch_kv_append(*dims, n_layers, src, caches, ctx_len, ws, (cudaStream_t)stream), __func__);
+}
+
 tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,
                                   const int32_t *count, uint32_t *sel_bits, void *stream) {
     tb_status s;

@@ -247,10 +247,3 @@ def record_event(ev: torch.cuda.Event, stream: torch.cuda.Stream):
     if err != 0:
         raise RuntimeError(f"cudaEventRecordWithFlags failed ({err})")
 
-
-def memcpy2d_async(dst: int, dpitch: int, src: int, spitch: int, width: int, height: int, kind: int,
-                   stream: torch.cuda.Stream):
-    err = _rt().cudaMemcpy2DAsync(ctypes.c_void_p(dst), dpitch, ctypes.c_void_p(src), spitch, width, height, kind,
-                                  ctypes.c_void_p(stream.cuda_stream))
-    if err != 0:
-        raise RuntimeError(f"cudaMemcpy2DAsync failed ({err})")

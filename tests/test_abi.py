@@ -34,7 +34,7 @@ def test_exports_match_header(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.tb_abi_version() == 2
+    assert lib.tb_abi_version() == 3
     assert lib.tb_status_str(0) == b"TB_OK"
     assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
 
@@ -129,6 +129,20 @@ def test_select_group_rejects_bad_arguments(lib):
     assert call(qp=0) == _lib.TB_ERR_INVALID_ARG
     assert b"tb_score_select_group" in lib.tb_last_error() and b"qp" in lib.tb_last_error()
     assert call(reduce=1, idx_cap=3 * 8192 - 1) == _lib.TB_ERR_INVALID_ARG
+
+
+def test_kv_append_rejects_bad_arguments(lib):
+    d = _d()
+
+    def call(n_layers=32, src=FAKE, caches=FAKE, ctx=FAKE, ws=FAKE, ws_bytes=256):
+        return lib.tb_kv_append(ctypes.byref(d), n_layers, src, caches, ctx, ws, ws_bytes, None)
+
+    assert call(n_layers=0) == _lib.TB_ERR_INVALID_ARG
+    assert call(caches=0) == _lib.TB_ERR_INVALID_ARG
+    assert b"caches" in lib.tb_last_error()
+    assert call(caches=FAKE + 4) == _lib.TB_ERR_INVALID_ARG
+    assert call(src=FAKE + 8) == _lib.TB_ERR_INVALID_ARG
+    assert call(ws_bytes=255) == _lib.TB_ERR_WORKSPACE
 
 
 def test_predict_and_project_reject_bad_arguments(lib):

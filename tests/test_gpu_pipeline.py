@@ -41,7 +41,7 @@ class HostData:
         return parity.bits16(tb_inputs.query(self.w, i, l, DEV))
 
 
-def _setup(w):
+def _setup(w, selection="head"):
     K, V, Wk = [], [], []
     for l in range(w.n_layers):
         k, v = tb_inputs.kv_layer(w, l, DEV)
@@ -54,7 +54,7 @@ def _setup(w):
                         head_dim=w.head_dim, d_proj=w.d_proj, hidden=w.hidden, inter=w.inter, stride=stride,
                         sink=w.sink, window=w.window, budget=w.budget, nbr=w.nbr, interval=w.interval,
                         ctx_cap=w.ctx_cap)
-    dec = SparseDecoder(shape, K, V, Wk, mlp, w.ctx0_per_seq(), w.steps, DEV)
+    dec = SparseDecoder(shape, K, V, Wk, mlp, w.ctx0_per_seq(), w.steps, DEV, selection=selection)
     return dec, dict(K=K, V=V, Wk=Wk, mlp=mlp)
 
 
@@ -79,15 +79,17 @@ def test_projection_schedule_matches_oracle_schedule():
                 assert [(i, v[b]) for i, v in sorted(ev.items()) if v[b] >= 0] == oev
 
 
-def test_tiny300_end_to_end_bit_exact_selection():
+@pytest.mark.parametrize("selection", ["head", "group_max", "group_sum"])
+def test_tiny300_end_to_end_bit_exact_selection(selection):
+    # integer-valued inputs: every score is exact, so the sets must match bit for bit
     w = tb_inputs.WORKLOADS["tiny300"]
-    dec, run = _setup(w)
+    dec, run = _setup(w, selection)
     dec.prefill()
     Q, _, qd = _step_inputs(w, 0)
     out = torch.zeros(1, 1, w.n_q_heads, w.head_dim, device=DEV)
     dec.step(0, Q, out, qp_direct=qd)
     torch.cuda.synchronize()
-    ref = oschedule.run(w, HostData(w, run), layers=[0], steps=1)[(0, 0)]
+    ref = oschedule.run(w, HostData(w, run), layers=[0], steps=1, selection=selection)[(0, 0)]
     for h in range(w.n_q_heads):
         got = dec.idx[0][0, h, :dec.cnt[0][0, h]].cpu().numpy()
         assert np.array_equal(got, ref["idx"][0][h]), h

@@ -94,6 +94,25 @@ def test_run_tiny300_invariants():
     assert np.all(np.isfinite(r["out"]))
 
 
+def test_run_group_selection_shares_one_set_per_kv_head():
+    # the group-shared variant: the 4 heads of a KV head attend to one set, the
+    # top-B of the group score (max or fp32 sum of the head scores)
+    w = tb_inputs.WORKLOADS["tiny300"]
+    data = HostData(w)
+    T = w.ctx0 + 1
+    K, _ = data.kv(0)
+    qp = data.qp_direct(0, 0)
+    for red in ("max", "sum"):
+        r = schedule.run(w, data, layers=[0], steps=1, selection="group_" + red)[(0, 0)]
+        for g in range(w.n_kv_heads):
+            Kp = oracle.project_keys(K[0, g, :T - w.window], data.wk(0)[g])
+            s = oracle.group_scores(qp[0, 4 * g:4 * g + 4], Kp, w.sink, T - w.window, red)
+            want = oracle.select(s, T, w.sink, w.window, w.budget, w.nbr)
+            for h in range(4 * g, 4 * g + 4):
+                assert np.array_equal(r["idx"][0][h], want), (red, g, h)
+        assert np.all(np.isfinite(r["out"]))
+
+
 def test_run_reuses_selection_over_interval():
     w = _small_llama()
     res = schedule.run(w, HostData(w), layers=[0, 1], steps=w.steps)
