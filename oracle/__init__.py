@@ -51,6 +51,8 @@ def _bind(path: str):
     lib.orc_group_scores.restype = None
     lib.orc_select.argtypes = [P, i64, i64, i64, i64, i32, P]
     lib.orc_select.restype = i64
+    lib.orc_select_inclusive.argtypes = [P, i64, i64, i64, i64, i32, P]
+    lib.orc_select_inclusive.restype = i64
     lib.orc_attention_set.argtypes = [i64, i64, i64, P, i64, P]
     lib.orc_attention_set.restype = i64
     lib.orc_attention.argtypes = [P, P, P, i32, P, i64, f64, P]
@@ -174,6 +176,19 @@ def select(s_cand: np.ndarray, T: int, S: int, N: int, B: int, nbr: int, lib=Non
     assert s_cand.shape == (nC,)
     out = np.empty(max(nC, 1), dtype=np.int32)
     n = lib.orc_select(_ptr(s_cand), T, S, N, B, nbr, _ptr(out)) if nC else 0
+    return out[:n].copy()
+
+
+def select_inclusive(s_cand: np.ndarray, T: int, S: int, N: int, B: int, nbr: int, lib=None) -> np.ndarray:
+    """Budget-inclusive variant: candidates in (score desc, position asc) order
+    while the union of their +-nbr neighbourhoods, clipped to [S, T-N), holds
+    at most B positions; sorted int32 positions."""
+    lib = lib or load()
+    nC = max(0, T - N - S)
+    s_cand = np.ascontiguousarray(s_cand, dtype=np.float32)
+    assert s_cand.shape == (nC,)
+    out = np.empty(max(nC, 1), dtype=np.int32)
+    n = lib.orc_select_inclusive(_ptr(s_cand), T, S, N, B, nbr, _ptr(out)) if nC else 0
     return out[:n].copy()
 
 

@@ -249,6 +249,47 @@ int64_t orc_select(const float *s, int64_t T, int64_t S, int64_t N, int64_t B,
     return n;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Step 4, budget-inclusive variant (not on the pages).  An alternative to    */
+/* reading R3 in which the importance buffer itself holds at most B tokens:  */
+/* candidates are taken in the order of orc_select (score descending,        */
+/* position ascending) while the union of their [t-r, t+r] neighbourhoods,   */
+/* clipped to C, stays within B; the first candidate that would push it past */
+/* B ends the selection.  Every taken candidate belongs to the union, so at  */
+/* most B candidates are taken.                                               */
+/* ------------------------------------------------------------------------ */
+
+int64_t orc_select_inclusive(const float *s, int64_t T, int64_t S, int64_t N, int64_t B,
+                             int r, int32_t *idx)
+{
+    const int64_t lo = S, hi = T - N;
+    if (hi <= lo || B <= 0) return 0;
+    const int64_t n_cand = hi - lo;
+
+    orc_cand *order = (orc_cand *)malloc(sizeof(orc_cand) * (size_t)n_cand);
+    for (int64_t k = 0; k < n_cand; ++k) { order[k].s = s[k]; order[k].t = (int32_t)(lo + k); }
+    qsort(order, (size_t)n_cand, sizeof(orc_cand), orc_cand_cmp);
+
+    unsigned char *in_set = (unsigned char *)calloc((size_t)n_cand, 1);
+    int64_t size = 0;
+    for (int64_t k = 0; k < n_cand; ++k) {
+        const int64_t t = order[k].t;
+        const int64_t from = t - r < lo ? lo : t - r;
+        const int64_t to = t + r > hi - 1 ? hi - 1 : t + r;
+        int64_t fresh = 0;
+        for (int64_t u = from; u <= to; ++u) fresh += !in_set[u - lo];
+        if (size + fresh > B) break;
+        for (int64_t u = from; u <= to; ++u) in_set[u - lo] = 1;
+        size += fresh;
+    }
+    int64_t n = 0;
+    for (int64_t k = 0; k < n_cand; ++k)
+        if (in_set[k]) idx[n++] = (int32_t)(lo + k);
+    free(in_set);
+    free(order);
+    return n;
+}
+
 /* The attended set A = sink U window U I, sorted ascending ([ja] 推論戦略).
  * I must lie in C = [S, T-N), so the three parts are disjoint.  Returns |A|. */
 int64_t orc_attention_set(int64_t T, int64_t S, int64_t N,

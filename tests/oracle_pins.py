@@ -18,6 +18,9 @@ What pins what:
                      heads select what one head selects
   selection          hand-worked golden cases, and brute force by rank counting
                      on tiny inputs with many ties
+  inclusive budget   a hand-worked case, brute force (the union recomputed from
+                     scratch for every prefix of the score order), and r = 0,
+                     where it is the plain top-B
   attention set      sink/window/importance invariants
   attention          closed forms (two-logit softmax, equal logits, constant V),
                      torch float64 softmax as a witness, sparse == dense when the
@@ -257,6 +260,49 @@ def pin_select_brute_force(lib):
         assert got == want, (S, N, T, B, r, s.tolist(), got, want)
 
 
+def pin_select_inclusive_worked_case(lib):
+    # C = [10, 15), scores fall with position, B = 4, r = 1: t=10 brings {10, 11}
+    # (9 is the sink), 11 brings 12, 12 brings 13, and 13 would make 5 > 4.
+    s = np.array([5, 4, 3, 2, 1], np.float32)
+    assert oracle.select_inclusive(s, 20, 10, 5, 4, 1, lib=lib).tolist() == [10, 11, 12, 13]
+    # C = [0, 6), B = 5, r = 1, order 0, 2, 1, 3, 4, 5: t=0 brings {0, 1}, t=2
+    # brings {2, 3}, t=1 is already covered and costs nothing, t=3 brings 4,
+    # and t=4 would bring 5 (6 > 5).  Stopping at the free candidate would
+    # give [0, 1, 2, 3].
+    s = np.array([9, 6, 8, 1, 1, 1], np.float32)
+    assert oracle.select_inclusive(s, 6, 0, 0, 5, 1, lib=lib).tolist() == [0, 1, 2, 3, 4]
+
+
+def _brute_select_inclusive(s, T, S, N, B, r):
+    lo, hi = S, T - N
+    order = sorted(range(lo, hi), key=lambda t: (-float(s[t - lo]), t))
+    best = []
+    for k in range(len(order) + 1):
+        union = sorted({u for t in order[:k] for u in range(t - r, t + r + 1) if lo <= u < hi})
+        if len(union) > B:
+            break
+        best = union
+    return best
+
+
+def pin_select_inclusive_brute_force(lib):
+    rng = np.random.default_rng(13)
+    for trial in range(300):
+        S = int(rng.integers(0, 5))
+        N = int(rng.integers(1, 6))
+        T = int(rng.integers(1, 40))
+        B = int(rng.integers(1, 14))
+        r = int(rng.integers(0, 3))
+        nC = max(0, T - N - S)
+        s = rng.integers(-3, 4, nC).astype(np.float32)
+        if trial % 3 == 0:
+            s = rng.standard_normal(nC).astype(np.float32)
+        got = oracle.select_inclusive(s, T, S, N, B, r, lib=lib).tolist()
+        assert got == _brute_select_inclusive(s, T, S, N, B, r), (S, N, T, B, r, s.tolist(), got)
+        if r == 0:
+            assert got == oracle.select(s, T, S, N, B, 0, lib=lib).tolist()
+
+
 # ---------------------------------------------------------------------------
 # attention set and attention
 # ---------------------------------------------------------------------------
@@ -356,6 +402,8 @@ ALL_PINS = [
     pin_group_selection_identical_heads,
     pin_select_golden,
     pin_select_brute_force,
+    pin_select_inclusive_worked_case,
+    pin_select_inclusive_brute_force,
     pin_attention_set,
     pin_attention_golden,
     pin_attention_constant_v,

@@ -45,6 +45,9 @@ MUTANTS = [
     ("group_max_is_min", "g = sh > g ? sh : g;", "g = sh < g ? sh : g;"),
     ("group_drops_last_head", "for (int h = 0; h < G; ++h) {", "for (int h = 0; h < G - 1; ++h) {"),
     ("group_sum_in_double", "        float g = 0.0f;", "        double g = 0.0;"),
+    ("inclusive_allows_overshoot", "if (size + fresh > B) break;", "if (size + fresh > B + 1) break;"),
+    ("inclusive_skips_instead_of_stopping", "if (size + fresh > B) break;", "if (size + fresh > B) continue;"),
+    ("inclusive_counts_covered", "fresh += !in_set[u - lo];", "fresh += 1;"),
 ]
 
 
