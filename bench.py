@@ -463,7 +463,8 @@ def config_of(w: tb_inputs.Workload, decode_steps: int, world: int, selection: s
     return {"workload": w.name, "batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
             "layers": w.n_layers, "decode_steps_per_bench_step": decode_steps, "budget": w.budget,
             "interval": w.interval, "sink": w.sink, "window": w.window, "d_proj": w.d_proj,
-            "selection": "per query head" if selection == "head" else f"per KV head ({selection})",
+            "selection": {"head": "per query head", "inclusive": "per query head, budget includes neighbours"}.get(
+                selection, f"per KV head ({selection})"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -522,7 +523,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--selection", default="head", choices=list(SparseDecoder.SELECTIONS),
                     help="head: one importance set per query head (the default, the pages' reading); "
-                         "group_max / group_sum: one set per KV head (the group-shared variant)")
+                         "group_max / group_sum: one set per KV head (the group-shared variant); "
+                         "inclusive: at most B positions per head after neighbour fetch")
     args = ap.parse_args()
 
     if args.impl == "reference":

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 3
+#define TB_ABI_VERSION 4
 
 typedef uint16_t tb_bf16;
 
@@ -187,6 +187,22 @@ tb_status tb_score_select_group(const tb_dims *dims, const float *qp, int64_t qp
                                 int32_t budget, int32_t nbr, int32_t reduce, int32_t *idx, int32_t idx_cap,
                                 int32_t *count, uint32_t *sel_bits, void *ws, size_t ws_bytes,
                                 void *stream);
+
+/* Budget-inclusive variant (no counterpart on the pages; an alternative to
+ * counting the budget before neighbour fetch).  Per query head, the
+ * importance buffer itself holds at most `budget` positions: with the
+ * candidates of C in the order (s desc, t asc) defined above,
+ *
+ *   I = ( ∪_{t in P} [t - nbr, t + nbr] ) ∩ C
+ *
+ * for the longest prefix P of that order whose I has at most `budget`
+ * members (every member of P is in I, so |P| <= budget).  Arguments and
+ * layouts are those of tb_score_select, except idx_cap >= min(budget,
+ * ctx_cap) suffices; budget <= 8192 (larger is TB_ERR_UNSUPPORTED). */
+tb_status tb_score_select_inclusive(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
+                                    const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
+                                    int32_t budget, int32_t nbr, int32_t *idx, int32_t idx_cap, int32_t *count,
+                                    uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream);
 
 /* Build the sel_bits bitmap from index lists that came from elsewhere (e.g. a
  * host-side selection): bit t of row (b,h) is set iff t is among

@@ -24,7 +24,8 @@ EXPORTS = [
     "tb_score_select_workspace_bytes", "tb_attn_workspace_bytes",
     "tb_predict_queries_workspace_bytes", "tb_project_keys_workspace_bytes",
     "tb_workspace_init", "tb_workspace_check",
-    "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_select_bits_from_idx",
+    "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_score_select_inclusive",
+    "tb_select_bits_from_idx",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
 ]
 
@@ -69,6 +70,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_score_select": ([D, P, i64, P, P, i32, i32, i32, i32, P, i32, P, P, P, sz, P], ctypes.c_int),
         "tb_score_select_group": ([D, P, i64, P, P, i32, i32, i32, i32, i32, P, i32, P, P, P, sz, P],
                                   ctypes.c_int),
+        "tb_score_select_inclusive": ([D, P, i64, P, P, i32, i32, i32, i32, P, i32, P, P, P, sz, P], ctypes.c_int),
         "tb_select_bits_from_idx": ([D, P, i32, P, P, P], ctypes.c_int),
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
@@ -182,6 +184,16 @@ def score_select_group(d: TbDims, qp, qp_batch_stride: int, Kp, ctx_len, sink: i
     _check(load().tb_score_select_group(ctypes.byref(d), _ptr(qp), int(qp_batch_stride), _ptr(Kp), _ptr(ctx_len),
                                         sink, window, budget, nbr, TB_GROUP_REDUCE[reduce], _ptr(idx), idx_cap,
                                         _ptr(count), _ptr(sel_bits), _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def score_select_inclusive(d: TbDims, qp, qp_batch_stride: int, Kp, ctx_len, sink: int, window: int,
+                           budget: int, nbr: int, idx, count, sel_bits, ws, stream=None):
+    """tb_score_select_inclusive: per head, the importance buffer holds at most
+    `budget` positions after neighbour fetch."""
+    idx_cap = idx.shape[-1]
+    _check(load().tb_score_select_inclusive(ctypes.byref(d), _ptr(qp), int(qp_batch_stride), _ptr(Kp),
+                                            _ptr(ctx_len), sink, window, budget, nbr, _ptr(idx), idx_cap,
+                                            _ptr(count), _ptr(sel_bits), _ptr(ws), _bytes(ws), _stream(stream)))
 
 
 def select_bits_from_idx(d: TbDims, idx, count, sel_bits, stream=None):

@@ -23,6 +23,7 @@ void set_error(const char *fmt, ...) {
 namespace {
 
 constexpr int kMaxCtxSelect = 1 << 19;
+constexpr int kMaxInclusiveBudget = 8192;
 constexpr int kMaxCtxAttn = 1 << 22;
 
 tb_status fail(tb_status s, const char *fmt, ...) {
@@ -194,10 +195,13 @@ static tb_status score_select_impl(const char *fn, const tb_dims *dims, const fl
     if (sink < 0 || window < 1 || budget < 1)
         return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0, window >= 1, budget >= 1", fn);
     if (nbr < 0 || nbr > 16) return fail(TB_ERR_INVALID_ARG, "%s: nbr %d outside [0, 16]", fn, nbr);
-    const long long need_cap = (long long)(2 * nbr + 1) * budget;
+    // group_reduce 2 is the budget-inclusive mode: |I| <= budget
+    if (group_reduce == 2 && budget > kMaxInclusiveBudget)
+        return fail(TB_ERR_UNSUPPORTED, "%s: budget %d above %d", fn, budget, kMaxInclusiveBudget);
+    const long long need_cap = group_reduce == 2 ? (long long)budget : (long long)(2 * nbr + 1) * budget;
     const long long min_cap = need_cap < dims->ctx_cap ? need_cap : dims->ctx_cap;
     if (idx_cap < min_cap)
-        return fail(TB_ERR_INVALID_ARG, "%s: idx_cap %d < min((2*nbr+1)*budget, ctx_cap) = %lld", fn, idx_cap,
+        return fail(TB_ERR_INVALID_ARG, "%s: idx_cap %d < %lld (the largest possible selection)", fn, idx_cap,
                     min_cap);
     if ((s = check_ws(ws, ws_bytes, select_ws_bytes(*dims), fn)) != TB_OK) return s;
     return cuda_status(launch_score_select(*dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget, nbr,
@@ -235,6 +239,14 @@ tb_status tb_kv_append(const tb_dims *dims, int32_t n_layers, const tb_bf16 *src
         return fail(TB_ERR_INVALID_ARG, "%s: n_layers %d out of range", __func__, n_layers);
     if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
     return cuda_status(launch_kv_append(*dims, n_layers, src, caches, ctx_len, ws, (cudaStream_t)stream), __func__);
+}
+
+tb_status tb_score_select_inclusive(const tb_dims *dims, const float *qp, int64_t qp_batch_stride,
+                                    const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
+                                    int32_t budget, int32_t nbr, int32_t *idx, int32_t idx_cap, int32_t *count,
+                                    uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream) {
+    return score_select_impl(__func__, dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget, nbr, 2, idx,
+                             idx_cap, count, sel_bits, ws, ws_bytes, stream);
 }
 
 tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,

@@ -20,7 +20,8 @@ cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, 
 // ---- score + select (select.cu) ----
 size_t select_ws_bytes(const tb_dims &d);
 // group_reduce: -1 = one set per query head; 0 / 1 = one set per KV head from
-// the largest / the fp32 sum of the group's head scores.
+// the largest / the fp32 sum of the group's head scores; 2 = one set per query
+// head holding at most `budget` positions after neighbour fetch.
 cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_stride,
                                 const uint16_t *Kp, const int32_t *ctx_len, int32_t sink,
                                 int32_t window, int32_t budget, int32_t nbr, int32_t group_reduce,

@@ -44,7 +44,11 @@ enum : uint32_t { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
 // from the largest or the fp32 sum (heads in order) of the group's scores.
 // A group's set is kept in the rows of its first head until finalize copies
 // it to all 4 heads.
-enum : int { kSelHead = 0, kSelGroupMax = 1, kSelGroupSum = 2 };
+enum : int { kSelHead = 0, kSelGroupMax = 1, kSelGroupSum = 2, kSelInclusive = 3 };
+// kSelInclusive: per query head, but the importance buffer itself holds at
+// most B tokens (candidates in score order while the union of their
+// neighbourhoods fits); its budget is at most kCandCache.
+__host__ __device__ constexpr bool sel_is_group(int sel) { return sel == kSelGroupMax || sel == kSelGroupSum; }
 
 struct HeadState {   // 8 words per (b, query head)
     uint32_t mode, b1, k_rem, cand_count, n_in_bin, pad[3];
@@ -161,7 +165,7 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
     constexpr int PER = kChunk / kThreads;  // positions per thread
-    constexpr int NH = SEL == kSelHead ? kGroup : 1;  // score rows per (b, KV head)
+    constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
     __shared__ __align__(16) float qs[kGroup][DP];
     __shared__ uint32_t hist[NH][kBins1];
     __shared__ int s_last;
@@ -227,7 +231,7 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
             for (int k = 0; k < R; ++k) {
                 const int p = p0 + (k0 + k) * kThreads + tid;
                 const bool valid = p >= lo && p < hi;
-                if constexpr (SEL == kSelHead) {
+                if constexpr (!sel_is_group(SEL)) {
 #pragma unroll
                     for (int h = 0; h < kGroup; ++h) {
                         const uint32_t key = score_key(sc[k][h]);
@@ -315,7 +319,7 @@ __global__ void __launch_bounds__(kThreads)
 mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int W,
                     int sink, int window, SelWs ws) {
     constexpr int kWordsPerWarp = kChunk / 32 / (kThreads / 32);  // 4
-    constexpr int NH = SEL == kSelHead ? kGroup : 1;
+    constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;
     __shared__ uint32_t s_cnt[kGroup], s_base[kGroup];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
@@ -398,7 +402,7 @@ __device__ __forceinline__ uint32_t range_mask(int w, int lo, int hi) {
 template <int SEL>
 __global__ void __launch_bounds__(kFinThreads)
 finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int sink, int window,
-                int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
+                int budget, int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
                 uint32_t *__restrict__ sel_bits, SelWs ws) {
     extern __shared__ unsigned long long fsm8[];
     unsigned long long *cand_s = fsm8;                                  // [kCandCache]
@@ -408,7 +412,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
     __shared__ int scratch[kFinThreads / 32 + 3];
 
     // a group's set is computed in its first head's rows and written to all 4
-    constexpr int NOUT = SEL == kSelHead ? 1 : kGroup;
+    constexpr int NOUT = sel_is_group(SEL) ? kGroup : 1;
     const int tid = threadIdx.x;
     const int h = blockIdx.x * NOUT, b = blockIdx.y;
     const size_t row = (size_t)b * Hq + h;
@@ -482,6 +486,131 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         }
     }
     __syncthreads();
+
+    if constexpr (SEL == kSelInclusive) {
+        // top_s holds the exact top-B positions (B <= kCandCache).  Keep the
+        // longest prefix of them in score order whose neighbourhoods, clipped
+        // to C, cover at most B positions.
+        const int lane = tid & 31;
+        const uint32_t lt = (1u << lane) - 1u;
+        const uint32_t *keys = ws.keys + row * Tcap;
+        // rank of the k-th top position (position order): after the tie
+        // buffer, which now holds the per-word count of top positions before it
+        uint16_t *rank_by_idx = reinterpret_cast<uint16_t *>(tie_s + W);
+        uint32_t *wpref = tie_s;
+        // 1. gather (key, position) of the top positions, words in order
+        const int wpt = (W + kFinThreads - 1) / kFinThreads;
+        const int wb = tid * wpt, we = min(wb + wpt, W);
+        int mine = 0;
+        for (int w = wb; w < we; ++w) mine += __popc(top_s[w]);
+        int n_top;
+        const int base = block_excl_scan<kFinThreads>(mine, scratch, &n_top);
+        {
+            int acc = base;
+            for (int w = wb; w < we; ++w) {
+                wpref[w] = (uint32_t)acc;
+                acc += __popc(top_s[w]);
+            }
+        }
+        {
+            // lane = bit; the keys of 16 words are requested before any is used
+            constexpr int kWB = 16;
+            const int w_first = (tid - lane) * wpt, w_last = min(w_first + 32 * wpt, W);
+            int run = __shfl_sync(kFull, base, 0);
+            for (int w0 = w_first; w0 < w_last; w0 += kWB) {
+                uint32_t ev[kWB], kv[kWB];
+#pragma unroll
+                for (int u = 0; u < kWB; ++u) {
+                    const int w = w0 + u;
+                    ev[u] = w < w_last ? top_s[w] : 0u;
+                    kv[u] = ((ev[u] >> lane) & 1u) ? __ldcg(keys + (w << 5) + lane) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < kWB; ++u) {
+                    if ((ev[u] >> lane) & 1u) {
+                        const uint32_t p = (uint32_t)(((w0 + u) << 5) + lane);
+                        cand_s[run + __popc(ev[u] & lt)] = ((unsigned long long)kv[u] << 32) | (0xFFFFFFFFu - p);
+                    }
+                    run += __popc(ev[u]);
+                }
+            }
+        }
+        int P = 1;
+        while (P < n_top) P <<= 1;
+        for (int i = n_top + tid; i < P; i += kFinThreads) cand_s[i] = 0ull;  // sorts last
+        __syncthreads();
+        // 2. bitonic sort, descending: score key first, then the lower position
+        for (int k = 2; k <= P; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll 8
+                for (int i = tid; i < P; i += kFinThreads) {
+                    const int ixj = i ^ j;
+                    if (ixj > i) {
+                        const unsigned long long a = cand_s[i], c = cand_s[ixj];
+                        if (((i & k) == 0) ? (a < c) : (a > c)) {
+                            cand_s[i] = c;
+                            cand_s[ixj] = a;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        // 3. rank of each top position, looked up through its index among the
+        //    top positions (all in shared memory)
+        auto top_index = [&](uint32_t u) {
+            return wpref[u >> 5] + __popc(top_s[u >> 5] & ((1u << (u & 31)) - 1u));
+        };
+        for (int j = tid; j < n_top; j += kFinThreads)
+            rank_by_idx[top_index(0xFFFFFFFFu - (uint32_t)cand_s[j])] = (uint16_t)j;
+        __syncthreads();
+        // 4. positions each candidate adds: those of its neighbourhood (in C)
+        //    not within nbr of a better-ranked top position
+        auto is_top = [&](int u) { return (top_s[u >> 5] >> (u & 31)) & 1u; };
+        for (int j = tid; j < n_top; j += kFinThreads) {
+            const int p = (int)(0xFFFFFFFFu - (uint32_t)cand_s[j]);
+            uint32_t gain = 0;
+            for (int q = max(p - nbr, lo); q <= min(p + nbr, hi - 1); ++q) {
+                bool covered = false;
+                for (int u = max(q - nbr, lo); u <= min(q + nbr, hi - 1) && !covered; ++u)
+                    covered = is_top(u) && rank_by_idx[top_index((uint32_t)u)] < (uint32_t)j;
+                gain += covered ? 0u : 1u;
+            }
+            cand_s[j] = ((unsigned long long)gain << 32) | (uint32_t)cand_s[j];
+        }
+        __syncthreads();
+        // 5. the longest prefix whose running size stays within the budget:
+        //    thread t owns ranks [8t, 8t + 8); sizes only grow along the ranks
+        constexpr int kPer = kCandCache / kFinThreads;
+        int sum = 0;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int j = tid * kPer + e;
+            if (j < n_top) sum += (int)(cand_s[j] >> 32);
+        }
+        int tot;
+        int run = block_excl_scan<kFinThreads>(sum, scratch, &tot);
+        int keep_n = 0;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int j = tid * kPer + e;
+            if (j < n_top) {
+                run += (int)(cand_s[j] >> 32);
+                if (run <= budget) keep_n = e + 1;
+            }
+        }
+        // prefix sizes are monotone, so the kept ranks are [0, k*): count them
+        int kept;
+        (void)block_excl_scan<kFinThreads>(keep_n, scratch, &kept);
+        // 6. the Top bitmap becomes those k* positions; dilation and emission follow
+        for (int w = tid; w < W; w += kFinThreads) top_s[w] = 0u;
+        __syncthreads();
+        for (int j = tid; j < kept; j += kFinThreads) {
+            const uint32_t p = 0xFFFFFFFFu - (uint32_t)cand_s[j];
+            atomicOr(&top_s[p >> 5], 1u << (p & 31));
+        }
+        __syncthreads();
+    }
 
     // neighbour fetch, clip to C, emit bitmap and sorted index list
     const int wpt = (W + kFinThreads - 1) / kFinThreads;
@@ -567,16 +696,16 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
                                                         sink, window, s);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4;
+    const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4 + (SEL == kSelInclusive ? kCandCache * 2 : 0);
     static size_t configured = 0;
     if (fsm > 48 * 1024 && fsm > configured) {
         e = cudaFuncSetAttribute(finalize_kernel<SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
         if (e != cudaSuccess) return e;
         configured = fsm;
     }
-    const int rows = SEL == kSelHead ? d.n_q_heads : d.n_q_heads / kGroup;
+    const int rows = sel_is_group(SEL) ? d.n_q_heads / kGroup : d.n_q_heads;
     finalize_kernel<SEL><<<dim3(rows, d.batch), kFinThreads, fsm, st>>>(
-        ctx_len, d.n_q_heads, d.ctx_cap, W, sink, window, nbr, idx, idx_cap, count, sel_bits, s);
+        ctx_len, d.n_q_heads, d.ctx_cap, W, sink, window, budget, nbr, idx, idx_cap, count, sel_bits, s);
     return cudaGetLastError();
 }
 
@@ -592,6 +721,9 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
     if (group_reduce == 0)
         return launch_sel<kSelGroupMax>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap,
                                         count, sel_bits, ws, st);
+    if (group_reduce == 2)
+        return launch_sel<kSelInclusive>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap,
+                                         count, sel_bits, ws, st);
     if (group_reduce == 1)
         return launch_sel<kSelGroupSum>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap,
                                         count, sel_bits, ws, st);

@@ -100,10 +100,12 @@ class SparseDecoder:
     K[l], V[l]: [batch][Hkv][ctx_cap][d] bf16 caches (rows of future decode
     tokens may already be present; only rows < T are ever read).
     Wk[l]: [Hkv][d'][d] bf16.  mlp[p] = (W1, W2) for each producer layer p.
-    selection: "head" (one importance set per query head) or "group_max" /
-    "group_sum" (one set per KV head, tb_score_select_group)."""
+    selection: "head" (one importance set per query head), "group_max" /
+    "group_sum" (one set per KV head, tb_score_select_group) or "inclusive"
+    (per head, at most `budget` positions after neighbour fetch,
+    tb_score_select_inclusive)."""
 
-    SELECTIONS = ("head", "group_max", "group_sum")
+    SELECTIONS = ("head", "group_max", "group_sum", "inclusive")
 
     def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda",
                  selection: str = "head"):
@@ -172,6 +174,10 @@ class SparseDecoder:
         if self.selection == "head":
             L.score_select(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window, s.budget,
                            s.nbr, self.idx[layer], self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+        elif self.selection == "inclusive":
+            L.score_select_inclusive(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window,
+                                     s.budget, s.nbr, self.idx[layer], self.cnt[layer], self.bits[layer],
+                                     self.ws_sel, stream)
         else:
             L.score_select_group(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window,
                                  s.budget, s.nbr, self.selection[len("group_"):], self.idx[layer],

@@ -34,7 +34,7 @@ def test_exports_match_header(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.tb_abi_version() == 3
+    assert lib.tb_abi_version() == 4
     assert lib.tb_status_str(0) == b"TB_OK"
     assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
 
@@ -129,6 +129,19 @@ def test_select_group_rejects_bad_arguments(lib):
     assert call(qp=0) == _lib.TB_ERR_INVALID_ARG
     assert b"tb_score_select_group" in lib.tb_last_error() and b"qp" in lib.tb_last_error()
     assert call(reduce=1, idx_cap=3 * 8192 - 1) == _lib.TB_ERR_INVALID_ARG
+
+
+def test_select_inclusive_rejects_bad_arguments(lib):
+    d = _d()
+    wsb = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
+
+    def call(budget=8192, idx_cap=8192):
+        return lib.tb_score_select_inclusive(ctypes.byref(d), FAKE, 32 * 32, FAKE, FAKE, 16, 64, budget, 1, FAKE,
+                                             idx_cap, FAKE, FAKE, FAKE, wsb, None)
+
+    assert call(budget=8193, idx_cap=8193) == _lib.TB_ERR_UNSUPPORTED
+    assert call(idx_cap=8191) == _lib.TB_ERR_INVALID_ARG
+    assert b"idx_cap" in lib.tb_last_error() and b"tb_score_select_inclusive" in lib.tb_last_error()
 
 
 def test_kv_append_rejects_bad_arguments(lib):
