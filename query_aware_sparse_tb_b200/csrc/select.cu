@@ -494,9 +494,9 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         const int lane = tid & 31;
         const uint32_t lt = (1u << lane) - 1u;
         const uint32_t *keys = ws.keys + row * Tcap;
-        // rank of the k-th top position (position order): after the tie
+        // gain of the k-th top position (position order): after the tie
         // buffer, which now holds the per-word count of top positions before it
-        uint16_t *rank_by_idx = reinterpret_cast<uint16_t *>(tie_s + W);
+        uint16_t *gain_s = reinterpret_cast<uint16_t *>(tie_s + W);
         uint32_t *wpref = tie_s;
         // 1. gather (key, position) of the top positions, words in order
         const int wpt = (W + kFinThreads - 1) / kFinThreads;
@@ -535,80 +535,72 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
                 }
             }
         }
-        int P = 1;
-        while (P < n_top) P <<= 1;
-        for (int i = n_top + tid; i < P; i += kFinThreads) cand_s[i] = 0ull;  // sorts last
         __syncthreads();
-        // 2. bitonic sort, descending: score key first, then the lower position
-        for (int k = 2; k <= P; k <<= 1) {
-            for (int j = k >> 1; j > 0; j >>= 1) {
-#pragma unroll 8
-                for (int i = tid; i < P; i += kFinThreads) {
-                    const int ixj = i ^ j;
-                    if (ixj > i) {
-                        const unsigned long long a = cand_s[i], c = cand_s[ixj];
-                        if (((i & k) == 0) ? (a < c) : (a > c)) {
-                            cand_s[i] = c;
-                            cand_s[ixj] = a;
-                        }
-                    }
-                }
-                __syncthreads();
-            }
-        }
-        // 3. rank of each top position, looked up through its index among the
-        //    top positions (all in shared memory)
+        // 2. gains, in position order: a top position ranks ahead of p exactly
+        //    when its (key, inverted position) composite is larger, so no sort
+        //    is needed to tell which neighbours come first
         auto top_index = [&](uint32_t u) {
             return wpref[u >> 5] + __popc(top_s[u >> 5] & ((1u << (u & 31)) - 1u));
         };
-        for (int j = tid; j < n_top; j += kFinThreads)
-            rank_by_idx[top_index(0xFFFFFFFFu - (uint32_t)cand_s[j])] = (uint16_t)j;
-        __syncthreads();
-        // 4. positions each candidate adds: those of its neighbourhood (in C)
-        //    not within nbr of a better-ranked top position
         auto is_top = [&](int u) { return (top_s[u >> 5] >> (u & 31)) & 1u; };
+        uint32_t my_gain = 0;
         for (int j = tid; j < n_top; j += kFinThreads) {
-            const int p = (int)(0xFFFFFFFFu - (uint32_t)cand_s[j]);
+            const unsigned long long cp = cand_s[j];
+            const int p = (int)(0xFFFFFFFFu - (uint32_t)cp);
             uint32_t gain = 0;
             for (int q = max(p - nbr, lo); q <= min(p + nbr, hi - 1); ++q) {
                 bool covered = false;
                 for (int u = max(q - nbr, lo); u <= min(q + nbr, hi - 1) && !covered; ++u)
-                    covered = is_top(u) && rank_by_idx[top_index((uint32_t)u)] < (uint32_t)j;
+                    covered = is_top(u) && cand_s[top_index((uint32_t)u)] > cp;
                 gain += covered ? 0u : 1u;
             }
-            cand_s[j] = ((unsigned long long)gain << 32) | (uint32_t)cand_s[j];
+            gain_s[j] = (uint16_t)gain;
+            my_gain += gain;
         }
+        int total_gain;
+        (void)block_excl_scan<kFinThreads>((int)my_gain, scratch, &total_gain);
+        // 3. the first candidate in score order whose running gain exceeds B:
+        //    MSB-first radix over its 64-bit composite, weighted by the gains
+        //    (six passes of 11/11/11/11/10/10 bits); the kept candidates are
+        //    those ranked before it
+        unsigned long long cut = 0ull;  // keep composites > cut (all of them if none exceeds B)
+        if (total_gain > budget) {
+            uint32_t need = (uint32_t)budget + 1u;
+            unsigned long long prefix = 0ull;
+            int fixed = 0;
+#pragma unroll 1
+            for (int pass = 0; pass < 6; ++pass) {
+                const int dw = pass < 4 ? 11 : 10;
+                const int nb = 1 << dw;
+                const int shift = 64 - fixed - dw;
+                for (int i = tid; i < nb; i += kFinThreads) hist[i] = 0u;
+                __syncthreads();
+                for (int j = tid; j < n_top; j += kFinThreads) {
+                    const unsigned long long cp = cand_s[j];
+                    if (fixed == 0 || (cp >> (64 - fixed)) == prefix)
+                        atomicAdd(&hist[(uint32_t)(cp >> shift) & (uint32_t)(nb - 1)], (uint32_t)gain_s[j]);
+                }
+                __syncthreads();
+                uint32_t rem;
+                const uint32_t bin = (uint32_t)block_find_bin_desc<kFinThreads>(hist, nb, need, &rem, scratch, false);
+                prefix = (prefix << dw) | bin;
+                fixed += dw;
+                need = rem;
+            }
+            cut = prefix;
+        }
+        // the kept positions: composites above the cut (or all)
+        for (int w = tid; w < W; w += kFinThreads) tie_s[w] = 0u;
         __syncthreads();
-        // 5. the longest prefix whose running size stays within the budget:
-        //    thread t owns ranks [8t, 8t + 8); sizes only grow along the ranks
-        constexpr int kPer = kCandCache / kFinThreads;
-        int sum = 0;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) {
-            const int j = tid * kPer + e;
-            if (j < n_top) sum += (int)(cand_s[j] >> 32);
-        }
-        int tot;
-        int run = block_excl_scan<kFinThreads>(sum, scratch, &tot);
-        int keep_n = 0;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) {
-            const int j = tid * kPer + e;
-            if (j < n_top) {
-                run += (int)(cand_s[j] >> 32);
-                if (run <= budget) keep_n = e + 1;
+        for (int j = tid; j < n_top; j += kFinThreads) {
+            const unsigned long long cp = cand_s[j];
+            if (total_gain <= budget || cp > cut) {
+                const uint32_t p = 0xFFFFFFFFu - (uint32_t)cp;
+                atomicOr(&tie_s[p >> 5], 1u << (p & 31));
             }
         }
-        // prefix sizes are monotone, so the kept ranks are [0, k*): count them
-        int kept;
-        (void)block_excl_scan<kFinThreads>(keep_n, scratch, &kept);
-        // 6. the Top bitmap becomes those k* positions; dilation and emission follow
-        for (int w = tid; w < W; w += kFinThreads) top_s[w] = 0u;
         __syncthreads();
-        for (int j = tid; j < kept; j += kFinThreads) {
-            const uint32_t p = 0xFFFFFFFFu - (uint32_t)cand_s[j];
-            atomicOr(&top_s[p >> 5], 1u << (p & 31));
-        }
+        for (int w = tid; w < W; w += kFinThreads) top_s[w] = tie_s[w];
         __syncthreads();
     }
 
