@@ -14,10 +14,11 @@
 // query heads.  Warp roles:
 //   * 4 load warps build the slice's row list (sparse: union over the group's
 //     heads of their selected bits, plus sink and window rows, each row
-//     tagged with a 4-bit head mask) and stream 128-row K and V tiles into a
-//     3-stage shared-memory ring with cp.async, in the 128-byte-swizzled
-//     layout the tensor cores read;
-//   * 1 MMA warp issues, per tile, S^T = K Q^T (M = 128 rows, N = 16 with the
+//     tagged with a 4-bit head mask; compacted just ahead of the tiles that
+//     read it) and stream 128-row K and V tiles into a 3-stage shared-memory
+//     ring with cp.async, in the 128-byte-swizzled layout the tensor cores
+//     read;
+//   * 2 MMA warps issue (one the S products, one the PV products), per tile, S^T = K Q^T (M = 128 rows, N = 16 with the
 //     4 heads in columns 0..3) and O^T = V^T P^T (M = 128 head dims, N = 16:
 //     columns 0..3 take the bf16 high parts of the softmax weights, 4..7 the
 //     bf16 remainders, so the weights keep ~16 significant bits), both bf16
