@@ -22,6 +22,14 @@
 //                   ties on it are taken in position order, and the Top bitmap
 //                   is dilated by +-nbr, clipped to C, and written out both as
 //                   the bitmap and as the sorted index list.
+//
+// Two variants share the kernels through a template mode (no counterpart on
+// the pages): one set per KV head from the max or the fp32 sum of the
+// group's head scores (the kernels then work on one row per group and
+// finalize copies the set to the group's 4 heads), and a budget that includes
+// the neighbours (finalize keeps the longest prefix of the top-B, in score
+// order, whose neighbourhoods cover at most B positions, found with a radix
+// select over the candidates' composites weighted by what each one adds).
 #include "common.cuh"
 #include "internal.h"
 
