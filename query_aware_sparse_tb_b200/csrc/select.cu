@@ -37,7 +37,8 @@ namespace tb {
 namespace {
 
 constexpr int kGroup = 4;
-constexpr int kChunk = 1024;          // positions per CTA in the streaming kernels
+constexpr int kChunk = 1024;          // positions per CTA of mark_collect
+constexpr int kHistChunk = 2048;      // positions per CTA of score_hist (one wave at 64K)
 constexpr int kThreads = 256;
 constexpr int kBins1 = 2048;          // key bits 31..21
 constexpr int kBins2 = 2048;          // key bits 20..10
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
-    constexpr int PER = kChunk / kThreads;  // positions per thread
+    constexpr int PER = kHistChunk / kThreads;  // positions per thread
     constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
     __shared__ __align__(16) float qs[kGroup][DP];
     __shared__ uint32_t hist[NH][kBins1];
@@ -182,14 +183,14 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
     const int lo = sink, hi = T - window;
-    const int p0 = ch * kChunk;
+    const int p0 = ch * kHistChunk;
 
     for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
     if (tid < kGroup * DP) (&qs[0][0])[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
     __syncthreads();
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
-    if (hi > lo && p0 < hi && p0 + kChunk > lo) {
+    if (hi > lo && p0 < hi && p0 + kHistChunk > lo) {
         // four rows per batch: all rows' loads (clamped into C) first, then
         // the arithmetic straight from the packed bf16 pairs, with the 4
         // heads' q' read from shared memory once per 8 dims
@@ -684,11 +685,12 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
     const int W = (d.ctx_cap + 31) / 32;
     const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
     dim3 grid(nch, d.n_kv_heads, d.batch);
+    dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
     if (d.d_proj == 32)
-        score_hist_kernel<32, SEL><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
+        score_hist_kernel<32, SEL><<<grid_h, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
                                                               d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
     else
-        score_hist_kernel<16, SEL><<<grid, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
+        score_hist_kernel<16, SEL><<<grid_h, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
                                                               d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
