@@ -87,6 +87,21 @@ def test_full_size_sampled(name):
         for hh in range(4 * g + 1, 4 * g + 4):
             assert np.array_equal(idx[b, hh, :cnt[b, hh]].cpu().numpy(), got)
 
+    # (c'') the budget-inclusive variant (at most B positions per head after neighbour
+    # fetch), same inputs; the GPU's fp32 scores may order near-ties differently,
+    # which can move the cut, so the sets must agree almost fully
+    if w.budget <= 8192:
+        tb.score_select_inclusive(dm, qpt, w.n_q_heads * w.d_proj, Kp_in, dec.ctx[0], w.sink, w.window, w.budget,
+                                  w.nbr, idx, cnt, bits, dec.ws_sel)
+        torch.cuda.synchronize()
+        assert tb.workspace_check(dec.ws_sel) == 0
+        for (b, hh), (s, _) in refs.items():
+            T = ctx0[b] + 1
+            ref = oracle.select_inclusive(s, T, w.sink, w.window, w.budget, w.nbr)
+            got = idx[b, hh, :cnt[b, hh]].cpu().numpy()
+            assert got.size <= w.budget and np.all(np.diff(got) > 0), (name, b, hh)
+            assert np.intersect1d(got, ref).size >= 0.98 * max(ref.size, 1), (name, b, hh, got.size, ref.size)
+
     # (d) sparse attention on the oracle's sets, dense attention
     W = dec.shape.words
     sets = [[refs.get((b, hh), (None, np.zeros(0, np.int32)))[1] for hh in range(w.n_q_heads)]
