@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 4
+#define TB_ABI_VERSION 5
 
 typedef uint16_t tb_bf16;
 
@@ -230,6 +230,16 @@ tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32
  * write, gathered into one call. */
 tb_status tb_kv_append(const tb_dims *dims, int32_t n_layers, const tb_bf16 *src, const uint64_t *caches,
                        const int32_t *ctx_len, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- failure detection self-test ----------------------------------------- */
+/* Every wait inside the kernels is bounded by a clock budget; when one runs
+ * out the kernel raises TB_FLAG_TIMEOUT in the workspace flag word, leaves its
+ * loops and returns, so the context stays usable.  This call exercises that
+ * path on purpose: one thread waits on an mbarrier that nothing ever arrives
+ * on, gives up after budget_cycles (1 .. 4e9) SM clock cycles and raises
+ * TB_FLAG_TIMEOUT in ws (>= 256 bytes).  tb_workspace_check then reports it.
+ * No counterpart on the pages. */
+tb_status tb_selftest_bounded_wait(void *ws, size_t ws_bytes, int64_t budget_cycles, void *stream);
 
 /* ---- 5. sparse GQA decode attention --------------------------------------- */
 /* The full KV cache stays resident and only the selected tokens are read

@@ -27,6 +27,7 @@ EXPORTS = [
     "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_score_select_inclusive",
     "tb_select_bits_from_idx",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
+    "tb_selftest_bounded_wait",
 ]
 
 
@@ -76,6 +77,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_sparse_decode_attn_noalloc": ([D, P, P, P, P, i32, i32, P, f32, P, P], ctypes.c_int),
         "tb_kv_append": ([D, i32, P, P, P, P, sz, P], ctypes.c_int),
+        "tb_selftest_bounded_wait": ([P, sz, i64, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -227,3 +229,8 @@ def kv_append(d: TbDims, n_layers: int, src, caches, ctx_len, ws, stream=None):
     addresses (K of layer l at 2l, V at 2l+1)."""
     _check(load().tb_kv_append(ctypes.byref(d), int(n_layers), _ptr(src), _ptr(caches), _ptr(ctx_len), _ptr(ws),
                                _bytes(ws), _stream(stream)))
+
+
+def selftest_bounded_wait(ws, budget_cycles: int, stream=None):
+    """tb_selftest_bounded_wait: a wait that runs out on purpose (raises TB_FLAG_TIMEOUT in ws)."""
+    _check(load().tb_selftest_bounded_wait(_ptr(ws), _bytes(ws), int(budget_cycles), _stream(stream)))

@@ -249,6 +249,14 @@ tb_status tb_score_select_inclusive(const tb_dims *dims, const float *qp, int64_
                              idx_cap, count, sel_bits, ws, ws_bytes, stream);
 }
 
+tb_status tb_selftest_bounded_wait(void *ws, size_t ws_bytes, int64_t budget_cycles, void *stream) {
+    tb_status s;
+    if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
+    if (budget_cycles < 1 || budget_cycles > 4000000000LL)
+        return fail(TB_ERR_INVALID_ARG, "%s: budget_cycles %lld outside [1, 4e9]", __func__, (long long)budget_cycles);
+    return cuda_status(launch_bounded_wait_selftest(ws, budget_cycles, (cudaStream_t)stream), __func__);
+}
+
 tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,
                                   const int32_t *count, uint32_t *sel_bits, void *stream) {
     tb_status s;

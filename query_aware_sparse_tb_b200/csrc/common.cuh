@@ -113,13 +113,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
         : "memory");
     return ok != 0;
 }
-// Wait for phase `parity` of the barrier, giving up after the clock budget.
-// Returns false (and flags TB_FLAG_TIMEOUT) on expiry.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *flags) {
+// Wait for phase `parity` of the barrier, giving up after `budget` clock
+// cycles (default: the library-wide budget).  Returns false (and flags
+// TB_FLAG_TIMEOUT) on expiry.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *flags,
+                                                  long long budget = kWaitBudgetCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitBudgetCycles) {
+        if (clock64() - t0 > budget) {
             raise_flag(flags, TB_FLAG_TIMEOUT);
             return false;
         }

@@ -43,6 +43,8 @@ cudaError_t launch_predict_queries(const uint16_t *h, const uint16_t *W1, const 
 cudaError_t launch_kv_append(const tb_dims &d, int32_t n_layers, const uint16_t *src, const uint64_t *caches,
                              const int32_t *ctx_len, void *ws, cudaStream_t st);
 
+cudaError_t launch_bounded_wait_selftest(void *ws, long long budget_cycles, cudaStream_t st);
+
 // Host error text for the calling thread (api.cu).
 void set_error(const char *fmt, ...);
 

@@ -43,7 +43,26 @@ kv_append_kernel(const uint4 *__restrict__ src, const uint64_t *__restrict__ cac
     dst[c] = src[(size_t)r * V16 + c];
 }
 
+// A wait that runs out on purpose: one thread waits on an mbarrier that no
+// one ever arrives on, with a short clock budget; the bounded wait gives up,
+// raises TB_FLAG_TIMEOUT and the kernel returns.  Checks, on the device, the
+// path every pipeline wait takes when a peer stops making progress.
+__global__ void bounded_wait_selftest_kernel(uint32_t *flags, long long budget) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_mbar_init();
+        (void)mbar_wait_bounded(b, 0, flags, budget);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_bounded_wait_selftest(void *ws, long long budget_cycles, cudaStream_t st) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t *>(ws), budget_cycles);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_kv_append(const tb_dims &d, int32_t n_layers, const uint16_t *src, const uint64_t *caches,
                              const int32_t *ctx_len, void *ws, cudaStream_t st) {

@@ -34,7 +34,7 @@ def test_exports_match_header(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.tb_abi_version() == 4
+    assert lib.tb_abi_version() == 5
     assert lib.tb_status_str(0) == b"TB_OK"
     assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
 
@@ -156,6 +156,12 @@ def test_kv_append_rejects_bad_arguments(lib):
     assert call(caches=FAKE + 4) == _lib.TB_ERR_INVALID_ARG
     assert call(src=FAKE + 8) == _lib.TB_ERR_INVALID_ARG
     assert call(ws_bytes=255) == _lib.TB_ERR_WORKSPACE
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    assert lib.tb_selftest_bounded_wait(FAKE, 256, 0, None) == _lib.TB_ERR_INVALID_ARG
+    assert lib.tb_selftest_bounded_wait(FAKE, 255, 1000, None) == _lib.TB_ERR_WORKSPACE
+    assert lib.tb_selftest_bounded_wait(0, 256, 1000, None) == _lib.TB_ERR_INVALID_ARG
 
 
 def test_predict_and_project_reject_bad_arguments(lib):
