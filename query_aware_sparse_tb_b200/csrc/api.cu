@@ -137,9 +137,11 @@ tb_status tb_workspace_check(void *ws, size_t ws_bytes, uint32_t *flags, void *s
     cudaStream_t st = (cudaStream_t)stream;
     uint32_t v = 0;
     tb_status s;
+    // read and clear the word in the caller's stream order, so that a kernel
+    // queued after this call can never have its flag cleared
+    if ((s = cuda_status(cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st), __func__)) != TB_OK) return s;
+    if ((s = cuda_status(cudaMemsetAsync(ws, 0, 4, st), __func__)) != TB_OK) return s;
     if ((s = cuda_status(cudaStreamSynchronize(st), __func__)) != TB_OK) return s;
-    if ((s = cuda_status(cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost), __func__)) != TB_OK) return s;
-    if ((s = cuda_status(cudaMemset(ws, 0, 4), __func__)) != TB_OK) return s;
     *flags = v;
     return v ? fail(TB_ERR_DEVICE_FLAG, "device flags 0x%x", v) : TB_OK;
 }

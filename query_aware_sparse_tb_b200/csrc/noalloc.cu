@@ -61,7 +61,10 @@ tb_status scratch_for_current_device(void **out) {
             tb::set_error("tb_sparse_decode_attn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
             return TB_ERR_CUDA;
         }
+        // a memset of device memory may return before it is done, and the
+        // caller's stream need not be ordered after the legacy stream
         e = cudaMemset(p, 0, kNoAllocScratchBytes);
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
         if (e != cudaSuccess) {
             tb::set_error("tb_sparse_decode_attn_noalloc: clearing the scratch: %s", cudaGetErrorString(e));
             return TB_ERR_CUDA;
