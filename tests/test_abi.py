@@ -33,6 +33,27 @@ def test_exports_match_header(lib):
     assert sorted(_lib.EXPORTS) == declared
 
 
+def _header_constants():
+    src = open(os.path.join(ROOT, "include", "tb.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    consts = {m.group(1): int(m.group(2), 0)
+              for m in re.finditer(r"^#define (TB_[A-Z_]+)\s+(0x[0-9a-fA-F]+|\d+)u?\s*$", src, flags=re.M)}
+    consts.update({m.group(1): int(m.group(2)) for m in re.finditer(r"\b(TB_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", src)})
+    return consts
+
+
+def test_binding_constants_match_header(lib):
+    h = _header_constants()
+    for name in ("TB_OK", "TB_ERR_INVALID_ARG", "TB_ERR_UNSUPPORTED", "TB_ERR_CUDA", "TB_ERR_WORKSPACE",
+                 "TB_ERR_DEVICE_FLAG", "TB_FLAG_CTX_RANGE", "TB_FLAG_TIMEOUT", "TB_FLAG_IDX_OVERFLOW",
+                 "TB_FLAG_BAD_CACHE"):
+        assert getattr(_lib, name) == h[name], name
+        if name.startswith(("TB_OK", "TB_ERR")):
+            assert lib.tb_status_str(h[name]) == name.encode()
+    assert _lib.TB_GROUP_REDUCE == {"max": h["TB_GROUP_MAX"], "sum": h["TB_GROUP_SUM"]}
+    assert lib.tb_abi_version() == h["TB_ABI_VERSION"]
+
+
 def test_version_and_strings(lib):
     assert lib.tb_abi_version() == 5
     assert lib.tb_status_str(0) == b"TB_OK"
