@@ -24,12 +24,18 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 
-def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
-    """Compile the C oracle with gcc (plain -O2, no fast-math)."""
+_SAN_LIB_PATH = os.path.join(_HERE, "liboracle_san.so")
+_SAN_FLAGS = ["-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all", "-fno-omit-frame-pointer"]
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH, sanitize: bool = False) -> str:
+    """Compile the C oracle with gcc (plain -O2, no fast-math).  sanitize=True
+    adds AddressSanitizer and UBSan, for checking the oracle's own memory
+    accesses (the process then needs the sanitizer runtimes preloaded)."""
     if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
         subprocess.check_call(
             ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
-             "-ffp-contract=off", "-o", out, src, "-lm"])
+             "-ffp-contract=off"] + (_SAN_FLAGS if sanitize else []) + ["-o", out, src, "-lm"])
     return out
 
 
@@ -66,7 +72,10 @@ def load(path: str | None = None):
     if path is not None:
         return _bind(path)
     if _lib is None:
-        _lib = _bind(build())
+        if os.environ.get("TB_ORACLE_SANITIZE") == "1":
+            _lib = _bind(build(out=_SAN_LIB_PATH, sanitize=True))
+        else:
+            _lib = _bind(build())
     return _lib
 
 
