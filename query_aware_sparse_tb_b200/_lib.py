@@ -15,6 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtb.so")
 
+TB_ABI_VERSION = 5
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
 TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW, TB_FLAG_BAD_CACHE = 0x1, 0x2, 0x4, 0x8
 TB_GROUP_REDUCE = {"max": 0, "sum": 1}
@@ -83,6 +84,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = res
+    # the signatures above are those of this ABI version; a library built from
+    # other sources would be called with the wrong arguments
+    if lib.tb_abi_version() != TB_ABI_VERSION:
+        raise TbError(-1, f"{path} has ABI version {lib.tb_abi_version()}, this binding needs {TB_ABI_VERSION}: "
+                          "rebuild it with `python -m query_aware_sparse_tb_b200.build`")
     if path == LIB_PATH:
         _lib = lib
     return lib

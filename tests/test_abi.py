@@ -51,7 +51,7 @@ def test_binding_constants_match_header(lib):
         if name.startswith(("TB_OK", "TB_ERR")):
             assert lib.tb_status_str(h[name]) == name.encode()
     assert _lib.TB_GROUP_REDUCE == {"max": h["TB_GROUP_MAX"], "sum": h["TB_GROUP_SUM"]}
-    assert lib.tb_abi_version() == h["TB_ABI_VERSION"]
+    assert lib.tb_abi_version() == h["TB_ABI_VERSION"] == _lib.TB_ABI_VERSION
 
 
 def test_version_and_strings(lib):
@@ -208,3 +208,11 @@ def test_binding_refuses_host_tensors(lib):
     t = torch.zeros(16, dtype=torch.bfloat16)
     with pytest.raises(_lib.TbError):
         _lib.decode_attn(d, t, t, t, torch.zeros(1, dtype=torch.int32), 0.1, torch.zeros(4), t)
+
+
+def test_binding_refuses_another_abi_version(lib, monkeypatch):
+    monkeypatch.setattr(_lib, "TB_ABI_VERSION", _lib.TB_ABI_VERSION - 1)
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(_lib.TbError, match="ABI version"):
+        _lib.load()
+    assert _lib._lib is None            # nothing cached from the refused load
