@@ -22,7 +22,9 @@
  *    workspaces.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  *    asynchronous: it validates its arguments on the host, launches, and
- *    returns; it never synchronises the device.
+ *    returns; it never synchronises the device.  The exceptions say so:
+ *    tb_workspace_check synchronises its stream, and the first
+ *    tb_sparse_decode_attn_noalloc call on a device waits for its set-up.
  *  - bf16 values are passed as raw 16-bit patterns (`tb_bf16`).
  *  - Caches use the layout [batch][n_kv_heads][ctx_cap][dim], row-contiguous
  *    per (sequence, KV head).  Query-head h belongs to KV head h / (Hq/Hkv).
@@ -153,7 +155,9 @@ tb_status tb_predict_queries(const tb_bf16 *h, const tb_bf16 *W1, const tb_bf16 
  *              (point at one slot of a [batch][G][Hq][d'] array; stride G*Hq*d')
  *   Kp         [batch][Hkv][ctx_cap][d'] bf16; rows of C must be projected
  *   ctx_len    [batch] int32 (device)
- *   idx        [batch][Hq][idx_cap] int32 out: I sorted ascending
+ *   idx        [batch][Hq][idx_cap] int32 out: I sorted ascending in
+ *              idx[b][h][0 .. count[b][h]); the slots after those are not
+ *              written
  *   count      [batch][Hq] int32 out: |I|
  *   sel_bits   [batch][Hq][ceil(ctx_cap/32)] uint32 out: bit t%32 of word t/32
  *              is 1 iff t in I (all other bits 0); this is what
@@ -252,7 +256,8 @@ tb_status tb_selftest_bounded_wait(void *ws, size_t ws_bytes, int64_t budget_cyc
  *   out[b][h] = sum_{t in A} softmax_t( scale * Q[b][h]·K[b][g][t] ) * V[b][g][t]
  *
  * fp32 logits, fp32 online softmax, fp32 accumulation; every (b, KV head, t)
- * row is read once for the whole GQA group of 4 query heads.
+ * row is read once for the whole GQA group of 4 query heads, and a row in no
+ * head's A is never read (its contents, NaN included, cannot reach out).
  *   Q    [batch][Hq][d] bf16;  K, V [batch][Hkv][ctx_cap][d] bf16
  *   out  [batch][Hq][d] fp32
  * Split over the context across CTAs; the last CTA of each (b, KV head) merges
@@ -264,7 +269,8 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
 
 /* ---- dense decode attention (comparator) ---------------------------------- */
 /* The same computation over A = [0, T): the dense attention baseline the
- * summaries' on-GPU speedup is measured against ("Contributions 4"). */
+ * summaries' on-GPU speedup is measured against ("Contributions 4").  Rows at
+ * or past T are never read. */
 tb_status tb_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
                          const tb_bf16 *V, const int32_t *ctx_len, float scale, float *out,
                          void *ws, size_t ws_bytes, void *stream);
