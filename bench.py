@@ -334,18 +334,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def profiled_traffic(kernel: str):
+def profiled_traffic(kernel: str, root: str = ROOT):
     """DRAM bytes per launch from the committed ncu capture of `kernel`, or
-    None when that kernel's source has changed since the capture."""
+    None when any of that kernel's source files has changed since the capture
+    (or the record is missing)."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        with open(os.path.join(root, "profiles", "traffic.json")) as f:
             rec = json.load(f)[kernel]
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
-                return None
+        if not rec["sources"]:
+            return None
+        for path, sha in rec["sources"].items():
+            with open(os.path.join(root, path), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != sha:
+                    return None
         return rec["dram_read_bytes"] + rec["dram_write_bytes"]
-    except Exception:
+    except (OSError, KeyError, TypeError, ValueError):
         return None
 
 
