@@ -149,15 +149,29 @@ def pin_predict_queries(lib):
     assert np.all(z == 0.0)
 
 
+def _bf16_rne(x: float) -> float:
+    """Round a double to the nearest bf16 value, ties to even (normal range)."""
+    if x == 0.0:
+        return 0.0
+    quantum = 2.0 ** (math.floor(math.log2(abs(x))) - 7)
+    return round(x / quantum) * quantum          # x / quantum is exact; round() ties to even
+
+
 def pin_predict_queries_silu_closed_form(lib):
-    # hidden 1, W1 = identity row, W2 = identity: q' = bf16(SiLU(h))
-    hvals = torch.tensor([[-2.0], [0.5], [3.0]])
+    # hidden 1, W1 = identity row, W2 = identity: q' = bf16_rne(SiLU(h)) exactly
+    # (reading R6: the activation is rounded to bf16 before the second product).
+    # Each SiLU value here lies at least 0.1 bf16 spacings from a rounding
+    # midpoint and is not itself a bf16 value, so the rounding is visible.
+    xs = [-2.0, 0.5, 3.0, -0.75, 5.5]
+    hvals = torch.tensor([[x] for x in xs])
     W1 = torch.ones(1, 1)
     W2 = torch.ones(1, 1)
     got = oracle.predict_queries(_bf16_bits(hvals), _bf16_bits(W1), _bf16_bits(W2), lib=lib)
-    for k, x in enumerate([-2.0, 0.5, 3.0]):
+    for k, x in enumerate(xs):
         silu = x / (1.0 + math.exp(-x))
-        assert abs(float(got[k, 0]) - silu) <= abs(silu) * 2.0 ** -8, (x, got[k, 0], silu)
+        want = _bf16_rne(silu)
+        assert want != silu
+        assert float(got[k, 0]) == want, (x, float(got[k, 0]), want)
 
 
 # ---------------------------------------------------------------------------
@@ -341,6 +355,9 @@ def pin_attention_golden(lib):
     assert np.allclose(o, [(4 * e2) / (1 + e2), (-2 * e2 + 2) / (1 + e2)], rtol=1e-7, atol=0)
     o = run(cases["row_subset"])
     assert np.allclose(o, [2.0, 3.0], rtol=1e-7, atol=0)
+    em16 = math.exp(-16.0)
+    o = run(cases["large_logits"])
+    assert np.allclose(o, [1 / (1 + em16), em16 / (1 + em16)], rtol=1e-7, atol=0)
 
 
 def pin_attention_constant_v(lib):

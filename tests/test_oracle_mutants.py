@@ -48,15 +48,34 @@ MUTANTS = [
     ("inclusive_allows_overshoot", "if (size + fresh > B) break;", "if (size + fresh > B + 1) break;"),
     ("inclusive_skips_instead_of_stopping", "if (size + fresh > B) break;", "if (size + fresh > B) continue;"),
     ("inclusive_counts_covered", "fresh += !in_set[u - lo];", "fresh += 1;"),
+    ("projection_drops_last_input", "for (int i = 0; i < d; ++i)\n                acc += orc_bf16_to_double(K[",
+     "for (int i = 0; i < d - 1; ++i)\n                acc += orc_bf16_to_double(K["),
+    ("w2_transposed", "W2[(int64_t)o * inter + i]", "W2[(int64_t)i * n_out + o]"),
+    ("predict_ignores_batch", "h[(int64_t)b * hidden + k]", "h[k]"),
+    ("activation_not_rounded", [
+        ("uint16_t *act = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)inter);",
+         "double *act = (double *)malloc(sizeof(double) * (size_t)inter);"),
+        ("act[i] = orc_double_to_bf16(silu);", "act[i] = silu;"),
+        ("q += orc_bf16_to_double(act[i]) *", "q += act[i] *"),
+    ], None),
+    ("neighbour_left_dropped", "for (int64_t u = t - r; u <= t + r; ++u)",
+     "for (int64_t u = t - r + 1; u <= t + r; ++u)"),
+    ("window_long", "int64_t win_begin = T - N > S ? T - N : S;",
+     "int64_t win_begin = T - N - 1 > S ? T - N - 1 : S;"),
+    ("softmax_no_max_shift", "z[k] = exp(z[k] - zmax);", "z[k] = exp(z[k]);"),
 ]
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(name, old, new, tmp_path):
+    # one (old, new) edit, or a list of edits that make one mistake together
+    edits = old if isinstance(old, list) else [(old, new)]
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not unique/found"
+    for o, n in edits:
+        assert src.count(o) == 1, f"mutation site for {name} not unique/found: {o!r}"
+        src = src.replace(o, n)
     mut_src = tmp_path / "tb_oracle_mut.c"
-    mut_src.write_text(src.replace(old, new))
+    mut_src.write_text(src)
     so = oracle.build(force=True, src=str(mut_src), out=str(tmp_path / "libmut.so"))
     lib = oracle.load(so)
     caught = []
