@@ -5,6 +5,7 @@ Each mutant is a textual edit of tb_oracle.c compiled into a temporary shared
 library: a transposed operand, a dropped term, a flipped sign, an off-by-one
 range, a reversed tie-break, a skipped rounding step.
 """
+import importlib.util
 import os
 import shutil
 
@@ -12,6 +13,7 @@ import pytest
 
 import oracle
 import oracle_pins
+import test_oracle_schedule
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "tb_oracle.c")
 
@@ -87,3 +89,46 @@ def test_pins_catch_mutant(name, old, new, tmp_path):
             break
     assert caught, f"no pin caught mutant {name}"
     shutil.rmtree(tmp_path, ignore_errors=True)
+
+
+# The decode-loop schedule (oracle/schedule.py): mutated copies are loaded as
+# a module of the oracle package and must fail one of the schedule tests.
+SCHEDULE_SRC = os.path.join(os.path.dirname(oracle.__file__), "schedule.py")
+
+SCHEDULE_MUTANTS = [
+    ("prediction_every_step", "    return step % interval == 0", "    return True"),
+    ("prefix_not_whole_batches", "    proj = (ctx0 // window) * window\n", "    proj = ctx0\n"),
+    ("slot_ignored", "qp = qp_cache[(k, p)][:, slot_of(layer, w.producer_stride)]", "qp = qp_cache[(k, p)][:, 0]"),
+    ("selection_length_off_by_one", "T = ctx0[b] + i + 1\n                    hi = T - w.window",
+     "T = ctx0[b] + i\n                    hi = T - w.window"),
+    ("window_frozen_at_prediction", "T = ctx0[b] + i + 1\n                    for h in heads:",
+     "T = ctx0[b] + last_prediction_step(i, w.interval) + 1\n                    for h in heads:"),
+]
+
+SCHEDULE_CHECKS = [getattr(test_oracle_schedule, n) for n in dir(test_oracle_schedule)
+                   if n.startswith("test_") and callable(getattr(test_oracle_schedule, n))]
+
+
+def _load_schedule(text, tmp_path):
+    path = tmp_path / "schedule_mut.py"
+    path.write_text(text)
+    spec = importlib.util.spec_from_file_location("oracle.schedule_mut", str(path))
+    mod = importlib.util.module_from_spec(spec)
+    mod.__package__ = "oracle"
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", SCHEDULE_MUTANTS, ids=[m[0] for m in SCHEDULE_MUTANTS])
+def test_schedule_checks_catch_mutant(name, old, new, tmp_path, monkeypatch):
+    src = open(SCHEDULE_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique/found"
+    monkeypatch.setattr(test_oracle_schedule, "schedule", _load_schedule(src.replace(old, new), tmp_path))
+    caught = []
+    for check in SCHEDULE_CHECKS:
+        try:
+            check()
+        except (AssertionError, ValueError, IndexError):
+            caught.append(check.__name__)
+            break
+    assert caught, f"no schedule check caught mutant {name}"

@@ -139,3 +139,46 @@ def test_run_budget_covering_context_equals_dense():
             g = h // w.group
             dense = oracle.attention(Q[0, h], K[0, g], V[0, g], np.arange(T, dtype=np.int32), scale)
             assert np.allclose(res[(i, 1)]["out"][0, h], dense, rtol=1e-6, atol=1e-7)
+
+
+def test_run_window_follows_current_length_between_predictions():
+    # Reading R5: sink and window follow the current length T at every step,
+    # the importance set is the one chosen at the last prediction, and tokens
+    # that leave the window mid-interval are not added back until the next
+    # prediction.  With a budget covering every candidate the set is exactly
+    # [S, T_p - N), so the attended rows are [0, T_p - N) U [T - N, T): the
+    # rows [T_p - N, T - N) are left out until the next prediction.
+    w = _small_llama(budget=10_000, interval=4, steps=6)
+    data = HostData(w)
+    res = schedule.run(w, data, layers=[0], steps=w.steps)
+    K, V = data.kv(0)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    S, N = w.sink, w.window
+    for i in range(w.steps):
+        p = schedule.last_prediction_step(i, w.interval)
+        T, Tp = w.ctx0 + i + 1, w.ctx0 + p + 1
+        A = np.concatenate([np.arange(0, Tp - N), np.arange(T - N, T)]).astype(np.int32)
+        assert (i == p) == (A.size == T), "rows leave the attended set only between predictions"
+        Q = data.q(i, 0)
+        for h in range(w.n_q_heads):
+            assert np.array_equal(res[(i, 0)]["idx"][0][h], np.arange(S, Tp - N))
+            g = h // w.group
+            want = oracle.attention(Q[0, h], K[0, g], V[0, g], A, scale)
+            assert np.allclose(res[(i, 0)]["out"][0, h], want, rtol=1e-6, atol=1e-7), (i, h)
+
+
+def test_run_layer_reads_its_producer_slot():
+    # slot j of the producer's G-slot output serves layer p + j (reading R2)
+    w = _small_llama(steps=1)
+    data = HostData(w)
+    res = schedule.run(w, data, layers=[0, 1], steps=1, want_attention=False)
+    W1, W2 = data.mlp(0)
+    qp = oracle.predict_queries(data.h(0, 0), W1, W2).reshape(w.batch, w.slots, w.n_q_heads, w.d_proj)
+    K, _ = data.kv(1)
+    T = w.ctx0 + 1
+    hi = T - w.window
+    Kp = oracle.project_keys(K[0, 0, :hi], data.wk(1)[0])
+    sets = [oracle.select(oracle.scores(qp[0, j, 0], Kp, w.sink, hi), T, w.sink, w.window, w.budget, w.nbr)
+            for j in range(w.slots)]
+    assert not np.array_equal(sets[0], sets[1]), "the two slots must select differently for this check"
+    assert np.array_equal(res[(0, 1)]["idx"][0][0], sets[1])
