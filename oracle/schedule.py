@@ -21,7 +21,8 @@ import math
 
 import numpy as np
 
-from . import attention, attention_set, group_scores, predict_queries, project_keys, scores, select
+from . import (attention, attention_set, group_scores, predict_queries, project_keys, scores, select,
+               select_inclusive)
 
 
 def is_prediction_step(step: int, interval: int) -> bool:
@@ -65,13 +66,15 @@ def run(w, data, layers, steps, want_attention=True, heads=None, selection="head
       data.h(pred_index, producer) -> [batch][hidden]
       data.qp_direct(pred_index, layer) -> [batch][Hq][d'] float32
       data.q(step, layer) -> [batch][Hq][d]
-    `selection` is "head" (one importance set per query head, reading R1) or
+    `selection` is "head" (one importance set per query head, reading R1),
     "group_max" / "group_sum" (one set per KV head from the largest or the
     fp32 sum of the group's head scores, the group-shared variant; every head
-    of the group then attends to that set).
+    of the group then attends to that set) or "inclusive" (per query head,
+    at most `budget` positions after neighbour fetch, the budget-inclusive
+    variant).
     Returns {(step, layer): {"idx": [[I_bh]], "out": [batch][Hq][d] or None}}.
     """
-    assert selection in ("head", "group_max", "group_sum")
+    assert selection in ("head", "group_max", "group_sum", "inclusive")
     B, Hq, grp = w.batch, w.n_q_heads, w.group
     heads = list(range(Hq)) if heads is None else list(heads)
     ctx0 = w.ctx0_per_seq()
@@ -106,7 +109,7 @@ def run(w, data, layers, steps, want_attention=True, heads=None, selection="head
                             per_head.append(None)
                             continue
                         g = h // grp
-                        if selection != "head" and g in group_sets:
+                        if selection not in ("head", "inclusive") and g in group_sets:
                             per_head.append(group_sets[g])
                             continue
                         if hi > w.sink:
@@ -114,15 +117,16 @@ def run(w, data, layers, steps, want_attention=True, heads=None, selection="head
                             have = kp_cache.get(key)
                             if have is None or have.shape[0] < hi:
                                 kp_cache[key] = project_keys(K[b, g, :hi], Wk[g])
-                            if selection == "head":
+                            if selection in ("head", "inclusive"):
                                 s = scores(qp[b, h], kp_cache[key], w.sink, hi)
                             else:
                                 s = group_scores(qp[b, g * grp:(g + 1) * grp], kp_cache[key], w.sink, hi,
                                                  selection[len("group_"):])
                         else:
                             s = np.zeros(0, np.float32)
-                        I = select(s, T, w.sink, w.window, w.budget, w.nbr)
-                        if selection != "head":
+                        pick = select_inclusive if selection == "inclusive" else select
+                        I = pick(s, T, w.sink, w.window, w.budget, w.nbr)
+                        if selection not in ("head", "inclusive"):
                             group_sets[g] = I
                         per_head.append(I)
                     sets.append(per_head)

@@ -182,3 +182,27 @@ def test_run_layer_reads_its_producer_slot():
             for j in range(w.slots)]
     assert not np.array_equal(sets[0], sets[1]), "the two slots must select differently for this check"
     assert np.array_equal(res[(0, 1)]["idx"][0][0], sets[1])
+
+
+def test_run_inclusive_selection_holds_at_most_budget():
+    # the budget-inclusive variant: per head, the importance set after
+    # neighbour fetch has at most B positions, is the one orc_select_inclusive
+    # gives on that head's scores, and is reused over the interval like any other
+    w = _small_llama(interval=4, steps=5)
+    data = HostData(w)
+    res = schedule.run(w, data, layers=[1], steps=w.steps, selection="inclusive")
+    K, _ = data.kv(1)
+    W1, W2 = data.mlp(0)
+    qp = oracle.predict_queries(data.h(0, 0), W1, W2).reshape(w.batch, w.slots, w.n_q_heads, w.d_proj)[:, 1]
+    T = w.ctx0 + 1
+    hi = T - w.window
+    for h in range(w.n_q_heads):
+        Kp = oracle.project_keys(K[0, h // w.group, :hi], data.wk(1)[h // w.group])
+        want = oracle.select_inclusive(oracle.scores(qp[0, h], Kp, w.sink, hi), T, w.sink, w.window, w.budget,
+                                       w.nbr)
+        got = res[(0, 1)]["idx"][0][h]
+        assert np.array_equal(got, want), h
+        assert 0 < got.size <= w.budget
+        for i in range(1, 4):
+            assert np.array_equal(res[(i, 1)]["idx"][0][h], got)
+    assert np.all(np.isfinite(res[(0, 1)]["out"]))
