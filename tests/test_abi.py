@@ -216,3 +216,40 @@ def test_binding_refuses_another_abi_version(lib, monkeypatch):
     with pytest.raises(_lib.TbError, match="ABI version"):
         _lib.load()
     assert _lib._lib is None            # nothing cached from the refused load
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "tb.h"
+int main(void) {
+    tb_dims d = {1, 32, 8, 96, 32, 4096};
+    if (tb_abi_version() != TB_ABI_VERSION) return 1;
+    if (strcmp(tb_status_str(TB_ERR_WORKSPACE), "TB_ERR_WORKSPACE") != 0) return 2;
+    if (tb_attn_workspace_bytes(&d) != 0) return 3;           /* head_dim 96 is not built */
+    d.head_dim = 128;
+    if (tb_attn_workspace_bytes(&d) == 0) return 4;
+    if (tb_decode_attn(&d, NULL, NULL, NULL, NULL, 0.1f, NULL, NULL, 0, NULL) != TB_ERR_INVALID_ARG) return 5;
+    printf("%s\n", tb_last_error());
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
+    # the boundary is a C ABI: tb.h compiles as strict C99 and a C program
+    # links against libtb.so and gets host-side validation without a GPU
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "main.c"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "main"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-L", libdir, "-ltb", f"-Wl,-rpath,{libdir}",
+                    "-o", str(exe)], check=True, capture_output=True, text=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0, (res.returncode, res.stdout, res.stderr)
+    assert "16-byte aligned" in res.stdout
