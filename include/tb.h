@@ -70,9 +70,9 @@ typedef enum {
 
 /* Shapes shared by the cache-facing calls. */
 typedef struct {
-    int32_t batch;       /* sequences */
+    int32_t batch;       /* sequences, <= 65535 */
     int32_t n_q_heads;   /* Hq  */
-    int32_t n_kv_heads;  /* Hkv; Hq / Hkv must be 4 */
+    int32_t n_kv_heads;  /* Hkv <= 65535; Hq / Hkv must be 4 */
     int32_t head_dim;    /* d:  64 or 128 */
     int32_t d_proj;      /* d': 16 or 32 */
     int32_t ctx_cap;     /* rows per (sequence, KV head) in K, V and K' */

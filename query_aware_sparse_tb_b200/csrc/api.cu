@@ -61,6 +61,10 @@ tb_status check_dims(const tb_dims *d, bool need_dproj, const char *fn) {
     if (d->n_q_heads % d->n_kv_heads != 0)
         return fail(TB_ERR_INVALID_ARG, "%s: n_q_heads (%d) not a multiple of n_kv_heads (%d)", fn,
                     d->n_q_heads, d->n_kv_heads);
+    // batch and KV heads index grid dimensions whose limit is 65535
+    if (d->batch > 65535 || d->n_kv_heads > 65535)
+        return fail(TB_ERR_UNSUPPORTED, "%s: batch (%d) and n_kv_heads (%d) must be <= 65535", fn, d->batch,
+                    d->n_kv_heads);
     if (d->n_q_heads / d->n_kv_heads != 4)
         return fail(TB_ERR_UNSUPPORTED, "%s: only GQA groups of 4 query heads are built (got %d)", fn,
                     d->n_q_heads / d->n_kv_heads);

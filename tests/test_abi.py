@@ -103,6 +103,9 @@ def test_attention_rejects_bad_arguments(lib):
     assert call(d, K=MIS) == _lib.TB_ERR_INVALID_ARG
     assert call(d, ws_bytes=ws_bytes - 1) == _lib.TB_ERR_WORKSPACE
     assert call(_d(batch=0)) == _lib.TB_ERR_INVALID_ARG
+    assert call(_d(batch=65536)) == _lib.TB_ERR_UNSUPPORTED           # a grid dimension limit
+    assert b"65535" in lib.tb_last_error()
+    assert lib.tb_attn_workspace_bytes(ctypes.byref(_d(batch=65536))) == 0
     st = lib.tb_sparse_decode_attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16, 0, FAKE, 0.088, FAKE, FAKE,
                                    ws_bytes, None)
     assert st == _lib.TB_ERR_INVALID_ARG and b"window" in lib.tb_last_error()
