@@ -239,9 +239,6 @@ def _rt():
         _cudart = ctypes.CDLL("libcudart.so.12")
         _cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
         _cudart.cudaEventRecordWithFlags.restype = ctypes.c_int
-        _cudart.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t,
-                                              ctypes.c_size_t, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
-        _cudart.cudaMemcpy2DAsync.restype = ctypes.c_int
     return _cudart
 
 
