@@ -100,17 +100,6 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
-def f64_to_bf16(x, lib=None) -> np.ndarray:
-    """Round each double to bf16 (nearest, ties to even) through the C oracle."""
-    lib = lib or load()
-    x = np.asarray(x, dtype=np.float64)
-    out = np.empty(x.shape, dtype=np.uint16)
-    flat_in, flat_out = x.reshape(-1), out.reshape(-1)
-    for k in range(flat_in.size):
-        flat_out[k] = lib.orc_double_to_bf16(float(flat_in[k]))
-    return out
-
-
 # --------------------------------------------------------------------------
 # the five steps, one head (or one KV head) at a time
 # --------------------------------------------------------------------------
