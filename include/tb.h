@@ -17,9 +17,12 @@
  * ---------------------------------------
  *  - Pointers are DEVICE pointers unless a comment says "host".  bf16 arrays
  *    (K, V, K', Q, W_k, W1, W2, h) and workspaces must be 16-byte aligned;
- *    int32, uint32 and float arrays 4-byte aligned.  Nothing here allocates,
- *    frees or keeps device memory; the caller owns every buffer, including
- *    workspaces.
+ *    int32, uint32 and float arrays 4-byte aligned.  No call allocates or
+ *    frees device memory; the caller owns every buffer, including
+ *    workspaces.  One exception holds memory: the fixed scratch of
+ *    tb_sparse_decode_attn_noalloc (TB_NOALLOC_SCRATCH_BYTES = 4 MiB), a
+ *    static device array that every GPU which loads libtb.so keeps until the
+ *    process exits, whether or not that entry point is ever called.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  *    asynchronous: it validates its arguments on the host, launches, and
  *    returns; it never synchronises the device.  The exceptions say so:
@@ -49,7 +52,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 5
+#define TB_ABI_VERSION 6
 
 typedef uint16_t tb_bf16;
 
@@ -207,6 +210,23 @@ tb_status tb_score_select_inclusive(const tb_dims *dims, const float *qp, int64_
                                     const tb_bf16 *Kp, const int32_t *ctx_len, int32_t sink, int32_t window,
                                     int32_t budget, int32_t nbr, int32_t *idx, int32_t idx_cap, int32_t *count,
                                     uint32_t *sel_bits, void *ws, size_t ws_bytes, void *stream);
+
+/* The fp32 importance scores behind the last tb_score_select,
+ * tb_score_select_group or tb_score_select_inclusive call made on `ws` with
+ * the same dims, ctx_len, sink and window (the scoring step of "Core
+ * architecture: scoring"), for inspection and for checking a selection
+ * against the scores it was taken from:
+ *
+ *   scores[b][h][t] = s[t] of sequence b, query head h   for t in C = [sink, T - window)
+ *                   = NaN                                 for every other t < ctx_cap
+ *
+ *   scores  [batch][Hq][ctx_cap] float (device)
+ * After tb_score_select_group only the first head row of each KV head (h %
+ * 4 == 0) holds the group scores; the other three rows are unspecified.  The
+ * scores are the exact fp32 values the selection ranked.  Another selection
+ * call on `ws` overwrites them. */
+tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_bytes, const int32_t *ctx_len,
+                                 int32_t sink, int32_t window, float *scores, void *stream);
 
 /* Build the sel_bits bitmap from index lists that came from elsewhere (e.g. a
  * host-side selection): bit t of row (b,h) is set iff t is among

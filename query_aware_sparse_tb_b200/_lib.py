@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtb.so")
 
-TB_ABI_VERSION = 5
+TB_ABI_VERSION = 6
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
 TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW, TB_FLAG_BAD_CACHE = 0x1, 0x2, 0x4, 0x8
 TB_GROUP_REDUCE = {"max": 0, "sum": 1}
@@ -26,7 +26,7 @@ EXPORTS = [
     "tb_predict_queries_workspace_bytes", "tb_project_keys_workspace_bytes",
     "tb_workspace_init", "tb_workspace_check",
     "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_score_select_inclusive",
-    "tb_select_bits_from_idx",
+    "tb_score_select_scores", "tb_select_bits_from_idx",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
     "tb_selftest_bounded_wait",
 ]
@@ -73,6 +73,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_score_select_group": ([D, P, i64, P, P, i32, i32, i32, i32, i32, P, i32, P, P, P, sz, P],
                                   ctypes.c_int),
         "tb_score_select_inclusive": ([D, P, i64, P, P, i32, i32, i32, i32, P, i32, P, P, P, sz, P], ctypes.c_int),
+        "tb_score_select_scores": ([D, P, sz, P, i32, i32, P, P], ctypes.c_int),
         "tb_select_bits_from_idx": ([D, P, i32, P, P, P], ctypes.c_int),
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
@@ -202,6 +203,13 @@ def score_select_inclusive(d: TbDims, qp, qp_batch_stride: int, Kp, ctx_len, sin
     _check(load().tb_score_select_inclusive(ctypes.byref(d), _ptr(qp), int(qp_batch_stride), _ptr(Kp),
                                             _ptr(ctx_len), sink, window, budget, nbr, _ptr(idx), idx_cap,
                                             _ptr(count), _ptr(sel_bits), _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def score_select_scores(d: TbDims, ws, ctx_len, sink: int, window: int, scores, stream=None):
+    """tb_score_select_scores: the fp32 scores the last selection on `ws` ranked
+    ([batch][Hq][ctx_cap] float32; NaN outside the candidates)."""
+    _check(load().tb_score_select_scores(ctypes.byref(d), _ptr(ws), _bytes(ws), _ptr(ctx_len), sink, window,
+                                         _ptr(scores), _stream(stream)))
 
 
 def select_bits_from_idx(d: TbDims, idx, count, sel_bits, stream=None):

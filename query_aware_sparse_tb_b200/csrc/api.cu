@@ -6,12 +6,16 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace tb {
 
 static thread_local char g_err[512] = "";
+static std::mutex g_state_mu;  // serialises one-time per-device kernel set-up
 
 void set_error(const char *fmt, ...) {
     va_list ap;
@@ -88,6 +92,54 @@ tb_status cuda_status(cudaError_t e, const char *fn) {
 }
 
 }  // namespace
+
+tb_status check_attn_args(const char *fn, const tb_dims *dims, const uint16_t *Q, const uint16_t *K,
+                          const uint16_t *V, const int32_t *ctx_len, float scale, float *out, bool sparse,
+                          const uint32_t *sel_bits, int32_t sink, int32_t window) {
+    tb_status s;
+    if ((s = check_dims(dims, false, fn)) != TB_OK) return s;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V))
+        return fail(TB_ERR_INVALID_ARG, "%s: Q, K and V must be non-null and 16-byte aligned", fn);
+    if (!aligned4(ctx_len) || !aligned4(out))
+        return fail(TB_ERR_INVALID_ARG, "%s: ctx_len and out must be non-null and 4-byte aligned", fn);
+    if (dims->ctx_cap > kMaxCtxAttn)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", fn, dims->ctx_cap, kMaxCtxAttn);
+    if (!isfinite(scale)) return fail(TB_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+    if (sparse) {
+        if (!aligned4(sel_bits))
+            return fail(TB_ERR_INVALID_ARG, "%s: pointer 'sel_bits' is null or not 4-byte aligned", fn);
+        if (sink < 0 || window < 1) return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0 and window >= 1", fn);
+    }
+    return TB_OK;
+}
+
+cudaError_t ensure_dynamic_smem(const void *fn, int bytes, std::atomic<int> *done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::atomic<int> &have = done[dev];
+    if (have.load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(g_state_mu);
+    if (have.load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) have.store(bytes, std::memory_order_release);
+    return e;
+}
+
+int num_sms() {
+    static std::atomic<int> sms[kMaxDevices];  // zero-initialised (static storage)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    std::atomic<int> &have = sms[dev];
+    int n = have.load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        have.store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
 }  // namespace tb
 
 using namespace tb;
@@ -263,6 +315,19 @@ tb_status tb_selftest_bounded_wait(void *ws, size_t ws_bytes, int64_t budget_cyc
     return cuda_status(launch_bounded_wait_selftest(ws, budget_cycles, (cudaStream_t)stream), __func__);
 }
 
+tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_bytes, const int32_t *ctx_len,
+                                 int32_t sink, int32_t window, float *scores, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
+    if (dims->ctx_cap > kMaxCtxSelect)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", __func__, dims->ctx_cap, kMaxCtxSelect);
+    TB_CHECK_PTR4(ctx_len); TB_CHECK_PTR4(scores);
+    if (sink < 0 || window < 1) return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0 and window >= 1", __func__);
+    if ((s = check_ws(const_cast<void *>(ws), ws_bytes, select_ws_bytes(*dims), __func__)) != TB_OK) return s;
+    return cuda_status(launch_export_scores(*dims, ws, ctx_len, sink, window, scores, (cudaStream_t)stream),
+                       __func__);
+}
+
 tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32_t idx_cap,
                                   const int32_t *count, uint32_t *sel_bits, void *stream) {
     tb_status s;
@@ -274,30 +339,13 @@ tb_status tb_select_bits_from_idx(const tb_dims *dims, const int32_t *idx, int32
     return cuda_status(launch_select_bits(*dims, idx, idx_cap, count, sel_bits, (cudaStream_t)stream), __func__);
 }
 
-static tb_status attn_common(const char *fn, const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
-                             const tb_bf16 *V, const int32_t *ctx_len, float scale, float *out, void *ws,
-                             size_t ws_bytes) {
-    tb_status s;
-    if ((s = check_dims(dims, false, fn)) != TB_OK) return s;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V))
-        return fail(TB_ERR_INVALID_ARG, "%s: Q, K and V must be non-null and 16-byte aligned", fn);
-    if (!aligned4(ctx_len) || !aligned4(out))
-        return fail(TB_ERR_INVALID_ARG, "%s: ctx_len and out must be non-null and 4-byte aligned", fn);
-    if (dims->ctx_cap > kMaxCtxAttn)
-        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", fn, dims->ctx_cap, kMaxCtxAttn);
-    if (!isfinite(scale)) return fail(TB_ERR_INVALID_ARG, "%s: scale is not finite", fn);
-    return check_ws(ws, ws_bytes, attn_ws_bytes(*dims), fn);
-}
-
 tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
                                 const int32_t *ctx_len, int32_t sink, int32_t window,
                                 const uint32_t *sel_bits, float scale, float *out, void *ws,
                                 size_t ws_bytes, void *stream) {
-    tb_status s = attn_common(__func__, dims, Q, K, V, ctx_len, scale, out, ws, ws_bytes);
+    tb_status s = check_attn_args(__func__, dims, Q, K, V, ctx_len, scale, out, true, sel_bits, sink, window);
     if (s != TB_OK) return s;
-    TB_CHECK_PTR4(sel_bits);
-    if (sink < 0 || window < 1)
-        return fail(TB_ERR_INVALID_ARG, "tb_sparse_decode_attn: need sink >= 0 and window >= 1");
+    if ((s = check_ws(ws, ws_bytes, attn_ws_bytes(*dims), __func__)) != TB_OK) return s;
     return cuda_status(launch_attn(*dims, Q, K, V, ctx_len, sink, window, sel_bits, true, scale, out, ws,
                                    (cudaStream_t)stream),
                        __func__);
@@ -306,8 +354,9 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
 tb_status tb_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
                          const int32_t *ctx_len, float scale, float *out, void *ws, size_t ws_bytes,
                          void *stream) {
-    tb_status s = attn_common(__func__, dims, Q, K, V, ctx_len, scale, out, ws, ws_bytes);
+    tb_status s = check_attn_args(__func__, dims, Q, K, V, ctx_len, scale, out, false, nullptr, 0, 1);
     if (s != TB_OK) return s;
+    if ((s = check_ws(ws, ws_bytes, attn_ws_bytes(*dims), __func__)) != TB_OK) return s;
     return cuda_status(launch_attn(*dims, Q, K, V, ctx_len, 0, 1, nullptr, false, scale, out, ws,
                                    (cudaStream_t)stream),
                        __func__);

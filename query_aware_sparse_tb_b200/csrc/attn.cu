@@ -613,31 +613,13 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     if (tid == 0) counters[b * Hkv + g] = 0u;  // leave the ticket zeroed for the next call
 }
 
-int g_num_sms = 0;
-
-int num_sms() {
-    if (g_num_sms == 0) {
-        int dev = 0, n = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-            g_num_sms = n;
-        else
-            g_num_sms = 148;
-    }
-    return g_num_sms;
-}
-
 template <int D, bool SPARSE>
 cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                      const int32_t *ctx_len, int32_t sink, int32_t window, const uint32_t *sel_bits,
                      float scale, float *out, void *ws, cudaStream_t st) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, SPARSE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::kBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<int> smem_set[kMaxDevices];
+    cudaError_t e = ensure_dynamic_smem((const void *)attn_kernel<D, SPARSE>, Smem::kBytes, smem_set);
+    if (e != cudaSuccess) return e;
     const int splits = attn_splits(d);
     uint8_t *w = static_cast<uint8_t *>(ws);
     uint32_t *flags = reinterpret_cast<uint32_t *>(w);

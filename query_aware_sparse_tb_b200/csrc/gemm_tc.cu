@@ -261,13 +261,9 @@ cudaError_t launch_pk(const tb_dims &d, const uint16_t *K, const uint16_t *Wk, u
         !make_map(&mW, Wk, D, (uint64_t)d.n_kv_heads * DP, DP))
         return cudaErrorInvalidValue;
     constexpr int smem = 1024 + (D / 64) * (kAtomA + DP * 128);
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(project_keys_kernel<D, DP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<int> smem_set[kMaxDevices];
+    cudaError_t e = ensure_dynamic_smem((const void *)project_keys_kernel<D, DP>, smem, smem_set);
+    if (e != cudaSuccess) return e;
     dim3 grid((max_tok + 127) / 128, d.n_kv_heads, d.batch);
     project_keys_kernel<D, DP><<<grid, 128, smem, st>>>(mK, mW, Kp, tok_begin, tok_count, d.n_kv_heads,
                                                        d.ctx_cap, flags);
@@ -281,13 +277,9 @@ cudaError_t launch_skinny(const uint16_t *A, const uint16_t *B, float *partial, 
     CUtensorMap mA, mB;
     if (!make_map(&mA, A, K, M, 128) || !make_map(&mB, B, K, n_rows, 16)) return cudaErrorInvalidValue;
     constexpr int smem = 1024 + kKB * (kAtomA + 16 * 128);
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<kKB>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<int> smem_set[kMaxDevices];
+    cudaError_t e = ensure_dynamic_smem((const void *)skinny_gemm_kernel<kKB>, smem, smem_set);
+    if (e != cudaSuccess) return e;
     dim3 grid(M / 128, K / (kKB * 64));
     skinny_gemm_kernel<kKB><<<grid, 128, smem, st>>>(mA, mB, partial, M, n_rows, flags);
     return cudaGetLastError();

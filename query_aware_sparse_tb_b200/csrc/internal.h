@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/tb.h"
 
 namespace tb {
@@ -27,6 +29,8 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                 int32_t window, int32_t budget, int32_t nbr, int32_t group_reduce,
                                 int32_t *idx, int32_t idx_cap, int32_t *count, uint32_t *sel_bits,
                                 void *ws, cudaStream_t st);
+cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t *ctx_len, int32_t sink,
+                                 int32_t window, float *scores, cudaStream_t st);
 cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx_cap,
                                const int32_t *count, uint32_t *sel_bits, cudaStream_t st);
 
@@ -47,5 +51,24 @@ cudaError_t launch_bounded_wait_selftest(void *ws, long long budget_cycles, cuda
 
 // Host error text for the calling thread (api.cu).
 void set_error(const char *fmt, ...);
+
+// Host-side argument checks of the attention entry points (api.cu), shared by
+// tb_sparse_decode_attn, tb_decode_attn and tb_sparse_decode_attn_noalloc so
+// that all of them accept exactly the same dims and pointers.  `sel_bits`,
+// `sink` and `window` are checked only when `sparse` is true.
+tb_status check_attn_args(const char *fn, const tb_dims *dims, const uint16_t *Q, const uint16_t *K,
+                          const uint16_t *V, const int32_t *ctx_len, float scale, float *out, bool sparse,
+                          const uint32_t *sel_bits, int32_t sink, int32_t window);
+
+// ---- per-device host state (api.cu) ----
+// Kernel attributes (the dynamic shared-memory limit) and the SM count belong
+// to a device, not to the process: a process may drive several GPUs.
+constexpr int kMaxDevices = 64;
+// Raise kernel `fn`'s dynamic shared-memory limit to at least `bytes` on the
+// current device; `done` is the caller's per-kernel record [kMaxDevices] of
+// the limit already set on each device.
+cudaError_t ensure_dynamic_smem(const void *fn, int bytes, std::atomic<int> *done);
+// Multiprocessors of the current device (148 when it cannot be queried).
+int num_sms();
 
 }  // namespace tb

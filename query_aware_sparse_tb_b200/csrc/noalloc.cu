@@ -23,8 +23,6 @@
 // threads without ordering between them) race on the scratch and produce
 // wrong outputs.
 #include <cuda_runtime.h>
-#include <math.h>
-
 #include <mutex>
 
 #include "common.cuh"
@@ -33,7 +31,7 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = TB_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
+using tb::kMaxDevices;
 
 // The scratch itself (zero at module load).
 static __device__ __align__(256) unsigned char tb_noalloc_scratch[kNoAllocScratchBytes];
@@ -75,9 +73,6 @@ tb_status scratch_for_current_device(void **out) {
     return TB_OK;
 }
 
-bool al16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool al4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
-
 }  // namespace
 
 extern "C" tb_status tb_sparse_decode_attn_noalloc(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
@@ -85,23 +80,9 @@ extern "C" tb_status tb_sparse_decode_attn_noalloc(const tb_dims *dims, const tb
                                                    int32_t window, const uint32_t *sel_bits, float scale,
                                                    float *out, void *stream) {
     const char *fn = "tb_sparse_decode_attn_noalloc";
-    if (!dims || dims->batch < 1 || dims->n_q_heads < 1 || dims->n_kv_heads < 1 || dims->ctx_cap < 1 ||
-        dims->n_q_heads % dims->n_kv_heads != 0) {
-        tb::set_error("%s: invalid dims", fn);
-        return TB_ERR_INVALID_ARG;
-    }
-    if (dims->n_q_heads / dims->n_kv_heads != 4 || (dims->head_dim != 64 && dims->head_dim != 128)) {
-        tb::set_error("%s: only GQA groups of 4 and head_dim 64 or 128 are built", fn);
-        return TB_ERR_UNSUPPORTED;
-    }
-    if (!al16(Q) || !al16(K) || !al16(V) || !al4(ctx_len) || !al4(out) || !al4(sel_bits)) {
-        tb::set_error("%s: null or misaligned pointer", fn);
-        return TB_ERR_INVALID_ARG;
-    }
-    if (sink < 0 || window < 1 || !isfinite(scale)) {
-        tb::set_error("%s: need sink >= 0, window >= 1 and a finite scale", fn);
-        return TB_ERR_INVALID_ARG;
-    }
+    // the checks of tb_sparse_decode_attn, so both entry points accept the same dims
+    tb_status st = tb::check_attn_args(fn, dims, Q, K, V, ctx_len, scale, out, true, sel_bits, sink, window);
+    if (st != TB_OK) return st;
     const size_t need = tb::attn_ws_bytes(*dims);
     if (need > kNoAllocScratchBytes) {
         tb::set_error("%s: these dims need %zu bytes of scratch but the fixed scratch holds %zu; "
@@ -109,8 +90,7 @@ extern "C" tb_status tb_sparse_decode_attn_noalloc(const tb_dims *dims, const tb
         return TB_ERR_WORKSPACE;
     }
     void *ws = nullptr;
-    tb_status s = scratch_for_current_device(&ws);
-    if (s != TB_OK) return s;
+    if ((st = scratch_for_current_device(&ws)) != TB_OK) return st;
     cudaError_t e = tb::launch_attn(*dims, Q, K, V, ctx_len, sink, window, sel_bits, true, scale, out, ws,
                                     (cudaStream_t)stream);
     if (e != cudaSuccess) {

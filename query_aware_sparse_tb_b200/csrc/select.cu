@@ -9,7 +9,7 @@
 // selected tokens are expanded by their spatial neighbours.
 //
 // Exact top-B on the fp32 scores, ties broken by the lower position:
-//   1. score_hist   one CTA per (b, KV head, 1024 positions): reads each K'
+//   1. score_hist   one CTA per (b, KV head, 2048 positions): reads each K'
 //                   row once for the 4 query heads of the group, writes the
 //                   order-preserving uint32 image of every score, and builds
 //                   a histogram of its top 11 bits per query head.  The last
@@ -676,6 +676,27 @@ bits_from_idx_kernel(const int32_t *__restrict__ idx, int idx_cap, const int32_t
     for (int w = tid; w < W; w += kFinThreads) sel_bits[row * W + w] = bsm[w];
 }
 
+// ------------------------------------------------------ scores of a call
+
+// The fp32 scores behind the last selection on a workspace, decoded from the
+// order-preserving key image score_hist left there: candidates of C get their
+// score, every other position NaN.
+__global__ void __launch_bounds__(kThreads)
+export_scores_kernel(const uint32_t *__restrict__ keys, const int32_t *__restrict__ ctx_len, int Hq, int Tcap,
+                     int sink, int window, float *__restrict__ out) {
+    const int p = blockIdx.x * kThreads + threadIdx.x;
+    const int h = blockIdx.y, b = blockIdx.z;
+    if (p >= Tcap) return;
+    const int T = clamp_ctx(ctx_len[b], Tcap, nullptr, false);
+    const size_t i = ((size_t)b * Hq + h) * Tcap + p;
+    float v = __int_as_float(0x7fc00000);
+    if (p >= sink && p < T - window) {
+        const uint32_t k = keys[i];
+        v = __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+    }
+    out[i] = v;
+}
+
 template <int SEL>
 cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
                        const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, int32_t nbr,
@@ -699,11 +720,10 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4 + (SEL == kSelInclusive ? kCandCache * 2 : 0);
-    static size_t configured = 0;
-    if (fsm > 48 * 1024 && fsm > configured) {
-        e = cudaFuncSetAttribute(finalize_kernel<SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
+    static std::atomic<int> smem_set[kMaxDevices];
+    if (fsm > 48 * 1024) {
+        e = ensure_dynamic_smem((const void *)finalize_kernel<SEL>, (int)fsm, smem_set);
         if (e != cudaSuccess) return e;
-        configured = fsm;
     }
     const int rows = sel_is_group(SEL) ? d.n_q_heads / kGroup : d.n_q_heads;
     finalize_kernel<SEL><<<dim3(rows, d.batch), kFinThreads, fsm, st>>>(
@@ -733,15 +753,22 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                 sel_bits, ws, st);
 }
 
+cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t *ctx_len, int32_t sink,
+                                 int32_t window, float *scores, cudaStream_t st) {
+    const SelWs s = carve(d, const_cast<void *>(ws));
+    dim3 grid((d.ctx_cap + kThreads - 1) / kThreads, d.n_q_heads, d.batch);
+    export_scores_kernel<<<grid, kThreads, 0, st>>>(s.keys, ctx_len, d.n_q_heads, d.ctx_cap, sink, window, scores);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx_cap,
                                const int32_t *count, uint32_t *sel_bits, cudaStream_t st) {
     const int W = (d.ctx_cap + 31) / 32;
     const size_t sm = (size_t)W * 4;
-    static size_t configured = 0;
-    if (sm > 48 * 1024 && sm > configured) {
-        cudaError_t e = cudaFuncSetAttribute(bits_from_idx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    static std::atomic<int> smem_set[kMaxDevices];
+    if (sm > 48 * 1024) {
+        cudaError_t e = ensure_dynamic_smem((const void *)bits_from_idx_kernel, (int)sm, smem_set);
         if (e != cudaSuccess) return e;
-        configured = sm;
     }
     bits_from_idx_kernel<<<dim3(d.n_q_heads, d.batch), kFinThreads, sm, st>>>(
         idx, idx_cap, count, d.n_q_heads, d.ctx_cap, W, sel_bits);

@@ -55,7 +55,7 @@ def test_binding_constants_match_header(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.tb_abi_version() == 5
+    assert lib.tb_abi_version() == 6
     assert lib.tb_status_str(0) == b"TB_OK"
     assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
 
@@ -256,3 +256,43 @@ def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
     res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0, (res.returncode, res.stdout, res.stderr)
     assert "16-byte aligned" in res.stdout
+
+
+def test_score_export_rejects_bad_arguments(lib):
+    d = _d()
+    wsb = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
+    call = lambda dims, ws=FAKE, nb=wsb, ctx=FAKE, sink=16, window=64, out=FAKE: lib.tb_score_select_scores(  # noqa: E731
+        ctypes.byref(dims), ws, nb, ctx, sink, window, out, None)
+    assert call(_d(d_proj=24)) == _lib.TB_ERR_UNSUPPORTED
+    assert call(d, nb=wsb - 1) == _lib.TB_ERR_WORKSPACE
+    assert call(d, out=0) == _lib.TB_ERR_INVALID_ARG
+    assert call(d, ctx=FAKE + 2) == _lib.TB_ERR_INVALID_ARG
+    assert call(d, window=0) == _lib.TB_ERR_INVALID_ARG
+    assert call(_d(ctx_cap=(1 << 19) + 1)) == _lib.TB_ERR_UNSUPPORTED
+
+
+def test_noalloc_accepts_exactly_the_workspace_entry_points_dims(lib):
+    # both sparse entry points run the same host checks; the no-alloc one then
+    # also bounds the scratch the dims need
+    def noalloc(dims, **kw):
+        a = dict(Q=FAKE, K=FAKE, V=FAKE, ctx=FAKE, sink=16, window=64, bits=FAKE, scale=0.088, out=FAKE)
+        a.update(kw)
+        return lib.tb_sparse_decode_attn_noalloc(ctypes.byref(dims), a["Q"], a["K"], a["V"], a["ctx"], a["sink"],
+                                                 a["window"], a["bits"], a["scale"], a["out"], None)
+
+    def with_ws(dims, **kw):
+        a = dict(Q=FAKE, K=FAKE, V=FAKE, ctx=FAKE, sink=16, window=64, bits=FAKE, scale=0.088, out=FAKE)
+        a.update(kw)
+        nb = lib.tb_attn_workspace_bytes(ctypes.byref(_d())) or 256
+        return lib.tb_sparse_decode_attn(ctypes.byref(dims), a["Q"], a["K"], a["V"], a["ctx"], a["sink"],
+                                         a["window"], a["bits"], a["scale"], a["out"], FAKE, nb, None)
+
+    cases = [(_d(ctx_cap=(1 << 22) + 1), {}), (_d(head_dim=96), {}), (_d(n_q_heads=24), {}),
+             (_d(batch=65536), {}), (_d(), dict(Q=MIS)), (_d(), dict(bits=0)), (_d(), dict(window=0)),
+             (_d(), dict(sink=-1)), (_d(), dict(scale=float("inf")))]
+    for dims, kw in cases:
+        want = with_ws(dims, **kw)
+        assert want in (_lib.TB_ERR_INVALID_ARG, _lib.TB_ERR_UNSUPPORTED), (dims.ctx_cap, kw)
+        assert noalloc(dims, **kw) == want, (dims.ctx_cap, kw)
+    # valid dims beyond the fixed scratch: rejected before any CUDA call
+    assert noalloc(_d(batch=16, ctx_cap=32896)) == _lib.TB_ERR_WORKSPACE

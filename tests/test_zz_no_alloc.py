@@ -2,9 +2,10 @@
 
 It exists for callers that cannot allocate device memory for the call (an
 operator boundary that is handed only its inputs and outputs, or a decode
-loop that must not call cudaMalloc).  Its output must match the workspace
-entry point's within the attention tolerance, on two calls in a row (the
-second call reuses the fixed scratch the first one left behind).  This file is
+loop that must not call cudaMalloc).  It runs the same kernel on the same
+inputs as the workspace entry point, so its output must equal that entry
+point's bit for bit, on two calls in a row (the second call reuses the fixed
+scratch the first one left behind).  This file is
 collected last on purpose."""
 import ctypes
 import math
@@ -48,7 +49,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
                                                out.data_ptr(), stream)
         assert st == _lib.TB_OK, lib.tb_last_error()
         torch.cuda.synchronize()
-        parity.assert_close(out.cpu().numpy(), ref.cpu().numpy(), f"no-alloc call {call}")
+        assert torch.equal(out, ref), f"no-alloc call {call} differs from tb_sparse_decode_attn"
 
 
 @pytest.mark.gpu
