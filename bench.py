@@ -334,15 +334,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def profiled_traffic(kernel: str, root: str = ROOT):
-    """DRAM bytes per launch from the committed ncu capture of `kernel`, or
-    None when any of that kernel's source files has changed since the capture
-    (or the record is missing)."""
+def profiled_traffic(kernel: str, workload: str, root: str = ROOT):
+    """DRAM bytes per launch from the committed ncu capture of `kernel` on
+    `workload`, or None when the record was taken on another workload, when any
+    of that kernel's source files has changed since the capture, or when the
+    record is missing."""
     import hashlib
     try:
         with open(os.path.join(root, "profiles", "traffic.json")) as f:
             rec = json.load(f)[kernel]
-        if not rec["sources"]:
+        if rec.get("workload_name") != workload or not rec["sources"]:
             return None
         for path, sha in rec["sources"].items():
             with open(os.path.join(root, path), "rb") as f:
@@ -367,12 +368,27 @@ def measured_peaks():
 # CPU oracle on a bounded sample
 # ----------------------------------------------------------------------------
 
+def host_info() -> dict:
+    """The host's logical core count and CPU model (for the CPU baseline)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
 class OracleSample:
     """The oracle on one layer of the workload: the key projection of the
-    prefilled context (setup), then decode steps of that layer in schedule
-    order; a prediction step runs the predictor MLP, scoring and selection for
-    every query head, every step runs attention for every query head.  The
-    per-layer times are scaled to a whole decode step (x n_layers)."""
+    prefilled context (setup, timed), then decode steps of that layer in
+    schedule order.  A prediction step scores and selects for every query head
+    from the layer's slot of its producer's predicted queries (the predictor
+    MLP itself is timed apart, once per producer call); every step runs
+    attention for every query head."""
 
     def __init__(self, w: tb_inputs.Workload, layer: int = 0):
         import numpy as np
@@ -395,19 +411,26 @@ class OracleSample:
                 self.Kp[(b, g)] = self.o.project_keys(self.K[b, g, :n + w.window], self.Wk[g])
         self.proj_s = time.perf_counter() - t0
         self.rows_projected = sum((t // w.window) * w.window + w.window for t in self.ctx0) * w.n_kv_heads
+        self.stride = w.producer_stride if w.hidden > 0 else 1
+        self.producer = layer - layer % self.stride
         if w.hidden > 0:
-            W1, W2 = tb_inputs.mlp_weights(w, 0, "cpu")
+            W1, W2 = tb_inputs.mlp_weights(w, self.producer, "cpu")
             self.W1 = W1.view(torch.int16).numpy().view(np.uint16)
             self.W2 = W2.view(torch.int16).numpy().view(np.uint16)
         self.I = None
+        self.mlp_s = []
 
     def step(self, i):
         np, o, w = self.np, self.o, self.w
         ctx = [t + i + 1 for t in self.ctx0]
         if is_prediction_step(i, w.interval):
             if w.hidden > 0:
-                h = tb_inputs.hidden_state(w, i // w.interval, 0, "cpu").view(torch.int16).numpy().view(np.uint16)
-                qp = o.predict_queries(h, self.W1, self.W2).reshape(w.batch, w.slots, w.n_q_heads, w.d_proj)[:, 0]
+                h = tb_inputs.hidden_state(w, i // w.interval, self.producer, "cpu").view(torch.int16).numpy().view(
+                    np.uint16)
+                t0 = time.perf_counter()
+                qp = o.predict_queries(h, self.W1, self.W2).reshape(w.batch, w.slots, w.n_q_heads, w.d_proj)
+                self.mlp_s.append(time.perf_counter() - t0)
+                qp = qp[:, self.layer % self.stride]
             else:
                 qp = tb_inputs.direct_qp(w, i // w.interval, self.layer, "cpu").numpy()
             self.I = []
@@ -425,41 +448,65 @@ class OracleSample:
                 A = o.attention_set(ctx[b], w.sink, w.window, self.I[b][h_])
                 o.attention(Q[b, h_], self.K[b, h_ // w.group], self.V[b, h_ // w.group], A, self.scale)
 
-    def per_decode_step_s(self, t_pred, t_reuse):
-        """Whole-model seconds per decode step from per-layer step times: every
-        layer pays attention each step and selection once per interval; the
-        predictor is paid by 1/stride of the layers (it was timed on every
-        prediction step of the sampled producer layer, so this over-counts
-        it); key projection is paid once per token."""
-        w = self.w
-        per_layer = (t_pred + (w.interval - 1) * t_reuse) / w.interval
-        rows_per_step = w.batch * w.n_kv_heads                 # one new row per (b, kv head) per step
-        proj = self.proj_s / self.rows_projected * rows_per_step
-        return w.n_layers * (per_layer + proj)
+
+def per_decode_step_s(w, layers: list[dict]) -> float:
+    """Whole-model oracle seconds per decode step from per-layer samples.  Each
+    sample holds the layer's mean prediction-step time (without the predictor
+    MLP), mean reuse-step time, predictor MLP time (producer layers; None
+    otherwise) and projection seconds per projected row.  Every layer pays
+    attention at every step and scoring + selection once per interval; the
+    predictor is paid once per producer layer per interval; key projection
+    once per new token."""
+    per_layer = statistics.mean((x["t_pred"] + (w.interval - 1) * x["t_reuse"]) / w.interval for x in layers)
+    mlps = [x["t_mlp"] for x in layers if x["t_mlp"] is not None]
+    n_prod = len(range(0, w.n_layers, w.producer_stride)) if w.hidden > 0 else 0
+    mlp = (statistics.mean(mlps) * n_prod / w.interval) if mlps else 0.0
+    proj_row = statistics.mean(x["proj_s_per_row"] for x in layers)
+    rows_per_step = w.batch * w.n_kv_heads                     # one new row per (sequence, KV head)
+    return w.n_layers * (per_layer + proj_row * rows_per_step) + mlp
 
 
-def cpu_baseline(w, budget_s=25.0):
-    smp = OracleSample(w)
+def sample_layers(w) -> list[int]:
+    return sorted({0, min(1, w.n_layers - 1), w.n_layers - 1})
+
+
+def oracle_layer_sample(w, layer: int, budget_s: float) -> dict:
+    """Time one layer: its projection setup, its first (prediction) step and
+    reuse steps until `budget_s` seconds of steps have passed."""
+    smp = OracleSample(w, layer)
     t_pred, t_reuse = [], []
     t_start = time.perf_counter()
     i = 0
-    while True:
+    while i < w.steps:
         t0 = time.perf_counter()
         smp.step(i)
         dt = time.perf_counter() - t0
-        (t_pred if is_prediction_step(i, w.interval) else t_reuse).append(dt)
+        if is_prediction_step(i, w.interval):
+            t_pred.append(dt - (smp.mlp_s[-1] if smp.mlp_s else 0.0))
+        else:
+            t_reuse.append(dt)
         i += 1
         if t_reuse and time.perf_counter() - t_start > budget_s:
             break
-        if i >= w.steps:
-            break
-    s_per_step = smp.per_decode_step_s(statistics.mean(t_pred), statistics.mean(t_reuse))
-    return {"value": w.batch / s_per_step, "unit": "decode steps/s", "cores": 1, "kind": "oracle",
-            "sample": (f"layer 0 of {w.name}: key projection of the prefilled context ({smp.proj_s:.1f} s), "
-                       f"{len(t_pred)} prediction + {len(t_reuse)} reuse decode steps of all {w.n_q_heads} query "
-                       f"heads; scaled x{w.n_layers} layers, selection amortised over the interval, projection "
-                       f"per token"),
-            "sample_seconds": round(time.perf_counter() - t_start + smp.proj_s, 1)}
+    return {"layer": layer, "t_pred": statistics.mean(t_pred), "t_reuse": statistics.mean(t_reuse or t_pred),
+            "t_mlp": statistics.mean(smp.mlp_s) if (smp.mlp_s and layer % smp.stride == 0) else None,
+            "proj_s_per_row": smp.proj_s / smp.rows_projected, "setup_s": smp.proj_s,
+            "n_pred": len(t_pred), "n_reuse": len(t_reuse)}
+
+
+def cpu_baseline(w, budget_s=6.0):
+    t0 = time.perf_counter()
+    layers = [oracle_layer_sample(w, l, budget_s) for l in sample_layers(w)]
+    s_per_step = per_decode_step_s(w, layers)
+    desc = "; ".join(f"layer {x['layer']}: setup {x['setup_s']:.1f} s, {x['n_pred']} prediction + {x['n_reuse']} "
+                     f"reuse steps" for x in layers)
+    return dict({"value": w.batch / s_per_step, "unit": "decode steps/s", "cores": 1, "kind": "oracle",
+                 "sample": (f"{w.name}, layers {[x['layer'] for x in layers]} of {w.n_layers}, every query head, "
+                            f"one thread ({desc}); key projection of the prefilled context timed as setup and "
+                            f"charged per new token; per-layer step times averaged over the sampled layers and "
+                            f"scaled to all layers, selection amortised over the {w.interval}-step interval, the "
+                            f"predictor MLP once per producer layer per interval"),
+                 "sample_seconds": round(time.perf_counter() - t0, 1)}, **host_info())
 
 
 def config_of(w: tb_inputs.Workload, decode_steps: int, world: int, selection: str = "head") -> dict:
@@ -477,31 +524,50 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = tb_inputs.WORKLOADS[args.workload]
-    smp = OracleSample(w)
-    t_pred, t_reuse = [], []
-    for i in range(args.warmup):        # step 0 predicts, so reuse steps have a selection
-        smp.step(i)
-    order = list(range(args.steps))
+    layers = sample_layers(w)
+    samples = {l: OracleSample(w, l) for l in layers}
+    for smp in samples.values():
+        for i in range(min(args.warmup, w.steps)):     # step 0 predicts, so reuse steps have a selection
+            smp.step(i)
     t_all0 = time.perf_counter()
-    for i in order:
-        t0 = time.perf_counter()
-        smp.step(i)
-        (t_pred if is_prediction_step(i, w.interval) else t_reuse).append(time.perf_counter() - t0)
+    per = {l: {"pred": [], "reuse": []} for l in layers}
+    for k in range(args.steps):
+        # each bench step: one decode step of every sampled layer, cycling
+        # through the schedule so prediction steps come in their proportion
+        i = k % w.steps
+        for l, smp in samples.items():
+            t0 = time.perf_counter()
+            smp.step(i)
+            dt = time.perf_counter() - t0
+            if is_prediction_step(i, w.interval):
+                per[l]["pred"].append(dt - (smp.mlp_s[-1] if smp.mlp_s else 0.0))
+            else:
+                per[l]["reuse"].append(dt)
     wall = time.perf_counter() - t_all0
-    if not t_reuse:
-        t_reuse = t_pred
-    s_per_step = smp.per_decode_step_s(statistics.mean(t_pred), statistics.mean(t_reuse))
-    value = w.batch / s_per_step
-    sample = (f"each step: one decode step of layer 0 of {w.name} (all {w.n_q_heads} query heads; the first step "
-              f"also predicts and selects), scaled x{w.n_layers} layers with selection amortised over the "
-              f"{w.interval}-step interval")
+    stats = []
+    for l, smp in samples.items():
+        pr, ru = per[l]["pred"], per[l]["reuse"]
+        if not pr:                                       # no prediction step timed: the warm-up one
+            smp_w = OracleSample(w, l)
+            t0 = time.perf_counter()
+            smp_w.step(0)
+            pr = [time.perf_counter() - t0 - (smp_w.mlp_s[-1] if smp_w.mlp_s else 0.0)]
+            smp = smp_w
+        stats.append({"layer": l, "t_pred": statistics.mean(pr), "t_reuse": statistics.mean(ru or pr),
+                      "t_mlp": statistics.mean(smp.mlp_s) if (smp.mlp_s and l % smp.stride == 0) else None,
+                      "proj_s_per_row": smp.proj_s / smp.rows_projected})
+    value = w.batch / per_decode_step_s(w, stats)
+    sample = (f"each bench step: one decode step of layers {layers} of {w.name} (all {w.n_q_heads} query heads, one "
+              f"thread), in schedule order; per-layer times scaled to {w.n_layers} layers with selection amortised "
+              f"over the {w.interval}-step interval, the predictor once per producer layer")
+    cb = dict({"value": round(value, 4), "unit": "decode steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+              **host_info())
     line = {"impl": "reference", "metric": "sparse decode steps/s", "value": round(value, 4),
             "unit": "decode steps/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1000 * wall / max(1, len(order)), 3), "higher_is_better": True,
+            "ms_per_step": round(1000 * wall / max(1, args.steps), 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, args.decode_steps or w.steps, args.gpus),
-            "cpu_baseline": {"value": round(value, 4), "unit": "decode steps/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": cb,
             "e2e": {"value": round(value, 4), "unit": "decode steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -511,6 +577,85 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 # main
 # ----------------------------------------------------------------------------
+
+def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup: int, selection: str):
+    """Time one workload's sparse run, dense run and (optionally) the e2e run,
+    each replayed as one CUDA graph; returns the figures the JSON line needs."""
+    run = Run(w, device, steps=args.decode_steps, selection=selection)
+    run.dec.prefill()
+    torch.cuda.synchronize()
+
+    acct = run.bytes_model()       # eager pass: warms every kernel and counts the kept rows
+    stream = torch.cuda.Stream(device=device)
+    marks_s = Marks(run.steps)
+    marks_s.stream = stream
+    g_sparse = capture(lambda st: run.run_sparse(st, marks_s), stream)
+    marks_d = Marks(run.steps)
+    marks_d.stream = stream
+    g_dense = capture(lambda st: run.run_dense(st, marks_d), stream)
+    e2e = g_e2e = None
+    if with_e2e:
+        e2e = E2E(run)
+        g_e2e = capture(e2e.body, stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    ms_sparse = time_graph(g_sparse, warmup, steps, dist_on, device)
+    attn_ms = marks_s.attn_ms(run.steps)
+    ms_dense = time_graph(g_dense, warmup, steps, dist_on, device)
+    dense_attn_ms = marks_d.attn_ms(run.steps)
+    clk = clocks.stop()
+    ms_e2e = clk_e2e = None
+    if e2e is not None:
+        clocks = ClockSampler(torch.cuda.current_device())
+        ms_e2e = time_graph(g_e2e, warmup, steps, dist_on, device)
+        clk_e2e = clocks.stop()
+
+    flags = L.workspace_check(run.dec.ws_attn) | L.workspace_check(run.dec.ws_sel) | \
+        L.workspace_check(run.dec.ws_proj) | (L.workspace_check(run.dec.ws_pred) if run.dec.ws_pred is not None else 0)
+
+    tokens_per_run = run.steps * w.batch
+    per_step_sparse = ms_sparse / steps
+    per_step_dense = ms_dense / steps
+    n_attn = run.steps * w.n_layers
+    attn_launch_ms = sum(attn_ms) / n_attn
+    dense_launch_ms = sum(dense_attn_ms) / n_attn
+    res = dict(
+        run_steps=run.steps, tokens_per_run=tokens_per_run, acct=acct,
+        value=aggregate_rate(world, tokens_per_run, per_step_sparse),
+        dense_value=aggregate_rate(world, tokens_per_run, per_step_dense),
+        per_step_sparse=per_step_sparse, per_step_dense=per_step_dense,
+        attn_launch_ms=attn_launch_ms, attn_bytes_per_launch=acct["attn_bytes"] / n_attn,
+        dense_launch_ms=dense_launch_ms, dense_bytes_per_launch=(acct["dense_total"] / n_attn),
+        path_gbs=acct["sparse_total"] / (per_step_sparse / 1000.0) / 1e9,
+        dense_path_gbs=acct["dense_total"] / (per_step_dense / 1000.0) / 1e9,
+        launches=run.launches()[0], clocks=clk, flags=flags,
+        kv_gb=2 * sum(k.numel() for k in run.K) * 2 / 1e9)
+    if e2e is not None:
+        h2d, d2h = e2e.bytes_per_run()
+        res["e2e"] = {"value": round(aggregate_rate(world, tokens_per_run, ms_e2e / steps), 3),
+                      "unit": "decode steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": round(ms_e2e / steps, 4), "clocks": clk_e2e}
+    del g_sparse, g_dense, g_e2e, e2e, run
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def summary(w, r, peak):
+    """The compact per-workload figures of the extra workloads."""
+    achieved = r["attn_bytes_per_launch"] / (r["attn_launch_ms"] / 1000.0) / 1e9
+    return {"value": round(r["value"], 3), "unit": "decode steps/s", "ms_per_step": round(r["per_step_sparse"], 4),
+            "dense_value": round(r["dense_value"], 3), "speedup_vs_dense": round(r["value"] / r["dense_value"], 4),
+            "path_gbs": round(r["path_gbs"], 1), "path_frac_of_8tbs": round(r["path_gbs"] / HBM_NOMINAL_GBS, 4),
+            "attn_achieved_gbs": round(achieved, 1), "attn_frac": round(achieved / peak, 4),
+            "attn_launch_us": round(1000 * r["attn_launch_ms"], 3),
+            "dense_attn_frac": round(r["dense_bytes_per_launch"] / (r["dense_launch_ms"] / 1000.0) / 1e9 / peak, 4),
+            "decode_steps_per_bench_step": r["run_steps"], "clocks": r["clocks"], "device_flags": r["flags"],
+            "config": {"batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
+                       "layers": w.n_layers, "budget": w.budget, "interval": w.interval,
+                       "kv_gb": round(r["kv_gb"], 1)}}
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -525,6 +670,9 @@ def main():
                     help="override the prediction interval P (1: predict and select at every step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra workloads (batch16, long256k) timed after the headline one")
+    ap.add_argument("--extra-steps", type=int, default=3, help="timed bench steps of each extra workload")
     ap.add_argument("--selection", default="head", choices=list(SparseDecoder.SELECTIONS),
                     help="head: one importance set per query head (the default, the pages' reading); "
                          "group_max / group_sum: one set per KV head (the group-shared variant); "
@@ -545,91 +693,66 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device(device))
     L.load()
-    base = tb_inputs.WORKLOADS[args.workload]
-    w = replica(base, rank)                          # an independent replica per rank
-    if args.layers:
-        w = w.scaled(n_layers=args.layers)
-    if args.interval:
-        w = w.scaled(interval=args.interval)
-    run = Run(w, device, steps=args.decode_steps, selection=args.selection)
-    run.dec.prefill()
-    torch.cuda.synchronize()
 
-    acct = run.bytes_model()       # eager pass: warms every kernel and counts the kept rows
-    stream = torch.cuda.Stream(device=device)
-    marks_s = Marks(run.steps)
-    marks_s.stream = stream
-    g_sparse = capture(lambda st: run.run_sparse(st, marks_s), stream)
-    marks_d = Marks(run.steps)
-    marks_d.stream = stream
-    g_dense = capture(lambda st: run.run_dense(st, marks_d), stream)
-    e2e = None
-    if not args.no_e2e:
-        e2e = E2E(run)
-        g_e2e = capture(e2e.body, stream)
-    torch.cuda.synchronize()
+    def prepare(name):
+        w = replica(tb_inputs.WORKLOADS[name], rank)          # an independent replica per rank
+        if args.layers:
+            w = w.scaled(n_layers=args.layers)
+        if args.interval:
+            w = w.scaled(interval=args.interval)
+        return w
 
-    clocks = ClockSampler(local)
-    ms_sparse = time_graph(g_sparse, args.warmup, args.steps, dist_on, device)
-    attn_ms = marks_s.attn_ms(run.steps)
-    ms_dense = time_graph(g_dense, args.warmup, args.steps, dist_on, device)
-    dense_attn_ms = marks_d.attn_ms(run.steps)
-    clk = clocks.stop()
-    ms_e2e = time_graph(g_e2e, args.warmup, args.steps, dist_on, device) if e2e else None
+    w = prepare(args.workload)
+    r = measure(w, args, device, dist_on, world, not args.no_e2e, args.steps, args.warmup, args.selection)
+    extras = {}
+    if not args.no_extra and args.workload == "llama64k" and not args.layers and not args.decode_steps:
+        # the other two large workloads, each against the dense kernel on its own cache
+        for name in ("long256k", "batch16"):
+            wx = prepare(name)
+            extras[name] = summary(wx, measure(wx, args, device, dist_on, world, False, args.extra_steps,
+                                               max(3, args.warmup), args.selection), measured_peaks()[0])
 
-    flags = L.workspace_check(run.dec.ws_attn) | L.workspace_check(run.dec.ws_sel) | \
-        L.workspace_check(run.dec.ws_proj) | (L.workspace_check(run.dec.ws_pred) if run.dec.ws_pred is not None else 0)
-
-    tokens_per_run = run.steps * w.batch
-    per_step_sparse = ms_sparse / args.steps
-    per_step_dense = ms_dense / args.steps
-    value = aggregate_rate(world, tokens_per_run, per_step_sparse)
-    dense_value = aggregate_rate(world, tokens_per_run, per_step_dense)
     peak, peak_kind = measured_peaks()
-    n_attn = run.steps * w.n_layers
-    attn_launch_ms = sum(attn_ms) / n_attn
-    attn_bytes_per_launch = acct["attn_bytes"] / n_attn
-    achieved = attn_bytes_per_launch / (attn_launch_ms / 1000.0) / 1e9
-    dense_launch_ms = sum(dense_attn_ms) / n_attn
-    dense_achieved = (acct["dense_total"] / n_attn) / (dense_launch_ms / 1000.0) / 1e9
-    path_gbs = acct["sparse_total"] / (per_step_sparse / 1000.0) / 1e9
-    dense_path_gbs = acct["dense_total"] / (per_step_dense / 1000.0) / 1e9
-    sparse_launches, dense_launches = run.launches()
+    acct = r["acct"]
+    achieved = r["attn_bytes_per_launch"] / (r["attn_launch_ms"] / 1000.0) / 1e9
+    dense_achieved = r["dense_bytes_per_launch"] / (r["dense_launch_ms"] / 1000.0) / 1e9
 
     if rank != 0:
         if dist_on:
             torch.distributed.destroy_process_group()
         return 0
     line = {
-        "metric": "sparse decode steps/s", "value": round(value, 3), "unit": "decode steps/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_sparse, 4),
+        "metric": "sparse decode steps/s", "value": round(r["value"], 3), "unit": "decode steps/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["per_step_sparse"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; Llama-3.1-8B attention shapes, random weights)",
-        "config": dict(config_of(w, run.steps, world, args.selection),
-                       l2="inputs larger than L2 (KV %.1f GB)" % (2 * sum(k.numel() for k in run.K) * 2 / 1e9),
+        "config": dict(config_of(w, r["run_steps"], world, args.selection),
+                       l2="inputs larger than L2 (KV %.1f GB)" % r["kv_gb"],
                        graph="one CUDA graph per bench step"),
-        "speedup_vs_dense": round(value / dense_value, 4),
-        "dense": {"value": round(dense_value, 3), "unit": "decode steps/s", "ms_per_step": round(per_step_dense, 4),
-                  "path_gbs": round(dense_path_gbs, 1), "attn_launch_us": round(1000 * dense_launch_ms, 3),
+        "speedup_vs_dense": round(r["value"] / r["dense_value"], 4),
+        "dense": {"value": round(r["dense_value"], 3), "unit": "decode steps/s",
+                  "ms_per_step": round(r["per_step_dense"], 4), "path_gbs": round(r["dense_path_gbs"], 1),
+                  "attn_launch_us": round(1000 * r["dense_launch_ms"], 3),
                   "attn_achieved_gbs": round(dense_achieved, 1)},
-        "hbm": {"path_gbs": round(path_gbs, 1), "path_frac_of_8tbs": round(path_gbs / HBM_NOMINAL_GBS, 4),
-                "path_frac_of_measured": round(path_gbs / peak, 4), "bytes_per_bench_step": acct["sparse_total"],
+        "hbm": {"path_gbs": round(r["path_gbs"], 1), "path_frac_of_8tbs": round(r["path_gbs"] / HBM_NOMINAL_GBS, 4),
+                "path_frac_of_measured": round(r["path_gbs"] / peak, 4), "bytes_per_bench_step": acct["sparse_total"],
                 "attn_rows_union": acct["attn_rows"], "attn_rows_per_head_sum": acct["sum_head_rows"],
                 "dense_bytes_per_bench_step": acct["dense_total"]},
         "roofline": {"kernel": "attn_kernel<128,true> (sparse GQA decode attention)", "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic("attn_kernel<128,true>") if args.selection == "head" else None,
-                     "bytes_per_launch": round(attn_bytes_per_launch), "launch_us": round(1000 * attn_launch_ms, 3)},
-        "gpu_launches": (sparse_launches) * args.steps,
-        "clocks": clk,
-        "device_flags": flags,
+                     "traffic": (profiled_traffic("attn_kernel<128,true>", w.name)
+                                 if args.selection == "head" and not args.layers and not args.interval else None),
+                     "bytes_per_launch": round(r["attn_bytes_per_launch"]),
+                     "launch_us": round(1000 * r["attn_launch_ms"], 3)},
+        "gpu_launches": r["launches"] * args.steps,
+        "clocks": r["clocks"],
+        "device_flags": r["flags"],
     }
-    if e2e is not None:
-        h2d, d2h = e2e.bytes_per_run()
-        line["e2e"] = {"value": round(aggregate_rate(world, tokens_per_run, ms_e2e / args.steps), 3),
-                       "unit": "decode steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "ms_per_step": round(ms_e2e / args.steps, 4)}
+    if "e2e" in r:
+        line["e2e"] = r["e2e"]
+    if extras:
+        line["workloads"] = extras
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))

@@ -56,7 +56,8 @@ def projection_events(ctx0: int, window: int, steps: int):
     return (ctx0 // window) * window, events
 
 
-def run(w, data, layers, steps, want_attention=True, heads=None, selection="head"):
+def run(w, data, layers, steps, want_attention=True, heads=None, selection="head", seqs=None, attn_steps=None,
+        keep=False):
     """Run the oracle over decode steps [0, steps) for the given layers.
 
     `data` provides host arrays (numpy; bf16 as uint16):
@@ -72,11 +73,19 @@ def run(w, data, layers, steps, want_attention=True, heads=None, selection="head
     of the group then attends to that set) or "inclusive" (per query head,
     at most `budget` positions after neighbour fetch, the budget-inclusive
     variant).
+    `heads` and `seqs` restrict the work to some query heads and sequences
+    (the others get None), `attn_steps` to the steps whose attention output is
+    computed (default: every step).  With keep=True a prediction step's entry
+    also holds what the selection was taken from: "qp" [batch][Hq][d'] (the
+    layer's predicted queries), "scores" [b][h] (the fp32 scores of the
+    candidates [S, T-N); group scores in the group-shared modes) and "kp"
+    {(b, g): K' rows [0, T-N) of KV head g}.
     Returns {(step, layer): {"idx": [[I_bh]], "out": [batch][Hq][d] or None}}.
     """
     assert selection in ("head", "group_max", "group_sum", "inclusive")
     B, Hq, grp = w.batch, w.n_q_heads, w.group
     heads = list(range(Hq)) if heads is None else list(heads)
+    seqs = list(range(B)) if seqs is None else list(seqs)
     ctx0 = w.ctx0_per_seq()
     scale = 1.0 / math.sqrt(w.head_dim)
     res = {}
@@ -99,18 +108,23 @@ def run(w, data, layers, steps, want_attention=True, heads=None, selection="head
                 else:
                     qp = data.qp_direct(k, layer)
                 sets = []
+                kept_scores = []
                 for b in range(B):
                     T = ctx0[b] + i + 1
                     hi = T - w.window
                     per_head = []
+                    per_head_scores = []
                     group_sets = {}
+                    group_scores_ = {}
                     for h in range(Hq):
-                        if h not in heads:
+                        if h not in heads or b not in seqs:
                             per_head.append(None)
+                            per_head_scores.append(None)
                             continue
                         g = h // grp
                         if selection not in ("head", "inclusive") and g in group_sets:
                             per_head.append(group_sets[g])
+                            per_head_scores.append(group_scores_[g])
                             continue
                         if hi > w.sink:
                             key = (layer, b, g)
@@ -128,19 +142,28 @@ def run(w, data, layers, steps, want_attention=True, heads=None, selection="head
                         I = pick(s, T, w.sink, w.window, w.budget, w.nbr)
                         if selection not in ("head", "inclusive"):
                             group_sets[g] = I
+                            group_scores_[g] = s
                         per_head.append(I)
+                        per_head_scores.append(s)
                     sets.append(per_head)
+                    kept_scores.append(per_head_scores)
                 cur_idx[layer] = sets
+                if keep:
+                    kept = {"qp": qp, "scores": kept_scores,
+                            "kp": {(b, g): kp_cache[(layer, b, g)][:ctx0[b] + i + 1 - w.window]
+                                   for (l_, b, g) in kp_cache if l_ == layer and b in seqs}}
             out = None
-            if want_attention:
+            if want_attention and (attn_steps is None or i in attn_steps):
                 Q = data.q(i, layer)
                 out = np.zeros((B, Hq, w.head_dim), np.float32)
-                for b in range(B):
+                for b in seqs:
                     T = ctx0[b] + i + 1
                     for h in heads:
                         g = h // grp
                         A = attention_set(T, w.sink, w.window, cur_idx[layer][b][h])
                         out[b, h] = attention(Q[b, h], K[b, g], V[b, g], A, scale)
             res[(i, layer)] = {"idx": cur_idx[layer], "out": out}
+            if keep and is_prediction_step(i, w.interval):
+                res[(i, layer)].update(kept)
         kp_cache.clear()
     return res

@@ -193,7 +193,7 @@ class SparseDecoder:
                       stream)
 
     # -------------------------------------------------------------- one step
-    def step(self, step: int, Q, out, h=None, qp_direct=None, stream=None, marks=None):
+    def step(self, step: int, Q, out, h=None, qp_direct=None, stream=None, marks=None, on_select=None):
         """One decode step over all layers.
 
         Q: [n_layers][batch][Hq][d] bf16; out: [n_layers][batch][Hq][d] fp32;
@@ -201,7 +201,9 @@ class SparseDecoder:
         qp_direct: [n_layers][batch][Hq][d'] fp32 (shapes without an MLP).
         The selection work of a prediction step is issued before the step's
         attention launches; `marks(name)` is called between the two groups so
-        a caller can bracket them with events."""
+        a caller can bracket them with events.  `on_select(layer)`, if given,
+        is called right after each layer's selection is issued (while the
+        selection workspace still holds that layer's scores)."""
         s = self.shape
         if step in self.proj_begin:
             for l in range(s.n_layers):
@@ -211,6 +213,8 @@ class SparseDecoder:
                 if s.hidden > 0 and l in self.qp:
                     self.predict(l, h[self.producers.index(l)], stream)
                 self.select(step, l, None if qp_direct is None else qp_direct[l], stream)
+                if on_select:
+                    on_select(l)
         if marks:
             marks("attn_begin")
         for l in range(s.n_layers):
