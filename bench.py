@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 import tb_inputs  # noqa: E402
 from query_aware_sparse_tb_b200 import _lib as L  # noqa: E402
 from query_aware_sparse_tb_b200.decode import (DecodeShape, SparseDecoder, is_prediction_step,  # noqa: E402
-                                              record_event)
+                                              kv_head_shard, record_event, shard_w2)
 
 HBM_NOMINAL_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -48,25 +48,40 @@ ROW_BYTES_PER_DIM = 2 * 2      # K and V, bf16
 # ----------------------------------------------------------------------------
 
 class Run:
-    """All device buffers of one workload replica plus its decoder."""
+    """All device buffers of one workload replica plus its decoder.  With
+    shard=(rank, world) the run holds only the KV heads (and their query heads)
+    that rank owns under KV-head sharding, sliced from the same seeded data."""
 
-    def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head"):
+    def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head",
+                 shard: tuple[int, int] | None = None):
         self.w = w
         self.device = device
         self.steps = steps or w.steps
         self.ctx0 = w.ctx0_per_seq()
         nL = w.n_layers
+        if shard is None:
+            kvh, qh = range(w.n_kv_heads), range(w.n_q_heads)
+        else:
+            kvh, qh = kv_head_shard(w.n_kv_heads, w.group, *shard)
+        self.kv_heads, self.q_heads = kvh, qh
+        self.Hkv, self.Hq = len(kvh), len(qh)
+        gs, hs = slice(kvh.start, kvh.stop), slice(qh.start, qh.stop)
         self.K, self.V, self.Wk = [], [], []
         for l in range(nL):
             K, V = tb_inputs.kv_layer(w, l, device)
-            self.K.append(K)
-            self.V.append(V)
-            self.Wk.append(tb_inputs.wk_layer(w, l, device))
+            self.K.append(K[:, gs].contiguous() if shard else K)
+            self.V.append(V[:, gs].contiguous() if shard else V)
+            self.Wk.append(tb_inputs.wk_layer(w, l, device)[gs].contiguous())
+            del K, V
         stride = w.producer_stride if w.hidden > 0 else 1
         self.producers = [l for l in range(nL) if l % stride == 0]
-        self.mlp = {p: tb_inputs.mlp_weights(w, p, device) for p in self.producers} if w.hidden > 0 else {}
-        self.Q = torch.stack([torch.stack([tb_inputs.query(w, i, l, device) for l in range(nL)])
-                              for i in range(self.steps)])                       # [steps][L][B][Hq][d]
+        self.mlp = {}
+        if w.hidden > 0:
+            for p in self.producers:
+                W1, W2 = tb_inputs.mlp_weights(w, p, device)
+                self.mlp[p] = (W1, shard_w2(W2, w.slots, w.n_q_heads, w.d_proj, qh) if shard else W2)
+        self.Q = torch.stack([torch.stack([tb_inputs.query(w, i, l, device)[:, hs] for l in range(nL)])
+                              for i in range(self.steps)]).contiguous()          # [steps][L][B][Hq][d]
         self.n_pred = (self.steps + w.interval - 1) // w.interval
         if w.hidden > 0:
             self.h = torch.stack([torch.stack([tb_inputs.hidden_state(w, k, p, device) for p in self.producers])
@@ -74,15 +89,16 @@ class Run:
             self.qp_direct = None
         else:
             self.h = None
-            self.qp_direct = torch.stack([torch.stack([tb_inputs.direct_qp(w, k, l, device) for l in range(nL)])
-                                          for k in range(self.n_pred)])          # [npred][L][B][Hq][d']
-        self.shape = DecodeShape(batch=w.batch, n_layers=nL, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+            self.qp_direct = torch.stack([torch.stack([tb_inputs.direct_qp(w, k, l, device)[:, hs]
+                                                       for l in range(nL)])
+                                          for k in range(self.n_pred)]).contiguous()  # [npred][L][B][Hq][d']
+        self.shape = DecodeShape(batch=w.batch, n_layers=nL, n_q_heads=self.Hq, n_kv_heads=self.Hkv,
                                  head_dim=w.head_dim, d_proj=w.d_proj, hidden=w.hidden, inter=w.inter,
                                  stride=stride, sink=w.sink, window=w.window, budget=w.budget, nbr=w.nbr,
                                  interval=w.interval, ctx_cap=w.ctx_cap)
         self.dec = SparseDecoder(self.shape, self.K, self.V, self.Wk, self.mlp, self.ctx0, self.steps, device,
                                  selection=selection)
-        self.out = torch.zeros(nL, w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=device)
+        self.out = torch.zeros(nL, w.batch, self.Hq, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):
         k = i // self.w.interval
@@ -128,14 +144,14 @@ class Run:
                 u = []
                 s_ = []
                 for l in range(w.n_layers):
-                    b = dec.bits[l].view(w.batch, w.n_kv_heads, w.group, -1)
+                    b = dec.bits[l].view(w.batch, self.Hkv, w.group, -1)
                     orb = b[:, :, 0] | b[:, :, 1] | b[:, :, 2] | b[:, :, 3]
                     u.append(lut[orb.contiguous().view(torch.uint8).long()].sum())
                     s_.append(dec.cnt[l].sum())
                 union = torch.stack(u).cpu()
                 isets = torch.stack(s_).cpu()
             T = [t + i + 1 for t in self.ctx0]
-            keep = sum(min(w.sink, t) + (t - max(w.sink, t - w.window)) for t in T) * w.n_kv_heads
+            keep = sum(min(w.sink, t) + (t - max(w.sink, t - w.window)) for t in T) * self.Hkv
             rows[i] = union + keep
             sel_sizes[i] = isets
             cand[i] = sum(max(0, t - w.window - w.sink) for t in T)
@@ -150,19 +166,20 @@ class Run:
         rows, sel_sizes, cand = self.union_rows()
         attn_rows = rows.sum().item()
         row_b = d * ROW_BYTES_PER_DIM
-        qo = self.steps * w.n_layers * w.batch * w.n_q_heads * d * (2 + 4)
+        qo = self.steps * w.n_layers * w.batch * self.Hq * d * (2 + 4)
         attn_bytes = attn_rows * row_b
         sel_bytes = 0
         for i in range(self.steps):
             if is_prediction_step(i, w.interval):
-                sel_bytes += w.n_layers * (w.n_kv_heads * cand[i].item() * dp * 2)
+                sel_bytes += w.n_layers * (self.Hkv * cand[i].item() * dp * 2)
                 sel_bytes += 4 * sel_sizes[i].sum().item()
         mlp_bytes = 0
         if w.hidden > 0:
-            mlp_bytes = self.n_pred * len(self.producers) * (w.inter * w.hidden + w.n_out * w.inter) * 2
-        proj_bytes = len(self.dec.proj_steps) * w.n_layers * w.batch * w.window * w.n_kv_heads * (d + dp) * 2
+            n_out = w.slots * self.Hq * w.d_proj
+            mlp_bytes = self.n_pred * len(self.producers) * (w.inter * w.hidden + n_out * w.inter) * 2
+        proj_bytes = len(self.dec.proj_steps) * w.n_layers * w.batch * w.window * self.Hkv * (d + dp) * 2
         sparse_total = attn_bytes + qo + sel_bytes + mlp_bytes + proj_bytes
-        dense_rows = sum(sum(t + i + 1 for t in self.ctx0) for i in range(self.steps)) * w.n_kv_heads * w.n_layers
+        dense_rows = sum(sum(t + i + 1 for t in self.ctx0) for i in range(self.steps)) * self.Hkv * w.n_layers
         dense_total = dense_rows * row_b + qo
         return dict(attn_bytes=attn_bytes, attn_rows=attn_rows, sparse_total=sparse_total, dense_total=dense_total,
                     dense_rows=dense_rows, sel_bytes=sel_bytes, mlp_bytes=mlp_bytes, proj_bytes=proj_bytes,
@@ -213,11 +230,11 @@ class E2E:
         nL = w.n_layers
         pos = [[t + i for t in run.ctx0] for i in range(run.steps)]     # new token position T-1
         q_el = run.Q[0].numel()
-        kv_el = nL * 2 * w.batch * w.n_kv_heads * w.head_dim
+        kv_el = nL * 2 * w.batch * run.Hkv * w.head_dim
         packed = torch.empty(run.steps, q_el + kv_el, dtype=torch.bfloat16)
         for i in range(run.steps):
             packed[i, :q_el] = run.Q[i].reshape(-1).cpu()
-            kv = torch.empty(nL, 2, w.batch, w.n_kv_heads, w.head_dim, dtype=torch.bfloat16)
+            kv = torch.empty(nL, 2, w.batch, run.Hkv, w.head_dim, dtype=torch.bfloat16)
             for l in range(nL):
                 for b in range(w.batch):
                     kv[l, 0, b] = run.K[l][b, :, pos[i][b]].cpu()
@@ -509,14 +526,16 @@ def cpu_baseline(w, budget_s=6.0):
                  "sample_seconds": round(time.perf_counter() - t0, 1)}, **host_info())
 
 
-def config_of(w: tb_inputs.Workload, decode_steps: int, world: int, selection: str = "head") -> dict:
+def config_of(w: tb_inputs.Workload, decode_steps: int, world: int, selection: str = "head",
+              sharded: bool = False) -> dict:
     """The workload description both arms print."""
     return {"workload": w.name, "batch": w.batch, "ctx": w.ctx0 if not w.ragged else [w.ctx0_lo, w.ctx0_hi],
             "layers": w.n_layers, "decode_steps_per_bench_step": decode_steps, "budget": w.budget,
             "interval": w.interval, "sink": w.sink, "window": w.window, "d_proj": w.d_proj,
             "selection": {"head": "per query head", "inclusive": "per query head, budget includes neighbours"}.get(
                 selection, f"per KV head ({selection})"),
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+            "parallelism": (f"kv-head shards x{world}" if sharded else f"replicas x{world}") if world > 1
+            else "single GPU"}
 
 
 def run_reference(args):
@@ -578,10 +597,14 @@ def run_reference(args):
 # main
 # ----------------------------------------------------------------------------
 
-def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup: int, selection: str):
+def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup: int, selection: str,
+            shard=None):
     """Time one workload's sparse run, dense run and (optionally) the e2e run,
-    each replayed as one CUDA graph; returns the figures the JSON line needs."""
-    run = Run(w, device, steps=args.decode_steps, selection=selection)
+    each replayed as one CUDA graph; returns the figures the JSON line needs.
+    With shard=(rank, world) this rank runs only its KV heads of the one
+    workload (strong scaling: the job's tokens are the workload's tokens)."""
+    run = Run(w, device, steps=args.decode_steps, selection=selection, shard=shard)
+    copies = 1 if shard else world          # independent replicas count every rank's tokens
     run.dec.prefill()
     torch.cuda.synchronize()
 
@@ -622,8 +645,8 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
     dense_launch_ms = sum(dense_attn_ms) / n_attn
     res = dict(
         run_steps=run.steps, tokens_per_run=tokens_per_run, acct=acct,
-        value=aggregate_rate(world, tokens_per_run, per_step_sparse),
-        dense_value=aggregate_rate(world, tokens_per_run, per_step_dense),
+        value=aggregate_rate(copies, tokens_per_run, per_step_sparse),
+        dense_value=aggregate_rate(copies, tokens_per_run, per_step_dense),
         per_step_sparse=per_step_sparse, per_step_dense=per_step_dense,
         attn_launch_ms=attn_launch_ms, attn_bytes_per_launch=acct["attn_bytes"] / n_attn,
         dense_launch_ms=dense_launch_ms, dense_bytes_per_launch=(acct["dense_total"] / n_attn),
@@ -633,7 +656,7 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
         kv_gb=2 * sum(k.numel() for k in run.K) * 2 / 1e9)
     if e2e is not None:
         h2d, d2h = e2e.bytes_per_run()
-        res["e2e"] = {"value": round(aggregate_rate(world, tokens_per_run, ms_e2e / steps), 3),
+        res["e2e"] = {"value": round(aggregate_rate(copies, tokens_per_run, ms_e2e / steps), 3),
                       "unit": "decode steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": round(ms_e2e / steps, 4), "clocks": clk_e2e}
     del g_sparse, g_dense, g_e2e, e2e, run
@@ -673,6 +696,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the extra workloads (batch16, long256k) timed after the headline one")
     ap.add_argument("--extra-steps", type=int, default=3, help="timed bench steps of each extra workload")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "kv_heads"],
+                    help="with N > 1 ranks: replicas (each rank decodes its own seeded replica; weak scaling) or "
+                         "kv_heads (the ranks split one workload's KV heads; strong scaling)")
     ap.add_argument("--selection", default="head", choices=list(SparseDecoder.SELECTIONS),
                     help="head: one importance set per query head (the default, the pages' reading); "
                          "group_max / group_sum: one set per KV head (the group-shared variant); "
@@ -694,8 +720,12 @@ def main():
                                              device_id=torch.device(device))
     L.load()
 
+    sharded = args.shard == "kv_heads"
+    shard = (rank, world) if sharded else None
+
     def prepare(name):
-        w = replica(tb_inputs.WORKLOADS[name], rank)          # an independent replica per rank
+        # an independent replica per rank, or one workload split by KV heads
+        w = tb_inputs.WORKLOADS[name] if sharded else replica(tb_inputs.WORKLOADS[name], rank)
         if args.layers:
             w = w.scaled(n_layers=args.layers)
         if args.interval:
@@ -703,14 +733,14 @@ def main():
         return w
 
     w = prepare(args.workload)
-    r = measure(w, args, device, dist_on, world, not args.no_e2e, args.steps, args.warmup, args.selection)
+    r = measure(w, args, device, dist_on, world, not args.no_e2e, args.steps, args.warmup, args.selection, shard)
     extras = {}
     if not args.no_extra and args.workload == "llama64k" and not args.layers and not args.decode_steps:
         # the other two large workloads, each against the dense kernel on its own cache
         for name in ("long256k", "batch16"):
             wx = prepare(name)
             extras[name] = summary(wx, measure(wx, args, device, dist_on, world, False, args.extra_steps,
-                                               max(3, args.warmup), args.selection), measured_peaks()[0])
+                                               max(3, args.warmup), args.selection, shard), measured_peaks()[0])
 
     peak, peak_kind = measured_peaks()
     acct = r["acct"]
@@ -724,9 +754,9 @@ def main():
     line = {
         "metric": "sparse decode steps/s", "value": round(r["value"], 3), "unit": "decode steps/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["per_step_sparse"], 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; Llama-3.1-8B attention shapes, random weights)",
-        "config": dict(config_of(w, r["run_steps"], world, args.selection),
+        "config": dict(config_of(w, r["run_steps"], world, args.selection, sharded),
                        l2="inputs larger than L2 (KV %.1f GB)" % r["kv_gb"],
                        graph="one CUDA graph per bench step"),
         "speedup_vs_dense": round(r["value"] / r["dense_value"], 4),

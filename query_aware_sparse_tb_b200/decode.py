@@ -62,6 +62,45 @@ def projection_schedule(ctx0: list[int], window: int, steps: int):
     return prefill, events
 
 
+# --------------------------------------------------------------- KV-head sharding
+#
+# Tensor-parallel placement of the path: rank r of `world` owns a contiguous
+# block of KV heads and the query heads of their GQA groups, with those heads'
+# K, V, K' and W_k, and the rows of the predictor's second matrix that emit
+# their queries (the first matrix is replicated: every rank needs the whole
+# activation).  Projection, prediction, scoring, selection and attention are
+# independent per head, so a rank runs the unchanged entry points on its slice
+# and nothing crosses ranks on the way; the heads' outputs meet again only in
+# the model's output projection (a TP all-reduce outside this path), or in an
+# all-gather when the full [batch][Hq][d] output is wanted on every rank.
+
+def kv_head_shard(n_kv_heads: int, group: int, rank: int, world: int) -> tuple[range, range]:
+    """(KV heads, query heads) owned by `rank` of `world`: contiguous blocks."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside a world of {world}")
+    if n_kv_heads % world:
+        raise ValueError(f"{n_kv_heads} KV heads do not split over {world} ranks")
+    per = n_kv_heads // world
+    g0 = rank * per
+    return range(g0, g0 + per), range(g0 * group, (g0 + per) * group)
+
+
+def shard_w2(W2, slots: int, n_q_heads: int, d_proj: int, heads: range):
+    """Rows of the predictor's second matrix W2 [slots*Hq*d'][inter] that emit
+    the queries of `heads`, for every slot, in the [slot][head][d'] order of a
+    predictor whose output has len(heads) heads."""
+    inter = W2.shape[-1]
+    return W2.reshape(slots, n_q_heads, d_proj, inter)[:, heads.start:heads.stop].reshape(-1, inter).contiguous()
+
+
+def gather_head_outputs(parts, heads_of_rank):
+    """Reassemble [..][batch][Hq][d] from the ranks' [..][batch][Hq_local][d]
+    outputs (parts[r] holds rank r's query heads heads_of_rank[r])."""
+    import torch
+    order = sorted(range(len(parts)), key=lambda r: heads_of_rank[r].start)
+    return torch.cat([parts[r] for r in order], dim=-2)
+
+
 @dataclass(frozen=True)
 class DecodeShape:
     batch: int
