@@ -35,8 +35,8 @@ if ROOT not in sys.path:
 
 import tb_inputs  # noqa: E402
 from query_aware_sparse_tb_b200 import _lib as L  # noqa: E402
-from query_aware_sparse_tb_b200.decode import (DecodeShape, SparseDecoder, is_prediction_step,  # noqa: E402
-                                              kv_head_shard, record_event, shard_w2)
+from query_aware_sparse_tb_b200.decode import (DecodeShape, OffloadDecoder, SparseDecoder,  # noqa: E402
+                                              is_prediction_step, kv_head_shard, record_event, shard_w2)
 
 HBM_NOMINAL_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -53,7 +53,7 @@ class Run:
     that rank owns under KV-head sharding, sliced from the same seeded data."""
 
     def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head",
-                 shard: tuple[int, int] | None = None):
+                 shard: tuple[int, int] | None = None, offload: bool = False):
         self.w = w
         self.device = device
         self.steps = steps or w.steps
@@ -96,8 +96,9 @@ class Run:
                                  head_dim=w.head_dim, d_proj=w.d_proj, hidden=w.hidden, inter=w.inter,
                                  stride=stride, sink=w.sink, window=w.window, budget=w.budget, nbr=w.nbr,
                                  interval=w.interval, ctx_cap=w.ctx_cap)
-        self.dec = SparseDecoder(self.shape, self.K, self.V, self.Wk, self.mlp, self.ctx0, self.steps, device,
-                                 selection=selection)
+        cls = OffloadDecoder if offload else SparseDecoder
+        self.dec = cls(self.shape, list(self.K), list(self.V), self.Wk, self.mlp, self.ctx0, self.steps, device,
+                       selection=selection)
         self.out = torch.zeros(nL, w.batch, self.Hq, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):
@@ -665,6 +666,62 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
     return res
 
 
+def measure_offload(w, args, device, selection: str):
+    """Per-token decode latency with the KV cache in pinned host memory (the
+    CPU-offloading workload): the sparse path against dense attention over the
+    same host cache.  The prediction step, a reuse step, a projection step and
+    a dense step are each captured as a graph and timed apart; the sparse
+    per-token latency amortises prediction over the interval and projection
+    over its N-token batch."""
+    N, P = w.window, w.interval
+    steps = max(P, N)                                       # the first projection batch falls at step < N
+    run = Run(w, device, steps=steps, selection=selection, offload=True)
+    run.dec.prefill()
+    torch.cuda.synchronize()
+    t_off = time.perf_counter()
+    run.dec.offload()
+    run.K = run.V = None
+    torch.cuda.empty_cache()
+    t_off = time.perf_counter() - t_off
+    proj_step = run.dec.proj_steps[0] if run.dec.proj_steps else None
+    stream = torch.cuda.Stream(device=device)
+
+    def one(i, dense=False):
+        Q, h, qd = run.step_inputs(i)
+        if dense:
+            return capture(lambda st: run.dec.dense_step(i, Q, run.out, stream=st), stream)
+        return capture(lambda st: run.dec.step(i, Q, run.out, h=h, qp_direct=qd, stream=st), stream)
+
+    for i in range(steps):                                  # eager pass: every kernel warmed, sets in place
+        Q, h, qd = run.step_inputs(i)
+        run.dec.step(i, Q, run.out, h=h, qp_direct=qd)
+    torch.cuda.synchronize()
+    graphs = {"pred": one(0), "reuse": one(1), "dense": one(1, dense=True)}
+    if proj_step is not None and not is_prediction_step(proj_step, P):
+        graphs["proj"] = one(proj_step)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    ms = {k: time_graph(g, max(3, args.warmup), args.extra_steps, False, device) / args.extra_steps
+          for k, g in graphs.items()}
+    clk = clocks.stop()
+    flags = L.workspace_check(run.dec.ws_attn) | L.workspace_check(run.dec.ws_sel) | L.workspace_check(run.dec.ws_proj)
+    sparse_ms = (ms["pred"] + (P - 1) * ms["reuse"]) / P + ((ms["proj"] - ms["reuse"]) / N if "proj" in ms else 0.0)
+    host_gb = sum(hb.nbytes for hb in run.dec.K_host + run.dec.V_host) / 1e9
+    res = {"workload": w.name, "per_token_ms": round(sparse_ms, 3), "dense_per_token_ms": round(ms["dense"], 3),
+           "speedup_vs_dense": round(ms["dense"] / sparse_ms, 3),
+           "step_ms": {k: round(v, 3) for k, v in ms.items()},
+           "host_kv_gb": round(host_gb, 2), "offload_s": round(t_off, 1), "clocks": clk, "device_flags": flags,
+           "note": ("K and V in pinned host memory read by the attention kernels across the host link; K', "
+                    "the predictor, scoring and selection on the device; per-token = (prediction step + "
+                    f"{P - 1} reuse steps)/{P} + (projection step - reuse step)/{N}")}
+    for hb in run.dec.K_host + run.dec.V_host:
+        hb.free()
+    del graphs, run
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
 def summary(w, r, peak):
     """The compact per-workload figures of the extra workloads."""
     achieved = r["attn_bytes_per_launch"] / (r["attn_launch_ms"] / 1000.0) / 1e9
@@ -696,6 +753,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the extra workloads (batch16, long256k) timed after the headline one")
     ap.add_argument("--extra-steps", type=int, default=3, help="timed bench steps of each extra workload")
+    ap.add_argument("--offload", action="store_true",
+                    help="also time the CPU-offloaded KV cache on long256k (per-token latency against dense)")
+    ap.add_argument("--offload-only", action="store_true", help="time only the CPU-offloaded workload")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "kv_heads"],
                     help="with N > 1 ranks: replicas (each rank decodes its own seeded replica; weak scaling) or "
                          "kv_heads (the ranks split one workload's KV heads; strong scaling)")
@@ -732,6 +792,9 @@ def main():
             w = w.scaled(interval=args.interval)
         return w
 
+    if args.offload_only:
+        print(json.dumps({"offload": measure_offload(prepare("long256k"), args, device, args.selection)}))
+        return 0
     w = prepare(args.workload)
     r = measure(w, args, device, dist_on, world, not args.no_e2e, args.steps, args.warmup, args.selection, shard)
     extras = {}
@@ -742,6 +805,7 @@ def main():
             extras[name] = summary(wx, measure(wx, args, device, dist_on, world, False, args.extra_steps,
                                                max(3, args.warmup), args.selection, shard), measured_peaks()[0])
 
+    offload = measure_offload(prepare("long256k"), args, device, args.selection) if args.offload else None
     peak, peak_kind = measured_peaks()
     acct = r["acct"]
     achieved = r["attn_bytes_per_launch"] / (r["attn_launch_ms"] / 1000.0) / 1e9
@@ -783,6 +847,8 @@ def main():
         line["e2e"] = r["e2e"]
     if extras:
         line["workloads"] = extras
+    if offload:
+        line["offload"] = offload
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))

@@ -128,7 +128,8 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             const uint16_t *__restrict__ V, const int32_t *__restrict__ ctx_len,
             const uint32_t *__restrict__ sel_bits, int Hq, int Hkv, int Tcap, int W, int sink,
             int window, float qscale, int splits, float *__restrict__ part,
-            uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags) {
+            uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags,
+            int early_trigger) {
     constexpr int CPR = D / 8;      // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;   // rows per warp-wide copy instruction
     constexpr int kKSteps = D / 16; // MMA K steps of S^T
@@ -167,6 +168,36 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     // that a CTA's first positions are known before the length arrives
     const int chunk = ((Tcap + splits - 1) / splits + kRows - 1) / kRows * kRows;
     const int p_begin = split * chunk;
+
+    // ------------------------------------------------------------ set-up
+    // (touches only this CTA's shared memory and TMEM, so under a programmatic
+    // launch it overlaps the end of the previous kernel in the stream)
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full(s), kRoleThreads);
+            mbar_init(empty(s), 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(s_done(q), 1);
+            mbar_init(p_ready(q), kRoleThreads);
+            mbar_init(o_done(q), 1);
+            mbar_init(o_free(q), kRoleThreads);
+        }
+        mbar_init(drain, 2);
+        mbar_init(q_ready, kRoleThreads);
+        misc[kMiscAbort] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8) {  // the S-issue warp owns the TMEM allocation
+        tmem_alloc(sb + Smem::kMisc + 4 * kMiscTmem, kTmemCols);
+        tmem_relinquish();
+    }
+    // every input and the workspace may be written by the previous kernel
+    griddep_wait();
+    // a one-wave grid lets the next kernel's CTAs take the SMs it leaves idle
+    // and the ones its CTAs free; a longer grid only once this CTA is done
+    if (early_trigger) griddep_launch_dependents();
+
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
     const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
     const int p_end = min(p_begin + chunk, T);
@@ -194,27 +225,6 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     };
     if (SPARSE && loader) fetch_words(p_begin);
 
-    // ------------------------------------------------------------ set-up
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(full(s), kRoleThreads);
-            mbar_init(empty(s), 1);
-        }
-        for (int q = 0; q < 2; ++q) {
-            mbar_init(s_done(q), 1);
-            mbar_init(p_ready(q), kRoleThreads);
-            mbar_init(o_done(q), 1);
-            mbar_init(o_free(q), kRoleThreads);
-        }
-        mbar_init(drain, 2);
-        mbar_init(q_ready, kRoleThreads);
-        misc[kMiscAbort] = 0;
-        fence_mbar_init();
-    }
-    if (warp == 8) {  // the S-issue warp owns the TMEM allocation
-        tmem_alloc(sb + Smem::kMisc + 4 * kMiscTmem, kTmemCols);
-        tmem_relinquish();
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -542,6 +552,7 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     }
 
     // ---------------------------------------------------- release, ticket
+    if (!early_trigger) griddep_launch_dependents();
     __threadfence();
     tc_fence_before();
     __syncthreads();
@@ -628,11 +639,22 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
         w + kWsHeaderBytes + align_up((size_t)d.batch * d.n_kv_heads * 4, 256));
     const int W = (d.ctx_cap + 31) / 32;
     const float qscale = scale * 1.4426950408889634f;  // logits in log2 units for exp2
-    dim3 grid(splits, d.n_kv_heads, d.batch);
-    attn_kernel<D, SPARSE><<<grid, kThreads, Smem::kBytes, st>>>(
-        Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, qscale,
-        splits, part, counters, out, flags);
-    return cudaGetLastError();
+    // programmatic stream serialization: the launch may begin while the
+    // previous kernel in the stream finishes; the kernel waits for it
+    // (griddep_wait) before its first global read
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, d.n_kv_heads, d.batch);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Smem::kBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int early = (long long)splits * d.n_kv_heads * d.batch <= num_sms() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, attn_kernel<D, SPARSE>, Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads,
+                              d.ctx_cap, W, sink, window, qscale, splits, part, counters, out, flags, early);
 }
 
 }  // namespace

@@ -291,6 +291,20 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
+// ------------------------------------------- programmatic dependent launch ----
+
+// Wait until every grid this one depends on through a programmatic launch
+// edge has completed and its memory operations are visible; returns at once
+// when the grid was launched without that attribute.  A kernel launched with
+// programmatic stream serialization calls this before its first access to
+// memory an earlier kernel may write.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+// Let the next grid in the stream (if launched with programmatic stream
+// serialization) be scheduled before this one has finished.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ------------------------------------------------------ named barriers ----
 
 // Barrier `id` over `n` threads (whole warps) that also returns whether any of

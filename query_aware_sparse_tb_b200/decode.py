@@ -175,6 +175,7 @@ class SparseDecoder:
         self.ctx = torch.tensor([[t + i + 1 for t in ctx0] for i in range(steps)], dtype=torch.int32,
                                 device=device)
         prefill, events = projection_schedule(self.ctx0, s.window, steps)
+        self.proj_events = events
         self.prefill_len = prefill
         self.proj_steps = sorted(events)
         self.proj_begin = {i: torch.tensor(events[i], dtype=torch.int32, device=device) for i in events}
@@ -270,18 +271,134 @@ class SparseDecoder:
             marks("attn_end")
 
 
+# ------------------------------------------------------------------ offloaded KV
+
+class HostBuffer:
+    """Pinned host memory mapped into the device's address space, so kernels
+    read and write it directly across the host link.  `dev_ptr` is the address
+    to hand the library; `tensor` is a CPU tensor view of the same bytes."""
+
+    PORTABLE, MAPPED = 1, 2
+
+    def __init__(self, shape, dtype=torch.bfloat16):
+        rt = _rt()
+        self.shape, self.dtype = tuple(shape), dtype
+        nbytes = math.prod(self.shape) * torch.empty(0, dtype=dtype).element_size()
+        p = ctypes.c_void_p()
+        err = rt.cudaHostAlloc(ctypes.byref(p), ctypes.c_size_t(nbytes), self.PORTABLE | self.MAPPED)
+        if err != 0 or not p.value:
+            raise RuntimeError(f"cudaHostAlloc of {nbytes} bytes failed ({err})")
+        self.ptr = p.value
+        dp = ctypes.c_void_p()
+        err = rt.cudaHostGetDevicePointer(ctypes.byref(dp), ctypes.c_void_p(self.ptr), 0)
+        if err != 0 or not dp.value:
+            rt.cudaFreeHost(ctypes.c_void_p(self.ptr))
+            raise RuntimeError(f"cudaHostGetDevicePointer failed ({err}): host memory is not mapped")
+        self.dev_ptr = dp.value
+        self._raw = (ctypes.c_uint8 * nbytes).from_address(self.ptr)
+        self.tensor = torch.frombuffer(self._raw, dtype=torch.uint8).view(dtype).view(self.shape)
+        self.nbytes = nbytes
+
+    def free(self):
+        if getattr(self, "ptr", None):
+            self.tensor = None
+            self._raw = None
+            _rt().cudaFreeHost(ctypes.c_void_p(self.ptr))
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def memcpy2d(dst: int, dpitch: int, src: int, spitch: int, width: int, height: int, stream) -> None:
+    """cudaMemcpy2DAsync with the copy direction inferred from the addresses."""
+    err = _rt().cudaMemcpy2DAsync(ctypes.c_void_p(dst), ctypes.c_size_t(dpitch), ctypes.c_void_p(src),
+                                  ctypes.c_size_t(spitch), ctypes.c_size_t(width), ctypes.c_size_t(height), 4,
+                                  ctypes.c_void_p(L._stream(stream)))
+    if err != 0:
+        raise RuntimeError(f"cudaMemcpy2DAsync failed ({err})")
+
+
+class OffloadDecoder(SparseDecoder):
+    """The sparse path with the KV cache in host memory: the CPU-offloading
+    workload of the TokenButler summaries ("Contributions" (CPU offloading) and
+    "Results" (latency at 256K+ tokens)).  The projected keys, and with them
+    scoring and selection, the predictor and the queries stay on the device;
+    the attention entry points are given host-mapped K and V, so only the kept
+    rows cross the host link, read by the kernels themselves.  Construct with
+    device K and V, project the prefill, then offload(): the caches move to
+    pinned host memory and the device copies are dropped.  A batch of N new keys
+    is projected from a device staging copy of its rows (the projection reads
+    K through tensor maps over device memory)."""
+
+    def offload(self):
+        s = self.shape
+        self.K_host, self.V_host = [], []
+        for l in range(s.n_layers):
+            for src, dst in ((self.K, self.K_host), (self.V, self.V_host)):
+                hb = HostBuffer(src[l].shape)
+                hb.tensor.copy_(src[l])
+                dst.append(hb)
+                src[l] = None
+        self.K = [hb.dev_ptr for hb in self.K_host]
+        self.V = [hb.dev_ptr for hb in self.V_host]
+        torch.cuda.empty_cache()
+        B, Hq, Hkv, N = s.batch, s.n_q_heads, s.n_kv_heads, s.window
+        self.stage_dims = L.dims(B, Hq, Hkv, s.head_dim, s.d_proj, N)
+        self.K_stage = torch.zeros(B, Hkv, N, s.head_dim, dtype=torch.bfloat16, device=self.device)
+        self.Kp_stage = torch.zeros(B, Hkv, N, s.d_proj, dtype=torch.bfloat16, device=self.device)
+        self.stage_begin = {i: torch.tensor([0 if x >= 0 else -1 for x in ev], dtype=torch.int32, device=self.device)
+                            for i, ev in self.proj_events.items()}
+
+    @property
+    def offloaded(self) -> bool:
+        return hasattr(self, "K_host")
+
+    def project(self, step: int, layer: int, stream=None):
+        if not self.offloaded:
+            return super().project(step, layer, stream)
+        if step not in self.proj_begin:
+            return
+        s = self.shape
+        Hkv, N, d, dp, cap = s.n_kv_heads, s.window, s.head_dim, s.d_proj, s.ctx_cap
+        begins = self.proj_events[step]
+        for b, t0 in enumerate(begins):
+            if t0 >= 0:   # rows [t0, t0+N) of every KV head of sequence b -> stage
+                memcpy2d(self.K_stage[b].data_ptr(), N * d * 2, self.K_host[layer].ptr + (b * Hkv * cap + t0) * d * 2,
+                         cap * d * 2, N * d * 2, Hkv, stream)
+        L.project_keys(self.stage_dims, self.K_stage, self.Wk[layer], self.Kp_stage, self.stage_begin[step],
+                       self.proj_count[step], N, self.ws_proj, stream)
+        for b, t0 in enumerate(begins):
+            if t0 >= 0:   # stage -> K' rows [t0, t0+N)
+                memcpy2d(self.Kp[layer].data_ptr() + (b * Hkv * cap + t0) * dp * 2, cap * dp * 2,
+                         self.Kp_stage[b].data_ptr(), N * dp * 2, N * dp * 2, Hkv, stream)
+
+
 # ------------------------------------------------------------------ events
 
 _cudart = None
 
 
 def _rt():
-    """The CUDA runtime torch already loaded (for external event records)."""
+    """The CUDA runtime torch already loaded (event records, pinned host
+    memory, strided copies)."""
     global _cudart
     if _cudart is None:
         _cudart = ctypes.CDLL("libcudart.so.12")
-        _cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        P, sz = ctypes.c_void_p, ctypes.c_size_t
+        _cudart.cudaEventRecordWithFlags.argtypes = [P, P, ctypes.c_uint]
         _cudart.cudaEventRecordWithFlags.restype = ctypes.c_int
+        _cudart.cudaHostAlloc.argtypes = [ctypes.POINTER(P), sz, ctypes.c_uint]
+        _cudart.cudaHostAlloc.restype = ctypes.c_int
+        _cudart.cudaHostGetDevicePointer.argtypes = [ctypes.POINTER(P), P, ctypes.c_uint]
+        _cudart.cudaHostGetDevicePointer.restype = ctypes.c_int
+        _cudart.cudaFreeHost.argtypes = [P]
+        _cudart.cudaFreeHost.restype = ctypes.c_int
+        _cudart.cudaMemcpy2DAsync.argtypes = [P, sz, P, sz, sz, sz, ctypes.c_int, P]
+        _cudart.cudaMemcpy2DAsync.restype = ctypes.c_int
     return _cudart
 
 

@@ -36,6 +36,15 @@ from query_aware_sparse_tb_b200.decode import is_prediction_step, producer_layer
 DEV = "cuda"
 
 
+def host_kv(run, l):
+    """Layer l's K and V as host bf16 bits, from the device or, for an
+    offloaded run, from its pinned host cache."""
+    dec = run.dec
+    if getattr(dec, "offloaded", False):
+        return parity.bits16(dec.K_host[l].tensor), parity.bits16(dec.V_host[l].tensor)
+    return parity.bits16(dec.K[l]), parity.bits16(dec.V[l])
+
+
 class RunData:
     """Host copies (numpy, bf16 as uint16) of a bench.Run's device inputs, in
     the form oracle/schedule.py reads them."""
@@ -44,7 +53,7 @@ class RunData:
         self.run = run
 
     def kv(self, l):
-        return parity.bits16(self.run.K[l]), parity.bits16(self.run.V[l])
+        return host_kv(self.run, l)
 
     def wk(self, l):
         return parity.bits16(self.run.Wk[l])
@@ -99,7 +108,11 @@ def check_schedule(run, layers, steps, seqs, heads, attn_steps, selection="head"
     ref = oschedule.run(w, data, layers=layers, steps=steps, heads=heads, seqs=seqs, attn_steps=set(attn_steps),
                         selection=selection, keep=True)
     groups = sorted({hh // w.group for hh in heads})
-    K_host = {(l, b, g): parity.bits16(run.K[l][b, g]) for l in layers for b in seqs for g in groups}
+    K_host = {}
+    for l in layers:
+        Kl = host_kv(run, l)[0]
+        K_host.update({(l, b, g): Kl[b, g].copy() for b in seqs for g in groups})
+        del Kl
     Wk_host = {l: parity.bits16(run.Wk[l]) for l in layers}
     dm = dec.dims
     scores = torch.empty(w.batch, w.n_q_heads, w.ctx_cap, dtype=torch.float32, device=DEV)
@@ -212,7 +225,7 @@ def check_schedule(run, layers, steps, seqs, heads, attn_steps, selection="head"
                         for hh in heads:
                             sets[b][hh] = R["idx"][b][hh]
                     bits = torch.from_numpy(parity.pack_sets(sets, s_.words).view(np.int32)).to(DEV)
-                    tb.sparse_decode_attn(dm, Q[l], run.K[l], run.V[l], dec.ctx[i], S, N, bits, scale, out2,
+                    tb.sparse_decode_attn(dm, Q[l], dec.K[l], dec.V[l], dec.ctx[i], S, N, bits, scale, out2,
                                           dec.ws_attn)
                     torch.cuda.synchronize()
                     assert tb.workspace_check(dec.ws_attn) == 0
