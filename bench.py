@@ -97,8 +97,10 @@ class Run:
                                  stride=stride, sink=w.sink, window=w.window, budget=w.budget, nbr=w.nbr,
                                  interval=w.interval, ctx_cap=w.ctx_cap)
         cls = OffloadDecoder if offload else SparseDecoder
+        # the bench's streams run only libtb's kernels, the K/V append of the
+        # e2e loop and copies, so every attention launch may prefetch its rows
         self.dec = cls(self.shape, list(self.K), list(self.V), self.Wk, self.mlp, self.ctx0, self.steps, device,
-                       selection=selection)
+                       selection=selection, prefetch_kv=True)
         self.out = torch.zeros(nL, w.batch, self.Hq, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):

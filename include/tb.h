@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 6
+#define TB_ABI_VERSION 8
 
 typedef uint16_t tb_bf16;
 
@@ -228,6 +228,71 @@ tb_status tb_score_select_inclusive(const tb_dims *dims, const float *qp, int64_
 tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_bytes, const int32_t *ctx_len,
                                  int32_t sink, int32_t window, float *scores, void *stream);
 
+/* ---- context-parallel selection and attention ----------------------------- */
+/* One sequence's context split over R ranks (each holds the K, V and K' rows
+ * of a block of positions): the scale-out the survey of this path proposes
+ * for contexts past 256K tokens.  No counterpart on the pages, which run on
+ * one device; the result is the single-device result:
+ *   1. each rank runs tb_score_select (nbr = 0) on its block, with the block's
+ *      part of C as its candidates, so its set is exactly its local top-B;
+ *   2. tb_select_export_candidates turns that set into composites
+ *      (key << 32) | (0xFFFFFFFF - global position), key being the score's
+ *      order-preserving image, which rank first in the (score desc, position
+ *      asc) order; the ranks exchange them (an all-gather);
+ *   3. tb_select_merge_candidates takes the top-B of all ranks' composites
+ *      (every member of the global top-B is in its block's local top-B),
+ *      applies the neighbour fetch and the clip to C on global positions, and
+ *      gives each rank the rows of its block that the attention keeps;
+ *   4. tb_sparse_decode_attn_partial attends over exactly those rows and
+ *      returns each head's unnormalised softmax state; the ranks exchange
+ *      them and tb_attn_combine merges them into the output.
+ * Only per-head selection is supported (not the group-shared variant). */
+
+/* Step 2.  For each (sequence b, query head h) of a rank's selection (dims,
+ * ws and the idx/count it wrote, with nbr = 0), write its first
+ * min(count[b][h], budget) positions p as composites of their score key and
+ * p + pos_offset (the block's first global position):
+ *   cand  [batch][Hq][budget] uint64 (device, 8-byte aligned); unused slots 0 */
+tb_status tb_select_export_candidates(const tb_dims *dims, const void *ws, size_t ws_bytes, const int32_t *idx,
+                                      int32_t idx_cap, const int32_t *count, int32_t budget, int32_t pos_offset,
+                                      uint64_t *cand, void *stream);
+
+/* Step 3, on every rank.  dims are the global shapes (ctx_cap = the global
+ * capacity, a multiple of 32 is not needed); cand holds all ranks' exports,
+ * [n_ranks][batch][Hq][budget].  With T = ctx_len[b] (global), C = [sink,
+ * T - window):
+ *   Top = the `budget` composites of (b, h) that rank first among those whose
+ *         position lies in C (all of them if there are fewer)
+ *   I   = ( ∪_{t in Top} [t - nbr, t + nbr] ) ∩ C         (global positions)
+ *   idx [batch][Hq][idx_cap], count [batch][Hq]: I sorted, as tb_score_select
+ *   local_bits [batch][Hq][ceil(local_cap/32)] uint32: bit t - shard_begin set
+ *         for t in (sink ∪ window ∪ I) ∩ [shard_begin, shard_begin + shard_len)
+ *         ∩ [0, T) (the rows this rank's partial attention reads)
+ * shard_begin must be a multiple of 32; ws >= 256 bytes holds the flag word
+ * (TB_FLAG_IDX_OVERFLOW, TB_FLAG_CTX_RANGE). */
+tb_status tb_select_merge_candidates(const tb_dims *dims, const uint64_t *cand, int32_t n_ranks, int32_t budget,
+                                     const int32_t *ctx_len, int32_t sink, int32_t window, int32_t nbr,
+                                     int32_t *idx, int32_t idx_cap, int32_t *count, int32_t shard_begin,
+                                     int32_t shard_len, int32_t local_cap, uint32_t *local_bits, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/* Step 4a.  The attention of tb_sparse_decode_attn over exactly the rows
+ * whose bit is set (no sink or window of its own), rows[b] being the number
+ * of valid rows of sequence b in this rank's cache (1 <= rows[b] <= ctx_cap),
+ * returning per (b, h) the unnormalised state in log2 units:
+ *   part[b][h][0..d)  = sum_t 2^(l_t - M) v_t,  part[b][h][d] = M = max_t l_t,
+ *   part[b][h][d + 1] = sum_t 2^(l_t - M),      l_t = scale * log2(e) * q.k_t
+ * (M = -inf and zeros when no row is kept).  part: [batch][Hq][d + 2] float. */
+tb_status tb_sparse_decode_attn_partial(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
+                                        const int32_t *rows, const uint32_t *bits, float scale, float *part,
+                                        void *ws, size_t ws_bytes, void *stream);
+
+/* Step 4b.  out[b][h] = sum_p 2^(M_p - M*) o_p / sum_p 2^(M_p - M*) L_p over
+ * n_parts states parts[p][b][h] (tb_sparse_decode_attn_partial's layout),
+ * M* = max_p M_p; 0 when every part is empty.  out: [batch][Hq][head_dim]. */
+tb_status tb_attn_combine(const float *parts, int32_t n_parts, int32_t batch, int32_t n_q_heads, int32_t head_dim,
+                          float *out, void *stream);
+
 /* Build the sel_bits bitmap from index lists that came from elsewhere (e.g. a
  * host-side selection): bit t of row (b,h) is set iff t is among
  * idx[b][h][0 .. count[b][h]).  Entries outside [0, ctx_cap) are ignored. */
@@ -286,6 +351,41 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
                                 const tb_bf16 *V, const int32_t *ctx_len, int32_t sink,
                                 int32_t window, const uint32_t *sel_bits, float scale,
                                 float *out, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- attention launch mode ------------------------------------------------ */
+/* How the attention entry points (tb_sparse_decode_attn, tb_decode_attn,
+ * tb_sparse_decode_attn_noalloc) order their reads against the kernel that
+ * precedes them in the stream.  Every libtb kernel is launched with
+ * programmatic stream serialization, so its CTAs may start while that kernel
+ * is still finishing.  No counterpart on the pages: a launch option.
+ *
+ *   TB_ATTN_WAIT_ALL     (default) nothing in global memory is touched before
+ *                        the preceding kernel has completed.
+ *   TB_ATTN_PREFETCH_KV  ctx_len, sel_bits and the K and V rows below
+ *                        ctx_len[b] - 1 are read (and the first tiles of K/V
+ *                        streamed into shared memory) as soon as the kernel
+ *                        is resident; Q, row ctx_len[b] - 1, out and the
+ *                        workspace only after the preceding kernel has
+ *                        completed.  Valid only when no kernel that may still
+ *                        be running writes ctx_len, sel_bits or those K/V
+ *                        rows: the kernel that immediately precedes the call
+ *                        in its stream (a decode loop's Q/K/V projection
+ *                        writes Q and row ctx_len[b] - 1 only, which is
+ *                        allowed), and, if that kernel lets its own
+ *                        dependents start before it has waited for its
+ *                        predecessor, that predecessor too (libtb's kernels
+ *                        never do).  The reads of the next tiles then overlap
+ *                        the end of the preceding kernel.  A preceding kernel
+ *                        that runs longer than about 2 s makes the bounded
+ *                        waits give up (TB_FLAG_TIMEOUT).
+ *
+ * The mode belongs to the calling thread and is read when an attention call
+ * launches (a graph captures it with the launch).  Any other value is
+ * TB_ERR_INVALID_ARG. */
+#define TB_ATTN_WAIT_ALL 0
+#define TB_ATTN_PREFETCH_KV 1
+tb_status tb_attn_set_launch_mode(int32_t mode);
+int32_t   tb_attn_launch_mode(void);
 
 /* ---- dense decode attention (comparator) ---------------------------------- */
 /* The same computation over A = [0, T): the dense attention baseline the

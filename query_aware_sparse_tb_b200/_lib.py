@@ -15,10 +15,11 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtb.so")
 
-TB_ABI_VERSION = 6
+TB_ABI_VERSION = 8
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
 TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW, TB_FLAG_BAD_CACHE = 0x1, 0x2, 0x4, 0x8
 TB_GROUP_REDUCE = {"max": 0, "sum": 1}
+TB_ATTN_WAIT_ALL, TB_ATTN_PREFETCH_KV = 0, 1
 
 EXPORTS = [
     "tb_abi_version", "tb_status_str", "tb_last_error",
@@ -27,8 +28,9 @@ EXPORTS = [
     "tb_workspace_init", "tb_workspace_check",
     "tb_project_keys", "tb_predict_queries", "tb_score_select", "tb_score_select_group", "tb_score_select_inclusive",
     "tb_score_select_scores", "tb_select_bits_from_idx",
+    "tb_select_export_candidates", "tb_select_merge_candidates", "tb_sparse_decode_attn_partial", "tb_attn_combine",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
-    "tb_selftest_bounded_wait",
+    "tb_selftest_bounded_wait", "tb_attn_set_launch_mode", "tb_attn_launch_mode",
 ]
 
 
@@ -75,11 +77,18 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_score_select_inclusive": ([D, P, i64, P, P, i32, i32, i32, i32, P, i32, P, P, P, sz, P], ctypes.c_int),
         "tb_score_select_scores": ([D, P, sz, P, i32, i32, P, P], ctypes.c_int),
         "tb_select_bits_from_idx": ([D, P, i32, P, P, P], ctypes.c_int),
+        "tb_select_export_candidates": ([D, P, sz, P, i32, P, i32, i32, P, P], ctypes.c_int),
+        "tb_select_merge_candidates": ([D, P, i32, i32, P, i32, i32, i32, P, i32, P, i32, i32, i32, P, P, sz, P],
+                                       ctypes.c_int),
+        "tb_sparse_decode_attn_partial": ([D, P, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
+        "tb_attn_combine": ([P, i32, i32, i32, i32, P, P], ctypes.c_int),
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_sparse_decode_attn_noalloc": ([D, P, P, P, P, i32, i32, P, f32, P, P], ctypes.c_int),
         "tb_kv_append": ([D, i32, P, P, P, P, sz, P], ctypes.c_int),
         "tb_selftest_bounded_wait": ([P, sz, i64, P], ctypes.c_int),
+        "tb_attn_set_launch_mode": ([i32], ctypes.c_int),
+        "tb_attn_launch_mode": ([], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -212,6 +221,37 @@ def score_select_scores(d: TbDims, ws, ctx_len, sink: int, window: int, scores, 
                                          _ptr(scores), _stream(stream)))
 
 
+def select_export_candidates(d: TbDims, ws, idx, count, budget: int, pos_offset: int, cand, stream=None):
+    """tb_select_export_candidates: a rank's top-B (a selection with nbr = 0)
+    as (score key, global position) composites, cand [batch][Hq][budget] int64."""
+    _check(load().tb_select_export_candidates(ctypes.byref(d), _ptr(ws), _bytes(ws), _ptr(idx), idx.shape[-1],
+                                              _ptr(count), int(budget), int(pos_offset), _ptr(cand), _stream(stream)))
+
+
+def select_merge_candidates(d: TbDims, cand, n_ranks: int, budget: int, ctx_len, sink: int, window: int, nbr: int,
+                            idx, count, shard_begin: int, shard_len: int, local_bits, local_cap: int, ws,
+                            stream=None):
+    """tb_select_merge_candidates: the global selection from every rank's
+    candidates, and this rank's attended-row bitmap."""
+    _check(load().tb_select_merge_candidates(ctypes.byref(d), _ptr(cand), int(n_ranks), int(budget), _ptr(ctx_len),
+                                             sink, window, nbr, _ptr(idx), idx.shape[-1], _ptr(count),
+                                             int(shard_begin), int(shard_len), int(local_cap), _ptr(local_bits),
+                                             _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def sparse_decode_attn_partial(d: TbDims, Q, K, V, rows, bits, scale: float, part, ws, stream=None):
+    """tb_sparse_decode_attn_partial: unnormalised attention state over the
+    rows of `bits` (part [batch][Hq][d+2] float32)."""
+    _check(load().tb_sparse_decode_attn_partial(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(rows), _ptr(bits),
+                                                float(scale), _ptr(part), _ptr(ws), _bytes(ws), _stream(stream)))
+
+
+def attn_combine(parts, out, stream=None):
+    """tb_attn_combine: parts [n][batch][Hq][d+2] -> out [batch][Hq][d]."""
+    n, batch, hq, dd = parts.shape
+    _check(load().tb_attn_combine(_ptr(parts), n, batch, hq, dd - 2, _ptr(out), _stream(stream)))
+
+
 def select_bits_from_idx(d: TbDims, idx, count, sel_bits, stream=None):
     _check(load().tb_select_bits_from_idx(ctypes.byref(d), _ptr(idx), idx.shape[-1], _ptr(count),
                                           _ptr(sel_bits), _stream(stream)))
@@ -230,6 +270,12 @@ def sparse_decode_attn_noalloc(d: TbDims, Q, K, V, ctx_len, sink: int, window: i
     workspace (for callers that cannot allocate; see include/tb.h)."""
     _check(load().tb_sparse_decode_attn_noalloc(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), sink,
                                                 window, _ptr(sel_bits), float(scale), _ptr(out), _stream(stream)))
+
+
+def attn_set_launch_mode(mode: int):
+    """tb_attn_set_launch_mode for the calling thread (TB_ATTN_WAIT_ALL or
+    TB_ATTN_PREFETCH_KV; see include/tb.h for the contract of the latter)."""
+    _check(load().tb_attn_set_launch_mode(int(mode)))
 
 
 def decode_attn(d: TbDims, Q, K, V, ctx_len, scale: float, out, ws, stream=None):

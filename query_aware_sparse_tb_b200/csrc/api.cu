@@ -15,6 +15,9 @@
 namespace tb {
 
 static thread_local char g_err[512] = "";
+static thread_local int g_attn_mode = TB_ATTN_WAIT_ALL;
+
+int attn_launch_mode() { return g_attn_mode; }
 static std::mutex g_state_mu;  // serialises one-time per-device kernel set-up
 
 void set_error(const char *fmt, ...) {
@@ -161,6 +164,15 @@ const char *tb_status_str(tb_status s) {
 }
 
 const char *tb_last_error(void) { return g_err; }
+
+tb_status tb_attn_set_launch_mode(int32_t mode) {
+    if (mode != TB_ATTN_WAIT_ALL && mode != TB_ATTN_PREFETCH_KV)
+        return fail(TB_ERR_INVALID_ARG, "tb_attn_set_launch_mode: unknown mode %d", mode);
+    g_attn_mode = mode;
+    return TB_OK;
+}
+
+int32_t tb_attn_launch_mode(void) { return g_attn_mode; }
 
 size_t tb_score_select_workspace_bytes(const tb_dims *dims) {
     if (check_dims(dims, true, __func__) != TB_OK || dims->ctx_cap > kMaxCtxSelect) return 0;
@@ -325,6 +337,78 @@ tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_
     if (sink < 0 || window < 1) return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0 and window >= 1", __func__);
     if ((s = check_ws(const_cast<void *>(ws), ws_bytes, select_ws_bytes(*dims), __func__)) != TB_OK) return s;
     return cuda_status(launch_export_scores(*dims, ws, ctx_len, sink, window, scores, (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_select_export_candidates(const tb_dims *dims, const void *ws, size_t ws_bytes, const int32_t *idx,
+                                      int32_t idx_cap, const int32_t *count, int32_t budget, int32_t pos_offset,
+                                      uint64_t *cand, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
+    if (dims->ctx_cap > kMaxCtxSelect)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", __func__, dims->ctx_cap, kMaxCtxSelect);
+    TB_CHECK_PTR4(idx); TB_CHECK_PTR4(count);
+    if (!cand || (reinterpret_cast<uintptr_t>(cand) & 7u) != 0)
+        return fail(TB_ERR_INVALID_ARG, "%s: cand is null or not 8-byte aligned", __func__);
+    if (idx_cap < 1 || budget < 1) return fail(TB_ERR_INVALID_ARG, "%s: need idx_cap >= 1 and budget >= 1", __func__);
+    if (pos_offset < 0 || (long long)pos_offset + dims->ctx_cap > 0x7fffffffLL)
+        return fail(TB_ERR_INVALID_ARG, "%s: pos_offset %d out of range", __func__, pos_offset);
+    if ((s = check_ws(const_cast<void *>(ws), ws_bytes, select_ws_bytes(*dims), __func__)) != TB_OK) return s;
+    return cuda_status(launch_export_candidates(*dims, ws, idx, idx_cap, count, budget, pos_offset, cand,
+                                                (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_select_merge_candidates(const tb_dims *dims, const uint64_t *cand, int32_t n_ranks, int32_t budget,
+                                     const int32_t *ctx_len, int32_t sink, int32_t window, int32_t nbr,
+                                     int32_t *idx, int32_t idx_cap, int32_t *count, int32_t shard_begin,
+                                     int32_t shard_len, int32_t local_cap, uint32_t *local_bits, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, true, __func__)) != TB_OK) return s;
+    if (dims->ctx_cap > kMaxCtxSelect)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", __func__, dims->ctx_cap, kMaxCtxSelect);
+    if (!cand || (reinterpret_cast<uintptr_t>(cand) & 7u) != 0)
+        return fail(TB_ERR_INVALID_ARG, "%s: cand is null or not 8-byte aligned", __func__);
+    TB_CHECK_PTR4(ctx_len); TB_CHECK_PTR4(idx); TB_CHECK_PTR4(count); TB_CHECK_PTR4(local_bits);
+    if (n_ranks < 1 || budget < 1 || (long long)n_ranks * budget > (1LL << 24))
+        return fail(TB_ERR_INVALID_ARG, "%s: need n_ranks >= 1, budget >= 1, n_ranks*budget <= 2^24", __func__);
+    if (sink < 0 || window < 1 || nbr < 0 || nbr > 16)
+        return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0, window >= 1, 0 <= nbr <= 16", __func__);
+    const long long need_cap = (long long)(2 * nbr + 1) * budget;
+    if (idx_cap < (need_cap < dims->ctx_cap ? need_cap : dims->ctx_cap))
+        return fail(TB_ERR_INVALID_ARG, "%s: idx_cap %d smaller than the largest possible selection", __func__, idx_cap);
+    if (shard_begin < 0 || shard_begin % 32 != 0 || shard_len < 0 || local_cap < 1 || local_cap < shard_len ||
+        (long long)shard_begin + shard_len > dims->ctx_cap)
+        return fail(TB_ERR_INVALID_ARG, "%s: need 0 <= shard_begin (a multiple of 32), 0 <= shard_len <= local_cap, "
+                    "and the shard inside ctx_cap", __func__);
+    if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
+    return cuda_status(launch_merge_candidates(*dims, cand, n_ranks, budget, ctx_len, sink, window, nbr, idx, idx_cap,
+                                               count, shard_begin, shard_len, local_cap, local_bits,
+                                               static_cast<uint32_t *>(ws), (cudaStream_t)stream),
+                       __func__);
+}
+
+tb_status tb_sparse_decode_attn_partial(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
+                                        const int32_t *rows, const uint32_t *bits, float scale, float *part,
+                                        void *ws, size_t ws_bytes, void *stream) {
+    tb_status s = check_attn_args(__func__, dims, Q, K, V, rows, scale, part, true, bits, 0, 1);
+    if (s != TB_OK) return s;
+    if ((s = check_ws(ws, ws_bytes, attn_ws_bytes(*dims), __func__)) != TB_OK) return s;
+    // sink 0 and window 0: no row is kept unless its bit is set
+    return cuda_status(launch_attn(*dims, Q, K, V, rows, 0, 0, bits, true, scale, nullptr, ws, (cudaStream_t)stream,
+                                   part),
+                       __func__);
+}
+
+tb_status tb_attn_combine(const float *parts, int32_t n_parts, int32_t batch, int32_t n_q_heads, int32_t head_dim,
+                          float *out, void *stream) {
+    TB_CHECK_PTR4(parts); TB_CHECK_PTR4(out);
+    if (n_parts < 1 || batch < 1 || n_q_heads < 1 || (long long)batch * n_q_heads > 0x7fffffffLL)
+        return fail(TB_ERR_INVALID_ARG, "%s: need n_parts, batch and n_q_heads >= 1", __func__);
+    if (head_dim != 64 && head_dim != 128)
+        return fail(TB_ERR_UNSUPPORTED, "%s: head_dim %d not built (64, 128)", __func__, head_dim);
+    return cuda_status(launch_combine(parts, n_parts, batch * n_q_heads, head_dim, out, (cudaStream_t)stream),
                        __func__);
 }
 

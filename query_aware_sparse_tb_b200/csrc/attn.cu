@@ -129,7 +129,7 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             const uint32_t *__restrict__ sel_bits, int Hq, int Hkv, int Tcap, int W, int sink,
             int window, float qscale, int splits, float *__restrict__ part,
             uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags,
-            int early_trigger) {
+            int early_trigger, int prefetch, float *__restrict__ part_out) {
     constexpr int CPR = D / 8;      // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;   // rows per warp-wide copy instruction
     constexpr int kKSteps = D / 16; // MMA K steps of S^T
@@ -164,10 +164,6 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
-    // the capacity split evenly over the CTAs of (b, g), in 128-row units, so
-    // that a CTA's first positions are known before the length arrives
-    const int chunk = ((Tcap + splits - 1) / splits + kRows - 1) / kRows * kRows;
-    const int p_begin = split * chunk;
 
     // ------------------------------------------------------------ set-up
     // (touches only this CTA's shared memory and TMEM, so under a programmatic
@@ -192,13 +188,26 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
         tmem_alloc(sb + Smem::kMisc + 4 * kMiscTmem, kTmemCols);
         tmem_relinquish();
     }
-    // every input and the workspace may be written by the previous kernel
-    griddep_wait();
-    // a one-wave grid lets the next kernel's CTAs take the SMs it leaves idle
-    // and the ones its CTAs free; a longer grid only once this CTA is done
-    if (early_trigger) griddep_launch_dependents();
+    // Without prefetch, every input and the workspace may be written by the
+    // previous kernel: wait for it before any global access.  With prefetch,
+    // the lengths, the selection words and the K/V rows below T-1 are not
+    // written by it (the caller's contract), so the load warps start on them
+    // at once; Q, row T-1, the output and the workspace wait for it.
+    if (!prefetch) {
+        griddep_wait();
+        // a one-wave grid lets the next kernel's CTAs take the SMs it leaves
+        // idle and the ones its CTAs free; a longer grid only once this CTA
+        // is done
+        if (early_trigger) griddep_launch_dependents();
+    }
 
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
+    // the context split evenly over the CTAs of (b, g), in whole selection
+    // words; with prefetch by the length itself, otherwise by the capacity so
+    // that a CTA's first positions are known before the length arrives
+    const int span = prefetch ? T : Tcap;
+    const int chunk = ((span + splits - 1) / splits + 31) / 32 * 32;
+    const int p_begin = split * chunk;
     const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
     const int p_end = min(p_begin + chunk, T);
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
@@ -301,6 +310,10 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             const int n_tiles = (n_rows + kRows - 1) / kRows;
             for (int t = 0; t < n_tiles; ++t, ++it) {
                 const int s = it % kStages;
+                // row T-1 (always kept: the window's last row) is the last row
+                // of the last tile of the CTA whose slice ends at T; the
+                // previous kernel may be writing it
+                if (prefetch && p1 == T && t == n_tiles - 1) griddep_wait();
                 if constexpr (SPARSE) compact_upto(min((t + 1) * kRows, n_rows));
                 bool ok = true;
                 if (it >= kStages) ok = wait_role(empty(s), ((it / kStages) + 1) & 1, abort_flag, flags);
@@ -405,6 +418,10 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
         const int mt = tid;  // tile row, then head dim
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         {
+            if (prefetch) {
+                griddep_wait();  // Q may come from the previous kernel
+                if (early_trigger) griddep_launch_dependents();
+            }
             // Q operand (K-major, 16 rows: the group's 4 query heads, then
             // zeros); P operands: rows 8..15 stay zero
             const uint16_t *Qg = Q + ((size_t)b * Hq + (size_t)g * kGroup) * D;
@@ -552,8 +569,8 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     }
 
     // ---------------------------------------------------- release, ticket
+    if (prefetch) griddep_wait();  // (roles that have not waited yet) before the workspace
     if (!early_trigger) griddep_launch_dependents();
-    __threadfence();
     tc_fence_before();
     __syncthreads();
     if (warp == 8) {
@@ -561,12 +578,13 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
         tmem_dealloc(tmem, kTmemCols);
     }
     if (tid == 0) {
-        const unsigned prev = atomicAdd(&counters[b * Hkv + g], 1u);
-        s_last = (prev == (unsigned)splits - 1u);
+        // one acquire-release ticket: its release publishes the CTA's partial
+        // states (every thread's stores are ordered before it by the barrier
+        // above), its acquire lets the last CTA read every other CTA's
+        s_last = (atom_add_acq_rel_gpu(&counters[b * Hkv + g], 1u) == (unsigned)splits - 1u);
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
 
     // ---------------------------------------------------- last CTA merges
     // One output group (head, 4 dims) per TPG threads; each thread folds its
@@ -589,11 +607,12 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             Ls = fmaf(Ls, a, l2 * c);
             M = Mn;
         };
-        for (int s0 = j; s0 < ns; s0 += 8 * TPG) {
-            float2 ml[8];
-            float4 v[8];
+        constexpr int kU = 16;  // states loaded per round: one round for up to 32 splits
+        for (int s0 = j; s0 < ns; s0 += kU * TPG) {
+            float2 ml[kU];
+            float4 v[kU];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < kU; ++u) {
                 const int s = s0 + u * TPG;
                 if (s < ns) {
                     const float *rec = src + (size_t)s * kPartStride;
@@ -605,7 +624,7 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) fold(ml[u].x, ml[u].y, v[u]);
+            for (int u = 0; u < kU; ++u) fold(ml[u].x, ml[u].y, v[u]);
         }
 #pragma unroll
         for (int off = 1; off < TPG; off <<= 1) {
@@ -616,18 +635,52 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             fold(m2, l2, o2);
         }
         if (j == 0) {  // scalar stores: `out` is only required to be 4-byte aligned
-            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-            float *dst = out + ((size_t)b * Hq + g * kGroup + h) * D + d4 * 4;
-            dst[0] = o.x * inv; dst[1] = o.y * inv; dst[2] = o.z * inv; dst[3] = o.w * inv;
+            if (part_out) {
+                // the unnormalised state (o relative to M, M, L) for a merge across shards
+                float *dst = part_out + ((size_t)b * Hq + g * kGroup + h) * (D + 2);
+                dst[d4 * 4] = o.x; dst[d4 * 4 + 1] = o.y; dst[d4 * 4 + 2] = o.z; dst[d4 * 4 + 3] = o.w;
+                if (d4 == 0) {
+                    dst[D] = M;
+                    dst[D + 1] = Ls;
+                }
+            } else {
+                const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+                float *dst = out + ((size_t)b * Hq + g * kGroup + h) * D + d4 * 4;
+                dst[0] = o.x * inv; dst[1] = o.y * inv; dst[2] = o.z * inv; dst[3] = o.w * inv;
+            }
         }
     }
     if (tid == 0) counters[b * Hkv + g] = 0u;  // leave the ticket zeroed for the next call
 }
 
+// out[b][h][:] = the merged state of n_parts unnormalised partial states
+// parts[p][b][h] = (o[D], M, L) (log2 units): sum_p 2^(M_p - M*) o_p / sum_p 2^(M_p - M*) L_p
+template <int D>
+__global__ void __launch_bounds__(D)
+combine_kernel(const float *__restrict__ parts, int n_parts, int rows, float *__restrict__ out) {
+    const int r = blockIdx.x, d = threadIdx.x;
+    griddep_wait();
+    griddep_launch_dependents();
+    float Mx = -INFINITY;
+    for (int p = 0; p < n_parts; ++p) Mx = fmaxf(Mx, parts[((size_t)p * rows + r) * (D + 2) + D]);
+    float o = 0.f, Ls = 0.f;
+    if (Mx != -INFINITY) {
+        for (int p = 0; p < n_parts; ++p) {
+            const float *st = parts + ((size_t)p * rows + r) * (D + 2);
+            const float m = st[D];
+            if (m == -INFINITY) continue;  // a shard with no attended row of this head
+            const float w = exp2f(m - Mx);
+            o = fmaf(st[d], w, o);
+            Ls = fmaf(st[D + 1], w, Ls);
+        }
+    }
+    out[(size_t)r * D + d] = Ls > 0.f ? o / Ls : 0.f;
+}
+
 template <int D, bool SPARSE>
 cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                      const int32_t *ctx_len, int32_t sink, int32_t window, const uint32_t *sel_bits,
-                     float scale, float *out, void *ws, cudaStream_t st) {
+                     float scale, float *out, void *ws, cudaStream_t st, float *part_out) {
     static std::atomic<int> smem_set[kMaxDevices];
     cudaError_t e = ensure_dynamic_smem((const void *)attn_kernel<D, SPARSE>, Smem::kBytes, smem_set);
     if (e != cudaSuccess) return e;
@@ -639,22 +692,13 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
         w + kWsHeaderBytes + align_up((size_t)d.batch * d.n_kv_heads * 4, 256));
     const int W = (d.ctx_cap + 31) / 32;
     const float qscale = scale * 1.4426950408889634f;  // logits in log2 units for exp2
-    // programmatic stream serialization: the launch may begin while the
-    // previous kernel in the stream finishes; the kernel waits for it
-    // (griddep_wait) before its first global read
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(splits, d.n_kv_heads, d.batch);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = Smem::kBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    // the launch may begin while the previous kernel in the stream finishes;
+    // the kernel waits for it (griddep_wait) before its first global access
     const int early = (long long)splits * d.n_kv_heads * d.batch <= num_sms() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, attn_kernel<D, SPARSE>, Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads,
-                              d.ctx_cap, W, sink, window, qscale, splits, part, counters, out, flags, early);
+    const int prefetch = attn_launch_mode() == TB_ATTN_PREFETCH_KV ? 1 : 0;
+    return launch_pdl(attn_kernel<D, SPARSE>, dim3(splits, d.n_kv_heads, d.batch), dim3(kThreads), Smem::kBytes,
+                      st, Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, qscale,
+                      splits, part, counters, out, flags, early, prefetch, part_out);
 }
 
 }  // namespace
@@ -688,13 +732,21 @@ size_t attn_ws_bytes(const tb_dims &d) {
 cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *ctx_len, int32_t sink, int32_t window,
                         const uint32_t *sel_bits, bool sparse, float scale, float *out, void *ws,
-                        cudaStream_t st) {
+                        cudaStream_t st, float *part_out) {
     if (d.head_dim == 128) {
-        return sparse ? launch_t<128, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st)
-                      : launch_t<128, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st);
+        return sparse ? launch_t<128, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out)
+                      : launch_t<128, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st,
+                                             part_out);
     }
-    return sparse ? launch_t<64, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st)
-                  : launch_t<64, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st);
+    return sparse ? launch_t<64, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out)
+                  : launch_t<64, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out);
+}
+
+cudaError_t launch_combine(const float *parts, int32_t n_parts, int32_t rows, int32_t head_dim, float *out,
+                           cudaStream_t st) {
+    if (head_dim == 128)
+        return launch_pdl(combine_kernel<128>, dim3(rows), dim3(128), 0, st, parts, n_parts, rows, out);
+    return launch_pdl(combine_kernel<64>, dim3(rows), dim3(64), 0, st, parts, n_parts, rows, out);
 }
 
 }  // namespace tb

@@ -65,6 +65,17 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// Atomic add at GPU scope with acquire-release semantics: the releasing
+// half publishes every store ordered before it (the calling thread's, and
+// other threads' ordered before it by a CTA barrier); the acquiring half
+// makes every store published by earlier releases on the same word visible
+// to the caller (and, after a CTA barrier, to its CTA).  Returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // ------------------------------------------------------------ cp.async ----
 
 // 16-byte global->shared copy; when `valid` is false nothing is read and the
@@ -303,6 +314,27 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 // serialization) be scheduled before this one has finished.
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// Launch `kernel` with programmatic stream serialization: its CTAs may start
+// while the previous kernel in the stream is finishing.  Every libtb kernel
+// calls griddep_wait() before its first access to global memory, so the
+// attribute only moves launch latency and shared-memory set-up off the
+// critical path.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
 }
 
 // ------------------------------------------------------ named barriers ----

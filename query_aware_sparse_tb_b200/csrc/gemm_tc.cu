@@ -74,6 +74,8 @@ project_keys_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
+    griddep_wait();
+    griddep_launch_dependents();
     const int begin = tok_begin[b], cnt = tok_count[b];
     if (begin < 0 || cnt <= tile * 128) return;
     const int t0 = begin + tile * 128;
@@ -185,6 +187,8 @@ skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    griddep_wait();
+    griddep_launch_dependents();
 
     if (tid == 0) {
         prefetch_tensormap(&tmA);
@@ -234,6 +238,8 @@ skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 // act[n][m] = bf16(SiLU(sum_s partial[s][n][m]))
 __global__ void silu_reduce_kernel(const float *__restrict__ partial, int splits, int n_rows, int M,
                                    uint16_t *__restrict__ act) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n_rows * M) return;
     float a = 0.f;
@@ -245,6 +251,8 @@ __global__ void silu_reduce_kernel(const float *__restrict__ partial, int splits
 // out[n][m] = sum_s partial[s][n][m]
 __global__ void sum_reduce_kernel(const float *__restrict__ partial, int splits, int n_rows, int M,
                                   float *__restrict__ out) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n_rows * M) return;
     float a = 0.f;
@@ -265,9 +273,8 @@ cudaError_t launch_pk(const tb_dims &d, const uint16_t *K, const uint16_t *Wk, u
     cudaError_t e = ensure_dynamic_smem((const void *)project_keys_kernel<D, DP>, smem, smem_set);
     if (e != cudaSuccess) return e;
     dim3 grid((max_tok + 127) / 128, d.n_kv_heads, d.batch);
-    project_keys_kernel<D, DP><<<grid, 128, smem, st>>>(mK, mW, Kp, tok_begin, tok_count, d.n_kv_heads,
-                                                       d.ctx_cap, flags);
-    return cudaGetLastError();
+    return launch_pdl(project_keys_kernel<D, DP>, grid, dim3(128), smem, st, mK, mW, Kp, tok_begin, tok_count,
+                      d.n_kv_heads, d.ctx_cap, flags);
 }
 
 constexpr int kKB = 4;  // 64-wide K blocks per CTA (256 of K)
@@ -280,9 +287,8 @@ cudaError_t launch_skinny(const uint16_t *A, const uint16_t *B, float *partial, 
     static std::atomic<int> smem_set[kMaxDevices];
     cudaError_t e = ensure_dynamic_smem((const void *)skinny_gemm_kernel<kKB>, smem, smem_set);
     if (e != cudaSuccess) return e;
-    dim3 grid(M / 128, K / (kKB * 64));
-    skinny_gemm_kernel<kKB><<<grid, 128, smem, st>>>(mA, mB, partial, M, n_rows, flags);
-    return cudaGetLastError();
+    return launch_pdl(skinny_gemm_kernel<kKB>, dim3(M / 128, K / (kKB * 64)), dim3(128), smem, st, mA, mB, partial,
+                      M, n_rows, flags);
 }
 
 struct PredWs {
@@ -331,13 +337,14 @@ cudaError_t launch_predict_queries(const uint16_t *h, const uint16_t *W1, const 
     cudaError_t e = launch_skinny(W1, h, w.p1, inter, hidden, batch, w.flags, st);
     if (e != cudaSuccess) return e;
     const int n1 = batch * inter;
-    silu_reduce_kernel<<<(n1 + 255) / 256, 256, 0, st>>>(w.p1, hidden / (kKB * 64), batch, inter, w.act);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(silu_reduce_kernel, dim3((n1 + 255) / 256), dim3(256), 0, st, (const float *)w.p1,
+                   hidden / (kKB * 64), batch, inter, w.act);
+    if (e != cudaSuccess) return e;
     e = launch_skinny(W2, w.act, w.p2, n_out, inter, batch, w.flags, st);
     if (e != cudaSuccess) return e;
     const int n2 = batch * n_out;
-    sum_reduce_kernel<<<(n2 + 255) / 256, 256, 0, st>>>(w.p2, inter / (kKB * 64), batch, n_out, qp);
-    return cudaGetLastError();
+    return launch_pdl(sum_reduce_kernel, dim3((n2 + 255) / 256), dim3(256), 0, st, (const float *)w.p2,
+                      inter / (kKB * 64), batch, n_out, qp);
 }
 
 }  // namespace tb

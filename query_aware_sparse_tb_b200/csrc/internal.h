@@ -17,7 +17,9 @@ int attn_splits(const tb_dims &d);
 cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *ctx_len, int32_t sink, int32_t window,
                         const uint32_t *sel_bits, bool sparse, float scale, float *out, void *ws,
-                        cudaStream_t st);
+                        cudaStream_t st, float *part_out = nullptr);
+cudaError_t launch_combine(const float *parts, int32_t n_parts, int32_t rows, int32_t head_dim, float *out,
+                           cudaStream_t st);
 
 // ---- score + select (select.cu) ----
 size_t select_ws_bytes(const tb_dims &d);
@@ -31,6 +33,13 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                 void *ws, cudaStream_t st);
 cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t *ctx_len, int32_t sink,
                                  int32_t window, float *scores, cudaStream_t st);
+cudaError_t launch_export_candidates(const tb_dims &d, const void *ws, const int32_t *idx, int32_t idx_cap,
+                                     const int32_t *count, int32_t budget, int32_t pos_offset, uint64_t *cand,
+                                     cudaStream_t st);
+cudaError_t launch_merge_candidates(const tb_dims &d, const uint64_t *cand, int32_t n_ranks, int32_t budget,
+                                    const int32_t *ctx_len, int32_t sink, int32_t window, int32_t nbr, int32_t *idx,
+                                    int32_t idx_cap, int32_t *count, int32_t shard_begin, int32_t shard_len,
+                                    int32_t local_cap, uint32_t *local_bits, uint32_t *flags, cudaStream_t st);
 cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx_cap,
                                const int32_t *count, uint32_t *sel_bits, cudaStream_t st);
 
@@ -51,6 +60,8 @@ cudaError_t launch_bounded_wait_selftest(void *ws, long long budget_cycles, cuda
 
 // Host error text for the calling thread (api.cu).
 void set_error(const char *fmt, ...);
+// The calling thread's attention launch mode (tb_attn_set_launch_mode, api.cu).
+int attn_launch_mode();
 
 // Host-side argument checks of the attention entry points (api.cu), shared by
 // tb_sparse_decode_attn, tb_decode_attn and tb_sparse_decode_attn_noalloc so

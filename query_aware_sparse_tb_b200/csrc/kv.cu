@@ -24,6 +24,8 @@ kv_append_kernel(const uint4 *__restrict__ src, const uint64_t *__restrict__ cac
                  const int32_t *__restrict__ ctx_len, int n_layers, int B, int Hkv, int Tcap,
                  uint32_t *__restrict__ flags) {
     constexpr int V16 = D / 8;  // 16-byte vectors per row
+    griddep_wait();
+    griddep_launch_dependents();
     const int rows = n_layers * 2 * B * Hkv;
     const int r = blockIdx.x * (kThreads / V16) + threadIdx.x / V16;
     const int c = threadIdx.x % V16;
@@ -72,12 +74,10 @@ cudaError_t launch_kv_append(const tb_dims &d, int32_t n_layers, const uint16_t 
     const dim3 grid((rows + per_block - 1) / per_block);
     const uint4 *s = reinterpret_cast<const uint4 *>(src);
     if (d.head_dim == 128)
-        kv_append_kernel<128><<<grid, kThreads, 0, st>>>(s, caches, ctx_len, n_layers, d.batch, d.n_kv_heads,
-                                                         d.ctx_cap, flags);
-    else
-        kv_append_kernel<64><<<grid, kThreads, 0, st>>>(s, caches, ctx_len, n_layers, d.batch, d.n_kv_heads,
-                                                        d.ctx_cap, flags);
-    return cudaGetLastError();
+        return launch_pdl(kv_append_kernel<128>, grid, dim3(kThreads), 0, st, s, caches, ctx_len, n_layers, d.batch,
+                          d.n_kv_heads, d.ctx_cap, flags);
+    return launch_pdl(kv_append_kernel<64>, grid, dim3(kThreads), 0, st, s, caches, ctx_len, n_layers, d.batch,
+                      d.n_kv_heads, d.ctx_cap, flags);
 }
 
 }  // namespace tb

@@ -181,11 +181,13 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     __shared__ int scratch[kThreads / 32 + 3];
     const int tid = threadIdx.x;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
-    const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
-    const int lo = sink, hi = T - window;
     const int p0 = ch * kHistChunk;
 
     for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
+    const int lo = sink, hi = T - window;
     if (tid < kGroup * DP) (&qs[0][0])[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
     __syncthreads();
 
@@ -332,10 +334,12 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
     __shared__ uint32_t s_cnt[kGroup], s_base[kGroup];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
+    if (tid < kGroup) s_cnt[tid] = 0u;
+    griddep_wait();
+    griddep_launch_dependents();
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, false);
     const int lo = sink, hi = T - window;
     const int w0 = ch * (kChunk / 32);
-    if (tid < kGroup) s_cnt[tid] = 0u;
 
     uint32_t mode[NH], b1[NH];
 #pragma unroll
@@ -424,6 +428,8 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
     constexpr int NOUT = sel_is_group(SEL) ? kGroup : 1;
     const int tid = threadIdx.x;
     const int h = blockIdx.x * NOUT, b = blockIdx.y;
+    griddep_wait();
+    griddep_launch_dependents();
     const size_t row = (size_t)b * Hq + h;
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, false);
     const int lo = sink, hi = T - window;
@@ -665,6 +671,8 @@ bits_from_idx_kernel(const int32_t *__restrict__ idx, int idx_cap, const int32_t
     const int tid = threadIdx.x;
     const size_t row = (size_t)blockIdx.y * Hq + blockIdx.x;
     for (int w = tid; w < W; w += kFinThreads) bsm[w] = 0u;
+    griddep_wait();
+    griddep_launch_dependents();
     __syncthreads();
     int n = count[row];
     n = n < 0 ? 0 : (n > idx_cap ? idx_cap : n);
@@ -674,6 +682,190 @@ bits_from_idx_kernel(const int32_t *__restrict__ idx, int idx_cap, const int32_t
     }
     __syncthreads();
     for (int w = tid; w < W; w += kFinThreads) sel_bits[row * W + w] = bsm[w];
+}
+
+// ------------------------------------------- context-parallel selection
+
+// A rank's local top-B as exchangeable candidates: for each selected local
+// position p (a selection with nbr = 0, so its set is exactly its top-B),
+// the composite (key << 32) | (0xFFFFFFFF - (p + pos_offset)) of its score's
+// order-preserving key and its global position.  Larger composites rank first
+// (score desc, position asc); 0 pads the unused slots.
+__global__ void __launch_bounds__(kThreads)
+export_candidates_kernel(const uint32_t *__restrict__ keys, const int32_t *__restrict__ idx, int idx_cap,
+                         const int32_t *__restrict__ count, int Hq, int Tcap, int budget, int pos_offset,
+                         unsigned long long *__restrict__ cand) {
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t row = (size_t)b * Hq + h;
+    griddep_wait();
+    griddep_launch_dependents();
+    int n = count[row];
+    n = n < 0 ? 0 : (n > idx_cap ? idx_cap : n);
+    n = n < budget ? n : budget;
+    for (int i = threadIdx.x; i < budget; i += kThreads) {
+        unsigned long long c = 0ull;
+        if (i < n) {
+            const int p = idx[row * idx_cap + i];
+            if (p >= 0 && p < Tcap)
+                c = ((unsigned long long)keys[row * Tcap + p] << 32) | (0xFFFFFFFFu - (uint32_t)(p + pos_offset));
+        }
+        cand[row * budget + i] = c;
+    }
+}
+
+// The global top-B of every rank's candidates, per (sequence, query head):
+// one CTA finds the budget-th largest composite with three radix passes over
+// the score keys (11/11/10 bits) and takes the ties on it by position, then
+// dilates the Top set by +-nbr, clips it to C = [sink, T - window), and writes
+// the global index list and count and this shard's attended-row bitmap: the
+// sink, window and selected positions in [shard_begin, shard_begin +
+// shard_len) ∩ [0, T), in local coordinates.
+__global__ void __launch_bounds__(kFinThreads)
+merge_candidates_kernel(const unsigned long long *__restrict__ cand, int n_ranks, int budget, int B, int Hq,
+                        const int32_t *__restrict__ ctx_len, int Tcap, int Wg, int sink, int window, int nbr,
+                        int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count, int shard_begin,
+                        int shard_len, int Wl, uint32_t *__restrict__ local_bits, uint32_t *__restrict__ flags) {
+    extern __shared__ uint32_t msm[];
+    uint32_t *top_s = msm;        // [Wg]
+    uint32_t *tie_s = msm + Wg;   // [Wg]
+    __shared__ uint32_t hist[kBins2];
+    __shared__ int scratch[kFinThreads / 32 + 3];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t row = (size_t)b * Hq + h;
+    for (int w = tid; w < Wg; w += kFinThreads) {
+        top_s[w] = 0u;
+        tie_s[w] = 0u;
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && h == 0 && b == 0);
+    const int lo = sink, hi = T - window;
+    const int n = n_ranks * budget;
+    auto cand_at = [&](int i) -> unsigned long long {
+        const int r = i / budget, k = i - r * budget;
+        return __ldcg(cand + (((size_t)r * B + b) * Hq + h) * budget + k);
+    };
+    // valid candidates (non-zero composites whose position is a candidate of C)
+    auto valid = [&](unsigned long long c, uint32_t *pos) {
+        const uint32_t p = 0xFFFFFFFFu - (uint32_t)c;
+        *pos = p;
+        return c != 0ull && (int)p >= lo && (int)p < hi;
+    };
+    int mine = 0;
+    for (int i = tid; i < n; i += kFinThreads) {
+        uint32_t p;
+        mine += valid(cand_at(i), &p) ? 1 : 0;
+    }
+    int n_valid;
+    (void)block_excl_scan<kFinThreads>(mine, scratch, &n_valid);
+    __syncthreads();
+    if (n_valid <= budget) {
+        for (int i = tid; i < n; i += kFinThreads) {
+            uint32_t p;
+            if (valid(cand_at(i), &p)) atomicOr(&top_s[p >> 5], 1u << (p & 31));
+        }
+    } else {
+        // the budget-th largest key: 11 + 11 + 10 bits, each pass over the
+        // candidates whose higher digits match the ones fixed so far
+        uint32_t need = (uint32_t)budget, prefix = 0u;
+        int fixed = 0;
+#pragma unroll 1
+        for (int pass = 0; pass < 3; ++pass) {
+            const int dw = pass < 2 ? 11 : 10;
+            const int nb = 1 << dw;
+            const int shift = 32 - fixed - dw;
+            for (int i = tid; i < nb; i += kFinThreads) hist[i] = 0u;
+            __syncthreads();
+            for (int i = tid; i < n; i += kFinThreads) {
+                uint32_t p;
+                const unsigned long long c = cand_at(i);
+                const uint32_t key = (uint32_t)(c >> 32);
+                if (valid(c, &p) && (fixed == 0 || (key >> (32 - fixed)) == prefix))
+                    atomicAdd(&hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
+            }
+            __syncthreads();
+            uint32_t rem;
+            const uint32_t bin = (uint32_t)block_find_bin_desc<kFinThreads>(hist, nb, need, &rem, scratch, false);
+            prefix = (prefix << dw) | bin;
+            fixed += dw;
+            need = rem;
+        }
+        const uint32_t tau = prefix;  // keys above it are Top; `need` of the keys equal to it, lowest positions first
+        for (int i = tid; i < n; i += kFinThreads) {
+            uint32_t p;
+            const unsigned long long c = cand_at(i);
+            if (!valid(c, &p)) continue;
+            const uint32_t key = (uint32_t)(c >> 32);
+            if (key > tau) atomicOr(&top_s[p >> 5], 1u << (p & 31));
+            else if (key == tau) atomicOr(&tie_s[p >> 5], 1u << (p & 31));
+        }
+        __syncthreads();
+        const int wpt = (Wg + kFinThreads - 1) / kFinThreads;
+        const int wb = tid * wpt, we = min(wb + wpt, Wg);
+        int tmine = 0;
+        for (int w = wb; w < we; ++w) tmine += __popc(tie_s[w]);
+        int tot;
+        int before = block_excl_scan<kFinThreads>(tmine, scratch, &tot);
+        for (int w = wb; w < we; ++w) {
+            uint32_t t = tie_s[w];
+            const int pc = __popc(t);
+            uint32_t keep = 0u;
+            if (before + pc <= (int)need) {
+                keep = t;
+            } else if (before < (int)need) {
+                for (int k = 0; k < (int)need - before; ++k) {
+                    const uint32_t low = t & (0u - t);
+                    keep |= low;
+                    t ^= low;
+                }
+            }
+            top_s[w] |= keep;
+            before += pc;
+        }
+    }
+    __syncthreads();
+    // neighbour fetch, clip to C, emit the global list; tie_s becomes I
+    const int wpt = (Wg + kFinThreads - 1) / kFinThreads;
+    const int wb = tid * wpt, we = min(wb + wpt, Wg);
+    int emine = 0;
+    for (int w = wb; w < we; ++w) {
+        const uint32_t t = top_s[w];
+        const uint32_t pv = w > 0 ? top_s[w - 1] : 0u, nx = w + 1 < Wg ? top_s[w + 1] : 0u;
+        uint32_t e = t;
+        for (int k = 1; k <= nbr; ++k) e |= (t << k) | (pv >> (32 - k)) | (t >> k) | (nx << (32 - k));
+        e &= range_mask(w, lo, hi);
+        emine += __popc(e);
+        tie_s[w] = e;
+    }
+    int total;
+    const int base = block_excl_scan<kFinThreads>(emine, scratch, &total);
+    {
+        const int lane = tid & 31;
+        const uint32_t lt = (1u << lane) - 1u;
+        int32_t *out = idx + row * (size_t)idx_cap;
+        const int w_first = (tid - lane) * wpt, w_last = min(w_first + 32 * wpt, Wg);
+        int run = __shfl_sync(kFull, base, 0);
+        for (int w = w_first; w < w_last; ++w) {
+            const uint32_t e = tie_s[w];
+            const int slot = run + __popc(e & lt);
+            if (((e >> lane) & 1u) && slot < idx_cap) out[slot] = (w << 5) + lane;
+            run += __popc(e);
+        }
+    }
+    if (tid == 0) {
+        if (total > idx_cap) raise_flag(flags, TB_FLAG_IDX_OVERFLOW);
+        count[row] = total < idx_cap ? total : idx_cap;
+    }
+    // this shard's attended rows: sink, window and I inside the shard (shard_begin % 32 == 0)
+    const int w0 = shard_begin >> 5;
+    const int shard_end = min(shard_begin + shard_len, T);
+    for (int wl = tid; wl < Wl; wl += kFinThreads) {
+        const int w = w0 + wl;
+        const uint32_t sel = w < Wg ? tie_s[w] : 0u;
+        const uint32_t kept = sel | range_mask(w, 0, min(sink, T)) | range_mask(w, max(sink, T - window), T);
+        local_bits[row * Wl + wl] = kept & range_mask(w, shard_begin, shard_end);
+    }
 }
 
 // ------------------------------------------------------ scores of a call
@@ -686,6 +878,8 @@ export_scores_kernel(const uint32_t *__restrict__ keys, const int32_t *__restric
                      int sink, int window, float *__restrict__ out) {
     const int p = blockIdx.x * kThreads + threadIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
+    griddep_wait();
+    griddep_launch_dependents();
     if (p >= Tcap) return;
     const int T = clamp_ctx(ctx_len[b], Tcap, nullptr, false);
     const size_t i = ((size_t)b * Hq + h) * Tcap + p;
@@ -707,17 +901,14 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
     const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
     dim3 grid(nch, d.n_kv_heads, d.batch);
     dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
-    if (d.d_proj == 32)
-        score_hist_kernel<32, SEL><<<grid_h, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
-                                                              d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
-    else
-        score_hist_kernel<16, SEL><<<grid_h, kThreads, 0, st>>>(qp, qp_stride, Kp, ctx_len, d.n_q_heads,
-                                                              d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = d.d_proj == 32
+        ? launch_pdl(score_hist_kernel<32, SEL>, grid_h, dim3(kThreads), 0, st, qp, qp_stride, Kp, ctx_len,
+                     d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s)
+        : launch_pdl(score_hist_kernel<16, SEL>, grid_h, dim3(kThreads), 0, st, qp, qp_stride, Kp, ctx_len,
+                     d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
     if (e != cudaSuccess) return e;
-    mark_collect_kernel<SEL><<<grid, kThreads, 0, st>>>(ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W,
-                                                        sink, window, s);
-    e = cudaGetLastError();
+    e = launch_pdl(mark_collect_kernel<SEL>, grid, dim3(kThreads), 0, st, ctx_len, d.n_q_heads, d.n_kv_heads,
+                   d.ctx_cap, W, sink, window, s);
     if (e != cudaSuccess) return e;
     const size_t fsm = (size_t)kCandCache * 8 + (size_t)2 * W * 4 + (SEL == kSelInclusive ? kCandCache * 2 : 0);
     static std::atomic<int> smem_set[kMaxDevices];
@@ -726,9 +917,8 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
         if (e != cudaSuccess) return e;
     }
     const int rows = sel_is_group(SEL) ? d.n_q_heads / kGroup : d.n_q_heads;
-    finalize_kernel<SEL><<<dim3(rows, d.batch), kFinThreads, fsm, st>>>(
-        ctx_len, d.n_q_heads, d.ctx_cap, W, sink, window, budget, nbr, idx, idx_cap, count, sel_bits, s);
-    return cudaGetLastError();
+    return launch_pdl(finalize_kernel<SEL>, dim3(rows, d.batch), dim3(kFinThreads), fsm, st, ctx_len, d.n_q_heads,
+                      d.ctx_cap, W, sink, window, budget, nbr, idx, idx_cap, count, sel_bits, s);
 }
 
 }  // namespace
@@ -757,8 +947,34 @@ cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t
                                  int32_t window, float *scores, cudaStream_t st) {
     const SelWs s = carve(d, const_cast<void *>(ws));
     dim3 grid((d.ctx_cap + kThreads - 1) / kThreads, d.n_q_heads, d.batch);
-    export_scores_kernel<<<grid, kThreads, 0, st>>>(s.keys, ctx_len, d.n_q_heads, d.ctx_cap, sink, window, scores);
-    return cudaGetLastError();
+    return launch_pdl(export_scores_kernel, grid, dim3(kThreads), 0, st, (const uint32_t *)s.keys, ctx_len,
+                      d.n_q_heads, d.ctx_cap, sink, window, scores);
+}
+
+cudaError_t launch_export_candidates(const tb_dims &d, const void *ws, const int32_t *idx, int32_t idx_cap,
+                                     const int32_t *count, int32_t budget, int32_t pos_offset, uint64_t *cand,
+                                     cudaStream_t st) {
+    const SelWs s = carve(d, const_cast<void *>(ws));
+    return launch_pdl(export_candidates_kernel, dim3(d.n_q_heads, d.batch), dim3(kThreads), 0, st,
+                      (const uint32_t *)s.keys, idx, idx_cap, count, d.n_q_heads, d.ctx_cap, budget, pos_offset,
+                      reinterpret_cast<unsigned long long *>(cand));
+}
+
+cudaError_t launch_merge_candidates(const tb_dims &d, const uint64_t *cand, int32_t n_ranks, int32_t budget,
+                                    const int32_t *ctx_len, int32_t sink, int32_t window, int32_t nbr, int32_t *idx,
+                                    int32_t idx_cap, int32_t *count, int32_t shard_begin, int32_t shard_len,
+                                    int32_t local_cap, uint32_t *local_bits, uint32_t *flags, cudaStream_t st) {
+    const int Wg = (d.ctx_cap + 31) / 32, Wl = (local_cap + 31) / 32;
+    const size_t sm = (size_t)2 * Wg * 4;
+    static std::atomic<int> smem_set[kMaxDevices];
+    if (sm > 48 * 1024) {
+        cudaError_t e = ensure_dynamic_smem((const void *)merge_candidates_kernel, (int)sm, smem_set);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(merge_candidates_kernel, dim3(d.n_q_heads, d.batch), dim3(kFinThreads), sm, st,
+                      reinterpret_cast<const unsigned long long *>(cand), n_ranks, budget, d.batch, d.n_q_heads,
+                      ctx_len, d.ctx_cap, Wg, sink, window, nbr, idx, idx_cap, count, shard_begin, shard_len, Wl,
+                      local_bits, flags);
 }
 
 cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx_cap,
@@ -770,9 +986,8 @@ cudaError_t launch_select_bits(const tb_dims &d, const int32_t *idx, int32_t idx
         cudaError_t e = ensure_dynamic_smem((const void *)bits_from_idx_kernel, (int)sm, smem_set);
         if (e != cudaSuccess) return e;
     }
-    bits_from_idx_kernel<<<dim3(d.n_q_heads, d.batch), kFinThreads, sm, st>>>(
-        idx, idx_cap, count, d.n_q_heads, d.ctx_cap, W, sel_bits);
-    return cudaGetLastError();
+    return launch_pdl(bits_from_idx_kernel, dim3(d.n_q_heads, d.batch), dim3(kFinThreads), sm, st, idx, idx_cap,
+                      count, d.n_q_heads, d.ctx_cap, W, sel_bits);
 }
 
 }  // namespace tb

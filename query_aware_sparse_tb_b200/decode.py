@@ -101,6 +101,132 @@ def gather_head_outputs(parts, heads_of_rank):
     return torch.cat([parts[r] for r in order], dim=-2)
 
 
+# --------------------------------------------------------------- context sharding
+#
+# One sequence's context split over ranks by position (the scale-out for
+# contexts past what one device should hold): rank r keeps the K, V and K'
+# rows of block [begin_r, end_r).  Each rank selects its block's local top-B,
+# the ranks exchange those candidates, every rank merges them into the global
+# selection (the global top-B is contained in the union of the blocks' top-B),
+# attends over its block's share of sink, window and selected rows, and the
+# ranks' unnormalised softmax states are combined.  The result is the
+# single-device result; tb.h (context-parallel selection and attention) has
+# the contract of each call.
+
+def context_blocks(ctx_cap: int, world: int, window: int) -> list[tuple[int, int]]:
+    """[begin, end) of each rank's block: equal blocks of whole windows (so
+    every block starts on a 32-position word and on a projection batch), the
+    last rank keeping everything from its begin to ctx_cap (where decoding
+    appends)."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    unit = window * 32 // math.gcd(window, 32)
+    per = max(unit, (ctx_cap // world) // unit * unit)
+    bounds = []
+    for r in range(world):
+        b0 = min(r * per, ctx_cap)
+        b1 = ctx_cap if r == world - 1 else min((r + 1) * per, ctx_cap)
+        bounds.append((b0, b1))
+    return bounds
+
+
+def block_capacity(block: tuple[int, int], window: int) -> int:
+    """Rows a rank's local caches hold: its block plus one window, the rows a
+    local selection may count as its window and never reads."""
+    return block[1] - block[0] + window
+
+
+def local_selection_params(T: int, block: tuple[int, int], sink: int, window: int) -> tuple[int, int]:
+    """(local T, local sink) for a selection over the block's part of the
+    candidates C = [sink, T - window): with window unchanged, the local
+    candidates [local sink, local T - window) are C ∩ block in local rows."""
+    b0, b1 = block
+    local_T = max(1, min(T, b1 + window) - b0)
+    return local_T, max(0, sink - b0)
+
+
+def local_rows(T: int, block: tuple[int, int]) -> int:
+    """Rows of the block that exist at length T (at least 1 for the call)."""
+    return max(1, min(T, block[1]) - block[0])
+
+
+class ContextShard:
+    """One rank's block of a context-sharded layer: its K, V (and K') rows,
+    the selection and attention workspaces, and the three phases of a
+    prediction step.  `exchange` between the phases is the caller's (an
+    all-gather over the ranks; stacking the ranks' tensors on one device
+    emulates it).  Per-head selection, queries given directly (q' of the
+    block's sequences, [batch][Hq][d']).
+
+      cand = shard.select_local(T, qp)              phase 1: local top-B
+      part = shard.merge_and_attend(T, cands, Q)    phase 2: global set, partial attention
+      combine_parts(parts, out)                     phase 3
+    """
+
+    def __init__(self, shape: "DecodeShape", block: tuple[int, int], K, V, Wk, device="cuda"):
+        s = self.shape = shape
+        self.block = block
+        self.cap = block_capacity(block, s.window)
+        assert K.shape[2] == self.cap and V.shape[2] == self.cap, "local caches hold block_capacity rows"
+        self.K, self.V, self.Wk = K, V, Wk
+        self.device = device
+        B, Hq, Hkv = s.batch, s.n_q_heads, s.n_kv_heads
+        self.dims = L.dims(B, Hq, Hkv, s.head_dim, s.d_proj, self.cap)
+        self.gdims = L.dims(B, Hq, Hkv, s.head_dim, s.d_proj, s.ctx_cap)
+        self.Kp = torch.zeros(B, Hkv, self.cap, s.d_proj, dtype=torch.bfloat16, device=device)
+        self.ws_sel = L.workspace(L.score_select_workspace_bytes(self.dims), device)
+        self.ws_attn = L.workspace(L.attn_workspace_bytes(self.dims), device)
+        self.ws_small = L.workspace(256, device)
+        self.local_idx = torch.zeros(B, Hq, min(s.budget, self.cap), dtype=torch.int32, device=device)
+        self.local_cnt = torch.zeros(B, Hq, dtype=torch.int32, device=device)
+        self.local_bits = torch.zeros(B, Hq, (self.cap + 31) // 32, dtype=torch.int32, device=device)
+        self.cand = torch.zeros(B, Hq, s.budget, dtype=torch.int64, device=device)
+        self.idx = torch.zeros(B, Hq, s.idx_cap, dtype=torch.int32, device=device)
+        self.cnt = torch.zeros(B, Hq, dtype=torch.int32, device=device)
+        self.bits = torch.zeros(B, Hq, (self.cap + 31) // 32, dtype=torch.int32, device=device)
+        self.part = torch.zeros(B, Hq, s.head_dim + 2, dtype=torch.float32, device=device)
+        self.scale = 1.0 / math.sqrt(s.head_dim)
+
+    def project(self, rows: list[int], stream=None):
+        """Project the first rows[b] local rows of every sequence."""
+        zero = torch.zeros(self.shape.batch, dtype=torch.int32, device=self.device)
+        cnt = torch.tensor(rows, dtype=torch.int32, device=self.device)
+        L.project_keys(self.dims, self.K, self.Wk, self.Kp, zero, cnt, max(max(rows), 1), self.ws_small, stream)
+
+    def select_local(self, T: list[int], qp, stream=None):
+        """Phase 1: this block's top-B per head (nbr = 0) as exchangeable
+        (score key, global position) candidates [batch][Hq][budget]."""
+        s = self.shape
+        params = [local_selection_params(t, self.block, s.sink, s.window) for t in T]
+        sinks = {p[1] for p in params}
+        assert len(sinks) == 1
+        self.sel_ctx = torch.tensor([p[0] for p in params], dtype=torch.int32, device=self.device)
+        L.score_select(self.dims, qp, s.n_q_heads * s.d_proj, self.Kp, self.sel_ctx, sinks.pop(), s.window,
+                       s.budget, 0, self.local_idx, self.local_cnt, self.local_bits, self.ws_sel, stream)
+        L.select_export_candidates(self.dims, self.ws_sel, self.local_idx, self.local_cnt, s.budget, self.block[0],
+                                   self.cand, stream)
+        return self.cand
+
+    def merge_and_attend(self, T: list[int], cands, Q, stream=None):
+        """Phase 2: the global selection from every rank's candidates
+        ([world][batch][Hq][budget]) and this block's unnormalised attention
+        state [batch][Hq][d+2]."""
+        s = self.shape
+        self.ctx_g = torch.tensor(T, dtype=torch.int32, device=self.device)
+        self.rows = torch.tensor([local_rows(t, self.block) for t in T], dtype=torch.int32, device=self.device)
+        L.select_merge_candidates(self.gdims, cands, cands.shape[0], s.budget, self.ctx_g, s.sink, s.window, s.nbr,
+                                  self.idx, self.cnt, self.block[0], self.block[1] - self.block[0], self.bits,
+                                  self.cap, self.ws_small, stream)
+        L.sparse_decode_attn_partial(self.dims, Q, self.K, self.V, self.rows, self.bits, self.scale, self.part,
+                                     self.ws_attn, stream)
+        return self.part
+
+
+def combine_parts(parts, out, stream=None):
+    """Phase 3: out [batch][Hq][d] from the ranks' states [world][batch][Hq][d+2]."""
+    L.attn_combine(parts, out, stream)
+
+
 @dataclass(frozen=True)
 class DecodeShape:
     batch: int
@@ -147,10 +273,17 @@ class SparseDecoder:
     SELECTIONS = ("head", "group_max", "group_sum", "inclusive")
 
     def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda",
-                 selection: str = "head"):
+                 selection: str = "head", prefetch_kv: bool = False):
         if selection not in self.SELECTIONS:
             raise ValueError(f"selection must be one of {self.SELECTIONS}")
         self.selection = selection
+        # TB_ATTN_PREFETCH_KV for the attention launches whose preceding
+        # kernel writes none of the lengths, selection words and K/V rows
+        # below T-1.  Inside a step that is every attention launch except the
+        # first one right after the selection of the same (only) layer; for
+        # the first launch of a step the caller vouches for the kernel it ran
+        # last (a K/V append of the new token's rows is fine).
+        self.prefetch_kv = prefetch_kv
         s = self.shape = shape
         self.K, self.V, self.Wk, self.mlp = K, V, Wk, mlp
         self.ctx0 = list(ctx0)
@@ -223,14 +356,22 @@ class SparseDecoder:
                                  s.budget, s.nbr, self.selection[len("group_"):], self.idx[layer],
                                  self.cnt[layer], self.bits[layer], self.ws_sel, stream)
 
-    def attend(self, step: int, layer: int, Q, out, stream=None):
+    def attend(self, step: int, layer: int, Q, out, stream=None, prefetch: bool = False):
         s = self.shape
-        L.sparse_decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], s.sink, s.window,
-                             self.bits[layer], self.scale, out, self.ws_attn, stream)
+        L.attn_set_launch_mode(L.TB_ATTN_PREFETCH_KV if prefetch else L.TB_ATTN_WAIT_ALL)
+        try:
+            L.sparse_decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], s.sink, s.window,
+                                 self.bits[layer], self.scale, out, self.ws_attn, stream)
+        finally:
+            L.attn_set_launch_mode(L.TB_ATTN_WAIT_ALL)
 
-    def attend_dense(self, step: int, layer: int, Q, out, stream=None):
-        L.decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], self.scale, out, self.ws_attn,
-                      stream)
+    def attend_dense(self, step: int, layer: int, Q, out, stream=None, prefetch: bool = False):
+        L.attn_set_launch_mode(L.TB_ATTN_PREFETCH_KV if prefetch else L.TB_ATTN_WAIT_ALL)
+        try:
+            L.decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], self.scale, out,
+                          self.ws_attn, stream)
+        finally:
+            L.attn_set_launch_mode(L.TB_ATTN_WAIT_ALL)
 
     # -------------------------------------------------------------- one step
     def step(self, step: int, Q, out, h=None, qp_direct=None, stream=None, marks=None, on_select=None):
@@ -257,8 +398,12 @@ class SparseDecoder:
                     on_select(l)
         if marks:
             marks("attn_begin")
+        # the first launch after a prediction follows the last layer's
+        # selection, which wrote that layer's selection words
+        after_own_select = is_prediction_step(step, s.interval) and s.n_layers == 1
         for l in range(s.n_layers):
-            self.attend(step, l, Q[l], out[l], stream)
+            self.attend(step, l, Q[l], out[l], stream,
+                        prefetch=self.prefetch_kv and not (l == 0 and after_own_select))
         if marks:
             marks("attn_end")
 
@@ -266,7 +411,7 @@ class SparseDecoder:
         if marks:
             marks("attn_begin")
         for l in range(self.shape.n_layers):
-            self.attend_dense(step, l, Q[l], out[l], stream)
+            self.attend_dense(step, l, Q[l], out[l], stream, prefetch=self.prefetch_kv)
         if marks:
             marks("attn_end")
 

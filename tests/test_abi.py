@@ -46,16 +46,16 @@ def test_binding_constants_match_header(lib):
     h = _header_constants()
     for name in ("TB_OK", "TB_ERR_INVALID_ARG", "TB_ERR_UNSUPPORTED", "TB_ERR_CUDA", "TB_ERR_WORKSPACE",
                  "TB_ERR_DEVICE_FLAG", "TB_FLAG_CTX_RANGE", "TB_FLAG_TIMEOUT", "TB_FLAG_IDX_OVERFLOW",
-                 "TB_FLAG_BAD_CACHE"):
+                 "TB_FLAG_BAD_CACHE", "TB_ATTN_WAIT_ALL", "TB_ATTN_PREFETCH_KV"):
         assert getattr(_lib, name) == h[name], name
-        if name.startswith(("TB_OK", "TB_ERR")):
+        if name.startswith(("TB_OK", "TB_ERR_")):
             assert lib.tb_status_str(h[name]) == name.encode()
     assert _lib.TB_GROUP_REDUCE == {"max": h["TB_GROUP_MAX"], "sum": h["TB_GROUP_SUM"]}
     assert lib.tb_abi_version() == h["TB_ABI_VERSION"] == _lib.TB_ABI_VERSION
 
 
 def test_version_and_strings(lib):
-    assert lib.tb_abi_version() == 6
+    assert lib.tb_abi_version() == 8
     assert lib.tb_status_str(0) == b"TB_OK"
     assert lib.tb_status_str(2) == b"TB_ERR_UNSUPPORTED"
 
@@ -296,3 +296,17 @@ def test_noalloc_accepts_exactly_the_workspace_entry_points_dims(lib):
         assert noalloc(dims, **kw) == want, (dims.ctx_cap, kw)
     # valid dims beyond the fixed scratch: rejected before any CUDA call
     assert noalloc(_d(batch=16, ctx_cap=32896)) == _lib.TB_ERR_WORKSPACE
+
+
+def test_attention_launch_mode_is_per_thread_and_checked(lib):
+    import threading
+    assert lib.tb_attn_launch_mode() == _lib.TB_ATTN_WAIT_ALL
+    assert lib.tb_attn_set_launch_mode(7) == _lib.TB_ERR_INVALID_ARG
+    assert lib.tb_attn_set_launch_mode(_lib.TB_ATTN_PREFETCH_KV) == _lib.TB_OK
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(lib.tb_attn_launch_mode()))
+    t.start()
+    t.join()
+    assert seen == [_lib.TB_ATTN_WAIT_ALL], "another thread keeps the default"
+    assert lib.tb_attn_launch_mode() == _lib.TB_ATTN_PREFETCH_KV
+    assert lib.tb_attn_set_launch_mode(_lib.TB_ATTN_WAIT_ALL) == _lib.TB_OK

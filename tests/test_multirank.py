@@ -1,6 +1,9 @@
-"""The multi-rank host logic of the benchmark on CPU with gloo (world size 2):
-every rank decodes its own seeded replica, the job time is the slowest
-rank's, and the reported rate counts every rank's tokens."""
+"""The multi-rank host logic on CPU with gloo (world sizes 2 and 3): every
+rank decodes its own seeded replica, the job time is the slowest rank's, and
+the reported rate counts every rank's tokens; KV-head sharding and context
+sharding reproduce the single-device oracle results from the ranks' shares
+and their exchanges."""
+import math
 import os
 import socket
 
@@ -179,3 +182,127 @@ def test_sharded_predictor_rows_give_the_sharded_queries():
         got = oracle.predict_queries(parity.bits16(h), parity.bits16(W1), parity.bits16(W2r)).reshape(
             w.batch, w.slots, len(qh), w.d_proj)
         assert np.array_equal(got, full[:, :, qh.start:qh.stop])
+
+
+# ------------------------------------------------------------ context sharding
+
+def _cp_case():
+    return tb_inputs.WORKLOADS["tiny300"].scaled(name="cp_tiny", ctx0=700, ctx0_lo=700, ctx0_hi=700, budget=40)
+
+
+def _cp_worker(rank, world, port, q):
+    # one rank's share of a context-sharded step, computed by the oracle on the
+    # rank's block: its local top-B, the exchange of candidates, the merge and
+    # its block's part of the attention as an unnormalised (m, l, o) state
+    import numpy as np
+
+    import oracle
+    import parity
+    from query_aware_sparse_tb_b200.decode import context_blocks, local_rows, local_selection_params
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = _cp_case()
+        T = w.ctx0 + 1
+        blk = context_blocks(w.ctx_cap, world, w.window)[rank]
+        K, V = tb_inputs.kv_layer(w, 0, "cpu")
+        Kb, Vb = parity.bits16(K), parity.bits16(V)
+        Wk = parity.bits16(tb_inputs.wk_layer(w, 0, "cpu"))
+        qp = tb_inputs.direct_qp(w, 0, 0, "cpu").numpy()
+        Q = parity.bits16(tb_inputs.query(w, 0, 0, "cpu"))
+        lT, lS = local_selection_params(T, blk, w.sink, w.window)
+        rows = local_rows(T, blk)
+        cands = {}
+        for h in range(w.n_q_heads):
+            g = h // w.group
+            Kp = oracle.project_keys(Kb[0, g, blk[0]:blk[0] + max(0, lT - w.window)], Wk[g])
+            s = oracle.scores(qp[0, h], Kp, lS, lT - w.window) if lT - w.window > lS else np.zeros(0, np.float32)
+            top = oracle.select(s, lT, lS, w.window, w.budget, 0)
+            cands[h] = [(float(s[t - lS]), int(t + blk[0])) for t in top]
+        allc = [None] * world
+        dist.all_gather_object(allc, cands)
+        parts = {}
+        for h in range(w.n_q_heads):
+            pool = sorted((c for rc in allc for c in rc[h]), key=lambda c: (-c[0], c[1]))[:w.budget]
+            lo, hi = w.sink, T - w.window
+            I = sorted({t + k for _, t in pool for k in range(-w.nbr, w.nbr + 1) if lo <= t + k < hi})
+            A = [t for t in oracle.attention_set(T, w.sink, w.window, np.array(I, np.int32))
+                 if blk[0] <= t < blk[0] + rows and t < T]
+            g = h // w.group
+            qv = parity.bf16_to_f64(Q[0, h])
+            if A:
+                kk = parity.bf16_to_f64(Kb[0, g, A])
+                vv = parity.bf16_to_f64(Vb[0, g, A])
+                logit = kk @ qv / math.sqrt(w.head_dim)
+                m = logit.max()
+                p = np.exp(logit - m)
+                parts[h] = (m, p.sum(), p @ vv, I)
+            else:
+                parts[h] = (-np.inf, 0.0, np.zeros(w.head_dim), I)
+        allp = [None] * world
+        dist.all_gather_object(allp, parts)
+        q.put((rank, allp))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_sharding_gloo(world):
+    # each rank holds one block of the context; the merged selection equals the
+    # single-device oracle selection exactly and the combined attention equals
+    # the single-device oracle attention
+    import numpy as np
+
+    import oracle
+    import parity
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    w = _cp_case()
+    T = w.ctx0 + 1
+    K, V = tb_inputs.kv_layer(w, 0, "cpu")
+    Kb, Vb = parity.bits16(K), parity.bits16(V)
+    Wk = parity.bits16(tb_inputs.wk_layer(w, 0, "cpu"))
+    qp = tb_inputs.direct_qp(w, 0, 0, "cpu").numpy()
+    Q = parity.bits16(tb_inputs.query(w, 0, 0, "cpu"))
+    for rank, allp in results:
+        for h in range(w.n_q_heads):
+            g = h // w.group
+            Kp = oracle.project_keys(Kb[0, g, :T], Wk[g])
+            I_ref = oracle.select(oracle.scores(qp[0, h], Kp, w.sink, T - w.window), T, w.sink, w.window, w.budget,
+                                  w.nbr)
+            states = [p[h] for p in allp]
+            for st in states:
+                assert np.array_equal(np.array(st[3], np.int64), I_ref), (rank, h)
+            M = max(st[0] for st in states)
+            num = sum(np.exp(st[0] - M) * st[2] for st in states if st[0] != -np.inf)
+            den = sum(np.exp(st[0] - M) * st[1] for st in states if st[0] != -np.inf)
+            ref = oracle.attention(Q[0, h], Kb[0, g], Vb[0, g], oracle.attention_set(T, w.sink, w.window, I_ref),
+                                   1 / math.sqrt(w.head_dim))
+            assert np.allclose(num / den, ref, atol=1e-6, rtol=0), (rank, h)
+
+
+def test_context_block_helpers():
+    from query_aware_sparse_tb_b200.decode import (block_capacity, context_blocks, local_rows,
+                                                   local_selection_params)
+    for cap, world, N in ((65792, 4, 64), (832, 3, 16), (300, 2, 16)):
+        blocks = context_blocks(cap, world, N)
+        assert blocks[0][0] == 0 and blocks[-1][1] == cap
+        for (a0, a1), (b0, b1) in zip(blocks, blocks[1:]):
+            assert a1 == b0 and a0 % 32 == 0 and a0 % N == 0
+        for T in (1, 17, cap // 2, cap):
+            covered = []
+            for blk in blocks:
+                lT, lS = local_selection_params(T, blk, 4, N)
+                assert 1 <= lT <= block_capacity(blk, N)
+                covered += [t + blk[0] for t in range(lS, lT - N)]   # the block's local candidates
+                assert 1 <= local_rows(T, blk) <= blk[1] - blk[0] or blk[1] == blk[0]
+            assert covered == list(range(4, max(4, T - N))), (cap, world, T)
