@@ -9,8 +9,9 @@
 // selected tokens are expanded by their spatial neighbours.
 //
 // Exact top-B on the fp32 scores, ties broken by the lower position:
-//   1. score_hist   one CTA per (b, KV head, 2048 positions): reads each K'
-//                   row once for the 4 query heads of the group, writes the
+//   1. score_hist   one CTA per (b, KV head, 2048 positions): brings the K'
+//                   rows in by double-buffered 1-D bulk copies (TMA), reads
+//                   each row once for the 4 query heads of the group, writes the
 //                   order-preserving uint32 image of every score, and builds
 //                   a histogram of its top 11 bits per query head.  The last
 //                   CTA of each (b, KV head) (atomic ticket, no waiting) finds
@@ -37,8 +38,9 @@ namespace tb {
 namespace {
 
 constexpr int kGroup = 4;
-constexpr int kChunk = 1024;          // positions per CTA of mark_collect
+constexpr int kChunk = 2048;          // positions per CTA of mark_collect (one wave at 64K)
 constexpr int kHistChunk = 2048;      // positions per CTA of score_hist (one wave at 64K)
+constexpr int kSubRows = 512;         // K' rows per bulk-copied sub-chunk of score_hist
 constexpr int kThreads = 256;
 constexpr int kBins1 = 2048;          // key bits 31..21
 constexpr int kBins2 = 2048;          // key bits 20..10
@@ -173,17 +175,29 @@ __global__ void __launch_bounds__(kThreads, 2)
 score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
-    constexpr int PER = kHistChunk / kThreads;  // positions per thread
     constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
+    constexpr int NSUB = kHistChunk / kSubRows;         // staged sub-chunks per CTA
+    constexpr int RPT = kSubRows / kThreads;            // rows per thread per sub-chunk
+    constexpr int ROWB = DP * 2;                        // bytes per K' row
+    constexpr int V16 = ROWB / 16;                      // 16-byte parts per row
+    extern __shared__ __align__(128) uint8_t stage[];   // [2][kSubRows][ROWB]: K' rows, double-buffered
     __shared__ __align__(16) float qs[kGroup][DP];
     __shared__ uint32_t hist[NH][kBins1];
+    __shared__ __align__(8) uint64_t bars[2];
     __shared__ int s_last;
     __shared__ int scratch[kThreads / 32 + 3];
     const int tid = threadIdx.x;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int p0 = ch * kHistChunk;
+    const uint32_t stage_s = smem_addr(stage);
+    auto bar = [&](int k) { return smem_addr(&bars[k]); };
 
     for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
+    if (tid == 0) {
+        mbar_init(bar(0), 1);
+        mbar_init(bar(1), 1);
+        fence_mbar_init();
+    }
     griddep_wait();
     griddep_launch_dependents();
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
@@ -193,68 +207,81 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     if (hi > lo && p0 < hi && p0 + kHistChunk > lo) {
-        // four rows per batch: all rows' loads (clamped into C) first, then
-        // the arithmetic straight from the packed bf16 pairs, with the 4
-        // heads' q' read from shared memory once per 8 dims
-        constexpr int R = 4;
+        // the chunk's K' rows (contiguous for one (b, g)) come in sub-chunks of
+        // kSubRows by 1-D bulk copies, two in flight: sub-chunk k+2 is
+        // requested as soon as sub-chunk k has been read.  Only sub-chunks
+        // that overlap C are fetched; rows outside C are scored and dropped.
+        const int j_lo = max(0, lo - p0) / kSubRows;
+        const int j_hi = min(NSUB, (hi - p0 + kSubRows - 1) / kSubRows);
+        auto issue = [&](int k) {  // sub-chunk j_lo + k into buffer k & 1 (thread 0)
+            const int r0 = p0 + (j_lo + k) * kSubRows;
+            const int nrows = min(kSubRows, Tcap - r0);
+            mbar_arrive_expect_tx(bar(k & 1), (uint32_t)(nrows * ROWB));
+            bulk_load(stage_s + (uint32_t)((k & 1) * kSubRows * ROWB), Kp + (slab + r0) * DP,
+                      (uint32_t)(nrows * ROWB), bar(k & 1));
+        };
+        const int n_sub = j_hi - j_lo;
+        if (tid == 0) {
+            issue(0);
+            if (n_sub > 1) issue(1);
+        }
+        int waited = 0;  // sub-chunks whose copy has been waited for
+        for (int k = 0; k < n_sub; ++k) {
+            const bool ok = __syncthreads_and(mbar_wait_bounded(bar(k & 1), (k >> 1) & 1, ws.flags));
+            waited = k + 1;
+            if (!ok) break;
+            const uint8_t *buf = stage + (k & 1) * kSubRows * ROWB;
+            const int pb = p0 + (j_lo + k) * kSubRows;
+            // rows tid + m * kThreads share one rotation of the 16-byte parts,
+            // which keeps a quarter-warp's reads on distinct banks
+            const int rot = (tid >> (V16 == 4 ? 1 : 2)) & (V16 - 1);
+            float sc[RPT][kGroup];
 #pragma unroll
-        for (int k0 = 0; k0 < PER; k0 += R) {
-            uint4 raw[R][DP / 8];
+            for (int m = 0; m < RPT; ++m)
 #pragma unroll
-            for (int k = 0; k < R; ++k) {
-                const int p = min(max(p0 + (k0 + k) * kThreads + tid, lo), hi - 1);
-                const uint4 *row = reinterpret_cast<const uint4 *>(Kp + (slab + p) * DP);
+                for (int h = 0; h < kGroup; ++h) sc[m][h] = 0.f;
 #pragma unroll
-                for (int v = 0; v < DP / 8; ++v) raw[k][v] = __ldg(row + v);
-            }
-            float sc[R][kGroup];
-#pragma unroll
-            for (int k = 0; k < R; ++k)
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) sc[k][h] = 0.f;
-#pragma unroll
-            for (int v = 0; v < DP / 8; ++v) {
+            for (int vv = 0; vv < V16; ++vv) {
+                const int pv = (vv + rot) & (V16 - 1);
                 float4 qv[kGroup][2];
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) {
-                    qv[h][0] = *reinterpret_cast<const float4 *>(&qs[h][8 * v]);
-                    qv[h][1] = *reinterpret_cast<const float4 *>(&qs[h][8 * v + 4]);
+                    qv[h][0] = *reinterpret_cast<const float4 *>(&qs[h][8 * pv]);
+                    qv[h][1] = *reinterpret_cast<const float4 *>(&qs[h][8 * pv + 4]);
                 }
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float kl[R], kh[R];
+                for (int m = 0; m < RPT; ++m) {
+                    const uint4 raw = *reinterpret_cast<const uint4 *>(buf + (tid + m * kThreads) * ROWB + pv * 16);
 #pragma unroll
-                    for (int k = 0; k < R; ++k) {
-                        const uint32_t wd = e == 0 ? raw[k][v].x : e == 1 ? raw[k][v].y : e == 2 ? raw[k][v].z : raw[k][v].w;
-                        kl[k] = bf16_lo(wd);
-                        kh[k] = bf16_hi(wd);
-                    }
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t wd = e == 0 ? raw.x : e == 1 ? raw.y : e == 2 ? raw.z : raw.w;
+                        const float kl = bf16_lo(wd), kh = bf16_hi(wd);
 #pragma unroll
-                    for (int h = 0; h < kGroup; ++h) {
-                        const float4 &q4 = qv[h][e >> 1];
-                        const float qa = (e & 1) ? q4.z : q4.x, qb = (e & 1) ? q4.w : q4.y;
-#pragma unroll
-                        for (int k = 0; k < R; ++k) sc[k][h] = fmaf(qb, kh[k], fmaf(qa, kl[k], sc[k][h]));
+                        for (int h = 0; h < kGroup; ++h) {
+                            const float4 &q4 = qv[h][e >> 1];
+                            const float qa = (e & 1) ? q4.z : q4.x, qb = (e & 1) ? q4.w : q4.y;
+                            sc[m][h] = fmaf(qb, kh, fmaf(qa, kl, sc[m][h]));
+                        }
                     }
                 }
             }
 #pragma unroll
-            for (int k = 0; k < R; ++k) {
-                const int p = p0 + (k0 + k) * kThreads + tid;
+            for (int m = 0; m < RPT; ++m) {
+                const int p = pb + tid + m * kThreads;
                 const bool valid = p >= lo && p < hi;
                 if constexpr (!sel_is_group(SEL)) {
 #pragma unroll
                     for (int h = 0; h < kGroup; ++h) {
-                        const uint32_t key = score_key(sc[k][h]);
+                        const uint32_t key = score_key(sc[m][h]);
                         if (valid) {
                             ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
                             atomicAdd(&hist[h][key >> 21], 1u);
                         }
                     }
                 } else {
-                    float gs = sc[k][0];
+                    float gs = sc[m][0];
 #pragma unroll
-                    for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, sc[k][h]) : gs + sc[k][h];
+                    for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, sc[m][h]) : gs + sc[m][h];
                     const uint32_t key = score_key(gs);
                     if (valid) {
                         ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
@@ -262,7 +289,15 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                     }
                 }
             }
+            __syncthreads();  // buffer k & 1 read by every thread before it is refilled
+            if (tid == 0 && k + 2 < n_sub) issue(k + 2);
         }
+        // a copy must not land after the CTA has gone: when a wait gave up on
+        // sub-chunk k, sub-chunk k + 1 may still be in flight; wait for it
+        // (bounded) before leaving
+        if (tid == 0)
+            for (int k = waited; k < min(n_sub, waited + 1); ++k)
+                (void)mbar_wait_bounded(bar(k & 1), (k >> 1) & 1, ws.flags);
     }
     __syncthreads();
     for (int i = tid; i < NH * kBins1; i += kThreads) {
@@ -412,17 +447,23 @@ __device__ __forceinline__ uint32_t range_mask(int w, int lo, int hi) {
     return upto & ~((1u << start) - 1u);
 }
 
+// One CTA per (b, query head) (per KV head in the group modes) of NT threads:
+// 1024 on the default path, 512 for the variants, which need more registers.
 template <int SEL>
-__global__ void __launch_bounds__(kFinThreads)
+__host__ __device__ constexpr int fin_threads() { return SEL == kSelHead ? kFinThreads : kFinThreads / 2; }
+
+template <int SEL>
+__global__ void __launch_bounds__(fin_threads<SEL>())
 finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int sink, int window,
                 int budget, int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
                 uint32_t *__restrict__ sel_bits, SelWs ws) {
+    constexpr int NT = fin_threads<SEL>();
     extern __shared__ unsigned long long fsm8[];
     unsigned long long *cand_s = fsm8;                                  // [kCandCache]
     uint32_t *top_s = reinterpret_cast<uint32_t *>(fsm8 + kCandCache);  // [W]
     uint32_t *tie_s = top_s + W;                                        // [W]
     __shared__ uint32_t hist[kBins2];
-    __shared__ int scratch[kFinThreads / 32 + 3];
+    __shared__ int scratch[NT / 32 + 3];
 
     // a group's set is computed in its first head's rows and written to all 4
     constexpr int NOUT = sel_is_group(SEL) ? kGroup : 1;
@@ -435,7 +476,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
     const int lo = sink, hi = T - window;
     const HeadState st = ws.state[row];
 
-    for (int w = tid; w < W; w += kFinThreads) {
+    for (int w = tid; w < W; w += NT) {
         top_s[w] = ws.top[row * W + w];
         tie_s[w] = 0u;
     }
@@ -445,31 +486,31 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         // when it fits
         const unsigned long long *cand = ws.cand + row * Tcap;
         if (n <= kCandCache) {
-            for (int i = tid; i < n; i += kFinThreads) cand_s[i] = cand[i];
+            for (int i = tid; i < n; i += NT) cand_s[i] = cand[i];
             cand = cand_s;
         }
         // digit 2: key bits 20..10 inside bin b1
-        for (int i = tid; i < kBins2; i += kFinThreads) hist[i] = 0u;
+        for (int i = tid; i < kBins2; i += NT) hist[i] = 0u;
         __syncthreads();
-        for (int i = tid; i < n; i += kFinThreads) {
+        for (int i = tid; i < n; i += NT) {
             const uint32_t key = (uint32_t)(cand[i] >> 32);
             atomicAdd(&hist[(key >> 10) & 0x7FFu], 1u);
         }
         __syncthreads();
         uint32_t k2;
-        const uint32_t b2 = (uint32_t)block_find_bin_desc<kFinThreads>(hist, kBins2, st.k_rem, &k2, scratch, false);
+        const uint32_t b2 = (uint32_t)block_find_bin_desc<NT>(hist, kBins2, st.k_rem, &k2, scratch, false);
         // digit 3: key bits 9..0 inside (b1, b2)
-        for (int i = tid; i < kBins3; i += kFinThreads) hist[i] = 0u;
+        for (int i = tid; i < kBins3; i += NT) hist[i] = 0u;
         __syncthreads();
-        for (int i = tid; i < n; i += kFinThreads) {
+        for (int i = tid; i < n; i += NT) {
             const uint32_t key = (uint32_t)(cand[i] >> 32);
             if (((key >> 10) & 0x7FFu) == b2) atomicAdd(&hist[key & 0x3FFu], 1u);
         }
         __syncthreads();
         uint32_t k3;  // keys equal to tau still to take, lowest positions first
-        const uint32_t b3 = (uint32_t)block_find_bin_desc<kFinThreads>(hist, kBins3, k2, &k3, scratch, false);
+        const uint32_t b3 = (uint32_t)block_find_bin_desc<NT>(hist, kBins3, k2, &k3, scratch, false);
         const uint32_t tau = (st.b1 << 21) | (b2 << 10) | b3;
-        for (int i = tid; i < n; i += kFinThreads) {
+        for (int i = tid; i < n; i += NT) {
             const unsigned long long e = cand[i];
             const uint32_t key = (uint32_t)(e >> 32), p = (uint32_t)e;
             if (key > tau) atomicOr(&top_s[p >> 5], 1u << (p & 31));
@@ -477,12 +518,12 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         }
         __syncthreads();
         // ties in position order: each thread owns a contiguous run of words
-        const int wpt = (W + kFinThreads - 1) / kFinThreads;
+        const int wpt = (W + NT - 1) / NT;
         const int wb = tid * wpt, we = min(wb + wpt, W);
         int mine = 0;
         for (int w = wb; w < we; ++w) mine += __popc(tie_s[w]);
         int tot;
-        int before = block_excl_scan<kFinThreads>(mine, scratch, &tot);
+        int before = block_excl_scan<NT>(mine, scratch, &tot);
         for (int w = wb; w < we; ++w) {
             uint32_t t = tie_s[w];
             const int pc = __popc(t);
@@ -514,12 +555,12 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         uint16_t *gain_s = reinterpret_cast<uint16_t *>(tie_s + W);
         uint32_t *wpref = tie_s;
         // 1. gather (key, position) of the top positions, words in order
-        const int wpt = (W + kFinThreads - 1) / kFinThreads;
+        const int wpt = (W + NT - 1) / NT;
         const int wb = tid * wpt, we = min(wb + wpt, W);
         int mine = 0;
         for (int w = wb; w < we; ++w) mine += __popc(top_s[w]);
         int n_top;
-        const int base = block_excl_scan<kFinThreads>(mine, scratch, &n_top);
+        const int base = block_excl_scan<NT>(mine, scratch, &n_top);
         {
             int acc = base;
             for (int w = wb; w < we; ++w) {
@@ -559,7 +600,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         };
         auto is_top = [&](int u) { return (top_s[u >> 5] >> (u & 31)) & 1u; };
         uint32_t my_gain = 0;
-        for (int j = tid; j < n_top; j += kFinThreads) {
+        for (int j = tid; j < n_top; j += NT) {
             const unsigned long long cp = cand_s[j];
             const int p = (int)(0xFFFFFFFFu - (uint32_t)cp);
             uint32_t gain = 0;
@@ -573,7 +614,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
             my_gain += gain;
         }
         int total_gain;
-        (void)block_excl_scan<kFinThreads>((int)my_gain, scratch, &total_gain);
+        (void)block_excl_scan<NT>((int)my_gain, scratch, &total_gain);
         // 3. the first candidate in score order whose running gain exceeds B:
         //    MSB-first radix over its 64-bit composite, weighted by the gains
         //    (six passes of 11/11/11/11/10/10 bits); the kept candidates are
@@ -588,16 +629,16 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
                 const int dw = pass < 4 ? 11 : 10;
                 const int nb = 1 << dw;
                 const int shift = 64 - fixed - dw;
-                for (int i = tid; i < nb; i += kFinThreads) hist[i] = 0u;
+                for (int i = tid; i < nb; i += NT) hist[i] = 0u;
                 __syncthreads();
-                for (int j = tid; j < n_top; j += kFinThreads) {
+                for (int j = tid; j < n_top; j += NT) {
                     const unsigned long long cp = cand_s[j];
                     if (fixed == 0 || (cp >> (64 - fixed)) == prefix)
                         atomicAdd(&hist[(uint32_t)(cp >> shift) & (uint32_t)(nb - 1)], (uint32_t)gain_s[j]);
                 }
                 __syncthreads();
                 uint32_t rem;
-                const uint32_t bin = (uint32_t)block_find_bin_desc<kFinThreads>(hist, nb, need, &rem, scratch, false);
+                const uint32_t bin = (uint32_t)block_find_bin_desc<NT>(hist, nb, need, &rem, scratch, false);
                 prefix = (prefix << dw) | bin;
                 fixed += dw;
                 need = rem;
@@ -605,9 +646,9 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
             cut = prefix;
         }
         // the kept positions: composites above the cut (or all)
-        for (int w = tid; w < W; w += kFinThreads) tie_s[w] = 0u;
+        for (int w = tid; w < W; w += NT) tie_s[w] = 0u;
         __syncthreads();
-        for (int j = tid; j < n_top; j += kFinThreads) {
+        for (int j = tid; j < n_top; j += NT) {
             const unsigned long long cp = cand_s[j];
             if (total_gain <= budget || cp > cut) {
                 const uint32_t p = 0xFFFFFFFFu - (uint32_t)cp;
@@ -615,12 +656,12 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
             }
         }
         __syncthreads();
-        for (int w = tid; w < W; w += kFinThreads) top_s[w] = tie_s[w];
+        for (int w = tid; w < W; w += NT) top_s[w] = tie_s[w];
         __syncthreads();
     }
 
     // neighbour fetch, clip to C, emit bitmap and sorted index list
-    const int wpt = (W + kFinThreads - 1) / kFinThreads;
+    const int wpt = (W + NT - 1) / NT;
     const int wb = tid * wpt, we = min(wb + wpt, W);
     int mine = 0;
     for (int w = wb; w < we; ++w) {
@@ -633,7 +674,7 @@ finalize_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, in
         mine += __popc(e);
     }
     int total;
-    const int base = block_excl_scan<kFinThreads>(mine, scratch, &total);
+    const int base = block_excl_scan<NT>(mine, scratch, &total);
     for (int w = wb; w < we; ++w)
 #pragma unroll
         for (int o = 0; o < NOUT; ++o) sel_bits[(row + o) * W + w] = tie_s[w];
@@ -901,11 +942,22 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
     const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
     dim3 grid(nch, d.n_kv_heads, d.batch);
     dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
-    cudaError_t e = d.d_proj == 32
-        ? launch_pdl(score_hist_kernel<32, SEL>, grid_h, dim3(kThreads), 0, st, qp, qp_stride, Kp, ctx_len,
-                     d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s)
-        : launch_pdl(score_hist_kernel<16, SEL>, grid_h, dim3(kThreads), 0, st, qp, qp_stride, Kp, ctx_len,
-                     d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    cudaError_t e;
+    const int hsm = 2 * kSubRows * d.d_proj * 2;  // two staged sub-chunks of K' rows
+    if (d.d_proj == 32) {
+        static std::atomic<int> smem_set32[kMaxDevices];
+        if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<32, SEL>, hsm, smem_set32)) != cudaSuccess)
+            return e;
+        e = launch_pdl(score_hist_kernel<32, SEL>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp, ctx_len,
+                       d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    } else {
+        // (with the static histogram the total is past the default 48 KB here too)
+        static std::atomic<int> smem_set16[kMaxDevices];
+        if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<16, SEL>, hsm, smem_set16)) != cudaSuccess)
+            return e;
+        e = launch_pdl(score_hist_kernel<16, SEL>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp, ctx_len,
+                       d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    }
     if (e != cudaSuccess) return e;
     e = launch_pdl(mark_collect_kernel<SEL>, grid, dim3(kThreads), 0, st, ctx_len, d.n_q_heads, d.n_kv_heads,
                    d.ctx_cap, W, sink, window, s);
@@ -917,7 +969,7 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
         if (e != cudaSuccess) return e;
     }
     const int rows = sel_is_group(SEL) ? d.n_q_heads / kGroup : d.n_q_heads;
-    return launch_pdl(finalize_kernel<SEL>, dim3(rows, d.batch), dim3(kFinThreads), fsm, st, ctx_len, d.n_q_heads,
+    return launch_pdl(finalize_kernel<SEL>, dim3(rows, d.batch), dim3(fin_threads<SEL>()), fsm, st, ctx_len, d.n_q_heads,
                       d.ctx_cap, W, sink, window, budget, nbr, idx, idx_cap, count, sel_bits, s);
 }
 
