@@ -418,22 +418,31 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
         const int mt = tid;  // tile row, then head dim
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         {
+            // P operands: rows 8..15 stay zero (shared memory only: before the wait)
+            uint4 *pz = reinterpret_cast<uint4 *>(sm + Smem::kP);
+            for (int e = mt; e < 2 * 4096 / 16; e += kRoleThreads) pz[e] = make_uint4(0u, 0u, 0u, 0u);
             if (prefetch) {
                 griddep_wait();  // Q may come from the previous kernel
                 if (early_trigger) griddep_launch_dependents();
             }
             // Q operand (K-major, 16 rows: the group's 4 query heads, then
-            // zeros); P operands: rows 8..15 stay zero
+            // zeros), one 16-byte chunk (8 dims) per load and per swizzled
+            // store: all of a thread's loads are in flight at once
             const uint16_t *Qg = Q + ((size_t)b * Hq + (size_t)g * kGroup) * D;
-            for (int e = mt; e < 2 * kN * 64; e += kRoleThreads) {
-                const int hf = e >> 10, n = (e >> 6) & 15, dd = e & 63, d = hf * 64 + dd;
-                uint16_t v = 0;
-                if (n < kGroup && d < D) v = Qg[(size_t)n * D + d];
-                *reinterpret_cast<uint16_t *>(sm + Smem::kQ + hf * 2048 + (n >> 3) * 1024 +
-                                              sw128_off(n & 7, dd >> 3) + (dd & 7) * 2) = v;
+            constexpr int kQChunks = kN * 16;  // 16 rows x (2 halves x 8 chunks of 8 dims)
+            uint4 qv[kQChunks / kRoleThreads];
+#pragma unroll
+            for (int k = 0; k < kQChunks / kRoleThreads; ++k) {
+                const int e = mt + k * kRoleThreads, n = e >> 4, c = e & 15;
+                qv[k] = (n < kGroup && c * 8 < D) ? *reinterpret_cast<const uint4 *>(Qg + (size_t)n * D + c * 8)
+                                                  : make_uint4(0u, 0u, 0u, 0u);
             }
-            uint4 *pz = reinterpret_cast<uint4 *>(sm + Smem::kP);
-            for (int e = mt; e < 2 * 4096 / 16; e += kRoleThreads) pz[e] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int k = 0; k < kQChunks / kRoleThreads; ++k) {
+                const int e = mt + k * kRoleThreads, n = e >> 4, c = e & 15;
+                *reinterpret_cast<uint4 *>(sm + Smem::kQ + (c >> 3) * 2048 + (n >> 3) * 1024 + sw128_off(n & 7, c & 7)) =
+                    qv[k];
+            }
             fence_proxy_async_smem();
             mbar_arrive(q_ready);
         }
@@ -587,9 +596,10 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     if (!s_last) return;
 
     // ---------------------------------------------------- last CTA merges
-    // One output group (head, 4 dims) per TPG threads; each thread folds its
-    // share of the ns <= 64 partial states with an online rescale (all loads
-    // of a batch issued first), then the TPG lanes combine with shuffles.
+    // One output group (head, 4 dims) per TPG threads; each thread loads its
+    // share of the ns <= 64 partial states (one round for up to 32 splits),
+    // scales them to the round's largest reference and sums, then the TPG
+    // lanes combine with shuffles.
     constexpr int kGroups4 = kGroup * D / 4;
     constexpr int TPG = kMergeThreads / kGroups4;
     if (tid < kMergeThreads) {
@@ -623,8 +633,23 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                     v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
+            // the round's largest reference first, then every state scaled to
+            // it independently (no chain of dependent rescales)
+            float Mr = -INFINITY;
 #pragma unroll
-            for (int u = 0; u < kU; ++u) fold(ml[u].x, ml[u].y, v[u]);
+            for (int u = 0; u < kU; ++u) Mr = fmaxf(Mr, ml[u].x);
+            if (Mr != -INFINITY) {
+                float Lr = 0.f;
+                float4 orr = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const float c = exp2f(ml[u].x - Mr);  // 0 for a slice with no kept row (-inf)
+                    orr.x = fmaf(v[u].x, c, orr.x); orr.y = fmaf(v[u].y, c, orr.y);
+                    orr.z = fmaf(v[u].z, c, orr.z); orr.w = fmaf(v[u].w, c, orr.w);
+                    Lr = fmaf(ml[u].y, c, Lr);
+                }
+                fold(Mr, Lr, orr);
+            }
         }
 #pragma unroll
         for (int off = 1; off < TPG; off <<= 1) {
