@@ -310,3 +310,44 @@ def test_attention_launch_mode_is_per_thread_and_checked(lib):
     assert seen == [_lib.TB_ATTN_WAIT_ALL], "another thread keeps the default"
     assert lib.tb_attn_launch_mode() == _lib.TB_ATTN_PREFETCH_KV
     assert lib.tb_attn_set_launch_mode(_lib.TB_ATTN_WAIT_ALL) == _lib.TB_OK
+
+
+def test_context_parallel_calls_reject_bad_arguments(lib):
+    d = _d()
+    wsb = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
+    # export: misaligned candidates, bad budget, offset overflow, short workspace
+    exp = lambda dims=d, ws=FAKE, nb=wsb, idx=FAKE, cap=8192, cnt=FAKE, budget=8192, off=0, cand=FAKE: \
+        lib.tb_select_export_candidates(ctypes.byref(dims), ws, nb, idx, cap, cnt, budget, off, cand, None)  # noqa: E731
+    assert exp(cand=FAKE + 4) == _lib.TB_ERR_INVALID_ARG
+    assert exp(budget=0) == _lib.TB_ERR_INVALID_ARG
+    assert exp(off=-1) == _lib.TB_ERR_INVALID_ARG
+    assert exp(off=0x7fffffff) == _lib.TB_ERR_INVALID_ARG
+    assert exp(nb=wsb - 1) == _lib.TB_ERR_WORKSPACE
+    assert exp(dims=_d(d_proj=24)) == _lib.TB_ERR_UNSUPPORTED
+
+    def merge(**kw):
+        a = dict(dims=d, cand=FAKE, ranks=4, budget=8192, ctx=FAKE, sink=16, window=64, nbr=1, idx=FAKE,
+                 cap=24576, cnt=FAKE, sb=0, sl=16384, lcap=16448, bits=FAKE, ws=FAKE, nb=256)
+        a.update(kw)
+        return lib.tb_select_merge_candidates(ctypes.byref(a["dims"]), a["cand"], a["ranks"], a["budget"], a["ctx"],
+                                              a["sink"], a["window"], a["nbr"], a["idx"], a["cap"], a["cnt"], a["sb"],
+                                              a["sl"], a["lcap"], a["bits"], a["ws"], a["nb"], None)
+    assert merge(sb=16) == _lib.TB_ERR_INVALID_ARG            # shard_begin not a multiple of 32
+    assert merge(sl=20000) == _lib.TB_ERR_INVALID_ARG         # shard longer than its local capacity
+    assert merge(sb=65536, sl=16384, lcap=16448) == _lib.TB_ERR_INVALID_ARG   # past ctx_cap
+    assert merge(ranks=0) == _lib.TB_ERR_INVALID_ARG
+    assert merge(cap=100) == _lib.TB_ERR_INVALID_ARG          # idx_cap below the largest selection
+    assert merge(window=0) == _lib.TB_ERR_INVALID_ARG
+    assert merge(nb=255) == _lib.TB_ERR_WORKSPACE
+    assert merge(cand=FAKE + 4) == _lib.TB_ERR_INVALID_ARG
+    # partial attention and combine
+    ab = lib.tb_attn_workspace_bytes(ctypes.byref(d))
+    part = lambda dims=d, bits=FAKE, nb=ab, scale=0.088: lib.tb_sparse_decode_attn_partial(  # noqa: E731
+        ctypes.byref(dims), FAKE, FAKE, FAKE, FAKE, bits, scale, FAKE, FAKE, nb, None)
+    assert part(bits=0) == _lib.TB_ERR_INVALID_ARG
+    assert part(nb=ab - 1) == _lib.TB_ERR_WORKSPACE
+    assert part(dims=_d(head_dim=96)) == _lib.TB_ERR_UNSUPPORTED
+    assert part(scale=float("nan")) == _lib.TB_ERR_INVALID_ARG
+    assert lib.tb_attn_combine(FAKE, 0, 1, 32, 128, FAKE, None) == _lib.TB_ERR_INVALID_ARG
+    assert lib.tb_attn_combine(FAKE, 2, 1, 32, 96, FAKE, None) == _lib.TB_ERR_UNSUPPORTED
+    assert lib.tb_attn_combine(FAKE + 2, 2, 1, 32, 128, FAKE, None) == _lib.TB_ERR_INVALID_ARG
