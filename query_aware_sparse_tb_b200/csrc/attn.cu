@@ -202,29 +202,34 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     }
 
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && split == 0 && g == 0);
-    // the context split evenly over the CTAs of (b, g), in whole selection
-    // words; with prefetch by the length itself, otherwise by the capacity so
-    // that a CTA's first positions are known before the length arrives
-    const int span = prefetch ? T : Tcap;
-    const int chunk = ((span + splits - 1) / splits + 31) / 32 * 32;
-    const int p_begin = split * chunk;
-    const int ns = (T + chunk - 1) / chunk;  // CTAs of (b, g) that hold rows
-    const int p_end = min(p_begin + chunk, T);
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     const uint16_t *Kb = K + slab * D;
     const uint16_t *Vb = V + slab * D;
     float *part_bg = part + (size_t)(b * Hkv + g) * splits * kPartStride;
+    const int pt = tid - kRoleThreads, pw = warp - 4;
+    const bool loader = warp >= 4 && warp < 8;
+    const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
+    const int hi_c = T - window;  // candidates are [sink, hi_c)
+
+    // This CTA's slice [p_begin, p_end) of (b, g): equal shares of the length,
+    // cut at whole 32-position selection words (slice s opens at the word that
+    // holds position s * T / splits).  Sparse and dense use the same slices, so
+    // with every candidate selected they do identical arithmetic.  (Cutting
+    // the sparse slices at equal kept rows instead, counted from the group's
+    // selection words, balanced the tiles but cost more at the start than it
+    // saved: 42.3 against 38.7 us per 64K launch.)
+    const int p_begin = (int)(((long long)split * T / splits) >> 5) << 5;
+    const int p_end = split + 1 == splits
+                          ? T
+                          : max(p_begin, min((int)(((long long)(split + 1) * T / splits) >> 5) << 5, T));
+    const int ns = splits;  // every CTA writes a state, empty slices with M = -inf
 
     // sparse: load warp thread pt owns word pt (32 positions) of a sub-chunk;
     // the group's 4 selection words of the first sub-chunk are requested
     // before the set-up, those of the next one while the current is streamed
-    const int pt = tid - kRoleThreads, pw = warp - 4;
-    const bool loader = warp >= 4 && warp < 8;
-    const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
     uint32_t hw[kGroup] = {0u, 0u, 0u, 0u};
-    // (bounded by the slice and the capacity only: words past the length are
-    // masked when the list is built)
-    const int p_cap_end = min(p_begin + chunk, Tcap);
+    // (words past the length are masked when the list is built)
+    const int p_cap_end = min((p_end + 31) & ~31, Tcap);
     auto fetch_words = [&](int q0) {
         const int q1 = min(q0 + kSub, p_cap_end);
         if (q0 + 32 * pt < q1) {
@@ -247,7 +252,6 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
         int it = 0;
         bool fail = false;
         const int step = SPARSE ? kSub : max(p_end - p_begin, 1);
-        const int hi_c = T - window;  // candidates are [sink, hi_c)
         for (int p0 = p_begin; p0 < p_end && !fail; p0 += step) {
             const int p1 = min(p0 + step, p_end);
             int n_rows = p1 - p0;
@@ -561,7 +565,7 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
 #pragma unroll
         for (int h = 0; h < kGroup; ++h)
             L[h] = red[16 + h] + red[16 + kGroup + h] + red[16 + 2 * kGroup + h] + red[16 + 3 * kGroup + h];
-        if (p_begin < T) {
+        {
             float *pp = part_bg + (size_t)split * kPartStride;
             if (mt < D) {
 #pragma unroll

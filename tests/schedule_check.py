@@ -94,23 +94,25 @@ def _group_band(selection, bands, gk_bits, gqs):
     return np.sum(bands, 0) + 8 * 2.0 ** -24 * absum
 
 
-def check_schedule(run, layers, steps, seqs, heads, attn_steps, selection="head"):
+def check_schedule(run, layers, steps, seqs, heads, attn_steps, selection="head", data=None, before_step=None):
     """Run `steps` decode steps of bench.Run `run` (eagerly, through the
-    library) and check them against the oracle as described above.  Returns
-    counts of what was checked."""
+    library) and check them against the oracle as described above.  `data`
+    gives the oracle its inputs (default: the run's own buffers);
+    `before_step(i)`, if given, runs right before decode step i (e.g. a cache
+    append).  Returns counts of what was checked."""
     w, dec = run.w, run.dec
     s_ = dec.shape
     S, N, Bud, r = w.sink, w.window, w.budget, w.nbr
     group = selection in ("group_max", "group_sum")
     inclusive = selection == "inclusive"
     ctx0 = run.ctx0
-    data = RunData(run)
+    data = data or RunData(run)
     ref = oschedule.run(w, data, layers=layers, steps=steps, heads=heads, seqs=seqs, attn_steps=set(attn_steps),
                         selection=selection, keep=True)
     groups = sorted({hh // w.group for hh in heads})
     K_host = {}
     for l in layers:
-        Kl = host_kv(run, l)[0]
+        Kl = data.kv(l)[0]
         K_host.update({(l, b, g): Kl[b, g].copy() for b in seqs for g in groups})
         del Kl
     Wk_host = {l: parity.bits16(run.Wk[l]) for l in layers}
@@ -134,6 +136,8 @@ def check_schedule(run, layers, steps, seqs, heads, attn_steps, selection="head"
                 q_l = qd[l]
             snap[l] = (scores.cpu().numpy(), q_l.cpu().numpy(), {b: parity.bits16(dec.Kp[l][b]) for b in seqs})
 
+        if before_step:
+            before_step(i)
         dec.step(i, Q, run.out, h=h, qp_direct=qd, on_select=on_select)
         torch.cuda.synchronize()
         for ws in (dec.ws_attn, dec.ws_sel, dec.ws_proj, dec.ws_pred):

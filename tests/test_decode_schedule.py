@@ -29,3 +29,37 @@ def test_producers_and_slots_match_oracle_schedule():
             assert decode.producer_layer(layer, stride) == oschedule.producer_of(layer, stride)
             assert decode.query_slot(layer, stride) == oschedule.slot_of(layer, stride)
             assert decode.producer_layer(layer, stride) + decode.query_slot(layer, stride) == layer
+
+
+def test_attention_prefetch_only_where_the_contract_holds():
+    # the decoder asks for TB_ATTN_PREFETCH_KV on every attention launch except
+    # the first one right after the selection of the same (only) layer, whose
+    # selection words the preceding kernel has just written
+    from query_aware_sparse_tb_b200 import _lib as L
+
+    class Rec(decode.SparseDecoder):
+        def __init__(self, n_layers, interval, prefetch_kv):
+            self.shape = decode.DecodeShape(batch=1, n_layers=n_layers, n_q_heads=8, n_kv_heads=2, head_dim=64,
+                                            d_proj=16, hidden=0, inter=0, stride=1, sink=4, window=16, budget=8,
+                                            nbr=1, interval=interval, ctx_cap=512)
+            self.prefetch_kv = prefetch_kv
+            self.proj_begin, self.qp, self.calls = {}, {}, []
+
+        def select(self, step, layer, qp_direct=None, stream=None):
+            self.calls.append(("select", step, layer))
+
+        def attend(self, step, layer, Q, out, stream=None, prefetch=False):
+            self.calls.append(("attend", step, layer, prefetch))
+
+    for n_layers in (1, 3):
+        for interval in (1, 4):
+            for prefetch_kv in (False, True):
+                dec = Rec(n_layers, interval, prefetch_kv)
+                for i in range(6):
+                    dec.step(i, [None] * n_layers, [None] * n_layers, qp_direct=[None] * n_layers)
+                modes = [(c[1], c[2], c[3]) for c in dec.calls if c[0] == "attend"]
+                assert len(modes) == 6 * n_layers
+                for step, layer, pf in modes:
+                    right_after_own_select = n_layers == 1 and step % interval == 0
+                    assert pf == (prefetch_kv and not right_after_own_select), (n_layers, interval, step, layer)
+    assert L.TB_ATTN_WAIT_ALL == 0 and L.TB_ATTN_PREFETCH_KV == 1
