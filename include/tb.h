@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 8
+#define TB_ABI_VERSION 9
 
 typedef uint16_t tb_bf16;
 
@@ -227,6 +227,33 @@ tb_status tb_score_select_inclusive(const tb_dims *dims, const float *qp, int64_
  * call on `ws` overwrites them. */
 tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_bytes, const int32_t *ctx_len,
                                  int32_t sink, int32_t window, float *scores, void *stream);
+
+/* ---- selection algorithm -------------------------------------------------- */
+/* Which kernels carry out tb_score_select and tb_score_select_group (the
+ * result is the same, bit for bit: same scores, same set, same index list;
+ * no counterpart on the pages, a choice of route):
+ *
+ *   TB_SELECT_AUTO          (default) the cluster kernel where it applies,
+ *                           else the multi-kernel path.
+ *   TB_SELECT_MULTI_KERNEL  three kernels per call: scoring with a global
+ *                           histogram, marking and candidate collection, and
+ *                           a per-head finish (any ctx_cap).
+ *   TB_SELECT_CLUSTER       one kernel per call: a thread-block cluster per
+ *                           (sequence, KV head) holds all of its scores in
+ *                           shared memory.  It applies while ctx_cap fits
+ *                           (up to 81,920 positions for tb_score_select,
+ *                           327,680 for tb_score_select_group, on a device
+ *                           that places 16-CTA clusters); elsewhere the
+ *                           selection calls return TB_ERR_UNSUPPORTED.
+ *
+ * tb_score_select_inclusive always takes the multi-kernel path.  The
+ * algorithm belongs to the calling thread and is read when a selection call
+ * launches.  Any other value is TB_ERR_INVALID_ARG. */
+#define TB_SELECT_AUTO 0
+#define TB_SELECT_MULTI_KERNEL 1
+#define TB_SELECT_CLUSTER 2
+tb_status tb_select_set_algorithm(int32_t algorithm);
+int32_t   tb_select_algorithm(void);
 
 /* ---- context-parallel selection and attention ----------------------------- */
 /* One sequence's context split over R ranks (each holds the K, V and K' rows

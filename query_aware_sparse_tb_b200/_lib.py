@@ -15,11 +15,12 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtb.so")
 
-TB_ABI_VERSION = 8
+TB_ABI_VERSION = 9
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
 TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW, TB_FLAG_BAD_CACHE = 0x1, 0x2, 0x4, 0x8
 TB_GROUP_REDUCE = {"max": 0, "sum": 1}
 TB_ATTN_WAIT_ALL, TB_ATTN_PREFETCH_KV = 0, 1
+TB_SELECT_AUTO, TB_SELECT_MULTI_KERNEL, TB_SELECT_CLUSTER = 0, 1, 2
 
 EXPORTS = [
     "tb_abi_version", "tb_status_str", "tb_last_error",
@@ -31,6 +32,7 @@ EXPORTS = [
     "tb_select_export_candidates", "tb_select_merge_candidates", "tb_sparse_decode_attn_partial", "tb_attn_combine",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
     "tb_selftest_bounded_wait", "tb_attn_set_launch_mode", "tb_attn_launch_mode",
+    "tb_select_set_algorithm", "tb_select_algorithm",
 ]
 
 
@@ -89,6 +91,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_selftest_bounded_wait": ([P, sz, i64, P], ctypes.c_int),
         "tb_attn_set_launch_mode": ([i32], ctypes.c_int),
         "tb_attn_launch_mode": ([], i32),
+        "tb_select_set_algorithm": ([i32], ctypes.c_int),
+        "tb_select_algorithm": ([], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -276,6 +280,12 @@ def attn_set_launch_mode(mode: int):
     """tb_attn_set_launch_mode for the calling thread (TB_ATTN_WAIT_ALL or
     TB_ATTN_PREFETCH_KV; see include/tb.h for the contract of the latter)."""
     _check(load().tb_attn_set_launch_mode(int(mode)))
+
+
+def select_set_algorithm(algorithm: int):
+    """tb_select_set_algorithm for the calling thread (TB_SELECT_AUTO,
+    TB_SELECT_MULTI_KERNEL or TB_SELECT_CLUSTER; the result is the same)."""
+    _check(load().tb_select_set_algorithm(int(algorithm)))
 
 
 def decode_attn(d: TbDims, Q, K, V, ctx_len, scale: float, out, ws, stream=None):

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtb.so")
-SOURCES = ["api.cu", "attn.cu", "select.cu", "gemm_tc.cu", "noalloc.cu", "kv.cu"]
+SOURCES = ["api.cu", "attn.cu", "select.cu", "select_cluster.cu", "gemm_tc.cu", "noalloc.cu", "kv.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-cudart", "shared", "-I", os.path.join(ROOT, "include")]

@@ -16,8 +16,10 @@ namespace tb {
 
 static thread_local char g_err[512] = "";
 static thread_local int g_attn_mode = TB_ATTN_WAIT_ALL;
+static thread_local int g_select_algo = TB_SELECT_AUTO;
 
 int attn_launch_mode() { return g_attn_mode; }
+int select_algorithm() { return g_select_algo; }
 static std::mutex g_state_mu;  // serialises one-time per-device kernel set-up
 
 void set_error(const char *fmt, ...) {
@@ -174,6 +176,15 @@ tb_status tb_attn_set_launch_mode(int32_t mode) {
 
 int32_t tb_attn_launch_mode(void) { return g_attn_mode; }
 
+tb_status tb_select_set_algorithm(int32_t algorithm) {
+    if (algorithm != TB_SELECT_AUTO && algorithm != TB_SELECT_MULTI_KERNEL && algorithm != TB_SELECT_CLUSTER)
+        return fail(TB_ERR_INVALID_ARG, "tb_select_set_algorithm: unknown algorithm %d", algorithm);
+    g_select_algo = algorithm;
+    return TB_OK;
+}
+
+int32_t tb_select_algorithm(void) { return g_select_algo; }
+
 size_t tb_score_select_workspace_bytes(const tb_dims *dims) {
     if (check_dims(dims, true, __func__) != TB_OK || dims->ctx_cap > kMaxCtxSelect) return 0;
     return select_ws_bytes(*dims);
@@ -274,6 +285,9 @@ static tb_status score_select_impl(const char *fn, const tb_dims *dims, const fl
         return fail(TB_ERR_INVALID_ARG, "%s: idx_cap %d < %lld (the largest possible selection)", fn, idx_cap,
                     min_cap);
     if ((s = check_ws(ws, ws_bytes, select_ws_bytes(*dims), fn)) != TB_OK) return s;
+    if (g_select_algo == TB_SELECT_CLUSTER && group_reduce != 2 && !select_cluster_fits(*dims, group_reduce, false))
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d does not fit the cluster selection kernel", fn,
+                    dims->ctx_cap);
     return cuda_status(launch_score_select(*dims, qp, qp_batch_stride, Kp, ctx_len, sink, window, budget, nbr,
                                            group_reduce, idx, idx_cap, count, sel_bits, ws, (cudaStream_t)stream),
                        fn);

@@ -31,6 +31,14 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                 int32_t window, int32_t budget, int32_t nbr, int32_t group_reduce,
                                 int32_t *idx, int32_t idx_cap, int32_t *count, uint32_t *sel_bits,
                                 void *ws, cudaStream_t st);
+// The one-kernel cluster path of launch_score_select (select_cluster.cu) for
+// group_reduce -1, 0 and 1: whether it takes dims `d` (with one_wave: in one
+// wave of clusters, where it beats the multi-kernel path), and the launch.
+bool select_cluster_fits(const tb_dims &d, int32_t group_reduce, bool one_wave);
+cudaError_t launch_score_select_cluster(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
+                                        const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget,
+                                        int32_t nbr, int32_t group_reduce, int32_t *idx, int32_t idx_cap,
+                                        int32_t *count, uint32_t *sel_bits, void *ws, cudaStream_t st);
 cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t *ctx_len, int32_t sink,
                                  int32_t window, float *scores, cudaStream_t st);
 cudaError_t launch_export_candidates(const tb_dims &d, const void *ws, const int32_t *idx, int32_t idx_cap,
@@ -62,6 +70,8 @@ cudaError_t launch_bounded_wait_selftest(void *ws, long long budget_cycles, cuda
 void set_error(const char *fmt, ...);
 // The calling thread's attention launch mode (tb_attn_set_launch_mode, api.cu).
 int attn_launch_mode();
+// The calling thread's selection algorithm (tb_select_set_algorithm, api.cu).
+int select_algorithm();
 
 // Host-side argument checks of the attention entry points (api.cu), shared by
 // tb_sparse_decode_attn, tb_decode_attn and tb_sparse_decode_attn_noalloc so

@@ -33,140 +33,13 @@
 // select over the candidates' composites weighted by what each one adds).
 #include "common.cuh"
 #include "internal.h"
+#include "score.cuh"
+#include "select_common.cuh"
 
 namespace tb {
 namespace {
 
-constexpr int kGroup = 4;
-constexpr int kChunk = 2048;          // positions per CTA of mark_collect (one wave at 64K)
-constexpr int kHistChunk = 2048;      // positions per CTA of score_hist (one wave at 64K)
-constexpr int kSubRows = 512;         // K' rows per bulk-copied sub-chunk of score_hist
-constexpr int kThreads = 256;
-constexpr int kBins1 = 2048;          // key bits 31..21
-constexpr int kBins2 = 2048;          // key bits 20..10
-constexpr int kBins3 = 1024;          // key bits 9..0
-constexpr int kFinThreads = 1024;
-constexpr int kCandCache = 8192;      // candidates staged in shared memory by finalize
-constexpr unsigned kFull = 0xffffffffu;
-
-enum : uint32_t { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
-
-// What is selected: one set per query head, or one set per KV head (group)
-// from the largest or the fp32 sum (heads in order) of the group's scores.
-// A group's set is kept in the rows of its first head until finalize copies
-// it to all 4 heads.
-enum : int { kSelHead = 0, kSelGroupMax = 1, kSelGroupSum = 2, kSelInclusive = 3 };
-// kSelInclusive: per query head, but the importance buffer itself holds at
-// most B tokens (candidates in score order while the union of their
-// neighbourhoods fits); its budget is at most kCandCache.
-__host__ __device__ constexpr bool sel_is_group(int sel) { return sel == kSelGroupMax || sel == kSelGroupSum; }
-
-struct HeadState {   // 8 words per (b, query head)
-    uint32_t mode, b1, k_rem, cand_count, n_in_bin, pad[3];
-};
-
-struct SelWs {
-    uint32_t *flags, *keys, *hist, *counters;
-    HeadState *state;
-    unsigned long long *cand;
-    uint32_t *top;
-};
-
-SelWs carve(const tb_dims &d, void *ws) {
-    uint8_t *p = static_cast<uint8_t *>(ws);
-    const size_t rows = (size_t)d.batch * d.n_q_heads;
-    SelWs s;
-    size_t off = 0;
-    s.flags = reinterpret_cast<uint32_t *>(p);
-    off += kWsHeaderBytes;
-    s.keys = reinterpret_cast<uint32_t *>(p + off);
-    off += align_up(rows * d.ctx_cap * 4, 256);
-    s.hist = reinterpret_cast<uint32_t *>(p + off);
-    off += align_up(rows * kBins1 * 4, 256);
-    s.state = reinterpret_cast<HeadState *>(p + off);
-    off += align_up(rows * sizeof(HeadState), 256);
-    s.counters = reinterpret_cast<uint32_t *>(p + off);
-    off += align_up((size_t)d.batch * d.n_kv_heads * 4, 256);
-    s.cand = reinterpret_cast<unsigned long long *>(p + off);
-    off += align_up(rows * d.ctx_cap * 8, 256);
-    s.top = reinterpret_cast<uint32_t *>(p + off);
-    return s;
-}
-
-size_t carve_bytes(const tb_dims &d) {
-    const size_t rows = (size_t)d.batch * d.n_q_heads;
-    const size_t W = (d.ctx_cap + 31) / 32;
-    return kWsHeaderBytes + align_up(rows * d.ctx_cap * 4, 256) + align_up(rows * kBins1 * 4, 256) +
-           align_up(rows * sizeof(HeadState), 256) + align_up((size_t)d.batch * d.n_kv_heads * 4, 256) +
-           align_up(rows * d.ctx_cap * 8, 256) + align_up(rows * W * 4, 256);
-}
-
-// Exclusive prefix sum over the block (NT threads, in thread order); *total
-// gets the sum.  `scratch` holds NT/32 + 1 ints.  All threads must call.
-template <int NT>
-__device__ int block_excl_scan(int v, int *scratch, int *total) {
-    constexpr int NW = NT / 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < NW ? scratch[lane] : 0;
-        int wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(kFull, wi, o);
-            if (lane >= o) wi += t;
-        }
-        if (lane < NW) scratch[lane] = wi - w;
-        if (lane == NW - 1) scratch[NW] = wi;
-    }
-    __syncthreads();
-    const int res = scratch[warp] + incl - v;
-    *total = scratch[NW];
-    __syncthreads();
-    return res;
-}
-
-// The bin that holds the `need`-th largest key of a histogram (bins in key
-// order), searched from the top by the whole block: thread t owns the t-th
-// group of bins counted from the top, a block scan gives every thread the
-// count above its group, and the one thread whose group crosses `need` walks
-// it.  Returns the bin; *rem = how many keys of that bin are still needed.
-// `hist` may be global (read through L2) or shared; `scratch` holds NT/32 + 3
-// ints.  All threads must call; nbins is a multiple of NT.
-template <int NT>
-__device__ int block_find_bin_desc(const uint32_t *hist, int nbins, uint32_t need, uint32_t *rem,
-                                   int *scratch, bool from_global) {
-    const int per = nbins / NT;
-    const int hi = nbins - threadIdx.x * per;  // this thread's bins are [hi - per, hi)
-    int mine = 0;
-    for (int j = 1; j <= per; ++j) mine += (int)(from_global ? __ldcg(hist + hi - j) : hist[hi - j]);
-    int total;
-    const int above = block_excl_scan<NT>(mine, scratch, &total);
-    if ((uint32_t)above < need && need <= (uint32_t)(above + mine)) {
-        uint32_t acc = (uint32_t)above;
-        for (int j = 1; j <= per; ++j) {
-            const uint32_t v = from_global ? __ldcg(hist + hi - j) : hist[hi - j];
-            if (acc + v >= need) {
-                scratch[NT / 32 + 1] = hi - j;
-                scratch[NT / 32 + 2] = (int)(need - acc);
-                break;
-            }
-            acc += v;
-        }
-    }
-    __syncthreads();
-    const int bin = scratch[NT / 32 + 1];
-    *rem = (uint32_t)scratch[NT / 32 + 2];
-    __syncthreads();
-    return bin;
-}
+using namespace sel;
 
 // ------------------------------------------------------------------ kernel 1
 
@@ -177,16 +50,15 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                   int window, int budget, SelWs ws) {
     constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
     constexpr int NSUB = kHistChunk / kSubRows;         // staged sub-chunks per CTA
-    constexpr int RPT = kSubRows / kThreads;            // rows per thread per sub-chunk
-    constexpr int ROWB = DP * 2;                        // bytes per K' row
-    constexpr int V16 = ROWB / 16;                      // 16-byte parts per row
+    using Sc = RowScorer<DP>;
+    constexpr int ROWB = Sc::ROWB;                      // bytes per K' row
     extern __shared__ __align__(128) uint8_t stage[];   // [2][kSubRows][ROWB]: K' rows, double-buffered
     __shared__ __align__(16) float qs[kGroup][DP];
     __shared__ uint32_t hist[NH][kBins1];
     __shared__ __align__(8) uint64_t bars[2];
     __shared__ int s_last;
     __shared__ int scratch[kThreads / 32 + 3];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int p0 = ch * kHistChunk;
     const uint32_t stage_s = smem_addr(stage);
@@ -204,6 +76,8 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     const int lo = sink, hi = T - window;
     if (tid < kGroup * DP) (&qs[0][0])[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
     __syncthreads();
+    Sc scorer;
+    scorer.load_q(&qs[0][0], lane);
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     if (hi > lo && p0 < hi && p0 + kHistChunk > lo) {
@@ -232,60 +106,37 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
             if (!ok) break;
             const uint8_t *buf = stage + (k & 1) * kSubRows * ROWB;
             const int pb = p0 + (j_lo + k) * kSubRows;
-            // rows tid + m * kThreads share one rotation of the 16-byte parts,
-            // which keeps a quarter-warp's reads on distinct banks
-            const int rot = (tid >> (V16 == 4 ? 1 : 2)) & (V16 - 1);
-            float sc[RPT][kGroup];
+            // 32-row blocks, one warp each (rows past the copied ones hold
+            // stale bytes: they are scored and dropped)
+            for (int blk = warp; blk < kSubRows / 32 && pb + blk * 32 < hi; blk += kThreads / 32) {
+                const uint8_t *block = buf + blk * 32 * ROWB;
 #pragma unroll
-            for (int m = 0; m < RPT; ++m)
+                for (int ps = 0; ps < Sc::NPART; ++ps) {
+                    float out[Sc::HPL];
+                    scorer.pass(*Sc::part_ptr(block, ps, lane), lane, out);
+                    const int p = pb + blk * 32 + Sc::row_of(ps, lane);
+                    const bool valid = p >= lo && p < hi;
+                    if constexpr (!sel_is_group(SEL)) {
 #pragma unroll
-                for (int h = 0; h < kGroup; ++h) sc[m][h] = 0.f;
-#pragma unroll
-            for (int vv = 0; vv < V16; ++vv) {
-                const int pv = (vv + rot) & (V16 - 1);
-                float4 qv[kGroup][2];
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) {
-                    qv[h][0] = *reinterpret_cast<const float4 *>(&qs[h][8 * pv]);
-                    qv[h][1] = *reinterpret_cast<const float4 *>(&qs[h][8 * pv + 4]);
-                }
-#pragma unroll
-                for (int m = 0; m < RPT; ++m) {
-                    const uint4 raw = *reinterpret_cast<const uint4 *>(buf + (tid + m * kThreads) * ROWB + pv * 16);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t wd = e == 0 ? raw.x : e == 1 ? raw.y : e == 2 ? raw.z : raw.w;
-                        const float kl = bf16_lo(wd), kh = bf16_hi(wd);
-#pragma unroll
-                        for (int h = 0; h < kGroup; ++h) {
-                            const float4 &q4 = qv[h][e >> 1];
-                            const float qa = (e & 1) ? q4.z : q4.x, qb = (e & 1) ? q4.w : q4.y;
-                            sc[m][h] = fmaf(qb, kh, fmaf(qa, kl, sc[m][h]));
+                        for (int j = 0; j < Sc::HPL; ++j) {
+                            const int h = Sc::head0(lane) + j;
+                            const uint32_t key = score_key(out[j]);
+                            if (valid) {
+                                ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
+                                atomicAdd(&hist[h][key >> 21], 1u);
+                            }
                         }
-                    }
-                }
-            }
+                    } else {
+                        float s4[kGroup];
+                        Sc::gather_heads(out, s4);
+                        float gs = s4[0];
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) {
-                const int p = pb + tid + m * kThreads;
-                const bool valid = p >= lo && p < hi;
-                if constexpr (!sel_is_group(SEL)) {
-#pragma unroll
-                    for (int h = 0; h < kGroup; ++h) {
-                        const uint32_t key = score_key(sc[m][h]);
-                        if (valid) {
-                            ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
-                            atomicAdd(&hist[h][key >> 21], 1u);
+                        for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, s4[h]) : gs + s4[h];
+                        const uint32_t key = score_key(gs);
+                        if (valid && lane % Sc::NPART == 0) {
+                            ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
+                            atomicAdd(&hist[0][key >> 21], 1u);
                         }
-                    }
-                } else {
-                    float gs = sc[m][0];
-#pragma unroll
-                    for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, sc[m][h]) : gs + sc[m][h];
-                    const uint32_t key = score_key(gs);
-                    if (valid) {
-                        ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
-                        atomicAdd(&hist[0][key >> 21], 1u);
                     }
                 }
             }
@@ -439,13 +290,6 @@ mark_collect_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tc
 
 // ------------------------------------------------------------------ kernel 3
 
-__device__ __forceinline__ uint32_t range_mask(int w, int lo, int hi) {
-    if (hi <= lo) return 0u;
-    const int start = max(lo - (w << 5), 0), end = min(hi - (w << 5), 32);
-    if (end <= start) return 0u;
-    const uint32_t upto = end == 32 ? 0xffffffffu : ((1u << end) - 1u);
-    return upto & ~((1u << start) - 1u);
-}
 
 // One CTA per (b, query head) (per KV head in the group modes) of NT threads:
 // 1024 on the default path, 512 for the variants, which need more registers.
@@ -982,6 +826,11 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                 int32_t window, int32_t budget, int32_t nbr, int32_t group_reduce,
                                 int32_t *idx, int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
                                 cudaStream_t st) {
+    const int algo = select_algorithm();
+    if (group_reduce != 2 && algo != TB_SELECT_MULTI_KERNEL &&
+        select_cluster_fits(d, group_reduce, algo == TB_SELECT_AUTO))
+        return launch_score_select_cluster(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, group_reduce,
+                                           idx, idx_cap, count, sel_bits, ws, st);
     if (group_reduce == 0)
         return launch_sel<kSelGroupMax>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap,
                                         count, sel_bits, ws, st);

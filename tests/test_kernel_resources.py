@@ -40,5 +40,6 @@ def test_no_register_spills():
     for r in reports:
         spills.update(_spills(r))
     assert any("attn_kernel" in k for k in spills) and any("score_hist_kernel" in k for k in spills)
+    assert any("sel_cluster_kernel" in k for k in spills)
     bad = {k: v for k, v in spills.items() if v > 0}
     assert not bad, f"kernels that spill registers: {bad}"
