@@ -233,18 +233,20 @@ tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_
  * result is the same, bit for bit: same scores, same set, same index list;
  * no counterpart on the pages, a choice of route):
  *
- *   TB_SELECT_AUTO          (default) the cluster kernel where it applies,
- *                           else the multi-kernel path.
- *   TB_SELECT_MULTI_KERNEL  three kernels per call: scoring with a global
- *                           histogram, marking and candidate collection, and
- *                           a per-head finish (any ctx_cap).
- *   TB_SELECT_CLUSTER       one kernel per call: a thread-block cluster per
- *                           (sequence, KV head) holds all of its scores in
- *                           shared memory.  It applies while ctx_cap fits
- *                           (up to 81,920 positions for tb_score_select,
- *                           327,680 for tb_score_select_group, on a device
- *                           that places 16-CTA clusters); elsewhere the
- *                           selection calls return TB_ERR_UNSUPPORTED.
+ *   TB_SELECT_AUTO          (default) the cluster route where one wave of
+ *                           clusters holds the call with slices of at least
+ *                           4,096 positions (long single sequences), else the
+ *                           multi-kernel route.
+ *   TB_SELECT_MULTI_KERNEL  three kernels per call: scoring with a histogram,
+ *                           marking and candidate collection, and a per-head
+ *                           finish (any ctx_cap).
+ *   TB_SELECT_CLUSTER       two kernels per call: scoring on every SM, then a
+ *                           thread-block cluster per (sequence, KV head) that
+ *                           holds all of its scores on chip and selects.  It
+ *                           applies while ctx_cap fits 16 CTAs (up to 131,072
+ *                           positions for tb_score_select, 270,336 for
+ *                           tb_score_select_group); elsewhere the selection
+ *                           calls return TB_ERR_UNSUPPORTED.
  *
  * tb_score_select_inclusive always takes the multi-kernel path.  The
  * algorithm belongs to the calling thread and is read when a selection call

@@ -33,12 +33,18 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                 void *ws, cudaStream_t st);
 // The one-kernel cluster path of launch_score_select (select_cluster.cu) for
 // group_reduce -1, 0 and 1: whether it takes dims `d` (with one_wave: in one
-// wave of clusters, where it beats the multi-kernel path), and the launch.
+// wave of clusters of long slices, where it beats the multi-kernel path), and
+// the launch.
 bool select_cluster_fits(const tb_dims &d, int32_t group_reduce, bool one_wave);
 cudaError_t launch_score_select_cluster(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
                                         const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget,
                                         int32_t nbr, int32_t group_reduce, int32_t *idx, int32_t idx_cap,
                                         int32_t *count, uint32_t *sel_bits, void *ws, cudaStream_t st);
+// The scores of launch_score_select (group_reduce -1, 0, 1) as order-preserving
+// keys in the workspace, nothing else (select.cu; the cluster path's first step).
+cudaError_t launch_score_keys(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
+                              const int32_t *ctx_len, int32_t sink, int32_t window, int32_t group_reduce, void *ws,
+                              cudaStream_t st);
 cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t *ctx_len, int32_t sink,
                                  int32_t window, float *scores, cudaStream_t st);
 cudaError_t launch_export_candidates(const tb_dims &d, const void *ws, const int32_t *idx, int32_t idx_cap,

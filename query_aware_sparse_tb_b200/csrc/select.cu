@@ -9,9 +9,10 @@
 // selected tokens are expanded by their spatial neighbours.
 //
 // Exact top-B on the fp32 scores, ties broken by the lower position:
-//   1. score_hist   one CTA per (b, KV head, 2048 positions): brings the K'
-//                   rows in by double-buffered 1-D bulk copies (TMA), reads
-//                   each row once for the 4 query heads of the group, writes the
+//   1. score_hist   one CTA per (b, KV head, 2048 positions): each warp
+//                   streams 32-row blocks of K' through a cp.async ring of its
+//                   own and scores each row once for the 4 query heads of the
+//                   group (BlockScorer), writes the
 //                   order-preserving uint32 image of every score, and builds
 //                   a histogram of its top 11 bits per query head.  The last
 //                   CTA of each (b, KV head) (atomic ticket, no waiting) finds
@@ -43,113 +44,84 @@ using namespace sel;
 
 // ------------------------------------------------------------------ kernel 1
 
-template <int DP, int SEL>
+// HIST = false: the scores only (their keys in the workspace), for the
+// cluster kernel that selects from them.
+template <int DP, int SEL, bool HIST>
 __global__ void __launch_bounds__(kThreads, 2)
 score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
                   int window, int budget, SelWs ws) {
     constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
-    constexpr int NSUB = kHistChunk / kSubRows;         // staged sub-chunks per CTA
-    using Sc = RowScorer<DP>;
-    constexpr int ROWB = Sc::ROWB;                      // bytes per K' row
-    extern __shared__ __align__(128) uint8_t stage[];   // [2][kSubRows][ROWB]: K' rows, double-buffered
+    using Sc = BlockScorer<DP>;
+    constexpr int NW = kThreads / 32;
+    extern __shared__ __align__(128) uint8_t stage[];   // [warp][kHistRing][32-row block]
     __shared__ __align__(16) float qs[kGroup][DP];
-    __shared__ uint32_t hist[NH][kBins1];
-    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ uint32_t hist[HIST ? NH : 1][HIST ? kBins1 : 1];
     __shared__ int s_last;
     __shared__ int scratch[kThreads / 32 + 3];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
     const int p0 = ch * kHistChunk;
-    const uint32_t stage_s = smem_addr(stage);
-    auto bar = [&](int k) { return smem_addr(&bars[k]); };
 
-    for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
-    if (tid == 0) {
-        mbar_init(bar(0), 1);
-        mbar_init(bar(1), 1);
-        fence_mbar_init();
-    }
+    if constexpr (HIST)
+        for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
     griddep_wait();
     griddep_launch_dependents();
     const int T = clamp_ctx(ctx_len[b], Tcap, ws.flags, tid == 0 && ch == 0 && g == 0);
     const int lo = sink, hi = T - window;
     if (tid < kGroup * DP) (&qs[0][0])[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
     __syncthreads();
-    Sc scorer;
-    scorer.load_q(&qs[0][0], lane);
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     if (hi > lo && p0 < hi && p0 + kHistChunk > lo) {
-        // the chunk's K' rows (contiguous for one (b, g)) come in sub-chunks of
-        // kSubRows by 1-D bulk copies, two in flight: sub-chunk k+2 is
-        // requested as soon as sub-chunk k has been read.  Only sub-chunks
-        // that overlap C are fetched; rows outside C are scored and dropped.
-        const int j_lo = max(0, lo - p0) / kSubRows;
-        const int j_hi = min(NSUB, (hi - p0 + kSubRows - 1) / kSubRows);
-        auto issue = [&](int k) {  // sub-chunk j_lo + k into buffer k & 1 (thread 0)
-            const int r0 = p0 + (j_lo + k) * kSubRows;
-            const int nrows = min(kSubRows, Tcap - r0);
-            mbar_arrive_expect_tx(bar(k & 1), (uint32_t)(nrows * ROWB));
-            bulk_load(stage_s + (uint32_t)((k & 1) * kSubRows * ROWB), Kp + (slab + r0) * DP,
-                      (uint32_t)(nrows * ROWB), bar(k & 1));
+        // the chunk's 32-row blocks that overlap C, dealt to the warps in
+        // turn; each warp streams its blocks through a ring of its own
+        // (kHistRing - 1 in flight) and lane l scores row l of each
+        const int blo = max(0, lo - p0) / 32;
+        const int bhi = min(kHistChunk, hi - p0 + 31) / 32;
+        const int nb = blo + warp < bhi ? (bhi - blo - warp + NW - 1) / NW : 0;  // this warp's blocks
+        uint8_t *ring = stage + warp * kHistRing * Sc::BLKB;
+        const uint32_t ring_s = smem_addr(ring);
+        auto issue = [&](int i) {
+            const int r0 = p0 + (blo + warp + NW * i) * 32;
+            Sc::copy(ring_s + (uint32_t)((i % kHistRing) * Sc::BLKB), Kp + (slab + r0) * DP, hi - r0, lane);
         };
-        const int n_sub = j_hi - j_lo;
-        if (tid == 0) {
-            issue(0);
-            if (n_sub > 1) issue(1);
+        for (int i = 0; i < kHistRing - 1; ++i) {
+            if (i < nb) issue(i);
+            cp_async_commit();
         }
-        int waited = 0;  // sub-chunks whose copy has been waited for
-        for (int k = 0; k < n_sub; ++k) {
-            const bool ok = __syncthreads_and(mbar_wait_bounded(bar(k & 1), (k >> 1) & 1, ws.flags));
-            waited = k + 1;
-            if (!ok) break;
-            const uint8_t *buf = stage + (k & 1) * kSubRows * ROWB;
-            const int pb = p0 + (j_lo + k) * kSubRows;
-            // 32-row blocks, one warp each (rows past the copied ones hold
-            // stale bytes: they are scored and dropped)
-            for (int blk = warp; blk < kSubRows / 32 && pb + blk * 32 < hi; blk += kThreads / 32) {
-                const uint8_t *block = buf + blk * 32 * ROWB;
+        for (int i = 0; i < nb; ++i) {
+            if (i + kHistRing - 1 < nb) issue(i + kHistRing - 1);
+            cp_async_commit();
+            cp_async_wait_group<kHistRing - 1>();
+            __syncwarp();  // every lane's copies of block i have landed
+            float sc[kGroup];
+            Sc::score(ring + (i % kHistRing) * Sc::BLKB, &qs[0][0], lane, sc);
+            __syncwarp();  // block i is read before its slot is refilled
+            const int p = p0 + (blo + warp + NW * i) * 32 + lane;
+            const bool valid = p >= lo && p < hi;
+            if constexpr (!sel_is_group(SEL)) {
 #pragma unroll
-                for (int ps = 0; ps < Sc::NPART; ++ps) {
-                    float out[Sc::HPL];
-                    scorer.pass(*Sc::part_ptr(block, ps, lane), lane, out);
-                    const int p = pb + blk * 32 + Sc::row_of(ps, lane);
-                    const bool valid = p >= lo && p < hi;
-                    if constexpr (!sel_is_group(SEL)) {
-#pragma unroll
-                        for (int j = 0; j < Sc::HPL; ++j) {
-                            const int h = Sc::head0(lane) + j;
-                            const uint32_t key = score_key(out[j]);
-                            if (valid) {
-                                ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
-                                atomicAdd(&hist[h][key >> 21], 1u);
-                            }
-                        }
-                    } else {
-                        float s4[kGroup];
-                        Sc::gather_heads(out, s4);
-                        float gs = s4[0];
-#pragma unroll
-                        for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, s4[h]) : gs + s4[h];
-                        const uint32_t key = score_key(gs);
-                        if (valid && lane % Sc::NPART == 0) {
-                            ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
-                            atomicAdd(&hist[0][key >> 21], 1u);
-                        }
+                for (int h = 0; h < kGroup; ++h) {
+                    const uint32_t key = score_key(sc[h]);
+                    if (valid) {
+                        ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
+                        if constexpr (HIST) atomicAdd(&hist[h][key >> 21], 1u);
                     }
                 }
+            } else {
+                float gs = sc[0];
+#pragma unroll
+                for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, sc[h]) : gs + sc[h];
+                const uint32_t key = score_key(gs);
+                if (valid) {
+                    ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
+                    if constexpr (HIST) atomicAdd(&hist[0][key >> 21], 1u);
+                }
             }
-            __syncthreads();  // buffer k & 1 read by every thread before it is refilled
-            if (tid == 0 && k + 2 < n_sub) issue(k + 2);
         }
-        // a copy must not land after the CTA has gone: when a wait gave up on
-        // sub-chunk k, sub-chunk k + 1 may still be in flight; wait for it
-        // (bounded) before leaving
-        if (tid == 0)
-            for (int k = waited; k < min(n_sub, waited + 1); ++k)
-                (void)mbar_wait_bounded(bar(k & 1), (k >> 1) & 1, ws.flags);
     }
+    if constexpr (!HIST) return;
     __syncthreads();
     for (int i = tid; i < NH * kBins1; i += kThreads) {
         const uint32_t v = (&hist[0][0])[i];
@@ -776,6 +748,27 @@ export_scores_kernel(const uint32_t *__restrict__ keys, const int32_t *__restric
     out[i] = v;
 }
 
+template <int SEL, bool HIST>
+cudaError_t launch_score_hist(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
+                              const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, const SelWs &s,
+                              cudaStream_t st) {
+    dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
+    const int hsm = (kThreads / 32) * kHistRing * 32 * d.d_proj * 2;  // the warps' rings of 32-row blocks
+    cudaError_t e;
+    if (d.d_proj == 32) {
+        static std::atomic<int> smem_set32[kMaxDevices];
+        if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<32, SEL, HIST>, hsm, smem_set32)) != cudaSuccess)
+            return e;
+        return launch_pdl(score_hist_kernel<32, SEL, HIST>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp,
+                          ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+    }
+    static std::atomic<int> smem_set16[kMaxDevices];
+    if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<16, SEL, HIST>, hsm, smem_set16)) != cudaSuccess)
+        return e;
+    return launch_pdl(score_hist_kernel<16, SEL, HIST>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp, ctx_len,
+                      d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+}
+
 template <int SEL>
 cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
                        const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, int32_t nbr,
@@ -785,23 +778,7 @@ cudaError_t launch_sel(const tb_dims &d, const float *qp, int64_t qp_stride, con
     const int W = (d.ctx_cap + 31) / 32;
     const int nch = (d.ctx_cap + kChunk - 1) / kChunk;
     dim3 grid(nch, d.n_kv_heads, d.batch);
-    dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
-    cudaError_t e;
-    const int hsm = 2 * kSubRows * d.d_proj * 2;  // two staged sub-chunks of K' rows
-    if (d.d_proj == 32) {
-        static std::atomic<int> smem_set32[kMaxDevices];
-        if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<32, SEL>, hsm, smem_set32)) != cudaSuccess)
-            return e;
-        e = launch_pdl(score_hist_kernel<32, SEL>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp, ctx_len,
-                       d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
-    } else {
-        // (with the static histogram the total is past the default 48 KB here too)
-        static std::atomic<int> smem_set16[kMaxDevices];
-        if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<16, SEL>, hsm, smem_set16)) != cudaSuccess)
-            return e;
-        e = launch_pdl(score_hist_kernel<16, SEL>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp, ctx_len,
-                       d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
-    }
+    cudaError_t e = launch_score_hist<SEL, true>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, s, st);
     if (e != cudaSuccess) return e;
     e = launch_pdl(mark_collect_kernel<SEL>, grid, dim3(kThreads), 0, st, ctx_len, d.n_q_heads, d.n_kv_heads,
                    d.ctx_cap, W, sink, window, s);
@@ -842,6 +819,17 @@ cudaError_t launch_score_select(const tb_dims &d, const float *qp, int64_t qp_st
                                         count, sel_bits, ws, st);
     return launch_sel<kSelHead>(d, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap, count,
                                 sel_bits, ws, st);
+}
+
+cudaError_t launch_score_keys(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
+                              const int32_t *ctx_len, int32_t sink, int32_t window, int32_t group_reduce, void *ws,
+                              cudaStream_t st) {
+    const SelWs s = carve(d, ws);
+    if (group_reduce == 0)
+        return launch_score_hist<kSelGroupMax, false>(d, qp, qp_stride, Kp, ctx_len, sink, window, 1, s, st);
+    if (group_reduce == 1)
+        return launch_score_hist<kSelGroupSum, false>(d, qp, qp_stride, Kp, ctx_len, sink, window, 1, s, st);
+    return launch_score_hist<kSelHead, false>(d, qp, qp_stride, Kp, ctx_len, sink, window, 1, s, st);
 }
 
 cudaError_t launch_export_scores(const tb_dims &d, const void *ws, const int32_t *ctx_len, int32_t sink,

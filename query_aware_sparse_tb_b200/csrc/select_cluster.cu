@@ -1,6 +1,5 @@
-// Importance scoring and exact top-B selection in one kernel: one
-// thread-block cluster per (sequence, KV head) keeps all of the group's
-// scores on chip.
+// Exact top-B selection on thread-block clusters: one cluster per (sequence,
+// KV head) holds all of the group's scores on chip and selects in one kernel.
 //
 // TokenButler technical summary (gist.science), "Core architecture: scoring":
 // predicted queries dotted with projected keys give per-token importance
@@ -10,18 +9,17 @@
 // selected tokens are expanded by their neighbours.
 //
 // The result is the one the multi-kernel path (score_hist, mark_collect,
-// finalize) computes, bit for bit: the same scores (RowScorer), the B largest
+// finalize) computes, bit for bit: the same scores, the B largest
 // order-preserving keys with ties on the B-th taken in position order, dilated
-// by +-nbr and clipped to C.  Only the route differs.  CTA r of a cluster of
-// CS owns the positions [r*L, (r+1)*L), L a multiple of 32, and warp w of it
-// the 32-position words w, w + 16, w + 32, ... of that slice:
-//   1. score  each warp streams its words' K' rows through a private ring in
-//             shared memory (16-byte cp.async, a few blocks in flight; a lane
-//             reads back only the parts it copied, so no barrier is needed),
-//             scores them with RowScorer and keeps the keys in registers, lane
-//             = position in the word; a histogram of key bits 31..21 per head
-//             is built in shared memory on the way.  The keys also go to the
-//             workspace, where the score and candidate exports read them.
+// by +-nbr and clipped to C.  Only the route differs.  The scores come first,
+// from score_hist's keys-only variant on every SM (scoring streams K', which
+// wants all of them); then one cluster per (sequence, KV head) selects.  CTA r
+// of a cluster of CS owns the positions [r*L, (r+1)*L), L a multiple of 32,
+// and warp w of it the 32-position words w, w + 16, w + 32, ... of that slice:
+//   1. keys   each lane loads the keys of its positions from the workspace
+//             (just written, so from L2) into registers, lane = position in
+//             the word; a histogram of key bits 31..21 per head is built on
+//             the way.
 //   2. radix  three passes (key bits 31..21, 20..10, 9..0) fix the B-th
 //             largest key tau and k, how many keys equal to it are taken.  In
 //             each, a CTA histograms its keys that match the digits fixed so
@@ -47,7 +45,6 @@
 
 #include "common.cuh"
 #include "internal.h"
-#include "score.cuh"
 #include "select_common.cuh"
 
 namespace tb {
@@ -60,16 +57,13 @@ constexpr int kCWarps = kCThreads / 32;
 constexpr int kHistWords = 2048 + 64; // per head: up to 2048 bins, then up to 64 group sums
 constexpr int kCDynMax = 227 * 1024 - 4096;
 constexpr int kMaxCluster = 16;
+constexpr int kMinAutoSlice = 4096;   // the automatic route takes the cluster kernel from this slice length
 
 template <int SEL>
 __host__ __device__ constexpr int rows_per_group() { return sel_is_group(SEL) ? 1 : kGroup; }
-// Words of the slice each warp owns (keys held in registers: 64 or 24 per thread).
+// Words of the slice each warp owns (keys held in registers: 64 or 33 per thread).
 template <int SEL>
-__host__ __device__ constexpr int words_per_warp() { return sel_is_group(SEL) ? 24 : 16; }
-// Blocks (32 rows) in each warp's shared-memory ring.
-template <int DP>
-__host__ __device__ constexpr int ring_blocks() { return DP == 32 ? 5 : 8; }
-
+__host__ __device__ constexpr int words_per_warp() { return sel_is_group(SEL) ? 33 : 16; }
 // Sum of the word at `local` over the shared memory of cluster CTAs 0 .. cs-1
 // (every read issued before the first is added).
 __device__ __forceinline__ uint32_t cluster_sum(const uint32_t *local, int cs) {
@@ -160,7 +154,7 @@ __device__ void cluster_find_digit(const uint32_t *hist, int nb, int dbits, int 
 template <int NH>
 __device__ void group_sums(uint32_t *hist) {
     constexpr int kChunks = 2048 / 4;  // per head
-    static_assert((NH * kChunks) % kCThreads == 0, "whole warps in every round");
+    static_assert((NH * kChunks) % 32 == 0 && kCThreads % 32 == 0, "whole warps in every round");
     for (int i = threadIdx.x; i < NH * kChunks; i += kCThreads) {
         const int h = i / kChunks, c = i % kChunks;
         const uint4 v = *reinterpret_cast<const uint4 *>(hist + h * kHistWords + 4 * c);
@@ -172,20 +166,14 @@ __device__ void group_sums(uint32_t *hist) {
     }
 }
 
-template <int DP, int SEL>
+template <int SEL>
 __global__ void __launch_bounds__(kCThreads, 1)
-sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
-                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int W, int L, int sink,
-                   int window, int budget, int nbr, int32_t *__restrict__ idx, int idx_cap,
-                   int32_t *__restrict__ count, uint32_t *__restrict__ sel_bits, uint32_t *__restrict__ gkeys,
-                   uint32_t *__restrict__ flags) {
-    using Sc = RowScorer<DP>;
+sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int L, int sink, int window,
+                   int budget, int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
+                   uint32_t *__restrict__ sel_bits, const uint32_t *__restrict__ gkeys, uint32_t *__restrict__ flags) {
     constexpr int NH = rows_per_group<SEL>();
     constexpr int NOUT = sel_is_group(SEL) ? kGroup : 1;  // output rows per score row
     constexpr int JMAX = words_per_warp<SEL>();
-    constexpr int NST = ring_blocks<DP>();
-    constexpr int BLKB = 32 * Sc::ROWB;                   // bytes of a 32-row block
-    constexpr int NPART = Sc::NPART, RPP = Sc::RPP, HPL = Sc::HPL;
     const int LW = L / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lt = (1u << lane) - 1u;
@@ -194,113 +182,52 @@ sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16
     const uint32_t r = cluster_ctarank();
     const int s0 = (int)r * L;
 
-    // dynamic shared memory: [per-warp rings | radix pass 2 histogram] [histogram A] [Top] [aux] [word prefix]
+    // dynamic shared memory: [radix pass 2 histogram] [histogram A] [Top] [aux] [word prefix]
     extern __shared__ __align__(128) uint8_t csm[];
-    constexpr int kRing = kCWarps * NST * BLKB;
-    static_assert(kRing >= NH * kHistWords * 4, "the pass-2 histogram lives in the rings");
-    uint8_t *ring = csm + warp * NST * BLKB;
     uint32_t *histB = reinterpret_cast<uint32_t *>(csm);
-    uint32_t *histA = reinterpret_cast<uint32_t *>(csm + kRing);
+    uint32_t *histA = histB + NH * kHistWords;
     uint32_t *top_s = histA + NH * kHistWords;
     uint32_t *aux_s = top_s + NH * LW;
     uint32_t *wpre_s = aux_s + NH * LW;
-    __shared__ __align__(16) float qs[kGroup * DP];
     __shared__ uint32_t edge_s[2][NH][32];  // keys of this slice's first and last word
     __shared__ uint32_t gco[4 * 64];
     __shared__ uint32_t prefix[4], need[4], x_cnt[4], base_s[4], total_s[4], take_s[4], nb_top[2][4];
     __shared__ int scratch[kCThreads / 32 + 3];
 
-    for (int i = tid; i < NH * kHistWords; i += kCThreads) histA[i] = 0u;
+    for (int i = tid; i < NH * kHistWords; i += kCThreads) {
+        histA[i] = 0u;
+        histB[i] = 0u;
+    }
     if (tid < 4) x_cnt[tid] = 0u;
-    griddep_wait();
+    griddep_wait();  // the keys come from the kernel before
     griddep_launch_dependents();
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && r == 0 && g == 0);
     const int lo = sink, hi = T - window;
     const int nC = hi > lo ? hi - lo : 0;
     const uint32_t mode = nC == 0 ? kModeEmpty : (nC <= budget ? kModeAll : kModeSelect);
     const int a = max(lo, s0), e = min(hi, s0 + L);  // this slice's part of C
-    if (tid < kGroup * DP) qs[tid] = qp[(int64_t)b * qp_stride + (int64_t)g * kGroup * DP + tid];
-    __syncthreads();
-
-    // ---- 1. scores: keys in registers, key[j][h] = word warp + 16 j, bit lane
-    const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
     const size_t krow0 = (size_t)b * Hq + (size_t)g * kGroup;  // first workspace key row of the group
+
+    // ---- 1. keys in registers, key[j][h] = word warp + 16 j, bit lane; 0
+    // marks a position outside C (no score has key 0: score_key maps every
+    // float, NaNs included, to a key of at least 0x007fffff)
     uint32_t key[JMAX][NH];
-    uint64_t vbits = 0;  // bit j: this lane's position of word j is a candidate
-    {
-        const uint32_t ring_s = smem_addr(ring);
-        auto active = [&](int j) {
-            const int w0 = s0 + 32 * (warp + kCWarps * j);
-            return warp + kCWarps * j < LW && w0 + 32 > a && w0 < e;
-        };
-        auto issue = [&](int j) {  // block j into slot j % NST: the lane's own 16-byte parts
-            const int r0 = s0 + 32 * (warp + kCWarps * j);
-            const uint32_t dst = ring_s + (uint32_t)((j % NST) * BLKB);
 #pragma unroll
-            for (int ps = 0; ps < NPART; ++ps) {
-                const int c = ps * 32 + lane;
-                const int row = r0 + c / NPART;
-                cp_async16(dst + c * 16, Kp + (slab + row) * DP + (c % NPART) * 8, row < e);
-            }
-        };
+    for (int j = 0; j < JMAX; ++j) {
+        const int wi = warp + kCWarps * j;
+        const int p = s0 + 32 * wi + lane;
+        const bool v = wi < LW && p >= a && p < e;
 #pragma unroll
-        for (int j = 0; j < NST - 1; ++j) {
-            if (j < JMAX && active(j)) issue(j);
-            cp_async_commit();
-        }
+        for (int h = 0; h < NH; ++h) key[j][h] = v ? __ldcg(gkeys + (krow0 + h) * Tcap + p) : 0u;
+    }
 #pragma unroll
-        for (int j = 0; j < JMAX; ++j) {
-            if (j + NST - 1 < JMAX && active(j + NST - 1)) issue(j + NST - 1);
-            cp_async_commit();
-            cp_async_wait_group<NST - 1>();
+    for (int j = 0; j < JMAX; ++j) {
+        const int wi = warp + kCWarps * j;
 #pragma unroll
-            for (int h = 0; h < NH; ++h) key[j][h] = 0u;
-            if (!active(j)) continue;  // warp-uniform
-            const uint8_t *blk = ring + (j % NST) * BLKB;
-            float out[NPART][HPL];
-#pragma unroll
-            for (int ps = 0; ps < NPART; ++ps) Sc::pass_q(qs, *Sc::part_ptr(blk, ps, lane), lane, out[ps]);
-            // lane l held row ps * RPP + l / NPART after pass ps; bring row l to lane l
-            const int src_row = lane % RPP, src_ps = lane / RPP;
-            if constexpr (!sel_is_group(SEL)) {
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) {
-                    uint32_t kv = 0u;
-#pragma unroll
-                    for (int ps = 0; ps < NPART; ++ps) {
-                        const uint32_t v =
-                            __shfl_sync(kFull, score_key(out[ps][h % HPL]), src_row * NPART + h / HPL);
-                        kv = ps == src_ps ? v : kv;
-                    }
-                    key[j][h] = kv;
-                }
-            } else {
-                uint32_t kv = 0u;
-#pragma unroll
-                for (int ps = 0; ps < NPART; ++ps) {
-                    float s4[kGroup];
-                    Sc::gather_heads(out[ps], s4);
-                    float gs = s4[0];
-#pragma unroll
-                    for (int h = 1; h < kGroup; ++h) gs = SEL == kSelGroupMax ? fmaxf(gs, s4[h]) : gs + s4[h];
-                    const uint32_t v = __shfl_sync(kFull, score_key(gs), src_row * NPART);
-                    kv = ps == src_ps ? v : kv;
-                }
-                key[j][0] = kv;
-            }
-            const int wi = warp + kCWarps * j;
-            const int p = s0 + 32 * wi + lane;
-            const bool v = p >= a && p < e;
-            vbits |= (uint64_t)v << j;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                if (v) {
-                    atomicAdd(&histA[h * kHistWords + (key[j][h] >> 21)], 1u);
-                    gkeys[(krow0 + h) * Tcap + p] = key[j][h];
-                }
-                if (wi == 0) edge_s[0][h][lane] = key[j][h];
-                if (wi == LW - 1) edge_s[1][h][lane] = key[j][h];
-            }
+        for (int h = 0; h < NH; ++h) {
+            if (key[j][h] != 0u) atomicAdd(&histA[h * kHistWords + (key[j][h] >> 21)], 1u);
+            if (wi == 0) edge_s[0][h][lane] = key[j][h];
+            if (wi == LW - 1) edge_s[1][h][lane] = key[j][h];
         }
     }
     __syncthreads();
@@ -312,8 +239,6 @@ sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16
             need[tid] = (uint32_t)budget;
         }
         group_sums<NH>(histA);
-        // (every copy into the rings has landed and been read: pass 2's histogram goes there)
-        for (int i = tid; i < NH * kHistWords; i += kCThreads) histB[i] = 0u;
         cluster_sync();
         cluster_find_digit<NH>(histA, 2048, 11, cs, gco, prefix, need);
         // key bits 20..10 of the keys whose bits 31..21 are prefix (few: counted with atomics)
@@ -322,7 +247,7 @@ sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16
             const uint32_t pf = prefix[h];
 #pragma unroll
             for (int j = 0; j < JMAX; ++j)
-                if (((vbits >> j) & 1u) && (key[j][h] >> 21) == pf) {
+                if (key[j][h] != 0u && (key[j][h] >> 21) == pf) {
                     const uint32_t d = (key[j][h] >> 10) & 0x7FFu;
                     atomicAdd(&histB[h * kHistWords + d], 1u);
                     atomicAdd(&histB[h * kHistWords + 2048 + (d >> 5)], 1u);
@@ -337,7 +262,7 @@ sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16
             const uint32_t pf = prefix[h];
 #pragma unroll
             for (int j = 0; j < JMAX; ++j)
-                if (((vbits >> j) & 1u) && (key[j][h] >> 10) == pf) {
+                if (key[j][h] != 0u && (key[j][h] >> 10) == pf) {
                     const uint32_t d = key[j][h] & 0x3FFu;
                     atomicAdd(&histA[h * kHistWords + d], 1u);
                     atomicAdd(&histA[h * kHistWords + 2048 + (d >> 5)], 1u);
@@ -345,9 +270,37 @@ sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16
         }
         cluster_sync();
         cluster_find_digit<NH>(histA, 1024, 10, cs, gco, prefix, need);
-        // now prefix[h] = tau, the B-th largest key, and need[h] = k.  Bin
-        // tau & 1023 of each CTA's last histogram counts its keys equal to
-        // tau: the ties each slice takes, in slice order, lowest first.
+        // now prefix[h] = tau, the B-th largest key, and need[h] = k
+    }
+
+    // ---- 3. Top and tie bitmaps of the slice ----------------------------------
+    {
+#pragma unroll
+        for (int j = 0; j < JMAX; ++j) {
+            const int wi = warp + kCWarps * j;
+            if (wi >= LW) break;  // warp-uniform
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const bool v = key[j][h] != 0u;
+                bool gt = false, eq = false;
+                if (mode == kModeSelect) {
+                    gt = v && key[j][h] > prefix[h];
+                    eq = v && key[j][h] == prefix[h];
+                } else if (mode == kModeAll) {
+                    gt = v;
+                }
+                const uint32_t tb = __ballot_sync(kFull, gt), eb = __ballot_sync(kFull, eq);
+                if (lane == 0) {
+                    top_s[h * LW + wi] = tb;
+                    aux_s[h * LW + wi] = eb;
+                }
+            }
+        }
+    }
+    __syncthreads();  // (the keys are dead from here on)
+    if (mode == kModeSelect) {
+        // bin tau & 1023 of each CTA's last histogram counts its keys equal
+        // to tau: the ties each slice takes, in slice order, lowest first
         if (warp < NH) {
             const int h = warp;
             const uint32_t tau = prefix[h], k = need[h];
@@ -402,31 +355,6 @@ sel_cluster_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16
         take_s[h] = 0u;
         nb_top[0][h] = (mode == kModeAll && r > 0) ? range_mask((s0 >> 5) - 1, lo, hi) : 0u;
         nb_top[1][h] = (mode == kModeAll && (int)r + 1 < cs) ? range_mask((s0 + L) >> 5, lo, hi) : 0u;
-    }
-
-    // ---- 3. Top and tie bitmaps of the slice ----------------------------------
-    {
-#pragma unroll
-        for (int j = 0; j < JMAX; ++j) {
-            const int wi = warp + kCWarps * j;
-            if (wi >= LW) break;  // warp-uniform
-            const bool v = (vbits >> j) & 1u;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                bool gt = false, eq = false;
-                if (mode == kModeSelect) {
-                    gt = v && key[j][h] > prefix[h];
-                    eq = v && key[j][h] == prefix[h];
-                } else if (mode == kModeAll) {
-                    gt = v;
-                }
-                const uint32_t tb = __ballot_sync(kFull, gt), eb = __ballot_sync(kFull, eq);
-                if (lane == 0) {
-                    top_s[h * LW + wi] = tb;
-                    aux_s[h * LW + wi] = eb;
-                }
-            }
-        }
     }
     __syncthreads();
     if (mode == kModeSelect && warp < NH) {
@@ -545,20 +473,19 @@ struct Plan {
     size_t smem = 0;
 };
 
-template <int DP, int SEL>
+template <int SEL>
 constexpr int max_slice() { return kCWarps * words_per_warp<SEL>() * 32; }
 
-template <int DP, int SEL>
+template <int SEL>
 size_t plan_smem(int L) {
     constexpr int NH = rows_per_group<SEL>();
-    return (size_t)kCWarps * ring_blocks<DP>() * 32 * DP * 2 + (size_t)NH * kHistWords * 4 +
-           (size_t)3 * NH * (L / 32) * 4;
+    return (size_t)2 * NH * kHistWords * 4 + (size_t)3 * NH * (L / 32) * 4;
 }
 
 // How many clusters of each size 1..16 the device holds at once (one CTA per
 // SM at the largest shared-memory size), queried once per device; nullptr
 // when the kernel cannot be set up.
-template <int DP, int SEL>
+template <int SEL>
 const int *active_clusters() {
     static std::atomic<int> state[kMaxDevices];  // 0 unknown, 1 ready, -1 unusable
     static int table[kMaxDevices][kMaxCluster + 1];
@@ -570,9 +497,9 @@ const int *active_clusters() {
         std::lock_guard<std::mutex> lock(mu);
         st = state[dev].load(std::memory_order_relaxed);
         if (st == 0) {
-            const void *fn = (const void *)sel_cluster_kernel<DP, SEL>;
+            const void *fn = (const void *)sel_cluster_kernel<SEL>;
             static std::atomic<int> smem_set[kMaxDevices];
-            const int smem = (int)plan_smem<DP, SEL>(max_slice<DP, SEL>());
+            const int smem = (int)plan_smem<SEL>(max_slice<SEL>());
             st = -1;
             if (ensure_dynamic_smem(fn, smem, smem_set) == cudaSuccess &&
                 cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
@@ -604,10 +531,10 @@ const int *active_clusters() {
 // Cluster size and slice length for dims `d`: the size that minimises waves x
 // slice length (the time of a latency-bound cluster grows with its slice),
 // larger clusters on ties; cs = 0 when no size holds a (sequence, KV head).
-template <int DP, int SEL>
+template <int SEL>
 Plan make_plan(const tb_dims &d) {
     Plan p;
-    const int *act = active_clusters<DP, SEL>();
+    const int *act = active_clusters<SEL>();
     if (!act) return p;
     const int Tcap = d.ctx_cap;
     const long long pairs = (long long)d.batch * d.n_kv_heads;
@@ -615,34 +542,36 @@ Plan make_plan(const tb_dims &d) {
     for (int cs = 1; cs <= kMaxCluster; ++cs) {
         const int L = ((Tcap + cs - 1) / cs + 31) / 32 * 32;
         const int used = (Tcap + L - 1) / L;  // CTAs that own positions
-        if (L > max_slice<DP, SEL>() || act[used] < 1 || plan_smem<DP, SEL>(L) > (size_t)kCDynMax) continue;
+        if (L > max_slice<SEL>() || act[used] < 1 || plan_smem<SEL>(L) > (size_t)kCDynMax) continue;
         const long long cost = (pairs + act[used] - 1) / act[used] * (long long)L;
         if (best < 0 || cost < best || (cost == best && used > p.cs)) {
             best = cost;
             p.cs = used;
             p.L = L;
             p.waves = (int)((pairs + act[used] - 1) / act[used]);
-            p.smem = plan_smem<DP, SEL>(L);
+            p.smem = plan_smem<SEL>(L);
         }
     }
     return p;
 }
 
-template <int DP, int SEL>
+template <int SEL>
 cudaError_t launch_cluster(const tb_dims &d, const Plan &p, const float *qp, int64_t qp_stride, const uint16_t *Kp,
                            const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, int32_t nbr,
                            int32_t *idx, int32_t idx_cap, int32_t *count, uint32_t *sel_bits, void *ws,
-                           cudaStream_t st) {
+                           cudaStream_t st, int32_t group_reduce) {
+    cudaError_t e = launch_score_keys(d, qp, qp_stride, Kp, ctx_len, sink, window, group_reduce, ws, st);
+    if (e != cudaSuccess) return e;
     const SelWs s = carve(d, ws);
     const int W = (d.ctx_cap + 31) / 32;
-    return launch_pdl_cluster(sel_cluster_kernel<DP, SEL>, dim3(p.cs, d.n_kv_heads, d.batch), dim3(kCThreads), p.cs,
-                              p.smem, st, qp, qp_stride, Kp, ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, p.L,
-                              sink, window, budget, nbr, idx, idx_cap, count, sel_bits, s.keys, s.flags);
+    return launch_pdl_cluster(sel_cluster_kernel<SEL>, dim3(p.cs, d.n_kv_heads, d.batch), dim3(kCThreads), p.cs,
+                              p.smem, st, ctx_len, d.n_q_heads, d.ctx_cap, W, p.L, sink, window, budget, nbr, idx,
+                              idx_cap, count, sel_bits, (const uint32_t *)s.keys, s.flags);
 }
 
 template <int SEL>
 Plan plan_for(const tb_dims &d) {
-    return d.d_proj == 32 ? make_plan<32, SEL>(d) : make_plan<16, SEL>(d);
+    return make_plan<SEL>(d);
 }
 
 }  // namespace
@@ -655,7 +584,9 @@ bool select_cluster_fits(const tb_dims &d, int32_t group_reduce, bool one_wave) 
         case 1: p = plan_for<kSelGroupSum>(d); break;
         default: return false;
     }
-    return p.cs > 0 && (!one_wave || p.waves == 1);
+    // (shorter slices leave the cluster kernel's fixed latency, ~30 barrier
+    // and exchange steps, larger than the multi-kernel path's whole cost)
+    return p.cs > 0 && (!one_wave || (p.waves == 1 && p.L >= kMinAutoSlice));
 }
 
 cudaError_t launch_score_select_cluster(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
@@ -666,10 +597,8 @@ cudaError_t launch_score_select_cluster(const tb_dims &d, const float *qp, int64
         constexpr int SEL = decltype(sel_tag)::value;
         const Plan p = plan_for<SEL>(d);
         if (p.cs == 0) return cudaErrorNotSupported;
-        return d.d_proj == 32 ? launch_cluster<32, SEL>(d, p, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr,
-                                                        idx, idx_cap, count, sel_bits, ws, st)
-                              : launch_cluster<16, SEL>(d, p, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr,
-                                                        idx, idx_cap, count, sel_bits, ws, st);
+        return launch_cluster<SEL>(d, p, qp, qp_stride, Kp, ctx_len, sink, window, budget, nbr, idx, idx_cap, count,
+                                   sel_bits, ws, st, group_reduce);
     };
     switch (group_reduce) {
         case -1: return go(std::integral_constant<int, kSelHead>());

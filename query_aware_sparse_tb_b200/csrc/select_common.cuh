@@ -11,7 +11,7 @@ namespace sel {
 constexpr int kGroup = 4;
 constexpr int kChunk = 2048;          // positions per CTA of mark_collect (one wave at 64K)
 constexpr int kHistChunk = 2048;      // positions per CTA of score_hist (one wave at 64K)
-constexpr int kSubRows = 512;         // K' rows per bulk-copied sub-chunk of score_hist
+constexpr int kHistRing = 4;          // 32-row blocks in each score_hist warp's ring (3 in flight)
 constexpr int kThreads = 256;
 constexpr int kBins1 = 2048;          // key bits 31..21
 constexpr int kBins2 = 2048;          // key bits 20..10
