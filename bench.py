@@ -19,6 +19,7 @@ max-over-ranks reduction of the device time use NCCL.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import math
 import os
@@ -121,14 +122,6 @@ class Run:
                                 marks=(lambda name, i=i: marks(name, i)) if marks else None)
 
     # ------------------------------------------------------------ accounting
-    def launches(self):
-        """(sparse kernel launches, dense kernel launches) of one run."""
-        nL = self.w.n_layers
-        n_proj = len(self.dec.proj_steps)
-        sel = 3 * nL * self.n_pred
-        pred = 4 * len(self.producers) * self.n_pred if self.w.hidden > 0 else 0
-        return self.steps * nL + sel + pred + n_proj * nL, self.steps * nL
-
     def union_rows(self):
         """Kept (b, kv-head, t) rows of every sparse attention launch of one run,
         counting a row once for the 4 query heads of its group: sink + window +
@@ -212,10 +205,48 @@ class Marks:
         return [self.ev[("attn_begin", i)].elapsed_time(self.ev[("attn_end", i)]) for i in range(steps)]
 
 
-def capture(fn, stream):
-    g = torch.cuda.CUDAGraph()
+class _KernelNodeParams(ctypes.Structure):
+    _fields_ = [("func", ctypes.c_void_p), ("grid", ctypes.c_uint * 3), ("block", ctypes.c_uint * 3),
+                ("shared_mem_bytes", ctypes.c_uint), ("kernel_params", ctypes.c_void_p), ("extra", ctypes.c_void_p)]
+
+
+def libtb_kernel_nodes(graph) -> int:
+    """Kernel nodes of a captured cudaGraph_t whose function is one of libtb's
+    (C++ namespace tb): the launches one replay makes."""
+    rt = ctypes.CDLL("libcudart.so.12")
+    P = ctypes.c_void_p
+    rt.cudaGraphGetNodes.argtypes = [P, P, ctypes.POINTER(ctypes.c_size_t)]
+    rt.cudaGraphNodeGetType.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
+    rt.cudaGraphKernelNodeGetParams.argtypes = [P, ctypes.POINTER(_KernelNodeParams)]
+    rt.cudaFuncGetName.argtypes = [ctypes.POINTER(ctypes.c_char_p), P]
+    n = ctypes.c_size_t(0)
+    if rt.cudaGraphGetNodes(P(graph), None, ctypes.byref(n)) != 0:
+        raise RuntimeError("cudaGraphGetNodes failed")
+    nodes = (P * n.value)()
+    if rt.cudaGraphGetNodes(P(graph), nodes, ctypes.byref(n)) != 0:
+        raise RuntimeError("cudaGraphGetNodes failed")
+    count = 0
+    for node in nodes:
+        t = ctypes.c_int(-1)
+        if rt.cudaGraphNodeGetType(P(node), ctypes.byref(t)) != 0 or t.value != 0:  # 0: kernel node
+            continue
+        prm = _KernelNodeParams()
+        name = ctypes.c_char_p()
+        if rt.cudaGraphKernelNodeGetParams(P(node), ctypes.byref(prm)) == 0 and \
+                rt.cudaFuncGetName(ctypes.byref(name), prm.func) == 0 and name.value and b"_ZN2tb" in name.value:
+            count += 1
+    return count
+
+
+def capture(fn, stream, count_kernels=False):
+    """Record fn(stream) into a CUDA graph; with count_kernels the graph also
+    carries `libtb_kernels`, the number of libtb kernels one replay launches."""
+    g = torch.cuda.CUDAGraph(keep_graph=count_kernels)
     with torch.cuda.graph(g, stream=stream):
         fn(stream)
+    if count_kernels:
+        g.libtb_kernels = libtb_kernel_nodes(g.raw_cuda_graph())
+        g.instantiate()
     return g
 
 
@@ -615,7 +646,7 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
     stream = torch.cuda.Stream(device=device)
     marks_s = Marks(run.steps)
     marks_s.stream = stream
-    g_sparse = capture(lambda st: run.run_sparse(st, marks_s), stream)
+    g_sparse = capture(lambda st: run.run_sparse(st, marks_s), stream, count_kernels=True)
     marks_d = Marks(run.steps)
     marks_d.stream = stream
     g_dense = capture(lambda st: run.run_dense(st, marks_d), stream)
@@ -655,7 +686,7 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
         dense_launch_ms=dense_launch_ms, dense_bytes_per_launch=(acct["dense_total"] / n_attn),
         path_gbs=acct["sparse_total"] / (per_step_sparse / 1000.0) / 1e9,
         dense_path_gbs=acct["dense_total"] / (per_step_dense / 1000.0) / 1e9,
-        launches=run.launches()[0], clocks=clk, flags=flags,
+        launches=g_sparse.libtb_kernels, clocks=clk, flags=flags,
         kv_gb=2 * sum(k.numel() for k in run.K) * 2 / 1e9)
     if e2e is not None:
         h2d, d2h = e2e.bytes_per_run()

@@ -235,7 +235,7 @@ tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_
  *
  *   TB_SELECT_AUTO          (default) the cluster route where one wave of
  *                           clusters holds the call with slices of at least
- *                           4,096 positions (long single sequences), else the
+ *                           512 positions (few long sequences), else the
  *                           multi-kernel route.
  *   TB_SELECT_MULTI_KERNEL  three kernels per call: scoring with a histogram,
  *                           marking and candidate collection, and a per-head
@@ -244,7 +244,7 @@ tb_status tb_score_select_scores(const tb_dims *dims, const void *ws, size_t ws_
  *                           thread-block cluster per (sequence, KV head) that
  *                           holds all of its scores on chip and selects.  It
  *                           applies while ctx_cap fits 16 CTAs (up to 131,072
- *                           positions for tb_score_select, 270,336 for
+ *                           positions for tb_score_select, 524,288 for
  *                           tb_score_select_group); elsewhere the selection
  *                           calls return TB_ERR_UNSUPPORTED.
  *

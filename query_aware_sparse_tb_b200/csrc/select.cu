@@ -54,7 +54,8 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
     using Sc = BlockScorer<DP>;
     constexpr int NW = kThreads / 32;
-    extern __shared__ __align__(128) uint8_t stage[];   // [warp][kHistRing][32-row block]
+    constexpr int RING = hist_ring(HIST);
+    extern __shared__ __align__(128) uint8_t stage[];   // [warp][RING][32-row block]
     __shared__ __align__(16) float qs[kGroup][DP];
     __shared__ uint32_t hist[HIST ? NH : 1][HIST ? kBins1 : 1];
     __shared__ int s_last;
@@ -76,27 +77,27 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     if (hi > lo && p0 < hi && p0 + kHistChunk > lo) {
         // the chunk's 32-row blocks that overlap C, dealt to the warps in
         // turn; each warp streams its blocks through a ring of its own
-        // (kHistRing - 1 in flight) and lane l scores row l of each
+        // (RING - 1 in flight) and lane l scores row l of each
         const int blo = max(0, lo - p0) / 32;
         const int bhi = min(kHistChunk, hi - p0 + 31) / 32;
         const int nb = blo + warp < bhi ? (bhi - blo - warp + NW - 1) / NW : 0;  // this warp's blocks
-        uint8_t *ring = stage + warp * kHistRing * Sc::BLKB;
+        uint8_t *ring = stage + warp * RING * Sc::BLKB;
         const uint32_t ring_s = smem_addr(ring);
         auto issue = [&](int i) {
             const int r0 = p0 + (blo + warp + NW * i) * 32;
-            Sc::copy(ring_s + (uint32_t)((i % kHistRing) * Sc::BLKB), Kp + (slab + r0) * DP, hi - r0, lane);
+            Sc::copy(ring_s + (uint32_t)((i % RING) * Sc::BLKB), Kp + (slab + r0) * DP, hi - r0, lane);
         };
-        for (int i = 0; i < kHistRing - 1; ++i) {
+        for (int i = 0; i < RING - 1; ++i) {
             if (i < nb) issue(i);
             cp_async_commit();
         }
         for (int i = 0; i < nb; ++i) {
-            if (i + kHistRing - 1 < nb) issue(i + kHistRing - 1);
+            if (i + RING - 1 < nb) issue(i + RING - 1);
             cp_async_commit();
-            cp_async_wait_group<kHistRing - 1>();
+            cp_async_wait_group<RING - 1>();
             __syncwarp();  // every lane's copies of block i have landed
             float sc[kGroup];
-            Sc::score(ring + (i % kHistRing) * Sc::BLKB, &qs[0][0], lane, sc);
+            Sc::score(ring + (i % RING) * Sc::BLKB, &qs[0][0], lane, sc);
             __syncwarp();  // block i is read before its slot is refilled
             const int p = p0 + (blo + warp + NW * i) * 32 + lane;
             const bool valid = p >= lo && p < hi;
@@ -753,7 +754,7 @@ cudaError_t launch_score_hist(const tb_dims &d, const float *qp, int64_t qp_stri
                               const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, const SelWs &s,
                               cudaStream_t st) {
     dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
-    const int hsm = (kThreads / 32) * kHistRing * 32 * d.d_proj * 2;  // the warps' rings of 32-row blocks
+    const int hsm = (kThreads / 32) * hist_ring(HIST) * 32 * d.d_proj * 2;  // the warps' rings of 32-row blocks
     cudaError_t e;
     if (d.d_proj == 32) {
         static std::atomic<int> smem_set32[kMaxDevices];

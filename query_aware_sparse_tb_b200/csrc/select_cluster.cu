@@ -14,12 +14,13 @@
 // by +-nbr and clipped to C.  Only the route differs.  The scores come first,
 // from score_hist's keys-only variant on every SM (scoring streams K', which
 // wants all of them); then one cluster per (sequence, KV head) selects.  CTA r
-// of a cluster of CS owns the positions [r*L, (r+1)*L), L a multiple of 32,
-// and warp w of it the 32-position words w, w + 16, w + 32, ... of that slice:
-//   1. keys   each lane loads the keys of its positions from the workspace
-//             (just written, so from L2) into registers, lane = position in
-//             the word; a histogram of key bits 31..21 per head is built on
-//             the way.
+// of a cluster of CS owns the positions [r*L, (r+1)*L), L a multiple of 32:
+//   1. keys   the CTA loads the keys of its slice from the workspace (just
+//             written, so from L2) into shared memory, a warp per 32-position
+//             word, lane = position; a histogram of key bits 31..21 per head
+//             is built on the way.  Every later step loops over these words
+//             (compact code: the kernel is otherwise bound by instruction
+//             fetch).
 //   2. radix  three passes (key bits 31..21, 20..10, 9..0) fix the B-th
 //             largest key tau and k, how many keys equal to it are taken.  In
 //             each, a CTA histograms its keys that match the digits fixed so
@@ -52,18 +53,18 @@ namespace {
 
 using namespace sel;
 
-constexpr int kCThreads = 512;        // 16 warps
+constexpr int kCThreads = 1024;       // 32 warps
 constexpr int kCWarps = kCThreads / 32;
 constexpr int kHistWords = 2048 + 64; // per head: up to 2048 bins, then up to 64 group sums
 constexpr int kCDynMax = 227 * 1024 - 4096;
 constexpr int kMaxCluster = 16;
-constexpr int kMinAutoSlice = 4096;   // the automatic route takes the cluster kernel from this slice length
+constexpr int kMinAutoSlice = 512;    // the automatic route takes the cluster kernel from this slice length
 
 template <int SEL>
 __host__ __device__ constexpr int rows_per_group() { return sel_is_group(SEL) ? 1 : kGroup; }
-// Words of the slice each warp owns (keys held in registers: 64 or 33 per thread).
+// Longest slice: its keys (4 bytes per position and score row) take 128 KB.
 template <int SEL>
-__host__ __device__ constexpr int words_per_warp() { return sel_is_group(SEL) ? 33 : 16; }
+__host__ __device__ constexpr int max_slice() { return sel_is_group(SEL) ? 32768 : 8192; }
 // Sum of the word at `local` over the shared memory of cluster CTAs 0 .. cs-1
 // (every read issued before the first is added).
 __device__ __forceinline__ uint32_t cluster_sum(const uint32_t *local, int cs) {
@@ -173,7 +174,6 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
                    uint32_t *__restrict__ sel_bits, const uint32_t *__restrict__ gkeys, uint32_t *__restrict__ flags) {
     constexpr int NH = rows_per_group<SEL>();
     constexpr int NOUT = sel_is_group(SEL) ? kGroup : 1;  // output rows per score row
-    constexpr int JMAX = words_per_warp<SEL>();
     const int LW = L / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lt = (1u << lane) - 1u;
@@ -182,9 +182,10 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
     const uint32_t r = cluster_ctarank();
     const int s0 = (int)r * L;
 
-    // dynamic shared memory: [radix pass 2 histogram] [histogram A] [Top] [aux] [word prefix]
+    // dynamic shared memory: [keys] [radix pass 2 histogram] [histogram A] [Top] [aux] [word prefix]
     extern __shared__ __align__(128) uint8_t csm[];
-    uint32_t *histB = reinterpret_cast<uint32_t *>(csm);
+    uint32_t *keys_s = reinterpret_cast<uint32_t *>(csm);  // [NH][L]
+    uint32_t *histB = keys_s + (size_t)NH * L;
     uint32_t *histA = histB + NH * kHistWords;
     uint32_t *top_s = histA + NH * kHistWords;
     uint32_t *aux_s = top_s + NH * LW;
@@ -208,26 +209,21 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
     const int a = max(lo, s0), e = min(hi, s0 + L);  // this slice's part of C
     const size_t krow0 = (size_t)b * Hq + (size_t)g * kGroup;  // first workspace key row of the group
 
-    // ---- 1. keys in registers, key[j][h] = word warp + 16 j, bit lane; 0
-    // marks a position outside C (no score has key 0: score_key maps every
-    // float, NaNs included, to a key of at least 0x007fffff)
-    uint32_t key[JMAX][NH];
-#pragma unroll
-    for (int j = 0; j < JMAX; ++j) {
-        const int wi = warp + kCWarps * j;
-        const int p = s0 + 32 * wi + lane;
-        const bool v = wi < LW && p >= a && p < e;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) key[j][h] = v ? __ldcg(gkeys + (krow0 + h) * Tcap + p) : 0u;
-    }
-#pragma unroll
-    for (int j = 0; j < JMAX; ++j) {
-        const int wi = warp + kCWarps * j;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            if (key[j][h] != 0u) atomicAdd(&histA[h * kHistWords + (key[j][h] >> 21)], 1u);
-            if (wi == 0) edge_s[0][h][lane] = key[j][h];
-            if (wi == LW - 1) edge_s[1][h][lane] = key[j][h];
+    // ---- 1. the slice's keys into shared memory, word wi of score row h at
+    // keys_s[h * L + 32 wi + lane]; 0 marks a position outside C (no score
+    // has key 0: score_key maps every float, NaNs included, to a key of at
+    // least 0x007fffff)
+#pragma unroll 1
+    for (int h = 0; h < NH; ++h) {
+        const uint32_t *src = gkeys + (krow0 + h) * Tcap;
+#pragma unroll 4
+        for (int wi = warp; wi < LW; wi += kCWarps) {
+            const int p = s0 + 32 * wi + lane;
+            const uint32_t k = (p >= a && p < e) ? __ldcg(src + p) : 0u;
+            keys_s[h * L + 32 * wi + lane] = k;
+            if (k != 0u) atomicAdd(&histA[h * kHistWords + (k >> 21)], 1u);
+            if (wi == 0) edge_s[0][h][lane] = k;
+            if (wi == LW - 1) edge_s[1][h][lane] = k;
         }
     }
     __syncthreads();
@@ -242,62 +238,66 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
         cluster_sync();
         cluster_find_digit<NH>(histA, 2048, 11, cs, gco, prefix, need);
         // key bits 20..10 of the keys whose bits 31..21 are prefix (few: counted with atomics)
-#pragma unroll
+#pragma unroll 1
         for (int h = 0; h < NH; ++h) {
             const uint32_t pf = prefix[h];
-#pragma unroll
-            for (int j = 0; j < JMAX; ++j)
-                if (key[j][h] != 0u && (key[j][h] >> 21) == pf) {
-                    const uint32_t d = (key[j][h] >> 10) & 0x7FFu;
+#pragma unroll 4
+            for (int i = tid; i < L; i += kCThreads) {
+                const uint32_t k = keys_s[h * L + i];
+                if (k != 0u && (k >> 21) == pf) {
+                    const uint32_t d = (k >> 10) & 0x7FFu;
                     atomicAdd(&histB[h * kHistWords + d], 1u);
                     atomicAdd(&histB[h * kHistWords + 2048 + (d >> 5)], 1u);
                 }
+            }
         }
+        __syncthreads();
         cluster_sync();  // (also: every CTA is past its reads of histogram A)
         cluster_find_digit<NH>(histB, 2048, 11, cs, gco, prefix, need);
         for (int i = tid; i < NH * kHistWords; i += kCThreads) histA[i] = 0u;
         __syncthreads();
-#pragma unroll
+#pragma unroll 1
         for (int h = 0; h < NH; ++h) {
             const uint32_t pf = prefix[h];
-#pragma unroll
-            for (int j = 0; j < JMAX; ++j)
-                if (key[j][h] != 0u && (key[j][h] >> 10) == pf) {
-                    const uint32_t d = key[j][h] & 0x3FFu;
+#pragma unroll 4
+            for (int i = tid; i < L; i += kCThreads) {
+                const uint32_t k = keys_s[h * L + i];
+                if (k != 0u && (k >> 10) == pf) {
+                    const uint32_t d = k & 0x3FFu;
                     atomicAdd(&histA[h * kHistWords + d], 1u);
                     atomicAdd(&histA[h * kHistWords + 2048 + (d >> 5)], 1u);
                 }
+            }
         }
+        __syncthreads();
         cluster_sync();
         cluster_find_digit<NH>(histA, 1024, 10, cs, gco, prefix, need);
         // now prefix[h] = tau, the B-th largest key, and need[h] = k
     }
 
     // ---- 3. Top and tie bitmaps of the slice ----------------------------------
-    {
-#pragma unroll
-        for (int j = 0; j < JMAX; ++j) {
-            const int wi = warp + kCWarps * j;
-            if (wi >= LW) break;  // warp-uniform
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                const bool v = key[j][h] != 0u;
-                bool gt = false, eq = false;
-                if (mode == kModeSelect) {
-                    gt = v && key[j][h] > prefix[h];
-                    eq = v && key[j][h] == prefix[h];
-                } else if (mode == kModeAll) {
-                    gt = v;
-                }
-                const uint32_t tb = __ballot_sync(kFull, gt), eb = __ballot_sync(kFull, eq);
-                if (lane == 0) {
-                    top_s[h * LW + wi] = tb;
-                    aux_s[h * LW + wi] = eb;
-                }
+#pragma unroll 1
+    for (int h = 0; h < NH; ++h) {
+        const uint32_t tau = prefix[h];
+#pragma unroll 2
+        for (int wi = warp; wi < LW; wi += kCWarps) {
+            const uint32_t k = keys_s[h * L + 32 * wi + lane];
+            const bool v = k != 0u;
+            bool gt = false, eq = false;
+            if (mode == kModeSelect) {
+                gt = v && k > tau;
+                eq = v && k == tau;
+            } else if (mode == kModeAll) {
+                gt = v;
+            }
+            const uint32_t tb = __ballot_sync(kFull, gt), eb = __ballot_sync(kFull, eq);
+            if (lane == 0) {
+                top_s[h * LW + wi] = tb;
+                aux_s[h * LW + wi] = eb;
             }
         }
     }
-    __syncthreads();  // (the keys are dead from here on)
+    __syncthreads();
     if (mode == kModeSelect) {
         // bin tau & 1023 of each CTA's last histogram counts its keys equal
         // to tau: the ties each slice takes, in slice order, lowest first
@@ -474,12 +474,9 @@ struct Plan {
 };
 
 template <int SEL>
-constexpr int max_slice() { return kCWarps * words_per_warp<SEL>() * 32; }
-
-template <int SEL>
 size_t plan_smem(int L) {
     constexpr int NH = rows_per_group<SEL>();
-    return (size_t)2 * NH * kHistWords * 4 + (size_t)3 * NH * (L / 32) * 4;
+    return (size_t)NH * L * 4 + (size_t)2 * NH * kHistWords * 4 + (size_t)3 * NH * (L / 32) * 4;
 }
 
 // How many clusters of each size 1..16 the device holds at once (one CTA per

@@ -11,7 +11,9 @@ namespace sel {
 constexpr int kGroup = 4;
 constexpr int kChunk = 2048;          // positions per CTA of mark_collect (one wave at 64K)
 constexpr int kHistChunk = 2048;      // positions per CTA of score_hist (one wave at 64K)
-constexpr int kHistRing = 4;          // 32-row blocks in each score_hist warp's ring (3 in flight)
+// 32-row blocks in each score_hist warp's ring: 3 in flight beside the
+// histogram, 5 when the kernel only writes keys (two CTAs per SM either way)
+__host__ __device__ constexpr int hist_ring(bool hist) { return hist ? 4 : 6; }
 constexpr int kThreads = 256;
 constexpr int kBins1 = 2048;          // key bits 31..21
 constexpr int kBins2 = 2048;          // key bits 20..10

@@ -107,3 +107,34 @@ def test_forced_cluster_route_refuses_what_does_not_fit():
     clus = _run(_lib.TB_SELECT_CLUSTER, dm, Kp, qp, [130_000], 16, 64, 1024, 1, "max")
     for a, b in zip(multi[:3], clus[:3]):
         assert np.array_equal(a, b)
+
+
+def test_graph_kernel_count_follows_the_route():
+    """bench.py reports the libtb kernels its graphs launch by counting the
+    graph's kernel nodes; one selection call is 3 kernels on the multi-kernel
+    route and 2 (scoring, then the cluster selection) on the cluster route."""
+    import bench
+    batch, hkv, dp, cap, ctx, sink, window, budget, nbr = CASES["ragged_modes"]
+    dm = tb.dims(batch=batch, n_q_heads=4 * hkv, n_kv_heads=hkv, head_dim=128, d_proj=dp, ctx_cap=cap)
+    Kp, qp = _inputs(3, batch, hkv, dp, cap, "normal")
+    hq, W = dm.n_q_heads, (cap + 31) // 32
+    idx = torch.zeros((batch, hq, min((2 * nbr + 1) * budget, cap)), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((batch, hq), dtype=torch.int32, device=DEV)
+    bits = torch.zeros((batch, hq, W), dtype=torch.int32, device=DEV)
+    ws = tb.workspace(tb.score_select_workspace_bytes(dm))
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device=DEV)
+    st = torch.cuda.Stream()
+    counts = {}
+    for algo in (_lib.TB_SELECT_MULTI_KERNEL, _lib.TB_SELECT_CLUSTER):
+        _lib.select_set_algorithm(algo)
+        try:
+            tb.score_select(dm, qp, hq * dp, Kp, ctx_t, sink, window, budget, nbr, idx, cnt, bits, ws)  # set-up
+            torch.cuda.synchronize()
+            g = bench.capture(lambda s: tb.score_select(dm, qp, hq * dp, Kp, ctx_t, sink, window, budget, nbr, idx,
+                                                        cnt, bits, ws, stream=s), st, count_kernels=True)
+        finally:
+            _lib.select_set_algorithm(_lib.TB_SELECT_AUTO)
+        g.replay()
+        torch.cuda.synchronize()
+        counts[algo] = g.libtb_kernels
+    assert counts == {_lib.TB_SELECT_MULTI_KERNEL: 3, _lib.TB_SELECT_CLUSTER: 2}
