@@ -405,6 +405,17 @@ __device__ __forceinline__ uint32_t ld_dsmem(const void *local, uint32_t rank) {
     return v;
 }
 
+// Generic address of the word at `local` (in this CTA's shared memory) in the
+// shared memory of cluster CTA `rank`; plain loads through it read
+// distributed shared memory, and several can be in flight at once.  The
+// mapping is ordered after earlier cluster barriers (volatile asm), so loads
+// through it are too.
+__device__ __forceinline__ const uint32_t *dsmem_ptr(const uint32_t *local, uint32_t rank) {
+    uint64_t g;
+    asm volatile("mapa.u64 %0, %1, %2;\n" : "=l"(g) : "l"(local), "r"(rank));
+    return reinterpret_cast<const uint32_t *>(g);
+}
+
 // ------------------------------------------------------ named barriers ----
 
 // Barrier `id` over `n` threads (whole warps) that also returns whether any of

@@ -9,7 +9,8 @@
 // selected tokens are expanded by their spatial neighbours.
 //
 // Exact top-B on the fp32 scores, ties broken by the lower position:
-//   1. score_hist   one CTA per (b, KV head, 2048 positions): each warp
+//   1. score_hist   one CTA per (b, KV head, 2048 positions; without the
+//                   histogram, chunks sized for two CTAs per SM): each warp
 //                   streams 32-row blocks of K' through a cp.async ring of its
 //                   own and scores each row once for the 4 query heads of the
 //                   group (BlockScorer), writes the
@@ -32,6 +33,8 @@
 // the neighbours (finalize keeps the longest prefix of the top-B, in score
 // order, whose neighbourhoods cover at most B positions, found with a radix
 // select over the candidates' composites weighted by what each one adds).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "score.cuh"
@@ -50,7 +53,7 @@ template <int DP, int SEL, bool HIST>
 __global__ void __launch_bounds__(kThreads, 2)
 score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_t *__restrict__ Kp,
                   const int32_t *__restrict__ ctx_len, int Hq, int Hkv, int Tcap, int sink,
-                  int window, int budget, SelWs ws) {
+                  int window, int budget, int chunk, SelWs ws) {
     constexpr int NH = sel_is_group(SEL) ? 1 : kGroup;  // score rows per (b, KV head)
     using Sc = BlockScorer<DP>;
     constexpr int NW = kThreads / 32;
@@ -62,7 +65,7 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     __shared__ int scratch[kThreads / 32 + 3];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, ch = blockIdx.x;
-    const int p0 = ch * kHistChunk;
+    const int p0 = ch * chunk;  // this CTA's positions: [p0, p0 + chunk), chunk a multiple of 32
 
     if constexpr (HIST)
         for (int i = tid; i < NH * kBins1; i += kThreads) (&hist[0][0])[i] = 0u;
@@ -74,12 +77,12 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     __syncthreads();
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
-    if (hi > lo && p0 < hi && p0 + kHistChunk > lo) {
+    if (hi > lo && p0 < hi && p0 + chunk > lo) {
         // the chunk's 32-row blocks that overlap C, dealt to the warps in
         // turn; each warp streams its blocks through a ring of its own
         // (RING - 1 in flight) and lane l scores row l of each
         const int blo = max(0, lo - p0) / 32;
-        const int bhi = min(kHistChunk, hi - p0 + 31) / 32;
+        const int bhi = min(chunk, hi - p0 + 31) / 32;
         const int nb = blo + warp < bhi ? (bhi - blo - warp + NW - 1) / NW : 0;  // this warp's blocks
         uint8_t *ring = stage + warp * RING * Sc::BLKB;
         const uint32_t ring_s = smem_addr(ring);
@@ -753,7 +756,15 @@ template <int SEL, bool HIST>
 cudaError_t launch_score_hist(const tb_dims &d, const float *qp, int64_t qp_stride, const uint16_t *Kp,
                               const int32_t *ctx_len, int32_t sink, int32_t window, int32_t budget, const SelWs &s,
                               cudaStream_t st) {
-    dim3 grid_h((d.ctx_cap + kHistChunk - 1) / kHistChunk, d.n_kv_heads, d.batch);
+    // with the histogram: 2048 positions a CTA; keys only: chunks that make
+    // the grid about two CTAs per SM, so every SM streams its share of K'
+    int chunk = kHistChunk;
+    if (!HIST) {
+        const long long pairs = (long long)d.batch * d.n_kv_heads;
+        const long long want = (long long)d.ctx_cap * pairs / (2LL * num_sms());
+        chunk = (int)std::max(512LL, (want + 31) / 32 * 32);
+    }
+    dim3 grid_h((d.ctx_cap + chunk - 1) / chunk, d.n_kv_heads, d.batch);
     const int hsm = (kThreads / 32) * hist_ring(HIST) * 32 * d.d_proj * 2;  // the warps' rings of 32-row blocks
     cudaError_t e;
     if (d.d_proj == 32) {
@@ -761,13 +772,13 @@ cudaError_t launch_score_hist(const tb_dims &d, const float *qp, int64_t qp_stri
         if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<32, SEL, HIST>, hsm, smem_set32)) != cudaSuccess)
             return e;
         return launch_pdl(score_hist_kernel<32, SEL, HIST>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp,
-                          ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+                          ctx_len, d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, chunk, s);
     }
     static std::atomic<int> smem_set16[kMaxDevices];
     if ((e = ensure_dynamic_smem((const void *)score_hist_kernel<16, SEL, HIST>, hsm, smem_set16)) != cudaSuccess)
         return e;
     return launch_pdl(score_hist_kernel<16, SEL, HIST>, grid_h, dim3(kThreads), hsm, st, qp, qp_stride, Kp, ctx_len,
-                      d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, s);
+                      d.n_q_heads, d.n_kv_heads, d.ctx_cap, sink, window, budget, chunk, s);
 }
 
 template <int SEL>

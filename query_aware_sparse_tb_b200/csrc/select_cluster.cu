@@ -70,7 +70,7 @@ __host__ __device__ constexpr int max_slice() { return sel_is_group(SEL) ? 32768
 __device__ __forceinline__ uint32_t cluster_sum(const uint32_t *local, int cs) {
     uint32_t v[kMaxCluster];
 #pragma unroll
-    for (int q = 0; q < kMaxCluster; ++q) v[q] = q < cs ? ld_dsmem(local, (uint32_t)q) : 0u;
+    for (int q = 0; q < kMaxCluster; ++q) v[q] = q < cs ? *dsmem_ptr(local, (uint32_t)q) : 0u;
     uint32_t s = 0;
 #pragma unroll
     for (int q = 0; q < kMaxCluster; ++q) s += v[q];
@@ -213,17 +213,32 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
     // keys_s[h * L + 32 wi + lane]; 0 marks a position outside C (no score
     // has key 0: score_key maps every float, NaNs included, to a key of at
     // least 0x007fffff)
-#pragma unroll 1
-    for (int h = 0; h < NH; ++h) {
-        const uint32_t *src = gkeys + (krow0 + h) * Tcap;
-#pragma unroll 4
-        for (int wi = warp; wi < LW; wi += kCWarps) {
-            const int p = s0 + 32 * wi + lane;
-            const uint32_t k = (p >= a && p < e) ? __ldcg(src + p) : 0u;
-            keys_s[h * L + 32 * wi + lane] = k;
-            if (k != 0u) atomicAdd(&histA[h * kHistWords + (k >> 21)], 1u);
-            if (wi == 0) edge_s[0][h][lane] = k;
-            if (wi == LW - 1) edge_s[1][h][lane] = k;
+    {
+        // the thread's loads go out 8 at a time, each batch issued before
+        // its first key is used
+        constexpr int WPW = max_slice<SEL>() / 32 / kCWarps;  // words of a score row per warp, at most
+        constexpr int NLD = NH * WPW, BATCH = 8;
+        static_assert(NLD % BATCH == 0, "whole batches");
+#pragma unroll
+        for (int b0 = 0; b0 < NLD; b0 += BATCH) {
+            uint32_t kv[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                const int h = (b0 + i) / WPW, wi = warp + kCWarps * ((b0 + i) % WPW);
+                const int p = s0 + 32 * wi + lane;
+                kv[i] = (wi < LW && p >= a && p < e) ? __ldcg(gkeys + (krow0 + h) * Tcap + p) : 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                const int h = (b0 + i) / WPW, wi = warp + kCWarps * ((b0 + i) % WPW);
+                if (wi < LW) {  // warp-uniform
+                    const uint32_t k = kv[i];
+                    keys_s[h * L + 32 * wi + lane] = k;
+                    if (k != 0u) atomicAdd(&histA[h * kHistWords + (k >> 21)], 1u);
+                    if (wi == 0) edge_s[0][h][lane] = k;
+                    if (wi == LW - 1) edge_s[1][h][lane] = k;
+                }
+            }
         }
     }
     __syncthreads();
@@ -276,11 +291,15 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
     }
 
     // ---- 3. Top and tie bitmaps of the slice ----------------------------------
+    // (lane q keeps the ballots of the warp's q-th word and stores them after
+    // the loop: one store per lane, no branch per word)
 #pragma unroll 1
     for (int h = 0; h < NH; ++h) {
         const uint32_t tau = prefix[h];
+        uint32_t my_top = 0u, my_tie = 0u;
+        int q = 0;
 #pragma unroll 2
-        for (int wi = warp; wi < LW; wi += kCWarps) {
+        for (int wi = warp; wi < LW; wi += kCWarps, ++q) {
             const uint32_t k = keys_s[h * L + 32 * wi + lane];
             const bool v = k != 0u;
             bool gt = false, eq = false;
@@ -291,10 +310,13 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
                 gt = v;
             }
             const uint32_t tb = __ballot_sync(kFull, gt), eb = __ballot_sync(kFull, eq);
-            if (lane == 0) {
-                top_s[h * LW + wi] = tb;
-                aux_s[h * LW + wi] = eb;
-            }
+            my_top = lane == q ? tb : my_top;
+            my_tie = lane == q ? eb : my_tie;
+        }
+        const int wi = warp + kCWarps * lane;
+        if (lane < q && wi < LW) {
+            top_s[h * LW + wi] = my_top;
+            aux_s[h * LW + wi] = my_tie;
         }
     }
     __syncthreads();
@@ -445,6 +467,7 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
             const uint32_t base = base_s[h];
+#pragma unroll 4
             for (int wi = warp; wi < LW; wi += kCWarps) {
                 const uint32_t ev = aux_s[h * LW + wi];
                 const uint32_t slot = base + (wpre_s[h * LW + wi] - hstart) + __popc(ev & lt);
