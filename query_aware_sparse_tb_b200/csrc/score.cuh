@@ -96,6 +96,41 @@ struct BlockScorer {
 #pragma unroll
         for (int h = 0; h < 4; ++h) s[h] = sum_f32x2(acc[h]);
     }
+
+    // score() for row `lane` of two staged blocks at once: every query load
+    // serves both rows (the operations on each row are those of score()).
+    __device__ __forceinline__ static void score2(const uint8_t *slot_a, const uint8_t *slot_b, const float *qs,
+                                                  int lane, float sa[4], float sb[4]) {
+        const uint8_t *row_a = slot_a + lane * ROWB;
+        const uint8_t *row_b = slot_b + lane * ROWB;
+        const int rt = rot(lane);
+        uint64_t acc_a[4] = {0ull, 0ull, 0ull, 0ull}, acc_b[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int v = 0; v < NPART; ++v) {
+            const uint4 ra = *reinterpret_cast<const uint4 *>(row_a + ((v + rt) % NPART) * 16);
+            const uint4 rb = *reinterpret_cast<const uint4 *>(row_b + ((v + rt) % NPART) * 16);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float4 qa = *reinterpret_cast<const float4 *>(qs + h * DP + 8 * v);
+                const float4 qb = *reinterpret_cast<const float4 *>(qs + h * DP + 8 * v + 4);
+                const uint64_t q0 = pack_f32x2(qa.x, qa.y), q1 = pack_f32x2(qa.z, qa.w);
+                const uint64_t q2 = pack_f32x2(qb.x, qb.y), q3 = pack_f32x2(qb.z, qb.w);
+                acc_a[h] = fma_f32x2(q0, bf16x2_to_f32x2(ra.x), acc_a[h]);
+                acc_a[h] = fma_f32x2(q1, bf16x2_to_f32x2(ra.y), acc_a[h]);
+                acc_a[h] = fma_f32x2(q2, bf16x2_to_f32x2(ra.z), acc_a[h]);
+                acc_a[h] = fma_f32x2(q3, bf16x2_to_f32x2(ra.w), acc_a[h]);
+                acc_b[h] = fma_f32x2(q0, bf16x2_to_f32x2(rb.x), acc_b[h]);
+                acc_b[h] = fma_f32x2(q1, bf16x2_to_f32x2(rb.y), acc_b[h]);
+                acc_b[h] = fma_f32x2(q2, bf16x2_to_f32x2(rb.z), acc_b[h]);
+                acc_b[h] = fma_f32x2(q3, bf16x2_to_f32x2(rb.w), acc_b[h]);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            sa[h] = sum_f32x2(acc_a[h]);
+            sb[h] = sum_f32x2(acc_b[h]);
+        }
+    }
 };
 
 }  // namespace tb

@@ -90,18 +90,13 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
             const int r0 = p0 + (blo + warp + NW * i) * 32;
             Sc::copy(ring_s + (uint32_t)((i % RING) * Sc::BLKB), Kp + (slab + r0) * DP, hi - r0, lane);
         };
-        for (int i = 0; i < RING - 1; ++i) {
+        // blocks go in pairs: RING - 2 in flight beside the pair being scored
+        static_assert(RING % 2 == 0, "pairs of slots");
+        for (int i = 0; i < RING - 2; ++i) {
             if (i < nb) issue(i);
             cp_async_commit();
         }
-        for (int i = 0; i < nb; ++i) {
-            if (i + RING - 1 < nb) issue(i + RING - 1);
-            cp_async_commit();
-            cp_async_wait_group<RING - 1>();
-            __syncwarp();  // every lane's copies of block i have landed
-            float sc[kGroup];
-            Sc::score(ring + (i % RING) * Sc::BLKB, &qs[0][0], lane, sc);
-            __syncwarp();  // block i is read before its slot is refilled
+        auto emit = [&](int i, const float *sc) {  // block i's keys (and histogram)
             const int p = p0 + (blo + warp + NW * i) * 32 + lane;
             const bool valid = p >= lo && p < hi;
             if constexpr (!sel_is_group(SEL)) {
@@ -123,6 +118,23 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                     if constexpr (HIST) atomicAdd(&hist[0][key >> 21], 1u);
                 }
             }
+        };
+        for (int i = 0; i < nb; i += 2) {
+            if (i + RING - 2 < nb) issue(i + RING - 2);
+            cp_async_commit();
+            if (i + RING - 1 < nb) issue(i + RING - 1);
+            cp_async_commit();
+            cp_async_wait_group<RING - 2>();
+            __syncwarp();  // every lane's copies of blocks i and i + 1 have landed
+            float sa[kGroup], sb[kGroup];
+            if (i + 1 < nb) {
+                Sc::score2(ring + (i % RING) * Sc::BLKB, ring + ((i + 1) % RING) * Sc::BLKB, &qs[0][0], lane, sa, sb);
+            } else {
+                Sc::score(ring + (i % RING) * Sc::BLKB, &qs[0][0], lane, sa);
+            }
+            __syncwarp();  // the blocks are read before their slots are refilled
+            emit(i, sa);
+            if (i + 1 < nb) emit(i + 1, sb);
         }
     }
     if constexpr (!HIST) return;
