@@ -256,7 +256,9 @@ class E2E:
     queries and the new token's K and V rows, packed), tb_kv_append writes the
     rows into every layer's cache in one launch, prediction steps also copy the
     producer hidden states, and one device->host copy returns all layers'
-    attention outputs."""
+    attention outputs.  The copies run on a stream of their own, double
+    buffered, as a serving loop would issue them: step i+1's inputs come in
+    and step i's outputs go out while step i+1 computes."""
 
     def __init__(self, run: Run):
         self.run = run
@@ -275,9 +277,11 @@ class E2E:
                     kv[l, 1, b] = run.V[l][b, :, pos[i][b]].cpu()
             packed[i, q_el:] = kv.reshape(-1)
         self.host = packed.pin_memory()
-        self.dev = torch.empty(q_el + kv_el, dtype=torch.bfloat16, device=run.device)
-        self.q_dev = self.dev[:q_el].view(run.Q[0].shape)
-        self.kv_dev = self.dev[q_el:]
+        self.dev = [torch.empty(q_el + kv_el, dtype=torch.bfloat16, device=run.device) for _ in range(2)]
+        self.q_dev = [d[:q_el].view(run.Q[0].shape) for d in self.dev]
+        self.kv_dev = [d[q_el:] for d in self.dev]
+        self.out = [run.out, torch.empty_like(run.out)]
+        self.copy_stream = torch.cuda.Stream(device=run.device)
         self.caches = torch.tensor([p for l in range(nL) for p in (run.K[l].data_ptr(), run.V[l].data_ptr())],
                                    dtype=torch.int64, device=run.device)
         self.ws = L.workspace(256, run.device)
@@ -294,16 +298,43 @@ class E2E:
 
     def body(self, stream):
         r, w = self.run, self.run.w
-        for i in range(r.steps):
-            self.dev.copy_(self.host[i], non_blocking=True)
-            L.kv_append(r.dec.dims, w.n_layers, self.kv_dev, self.caches, r.dec.ctx[i], self.ws, stream)
+        cs = self.copy_stream
+        n = r.steps
+        in_ready = [torch.cuda.Event() for _ in range(n)]   # step i's inputs are on the device
+        in_done = [torch.cuda.Event() for _ in range(n)]    # step i has read them (slot i % 2 free)
+        out_ready = [torch.cuda.Event() for _ in range(n)]  # step i's outputs are written
+        out_done = [torch.cuda.Event() for _ in range(n)]   # ... and copied to the host (slot i % 2 free)
+        self._events = (in_ready, in_done, out_ready, out_done)
+
+        def fetch(i):  # step i's inputs into slot i % 2, on the copy stream
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(in_done[i - 2])
+                self.dev[i % 2].copy_(self.host[i], non_blocking=True)
+                in_ready[i].record(cs)
+
+        cs.wait_stream(stream)
+        fetch(0)
+        for i in range(n):
+            if i + 1 < n:
+                fetch(i + 1)
+            stream.wait_event(in_ready[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])
+            L.kv_append(r.dec.dims, w.n_layers, self.kv_dev[i % 2], self.caches, r.dec.ctx[i], self.ws, stream)
             h = None
             if is_prediction_step(i, w.interval) and self.h_host is not None:
                 self.h_dev.copy_(self.h_host[i // w.interval], non_blocking=True)
                 h = self.h_dev
             qd = r.qp_direct[i // w.interval] if r.qp_direct is not None else None
-            r.dec.step(i, self.q_dev, r.out, h=h, qp_direct=qd, stream=stream)
-            self.out_host[i].copy_(r.out, non_blocking=True)
+            r.dec.step(i, self.q_dev[i % 2], self.out[i % 2], h=h, qp_direct=qd, stream=stream)
+            in_done[i].record(stream)
+            out_ready[i].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(out_ready[i])
+                self.out_host[i].copy_(self.out[i % 2], non_blocking=True)
+                out_done[i].record(cs)
+        stream.wait_stream(cs)
 
 
 def replica(base: tb_inputs.Workload, rank: int) -> tb_inputs.Workload:
