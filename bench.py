@@ -819,7 +819,7 @@ def main():
     ap.add_argument("--extra-steps", type=int, default=3, help="timed bench steps of each extra workload")
     ap.add_argument("--no-offload", action="store_true",
                     help="skip the CPU-offloaded KV cache on long256k (per-token latency against dense), which the "
-                         "default run times after the headline workload")
+                         "default single-GPU run times after the headline workload")
     ap.add_argument("--offload-only", action="store_true", help="time only the CPU-offloaded workload")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "kv_heads"],
                     help="with N > 1 ranks: replicas (each rank decodes its own seeded replica; weak scaling) or "
@@ -871,8 +871,10 @@ def main():
                                                max(3, args.warmup), args.selection, shard), measured_peaks()[0])
 
     offload = None
+    # (a per-token latency on one GPU: not run under torchrun, where every
+    # rank would pin its own 34 GB copy of the cache in host memory)
     if not args.no_offload and args.workload == "llama64k" and not args.layers and not args.decode_steps and \
-            not sharded:
+            world == 1:
         try:
             offload = measure_offload(prepare("long256k"), args, device, args.selection)
         except (RuntimeError, MemoryError) as e:   # e.g. the host cannot pin 34 GB
