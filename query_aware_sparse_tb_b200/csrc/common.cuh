@@ -142,8 +142,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 // ----------------------------------------------------------------- TMA ----
 
-// 2-D tiled bulk tensor load into this CTA's shared memory, completion counted
-// on `bar` in bytes.  No cluster multicast.
+// 2-D tiled bulk tensor load into this CTA's own shared memory only,
+// completion counted on `bar` in bytes.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int x, int y) {
     asm volatile(
@@ -151,14 +151,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%3, %4}], [%2];\n" ::"r"(dst),
         "l"(map), "r"(bar), "r"(x), "r"(y)
         : "memory");
-}
-// 1-D bulk copy of `bytes` from global memory into this CTA's shared memory
-// by the TMA engine, completion counted in bytes on `bar`.  Both addresses
-// 16-byte aligned, `bytes` a multiple of 16.  No cluster multicast.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
