@@ -54,7 +54,7 @@ class Run:
     that rank owns under KV-head sharding, sliced from the same seeded data."""
 
     def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head",
-                 shard: tuple[int, int] | None = None, offload: bool = False):
+                 shard: tuple[int, int] | None = None, offload: bool = False, balance: bool = True):
         self.w = w
         self.device = device
         self.steps = steps or w.steps
@@ -101,7 +101,7 @@ class Run:
         # the bench's streams run only libtb's kernels, the K/V append of the
         # e2e loop and copies, so every attention launch may prefetch its rows
         self.dec = cls(self.shape, list(self.K), list(self.V), self.Wk, self.mlp, self.ctx0, self.steps, device,
-                       selection=selection, prefetch_kv=True)
+                       selection=selection, prefetch_kv=True, balance=balance)
         self.out = torch.zeros(nL, w.batch, self.Hq, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):
@@ -668,7 +668,7 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
     each replayed as one CUDA graph; returns the figures the JSON line needs.
     With shard=(rank, world) this rank runs only its KV heads of the one
     workload (strong scaling: the job's tokens are the workload's tokens)."""
-    run = Run(w, device, steps=args.decode_steps, selection=selection, shard=shard)
+    run = Run(w, device, steps=args.decode_steps, selection=selection, shard=shard, balance=not args.no_balance)
     copies = 1 if shard else world          # independent replicas count every rank's tokens
     run.dec.prefill()
     torch.cuda.synchronize()
@@ -821,6 +821,8 @@ def main():
                     help="skip the CPU-offloaded KV cache on long256k (per-token latency against dense), which the "
                          "default single-GPU run times after the headline workload")
     ap.add_argument("--offload-only", action="store_true", help="time only the CPU-offloaded workload")
+    ap.add_argument("--no-balance", action="store_true",
+                    help="attention slices at equal shares of the length instead of the kept rows (no tb_attn_plan)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "kv_heads"],
                     help="with N > 1 ranks: replicas (each rank decodes its own seeded replica; weak scaling) or "
                          "kv_heads (the ranks split one workload's KV heads; strong scaling)")

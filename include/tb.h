@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define TB_ABI_VERSION 9
+#define TB_ABI_VERSION 10
 
 typedef uint16_t tb_bf16;
 
@@ -381,6 +381,39 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
                                 int32_t window, const uint32_t *sel_bits, float scale,
                                 float *out, void *ws, size_t ws_bytes, void *stream);
 
+/* ---- balanced attention slices -------------------------------------------- */
+/* The attention splits each (sequence, KV head) over several CTAs.  By
+ * default the slices are equal shares of the length T; the kept rows are not
+ * spread evenly over the positions, so some slices hold more rows than
+ * others and the launch lasts as long as the fullest.  A plan cuts the slices
+ * at equal shares of the kept rows instead.  No counterpart on the pages: a
+ * scheduling aid.
+ *
+ * tb_attn_plan counts, for each (b, KV head g), the kept rows of every
+ * 32-position word below T = ctx_len[b] (sink ∪ window ∪ the positions
+ * selected for any of the group's 4 query heads in sel_bits, as defined
+ * under tb_sparse_decode_attn) and writes the word index at which each slice
+ * opens:
+ *   plan  [batch][Hkv][TB_ATTN_PLAN_STRIDE] int32 (device, 4-byte aligned):
+ *         plan[b][g][s] for s = 0 .. splits, where splits is the attention's
+ *         CTA count per (b, g) for these dims; entries past it are not written
+ * The selection of an interval stays valid for its steps, and so does its
+ * plan (the window's few moving rows only shift the balance slightly): run
+ * tb_attn_plan once after each selection.
+ *
+ * tb_sparse_decode_attn_planned is tb_sparse_decode_attn with the slices of
+ * `plan` (from tb_attn_plan with the same dims).  The result is the same up to
+ * the order of the fp32 additions that merge the slices.  Under
+ * TB_ATTN_PREFETCH_KV the plan is read before the preceding kernel has
+ * completed, like sel_bits. */
+#define TB_ATTN_PLAN_STRIDE 65
+tb_status tb_attn_plan(const tb_dims *dims, const uint32_t *sel_bits, const int32_t *ctx_len, int32_t sink,
+                       int32_t window, int32_t *plan, void *ws, size_t ws_bytes, void *stream);
+tb_status tb_sparse_decode_attn_planned(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K,
+                                        const tb_bf16 *V, const int32_t *ctx_len, int32_t sink,
+                                        int32_t window, const uint32_t *sel_bits, const int32_t *plan,
+                                        float scale, float *out, void *ws, size_t ws_bytes, void *stream);
+
 /* ---- attention launch mode ------------------------------------------------ */
 /* How the attention entry points (tb_sparse_decode_attn, tb_decode_attn,
  * tb_sparse_decode_attn_noalloc) order their reads against the kernel that
@@ -390,14 +423,15 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
  *
  *   TB_ATTN_WAIT_ALL     (default) nothing in global memory is touched before
  *                        the preceding kernel has completed.
- *   TB_ATTN_PREFETCH_KV  ctx_len, sel_bits and the K and V rows below
+ *   TB_ATTN_PREFETCH_KV  ctx_len, sel_bits (and the plan, for the planned
+ *                        entry point) and the K and V rows below
  *                        ctx_len[b] - 1 are read (and the first tiles of K/V
  *                        streamed into shared memory) as soon as the kernel
  *                        is resident; Q, row ctx_len[b] - 1, out and the
  *                        workspace only after the preceding kernel has
  *                        completed.  Valid only when no kernel that may still
- *                        be running writes ctx_len, sel_bits or those K/V
- *                        rows: the kernel that immediately precedes the call
+ *                        be running writes ctx_len, sel_bits, the plan or
+ *                        those K/V rows: the kernel that immediately precedes the call
  *                        in its stream (a decode loop's Q/K/V projection
  *                        writes Q and row ctx_len[b] - 1 only, which is
  *                        allowed), and, if that kernel lets its own

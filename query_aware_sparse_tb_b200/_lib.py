@@ -15,12 +15,13 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtb.so")
 
-TB_ABI_VERSION = 9
+TB_ABI_VERSION = 10
 TB_OK, TB_ERR_INVALID_ARG, TB_ERR_UNSUPPORTED, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE_FLAG = range(6)
 TB_FLAG_CTX_RANGE, TB_FLAG_TIMEOUT, TB_FLAG_IDX_OVERFLOW, TB_FLAG_BAD_CACHE = 0x1, 0x2, 0x4, 0x8
 TB_GROUP_REDUCE = {"max": 0, "sum": 1}
 TB_ATTN_WAIT_ALL, TB_ATTN_PREFETCH_KV = 0, 1
 TB_SELECT_AUTO, TB_SELECT_MULTI_KERNEL, TB_SELECT_CLUSTER = 0, 1, 2
+TB_ATTN_PLAN_STRIDE = 65
 
 EXPORTS = [
     "tb_abi_version", "tb_status_str", "tb_last_error",
@@ -32,7 +33,7 @@ EXPORTS = [
     "tb_select_export_candidates", "tb_select_merge_candidates", "tb_sparse_decode_attn_partial", "tb_attn_combine",
     "tb_sparse_decode_attn", "tb_decode_attn", "tb_sparse_decode_attn_noalloc", "tb_kv_append",
     "tb_selftest_bounded_wait", "tb_attn_set_launch_mode", "tb_attn_launch_mode",
-    "tb_select_set_algorithm", "tb_select_algorithm",
+    "tb_select_set_algorithm", "tb_select_algorithm", "tb_attn_plan", "tb_sparse_decode_attn_planned",
 ]
 
 
@@ -85,6 +86,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tb_sparse_decode_attn_partial": ([D, P, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_attn_combine": ([P, i32, i32, i32, i32, P, P], ctypes.c_int),
         "tb_sparse_decode_attn": ([D, P, P, P, P, i32, i32, P, f32, P, P, sz, P], ctypes.c_int),
+        "tb_sparse_decode_attn_planned": ([D, P, P, P, P, i32, i32, P, P, f32, P, P, sz, P], ctypes.c_int),
+        "tb_attn_plan": ([D, P, P, i32, i32, P, P, sz, P], ctypes.c_int),
         "tb_decode_attn": ([D, P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "tb_sparse_decode_attn_noalloc": ([D, P, P, P, P, i32, i32, P, f32, P, P], ctypes.c_int),
         "tb_kv_append": ([D, i32, P, P, P, P, sz, P], ctypes.c_int),
@@ -266,6 +269,21 @@ def sparse_decode_attn(d: TbDims, Q, K, V, ctx_len, sink: int, window: int, sel_
     _check(load().tb_sparse_decode_attn(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), sink,
                                         window, _ptr(sel_bits), float(scale), _ptr(out), _ptr(ws), _bytes(ws),
                                         _stream(stream)))
+
+
+def attn_plan(d: TbDims, sel_bits, ctx_len, sink: int, window: int, plan, ws, stream=None):
+    """tb_attn_plan: slice cuts at equal shares of the kept rows,
+    plan [batch][Hkv][TB_ATTN_PLAN_STRIDE] int32."""
+    _check(load().tb_attn_plan(ctypes.byref(d), _ptr(sel_bits), _ptr(ctx_len), sink, window, _ptr(plan), _ptr(ws),
+                               _bytes(ws), _stream(stream)))
+
+
+def sparse_decode_attn_planned(d: TbDims, Q, K, V, ctx_len, sink: int, window: int, sel_bits, plan, scale: float,
+                               out, ws, stream=None):
+    """tb_sparse_decode_attn over the slices of a tb_attn_plan."""
+    _check(load().tb_sparse_decode_attn_planned(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(ctx_len), sink,
+                                                window, _ptr(sel_bits), _ptr(plan), float(scale), _ptr(out), _ptr(ws),
+                                                _bytes(ws), _stream(stream)))
 
 
 def sparse_decode_attn_noalloc(d: TbDims, Q, K, V, ctx_len, sink: int, window: int, sel_bits, scale: float,

@@ -449,6 +449,35 @@ tb_status tb_sparse_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_
                        __func__);
 }
 
+tb_status tb_sparse_decode_attn_planned(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
+                                        const int32_t *ctx_len, int32_t sink, int32_t window,
+                                        const uint32_t *sel_bits, const int32_t *plan, float scale, float *out,
+                                        void *ws, size_t ws_bytes, void *stream) {
+    tb_status s = check_attn_args(__func__, dims, Q, K, V, ctx_len, scale, out, true, sel_bits, sink, window);
+    if (s != TB_OK) return s;
+    TB_CHECK_PTR4(plan);
+    if ((s = check_ws(ws, ws_bytes, attn_ws_bytes(*dims), __func__)) != TB_OK) return s;
+    return cuda_status(launch_attn(*dims, Q, K, V, ctx_len, sink, window, sel_bits, true, scale, out, ws,
+                                   (cudaStream_t)stream, nullptr, plan),
+                       __func__);
+}
+
+tb_status tb_attn_plan(const tb_dims *dims, const uint32_t *sel_bits, const int32_t *ctx_len, int32_t sink,
+                       int32_t window, int32_t *plan, void *ws, size_t ws_bytes, void *stream) {
+    tb_status s;
+    if ((s = check_dims(dims, false, __func__)) != TB_OK) return s;
+    if (dims->ctx_cap > kMaxCtxAttn)
+        return fail(TB_ERR_UNSUPPORTED, "%s: ctx_cap %d above %d", __func__, dims->ctx_cap, kMaxCtxAttn);
+    TB_CHECK_PTR4(sel_bits);
+    TB_CHECK_PTR4(ctx_len);
+    TB_CHECK_PTR4(plan);
+    if (sink < 0 || window < 1) return fail(TB_ERR_INVALID_ARG, "%s: need sink >= 0 and window >= 1", __func__);
+    if ((s = check_ws(ws, ws_bytes, kWsHeaderBytes, __func__)) != TB_OK) return s;
+    return cuda_status(launch_attn_plan(*dims, sel_bits, ctx_len, sink, window, plan,
+                                        static_cast<uint32_t *>(ws), (cudaStream_t)stream),
+                       __func__);
+}
+
 tb_status tb_decode_attn(const tb_dims *dims, const tb_bf16 *Q, const tb_bf16 *K, const tb_bf16 *V,
                          const int32_t *ctx_len, float scale, float *out, void *ws, size_t ws_bytes,
                          void *stream) {

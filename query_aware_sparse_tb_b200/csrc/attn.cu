@@ -49,6 +49,8 @@ constexpr int kRows = 128;         // KV rows per tile (M of the S^T product)
 constexpr int kStages = 3;
 constexpr int kSub = 4096;         // positions per row list (sparse)
 constexpr int kMaxSplits = 64;     // partial states merged per (sequence, KV head)
+static_assert(TB_ATTN_PLAN_STRIDE == kMaxSplits + 1, "a plan row holds every cut");
+constexpr int kPlanThreads = 1024;
 constexpr int kN = 16;             // N of both products (padded)
 constexpr int kRoleThreads = 128;  // threads of the softmax role and of the load role
 constexpr int kThreads = 2 * kRoleThreads + 64;  // + an S-issue warp and a PV-issue warp
@@ -129,7 +131,7 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
             const uint32_t *__restrict__ sel_bits, int Hq, int Hkv, int Tcap, int W, int sink,
             int window, float qscale, int splits, float *__restrict__ part,
             uint32_t *__restrict__ counters, float *__restrict__ out, uint32_t *__restrict__ flags,
-            int early_trigger, int prefetch, float *__restrict__ part_out) {
+            int early_trigger, int prefetch, float *__restrict__ part_out, const int32_t *__restrict__ plan) {
     constexpr int CPR = D / 8;      // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;   // rows per warp-wide copy instruction
     constexpr int kKSteps = D / 16; // MMA K steps of S^T
@@ -211,17 +213,28 @@ attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
     const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
     const int hi_c = T - window;  // candidates are [sink, hi_c)
 
-    // This CTA's slice [p_begin, p_end) of (b, g): equal shares of the length,
-    // cut at whole 32-position selection words (slice s opens at the word that
-    // holds position s * T / splits).  Sparse and dense use the same slices, so
-    // with every candidate selected they do identical arithmetic.  (Cutting
-    // the sparse slices at equal kept rows instead, counted from the group's
-    // selection words, balanced the tiles but cost more at the start than it
-    // saved: 42.3 against 38.7 us per 64K launch.)
-    const int p_begin = (int)(((long long)split * T / splits) >> 5) << 5;
-    const int p_end = split + 1 == splits
-                          ? T
-                          : max(p_begin, min((int)(((long long)(split + 1) * T / splits) >> 5) << 5, T));
+    // This CTA's slice [p_begin, p_end) of (b, g), cut at whole 32-position
+    // selection words.  Without a plan: equal shares of the length (slice s
+    // opens at the word that holds position s * T / splits); sparse and dense
+    // use the same slices, so with every candidate selected they do identical
+    // arithmetic.  With a plan (tb_attn_plan: word indices at which equal
+    // shares of the kept rows begin, counted once per prediction): its cuts,
+    // clamped to [0, T), the first slice opening at 0 and the last closing at
+    // T.  (Counting the kept rows here, at every launch, cost more at the
+    // start than the balance saved: 42.3 against 38.7 us per 64K launch.)
+    int p_begin, p_end;
+    if (plan == nullptr) {
+        p_begin = (int)(((long long)split * T / splits) >> 5) << 5;
+        p_end = split + 1 == splits ? T
+                                    : max(p_begin, min((int)(((long long)(split + 1) * T / splits) >> 5) << 5, T));
+    } else {
+        // (a cut at or past T leaves an empty slice [T, T); every other cut is
+        // a whole word below T, and neighbouring slices share their cut)
+        const int32_t *pl = plan + (size_t)(b * Hkv + g) * TB_ATTN_PLAN_STRIDE;
+        const int nw = (T + 31) >> 5;
+        p_begin = split == 0 ? 0 : min(min(max(pl[split], 0), nw) << 5, T);
+        p_end = split + 1 == splits ? T : max(p_begin, min(min(max(pl[split + 1], 0), nw) << 5, T));
+    }
     const int ns = splits;  // every CTA writes a state, empty slices with M = -inf
 
     // sparse: load warp thread pt owns word pt (32 positions) of a sub-chunk;
@@ -709,7 +722,7 @@ combine_kernel(const float *__restrict__ parts, int n_parts, int rows, float *__
 template <int D, bool SPARSE>
 cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                      const int32_t *ctx_len, int32_t sink, int32_t window, const uint32_t *sel_bits,
-                     float scale, float *out, void *ws, cudaStream_t st, float *part_out) {
+                     float scale, float *out, void *ws, cudaStream_t st, float *part_out, const int32_t *plan) {
     static std::atomic<int> smem_set[kMaxDevices];
     cudaError_t e = ensure_dynamic_smem((const void *)attn_kernel<D, SPARSE>, Smem::kBytes, smem_set);
     if (e != cudaSuccess) return e;
@@ -727,7 +740,85 @@ cudaError_t launch_t(const tb_dims &d, const uint16_t *Q, const uint16_t *K, con
     const int prefetch = attn_launch_mode() == TB_ATTN_PREFETCH_KV ? 1 : 0;
     return launch_pdl(attn_kernel<D, SPARSE>, dim3(splits, d.n_kv_heads, d.batch), dim3(kThreads), Smem::kBytes,
                       st, Q, K, V, ctx_len, sel_bits, d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, qscale,
-                      splits, part, counters, out, flags, early, prefetch, part_out);
+                      splits, part, counters, out, flags, early, prefetch, part_out, plan);
+}
+
+// The plan of tb_attn_plan: one CTA per (b, g).  Word w of (b, g) weighs the
+// kept rows it holds (the sink, the window and the group's selected positions,
+// all below T); slice s of `splits` opens at the first word whose preceding
+// weight reaches s/splits of the total.
+__global__ void __launch_bounds__(kPlanThreads)
+attn_plan_kernel(const uint32_t *__restrict__ sel_bits, const int32_t *__restrict__ ctx_len, int Hq, int Hkv,
+                 int Tcap, int W, int sink, int window, int splits, int32_t *__restrict__ plan,
+                 uint32_t *__restrict__ flags) {
+    __shared__ int scratch[kPlanThreads / 32 + 1];
+    __shared__ int s_total;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = blockIdx.x, b = blockIdx.y;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int T = clamp_ctx(ctx_len[b], Tcap, flags, false);
+    const int nw = (T + 31) >> 5;
+    const uint32_t *sbits = sel_bits + ((size_t)b * Hq + (size_t)g * kGroup) * W;
+    const int lo_w = min(sink, T), hi_w = max(sink, T - window);
+    auto weight = [&](int w) {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) m |= sbits[(size_t)h * W + w];
+        const int base = w << 5;
+        auto range = [&](int a, int e) -> uint32_t {  // bits of [a, e) in word w
+            const int s0 = max(a - base, 0), s1 = min(e - base, 32);
+            if (s1 <= s0) return 0u;
+            return (s1 == 32 ? 0xffffffffu : ((1u << s1) - 1u)) & ~((1u << s0) - 1u);
+        };
+        m |= range(0, lo_w) | range(hi_w, T);
+        m &= range(0, T);
+        return __popc(m);
+    };
+    // contiguous runs of words per thread, an exclusive scan over the threads
+    const int per = (nw + kPlanThreads - 1) / kPlanThreads;
+    const int w0 = min(tid * per, nw), w1 = min(w0 + per, nw);
+    int mine = 0;
+    for (int w = w0; w < w1; ++w) mine += weight(w);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < kPlanThreads / 32 ? scratch[lane] : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += t;
+        }
+        if (lane < kPlanThreads / 32) scratch[lane] = x - v;
+        if (lane == kPlanThreads / 32 - 1) s_total = x;
+    }
+    __syncthreads();
+    const long long total = s_total;
+    int32_t *out = plan + (size_t)(b * Hkv + g) * TB_ATTN_PLAN_STRIDE;
+    // cut s (0 < s < splits) falls in the word where the running weight
+    // crosses s * total / splits; the slice opens after that word
+    int before = scratch[warp] + incl - mine;
+    for (int w = w0; w < w1; ++w) {
+        const int c = weight(w);
+        for (int s = 1; s < splits; ++s) {
+            const long long share = (long long)s * total;  // compared as weight * splits
+            if (share > (long long)before * splits && share <= (long long)(before + c) * splits) out[s] = w + 1;
+        }
+        before += c;
+    }
+    if (tid == 0) {
+        out[0] = 0;
+        out[splits] = nw;
+        if (total == 0)
+            for (int s = 1; s < splits; ++s) out[s] = 0;
+    }
 }
 
 }  // namespace
@@ -761,14 +852,24 @@ size_t attn_ws_bytes(const tb_dims &d) {
 cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *ctx_len, int32_t sink, int32_t window,
                         const uint32_t *sel_bits, bool sparse, float scale, float *out, void *ws,
-                        cudaStream_t st, float *part_out) {
+                        cudaStream_t st, float *part_out, const int32_t *plan) {
     if (d.head_dim == 128) {
-        return sparse ? launch_t<128, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out)
+        return sparse ? launch_t<128, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out,
+                                            plan)
                       : launch_t<128, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st,
-                                             part_out);
+                                             part_out, nullptr);
     }
-    return sparse ? launch_t<64, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out)
-                  : launch_t<64, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out);
+    return sparse ? launch_t<64, true>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out,
+                                       plan)
+                  : launch_t<64, false>(d, Q, K, V, ctx_len, sink, window, sel_bits, scale, out, ws, st, part_out,
+                                        nullptr);
+}
+
+cudaError_t launch_attn_plan(const tb_dims &d, const uint32_t *sel_bits, const int32_t *ctx_len, int32_t sink,
+                             int32_t window, int32_t *plan, uint32_t *flags, cudaStream_t st) {
+    const int W = (d.ctx_cap + 31) / 32;
+    return launch_pdl(attn_plan_kernel, dim3(d.n_kv_heads, d.batch), dim3(kPlanThreads), 0, st, sel_bits, ctx_len,
+                      d.n_q_heads, d.n_kv_heads, d.ctx_cap, W, sink, window, attn_splits(d), plan, flags);
 }
 
 cudaError_t launch_combine(const float *parts, int32_t n_parts, int32_t rows, int32_t head_dim, float *out,

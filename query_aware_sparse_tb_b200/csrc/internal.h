@@ -17,7 +17,9 @@ int attn_splits(const tb_dims &d);
 cudaError_t launch_attn(const tb_dims &d, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *ctx_len, int32_t sink, int32_t window,
                         const uint32_t *sel_bits, bool sparse, float scale, float *out, void *ws,
-                        cudaStream_t st, float *part_out = nullptr);
+                        cudaStream_t st, float *part_out = nullptr, const int32_t *plan = nullptr);
+cudaError_t launch_attn_plan(const tb_dims &d, const uint32_t *sel_bits, const int32_t *ctx_len, int32_t sink,
+                             int32_t window, int32_t *plan, uint32_t *flags, cudaStream_t st);
 cudaError_t launch_combine(const float *parts, int32_t n_parts, int32_t rows, int32_t head_dim, float *out,
                            cudaStream_t st);
 

@@ -273,10 +273,14 @@ class SparseDecoder:
     SELECTIONS = ("head", "group_max", "group_sum", "inclusive")
 
     def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda",
-                 selection: str = "head", prefetch_kv: bool = False):
+                 selection: str = "head", prefetch_kv: bool = False, balance: bool = True):
         if selection not in self.SELECTIONS:
             raise ValueError(f"selection must be one of {self.SELECTIONS}")
         self.selection = selection
+        # balance: after each selection, tb_attn_plan cuts the attention's
+        # slices at equal shares of the kept rows, and the attention launches
+        # of the interval use them (tb_sparse_decode_attn_planned)
+        self.balance = balance
         # TB_ATTN_PREFETCH_KV for the attention launches whose preceding
         # kernel writes none of the lengths, selection words and K/V rows
         # below T-1.  Inside a step that is every attention launch except the
@@ -300,6 +304,8 @@ class SparseDecoder:
         self.idx = [torch.zeros(B, Hq, s.idx_cap, dtype=torch.int32, device=device) for _ in range(s.n_layers)]
         self.cnt = [torch.zeros(B, Hq, dtype=torch.int32, device=device) for _ in range(s.n_layers)]
         self.bits = [torch.zeros(B, Hq, s.words, dtype=torch.int32, device=device) for _ in range(s.n_layers)]
+        self.plan = [torch.zeros(B, Hkv, L.TB_ATTN_PLAN_STRIDE, dtype=torch.int32, device=device)
+                     for _ in range(s.n_layers)] if balance else None
         self.ws_sel = L.workspace(L.score_select_workspace_bytes(self.dims), device)
         self.ws_attn = L.workspace(L.attn_workspace_bytes(self.dims), device)
         self.ws_proj = L.workspace(L.project_keys_workspace_bytes(), device)
@@ -355,13 +361,21 @@ class SparseDecoder:
             L.score_select_group(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window,
                                  s.budget, s.nbr, self.selection[len("group_"):], self.idx[layer],
                                  self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+        if self.balance:
+            L.attn_plan(self.dims, self.bits[layer], self.ctx[step], s.sink, s.window, self.plan[layer], self.ws_attn,
+                        stream)
 
     def attend(self, step: int, layer: int, Q, out, stream=None, prefetch: bool = False):
         s = self.shape
         L.attn_set_launch_mode(L.TB_ATTN_PREFETCH_KV if prefetch else L.TB_ATTN_WAIT_ALL)
         try:
-            L.sparse_decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], s.sink, s.window,
-                                 self.bits[layer], self.scale, out, self.ws_attn, stream)
+            if self.balance:
+                L.sparse_decode_attn_planned(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], s.sink,
+                                             s.window, self.bits[layer], self.plan[layer], self.scale, out,
+                                             self.ws_attn, stream)
+            else:
+                L.sparse_decode_attn(self.dims, Q, self.K[layer], self.V[layer], self.ctx[step], s.sink, s.window,
+                                     self.bits[layer], self.scale, out, self.ws_attn, stream)
         finally:
             L.attn_set_launch_mode(L.TB_ATTN_WAIT_ALL)
 
