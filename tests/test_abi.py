@@ -114,6 +114,26 @@ def test_attention_rejects_bad_arguments(lib):
     assert st == _lib.TB_ERR_INVALID_ARG
 
 
+def test_plan_and_planned_attention_reject_bad_arguments(lib):
+    d = _d()
+    ws_bytes = lib.tb_attn_workspace_bytes(ctypes.byref(d))
+    plan = lambda **kw: lib.tb_attn_plan(ctypes.byref(kw.get("d", d)), kw.get("bits", FAKE), kw.get("ctx", FAKE),  # noqa: E731
+                                         kw.get("sink", 16), kw.get("window", 64), kw.get("plan", FAKE),
+                                         kw.get("ws", FAKE), kw.get("ws_bytes", 256), None)
+    assert plan(bits=0) == _lib.TB_ERR_INVALID_ARG
+    assert plan(plan=FAKE + 2) == _lib.TB_ERR_INVALID_ARG  # int32 entries: 4-byte alignment
+    assert plan(window=0) == _lib.TB_ERR_INVALID_ARG and b"window" in lib.tb_last_error()
+    assert plan(sink=-1) == _lib.TB_ERR_INVALID_ARG
+    assert plan(ws_bytes=255) == _lib.TB_ERR_WORKSPACE
+    assert plan(d=_d(head_dim=96)) == _lib.TB_ERR_UNSUPPORTED
+    st = lib.tb_sparse_decode_attn_planned(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16, 64, FAKE, 0, 0.088, FAKE,
+                                           FAKE, ws_bytes, None)
+    assert st == _lib.TB_ERR_INVALID_ARG and b"plan" in lib.tb_last_error()
+    st = lib.tb_sparse_decode_attn_planned(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16, 0, FAKE, FAKE, 0.088,
+                                           FAKE, FAKE, ws_bytes, None)
+    assert st == _lib.TB_ERR_INVALID_ARG and b"window" in lib.tb_last_error()
+
+
 def test_select_rejects_bad_arguments(lib):
     d = _d()
     wsb = lib.tb_score_select_workspace_bytes(ctypes.byref(d))
