@@ -815,7 +815,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip the extra workloads (batch16, long256k) timed after the headline one")
+                    help="skip the extra workloads (batch16, long256k, llama64k at interval 1) timed after the "
+                         "headline one")
     ap.add_argument("--extra-steps", type=int, default=3, help="timed bench steps of each extra workload")
     ap.add_argument("--no-offload", action="store_true",
                     help="skip the CPU-offloaded KV cache on long256k (per-token latency against dense), which the "
@@ -871,6 +872,12 @@ def main():
             wx = prepare(name)
             extras[name] = summary(wx, measure(wx, args, device, dist_on, world, False, args.extra_steps,
                                                max(3, args.warmup), args.selection, shard), measured_peaks()[0])
+        # the headline workload with a prediction (and selection) at every
+        # decode step: what the interval amortises
+        wx = prepare("llama64k").scaled(interval=1)
+        extras["llama64k_interval1"] = summary(wx, measure(wx, args, device, dist_on, world, False, args.extra_steps,
+                                                           max(3, args.warmup), args.selection, shard),
+                                               measured_peaks()[0])
 
     offload = None
     # (a per-token latency on one GPU: not run under torchrun, where every

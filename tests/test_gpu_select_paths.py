@@ -25,6 +25,15 @@ def _inputs(seed, batch, hkv, dp, cap, kind):
     elif kind == "integer":  # small integers: many exactly equal scores
         Kp = torch.randint(-2, 3, (batch, hkv, cap, dp), generator=g).to(torch.bfloat16)
         qp = torch.randint(-1, 2, (batch, hq, dp), generator=g).float()
+    elif kind == "coarse":  # integer scores over a few hundred values: ties inside the B-th key's bin
+        Kp = torch.randint(-8, 9, (batch, hkv, cap, dp), generator=g).to(torch.bfloat16)
+        qp = torch.randint(-3, 4, (batch, hq, dp), generator=g).float()
+    elif kind == "outlier":  # a few huge scores squeeze the rest into the lowest score bins
+        Kp = torch.randn(batch, hkv, cap, dp, generator=g)
+        rows = torch.randint(0, cap, (batch, hkv, 3), generator=g)
+        Kp.scatter_(2, rows[..., None].expand(-1, -1, -1, dp), 3e4)
+        Kp = Kp.to(torch.bfloat16)
+        qp = torch.randn(batch, hq, dp, generator=g).abs()
     else:  # all scores zero: every candidate ties
         Kp = torch.zeros(batch, hkv, cap, dp, dtype=torch.bfloat16)
         qp = torch.randn(batch, hq, dp, generator=g)
@@ -67,12 +76,14 @@ CASES = {
 
 
 @pytest.mark.parametrize("reduce", [None, "max", "sum"])
-@pytest.mark.parametrize("kind", ["normal", "integer", "zeros"])
+@pytest.mark.parametrize("kind", ["normal", "integer", "zeros", "coarse", "outlier"])
 @pytest.mark.parametrize("case", list(CASES))
 def test_cluster_and_multi_kernel_routes_agree_bit_for_bit(case, kind, reduce):
     batch, hkv, dp, cap, ctx, sink, window, budget, nbr = CASES[case]
     if case in ("llama64k_layer", "batch16_ragged") and kind == "zeros" and reduce is not None:
         pytest.skip("all-ties at full size: covered per head")
+    if case == "batch16_ragged" and kind in ("coarse", "outlier") and reduce == "sum":
+        pytest.skip("covered by the per-head and max cases")
     if ctx is None:
         ctx = torch.randint(16384, 32769, (batch,), generator=torch.Generator().manual_seed(5)).tolist()
     dm = tb.dims(batch=batch, n_q_heads=4 * hkv, n_kv_heads=hkv, head_dim=128, d_proj=dp, ctx_cap=cap)
@@ -138,3 +149,41 @@ def test_graph_kernel_count_follows_the_route():
         torch.cuda.synchronize()
         counts[algo] = g.libtb_kernels
     assert counts == {_lib.TB_SELECT_MULTI_KERNEL: 3, _lib.TB_SELECT_CLUSTER: 2}
+
+
+def test_cluster_route_on_a_reused_workspace():
+    """The cluster route keeps each score row's key range in its workspace
+    between the scoring and the selection kernel and clears it again; calls
+    that reuse one workspace, with inputs of different ranges and with the
+    other route in between, must each give the multi-kernel route's result."""
+    batch, hkv, dp, cap, ctx, sink, window, budget, nbr = CASES["llama64k_layer"]
+    dm = tb.dims(batch=batch, n_q_heads=4 * hkv, n_kv_heads=hkv, head_dim=128, d_proj=dp, ctx_cap=cap)
+    hq, W = dm.n_q_heads, (cap + 31) // 32
+    icap = min((2 * nbr + 1) * budget, cap)
+    ws = tb.workspace(tb.score_select_workspace_bytes(dm))
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device=DEV)
+
+    def call(algo, Kp, qp):
+        idx = torch.full((batch, hq, icap), -7, dtype=torch.int32, device=DEV)
+        cnt = torch.full((batch, hq), -7, dtype=torch.int32, device=DEV)
+        bits = torch.full((batch, hq, W), -1, dtype=torch.int32, device=DEV)
+        _lib.select_set_algorithm(algo)
+        try:
+            tb.score_select(dm, qp, hq * dp, Kp, ctx_t, sink, window, budget, nbr, idx, cnt, bits, ws)
+        finally:
+            _lib.select_set_algorithm(_lib.TB_SELECT_AUTO)
+        torch.cuda.synchronize()
+        return idx.cpu().numpy(), cnt.cpu().numpy(), bits.cpu().numpy()
+
+    order = [("normal", _lib.TB_SELECT_CLUSTER), ("outlier", _lib.TB_SELECT_CLUSTER),
+             ("coarse", _lib.TB_SELECT_MULTI_KERNEL), ("normal", _lib.TB_SELECT_CLUSTER),
+             ("coarse", _lib.TB_SELECT_CLUSTER)]
+    for i, (kind, algo) in enumerate(order):
+        Kp, qp = _inputs(100 + i, batch, hkv, dp, cap, kind)
+        if kind == "normal":
+            qp = qp * (10.0 ** (i - 2))  # another score range on each call
+        got = call(algo, Kp, qp)
+        fresh = _run(_lib.TB_SELECT_MULTI_KERNEL, dm, Kp, qp, ctx, sink, window, budget, nbr, None)
+        for name, a, b in zip(("idx", "count", "sel_bits"), fresh[:3], got):
+            assert np.array_equal(a, b), f"call {i} ({kind}): {name} differs from a fresh multi-kernel call"
+    assert tb.workspace_check(ws) == 0
