@@ -15,7 +15,9 @@
 //                   own and scores each row once for the 4 query heads of the
 //                   group (BlockScorer), writes the
 //                   order-preserving uint32 image of every score, and builds
-//                   a histogram of its top 11 bits per query head.  The last
+//                   a histogram of its top 11 bits per query head (without
+//                   the histogram: the smallest and largest key of each score
+//                   row, for the cluster kernel's value route).  The last
 //                   CTA of each (b, KV head) (atomic ticket, no waiting) finds
 //                   the bin that holds the B-th largest key.
 //   2. mark_collect same grid: keys above that bin become bits of the Top

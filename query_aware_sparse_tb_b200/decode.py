@@ -279,8 +279,10 @@ class SparseDecoder:
         self.selection = selection
         # balance: after each selection, tb_attn_plan cuts the attention's
         # slices at equal shares of the kept rows, and the attention launches
-        # of the interval use them (tb_sparse_decode_attn_planned)
-        self.balance = balance
+        # of the interval use them (tb_sparse_decode_attn_planned).  A plan
+        # costs about what one launch saves, so it pays only when several
+        # launches share it: not at an interval of 1.
+        self.balance = balance and shape.interval > 1
         # TB_ATTN_PREFETCH_KV for the attention launches whose preceding
         # kernel writes none of the lengths, selection words and K/V rows
         # below T-1.  Inside a step that is every attention launch except the
