@@ -15,9 +15,7 @@
 //                   own and scores each row once for the 4 query heads of the
 //                   group (BlockScorer), writes the
 //                   order-preserving uint32 image of every score, and builds
-//                   a histogram of its top 11 bits per query head (without
-//                   the histogram: the smallest and largest key of each score
-//                   row, for the cluster kernel's value route).  The last
+//                   a histogram of its top 11 bits per query head.  The last
 //                   CTA of each (b, KV head) (atomic ticket, no waiting) finds
 //                   the bin that holds the B-th largest key.
 //   2. mark_collect same grid: keys above that bin become bits of the Top
@@ -79,13 +77,6 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
     __syncthreads();
 
     const size_t slab = ((size_t)b * Hkv + g) * (size_t)Tcap;
-    // the smallest and largest key this thread writes, per score row
-    uint32_t kmin[NH], kmax[NH];
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-        kmin[h] = 0xffffffffu;
-        kmax[h] = 0u;
-    }
     if (hi > lo && p0 < hi && p0 + chunk > lo) {
         // the chunk's 32-row blocks that overlap C, dealt to the warps in
         // turn; each warp streams its blocks through a ring of its own
@@ -115,8 +106,6 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                     if (valid) {
                         ws.keys[((size_t)b * Hq + g * kGroup + h) * Tcap + p] = key;
                         if constexpr (HIST) atomicAdd(&hist[h][key >> 21], 1u);
-                        kmin[h] = min(kmin[h], key);
-                        kmax[h] = max(kmax[h], key);
                     }
                 }
             } else {
@@ -127,8 +116,6 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
                 if (valid) {
                     ws.keys[((size_t)b * Hq + g * kGroup) * Tcap + p] = key;
                     if constexpr (HIST) atomicAdd(&hist[0][key >> 21], 1u);
-                    kmin[0] = min(kmin[0], key);
-                    kmax[0] = max(kmax[0], key);
                 }
             }
         };
@@ -150,22 +137,7 @@ score_hist_kernel(const float *__restrict__ qp, int64_t qp_stride, const uint16_
             if (i + 1 < nb) emit(i + 1, sb);
         }
     }
-    if constexpr (!HIST) {
-        // the range of the row's keys for the cluster kernel: words 0 and 1
-        // of the row's histogram (unused on this route) take the complement
-        // of the smallest key and the largest key by atomic max, so a zeroed
-        // workspace starts them empty; the cluster kernel zeroes them again
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            const uint32_t mn = __reduce_min_sync(kFull, kmin[h]), mx = __reduce_max_sync(kFull, kmax[h]);
-            if (lane == 0 && mx != 0u) {
-                uint32_t *rng = ws.hist + ((size_t)b * Hq + g * kGroup + h) * kBins1;
-                atomicMax(rng, ~mn);
-                atomicMax(rng + 1, mx);
-            }
-        }
-        return;
-    }
+    if constexpr (!HIST) return;
     __syncthreads();
     for (int i = tid; i < NH * kBins1; i += kThreads) {
         const uint32_t v = (&hist[0][0])[i];

@@ -15,48 +15,31 @@
 // from score_hist's keys-only variant on every SM (scoring streams K', which
 // wants all of them); then one cluster per (sequence, KV head) selects.  CTA r
 // of a cluster of CS owns the positions [r*L, (r+1)*L), L a multiple of 32:
-//   1. keys   the CTA copies the keys of its slice from the workspace (just
-//             written, so from L2) into shared memory with 16-byte cp.async,
-//             in four groups, and counts each group into a first histogram
-//             as it lands.  Every later step reads these keys (compact code:
-//             the kernel is otherwise bound by instruction fetch).
-//   2. tau    the B-th largest key tau and k, how many keys equal to it are
-//             taken, on one of two routes:
-//             value route (every row's scores span a finite, non-empty
-//               range): the first histogram's 2048 bins are linear in the
-//               score between the row's smallest and largest key (the
-//               scoring kernel leaves both in the workspace).  The cluster
-//               sums the histograms over distributed shared memory and finds
-//               the bin c that holds the B-th key; for Gaussian-like scores
-//               it holds a few dozen keys.  Each CTA marks the keys above c
-//               as Top and sends its keys in c to every CTA of the cluster;
-//               after one barrier every CTA ranks the same short list (by
-//               pairwise counts, or radix passes over the list when it is
-//               long) and knows tau, k and every CTA's count of keys equal
-//               to tau.  A bin of more than kVCap keys sends the cluster to
-//               the other route.
-//             radix route: three passes (key bits 31..21, 20..10, 9..0).  In
-//               each, a CTA histograms its keys that match the digits fixed
-//               so far, the cluster meets at a barrier, and every CTA sums
-//               the cluster's histograms over distributed shared memory:
-//               first per group of 32 bins, then the 32 bins of the group
-//               that holds the B-th key.  Every CTA finds the same digit; the
-//               last histogram's bin tau holds each CTA's count of keys equal
-//               to tau.
-//   3. ties   from the CTAs' counts of keys equal to tau every CTA knows how
-//             many of its own (and its neighbours') ties are taken, lowest
-//             positions first.
+//   1. keys   the CTA loads the keys of its slice from the workspace (just
+//             written, so from L2) into shared memory, a warp per 32-position
+//             word, lane = position; a histogram of key bits 31..21 per head
+//             is built on the way.  Every later step loops over these words
+//             (compact code: the kernel is otherwise bound by instruction
+//             fetch).
+//   2. radix  three passes (key bits 31..21, 20..10, 9..0) fix the B-th
+//             largest key tau and k, how many keys equal to it are taken.  In
+//             each, a CTA histograms its keys that match the digits fixed so
+//             far, the cluster meets at a barrier, and every CTA sums the
+//             cluster's histograms over distributed shared memory: first per
+//             group of 32 bins, then the 32 bins of the group that holds the
+//             B-th key.  Every CTA finds the same digit.
+//   3. ties   the last histogram's bin tau holds each CTA's count of keys
+//             equal to tau, so every CTA knows how many of its own (and its
+//             neighbours') ties are taken, lowest positions first.
 //   4. dilate the Top bitmap is dilated by +-nbr and clipped to C.  The edge
 //             words of the neighbouring slices are rebuilt from the keys their
 //             CTAs publish, so no extra barrier is needed for them.
 //   5. emit   each CTA writes its slice's bitmap words and, at the offset the
 //             lower slices' counts give, its part of the sorted index list.
-// Both routes rank the same keys exactly, so they select the same set.
 // The cluster barriers sit at the same points on every path of every CTA of
-// a cluster (the mode below depends only on the sequence's length, the route
-// only on workspace words and cluster-wide sums that every CTA reads alike),
-// and a CTA leaves only after a last barrier, so no CTA reads or writes the
-// shared memory of one that has exited.
+// a cluster (the mode below depends only on the sequence's length), and a CTA
+// leaves only after a last barrier, so no CTA reads the shared memory of one
+// that has exited.
 #include <algorithm>
 #include <mutex>
 #include <type_traits>
@@ -184,214 +167,11 @@ __device__ void group_sums(uint32_t *hist) {
     }
 }
 
-// The value route's cap on the keys of a crossing bin, per score row: they
-// are gathered into every CTA of the cluster and ranked there.
-constexpr int kVCap = 1024;
-// ... ranked by counting, pairwise, when no row's bin holds more than this
-constexpr int kRankMax = 256;
-static_assert(2 * kVCap <= kHistWords, "the gathered lists and this CTA's positions take histogram B");
-
-// 32-bit store of v to the word at `local` (an address in this CTA's shared
-// memory) in the shared memory of cluster CTA `rank`; visible there after the
-// next cluster barrier.
-__device__ __forceinline__ void st_dsmem(uint32_t *local, uint32_t rank, uint32_t v) {
-    uint32_t ra;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
-    asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(ra), "r"(v) : "memory");
-}
-
-// The score a key stands for (the inverse of score_key on finite scores).
-__device__ __forceinline__ float key_value(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Bin of a key on the value route: floor((s - smin) * scale) for the key's
-// score s, scale = 2048 / (smax - smin), clamped to 2047, for keys between
-// the row's smallest and largest key (finite scores; the smallest takes bin
-// 0, the largest 2047).  Each step (an fp32 subtraction and product rounded
-// to nearest, a truncation, a clamp) is monotone, so a larger key never takes
-// a lower bin, equal keys take the same bin, and every bin is a range of keys.
-__device__ __forceinline__ uint32_t value_bin(uint32_t k, float fmin, float scale) {
-    const float x = __fmul_rn(__fsub_rn(key_value(k), fmin), scale);
-    return min(__float2uint_rz(x), 2047u);
-}
-
-// The first key k in [kmin, kmax] with value_bin(k) >= t (kmax + 1 when t is
-// past the last bin), found by one warp: every round each lane probes one of
-// 32 points spread over the open range, and the range shrinks to the gap
-// between the last probe below t and the first at or above it.  All lanes
-// return it.
-__device__ uint64_t first_key_of_bin(uint32_t t, uint32_t kmin, uint32_t kmax, float fmin, float scale, int lane) {
-    if (t == 0u) return kmin;
-    if (t >= 2048u) return (uint64_t)kmax + 1u;
-    uint64_t lo = kmin, hi = kmax;  // value_bin(lo) = 0 < t <= 2047 = value_bin(hi)
-    while (hi - lo > 1u) {
-        const uint64_t p = lo + ((hi - lo) * (uint64_t)lane) / 32u;  // lane 0 probes lo
-        const unsigned m = __ballot_sync(kFull, value_bin((uint32_t)p, fmin, scale) >= t);
-        const int f = m ? __ffs(m) - 1 : 32;
-        const uint64_t nlo = __shfl_sync(kFull, p, f - 1);
-        if (m) hi = __shfl_sync(kFull, p, f);
-        lo = nlo;
-    }
-    return hi;
-}
-
-// cp.async.wait_group with a count known only at run time (0..3).
-__device__ __forceinline__ void cp_async_wait_upto(int n) {
-    switch (n) {
-        case 0: cp_async_wait_group<0>(); break;
-        case 1: cp_async_wait_group<1>(); break;
-        case 2: cp_async_wait_group<2>(); break;
-        default: cp_async_wait_group<3>(); break;
-    }
-}
-
-// cluster_find_digit for the value route's histogram (2048 bins per row):
-// per row, the bin that holds the need[h]-th largest key (xbin[h]), how many
-// of its keys are still needed (need[h]), its count in the cluster (xtot[h])
-// and in each CTA of the cluster (xcnt[h][q]).  Whole CTA; call after a
-// cluster barrier that follows the histogram and its group sums.
-template <int NH>
-__device__ void cluster_find_bin(const uint32_t *hist, int cs, uint32_t *gco, uint32_t *xbin, uint32_t *need,
-                                 uint32_t *xtot, uint32_t (*xcnt)[kMaxCluster]) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int ng = 2048 / 32;
-    if (tid < NH * ng) {
-        const int h = tid / ng, j = tid % ng;
-        gco[h * 64 + j] = cluster_sum(hist + h * kHistWords + 2048 + j, cs);
-    }
-    __syncthreads();
-    if (warp < NH) {
-        const int h = warp;
-        const uint32_t nd = need[h];
-        // the group of 32 bins that holds the nd-th largest key (2 groups per lane, from the top)
-        const uint32_t c0 = gco[h * 64 + ng - 1 - 2 * lane], c1 = gco[h * 64 + ng - 2 - 2 * lane];
-        const uint32_t v = c0 + c1;
-        uint32_t incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const uint32_t excl = incl - v;
-        const bool cross = excl < nd && nd <= incl;
-        int grp = 0;
-        uint32_t above = 0;
-        if (cross) {
-            const bool first = excl + c0 >= nd;
-            grp = ng - 1 - (2 * lane + (first ? 0 : 1));
-            above = first ? excl : excl + c0;
-        }
-        const unsigned m = __ballot_sync(kFull, cross);
-        const int src = m ? __ffs(m) - 1 : 0;
-        grp = __shfl_sync(kFull, grp, src);
-        above = __shfl_sync(kFull, above, src);
-        // its 32 bins, from the top, each CTA's count kept
-        const int bin = grp * 32 + 31 - lane;
-        uint32_t vq[kMaxCluster];
-        const uint32_t *loc = hist + h * kHistWords + bin;
-#pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) vq[q] = q < cs ? *dsmem_ptr(loc, (uint32_t)q) : 0u;
-        uint32_t bv = 0;
-#pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) bv += vq[q];
-        uint32_t bi = bv;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kFull, bi, o);
-            if (lane >= o) bi += t;
-        }
-        const uint32_t be = above + bi - bv;
-        const bool hit = be < nd && nd <= above + bi;
-        const unsigned hm = __ballot_sync(kFull, hit);
-        const int hsrc = hm ? __ffs(hm) - 1 : 0;
-        if (lane == hsrc) {
-            xbin[h] = (uint32_t)bin;
-            need[h] = nd - be;
-            xtot[h] = bv;
-#pragma unroll
-            for (int q = 0; q < kMaxCluster; ++q) xcnt[h][q] = vq[q];
-        }
-    }
-    __syncthreads();
-}
-
-// The need[h]-th largest of the n[h] keys list[h * kVCap + j] of each row
-// (the same lists in every CTA), by three radix passes (key bits 31..21,
-// 20..10, 9..0) over a histogram in `hist` (per row 2048 words at
-// h * kHistWords): prefix[h] becomes the key, need[h] how many keys equal to
-// it are taken.  A warp per row finds each digit.  Whole CTA.
-template <int NH>
-__device__ void list_select(const uint32_t *list, const uint32_t *n, uint32_t *hist, uint32_t *prefix,
-                            uint32_t *need) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
-        for (int i = tid; i < NH * 2048; i += kCThreads) hist[(i / 2048) * kHistWords + (i % 2048)] = 0u;
-        __syncthreads();
-        for (int i = tid; i < NH * kVCap; i += kCThreads) {
-            const int h = i / kVCap, j = i % kVCap;
-            if (j < (int)n[h]) {
-                const uint32_t k = list[i];
-                const bool match = pass == 0 || (k >> (shift + (pass == 1 ? 11 : 10))) == prefix[h];
-                if (match) atomicAdd(&hist[h * kHistWords + ((k >> shift) & (uint32_t)(nb - 1))], 1u);
-            }
-        }
-        __syncthreads();
-        if (warp < NH) {
-            const int h = warp;
-            const uint32_t nd = need[h];
-            const int per = nb / 32;  // bins per lane, lane l owning the l-th run from the top
-            const uint32_t *hb = hist + h * kHistWords;
-            uint32_t v = 0;
-            for (int j = 0; j < per; ++j) v += hb[nb - 1 - lane * per - ((j + lane) & (per - 1))];  // (rotated: no bank conflicts)
-            uint32_t incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += t;
-            }
-            const unsigned m = __ballot_sync(kFull, incl - v < nd && nd <= incl);
-            const int src = m ? __ffs(m) - 1 : 0;
-            uint32_t above = __shfl_sync(kFull, incl - v, src);
-            // the crossing run's bins, one or two per lane, from its top
-            const int top = nb - 1 - src * per;
-            const int k2 = per / 32;
-            uint32_t w = 0, w0 = 0;
-            for (int j = 0; j < k2; ++j) {
-                const uint32_t c = hb[top - lane * k2 - j];
-                if (j == 0) w0 = c;
-                w += c;
-            }
-            uint32_t wi = w;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(kFull, wi, o);
-                if (lane >= o) wi += t;
-            }
-            const uint32_t we = above + wi - w;
-            const bool hit = we < nd && nd <= above + wi;
-            const unsigned hm = __ballot_sync(kFull, hit);
-            if (hit && lane == __ffs(hm) - 1) {
-                const bool first = k2 == 1 || we + w0 >= nd;
-                const int bin = top - lane * k2 - (first ? 0 : 1);
-                const uint32_t bef = first ? we : we + w0;
-                prefix[h] = pass == 0 ? (uint32_t)bin : ((prefix[h] << (pass == 1 ? 11 : 10)) | (uint32_t)bin);
-                need[h] = nd - bef;
-            }
-        }
-        __syncthreads();
-    }
-}
-
 template <int SEL>
 __global__ void __launch_bounds__(kCThreads, 1)
 sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W, int L, int sink, int window,
                    int budget, int nbr, int32_t *__restrict__ idx, int idx_cap, int32_t *__restrict__ count,
-                   uint32_t *__restrict__ sel_bits, const uint32_t *__restrict__ gkeys, uint32_t *__restrict__ rng_words,
-                   uint32_t *__restrict__ flags) {
+                   uint32_t *__restrict__ sel_bits, const uint32_t *__restrict__ gkeys, uint32_t *__restrict__ flags) {
     constexpr int NH = rows_per_group<SEL>();
     constexpr int NOUT = sel_is_group(SEL) ? kGroup : 1;  // output rows per score row
     const int LW = L / 32;
@@ -414,125 +194,53 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
     __shared__ uint32_t gco[4 * 64];
     __shared__ uint32_t prefix[4], need[4], x_cnt[4], base_s[4], total_s[4], take_s[4], nb_top[2][4];
     __shared__ int scratch[kCThreads / 32 + 3];
-    // the value route: per row the key range, the crossing bin, its counts
-    __shared__ uint32_t v_kmin[4], v_kmax[4], v_bits, xbin[4], xtot[4], lcnt[4], v_klo[4], v_tau[4], v_take[4];
-    __shared__ unsigned long long v_khi[4];
-    __shared__ float v_fmin[4], v_scale[4];
-    __shared__ uint32_t xcnt[4][kMaxCluster], tieq[4][kMaxCluster];
 
     for (int i = tid; i < NH * kHistWords; i += kCThreads) {
         histA[i] = 0u;
         histB[i] = 0u;
     }
-    if (tid < 4) {
-        x_cnt[tid] = 0u;
-        lcnt[tid] = 0u;
-    }
-    if (tid == 0) v_bits = 0u;
-    griddep_wait();  // the keys come from the kernel before
+    if (tid < 4) x_cnt[tid] = 0u;
+    __syncthreads();  // the histograms are zero before any thread counts into them
+    griddep_wait();   // the keys come from the kernel before
     griddep_launch_dependents();
-    const size_t krow0 = (size_t)b * Hq + (size_t)g * kGroup;  // first workspace key row of the group
-
-    // ---- 1. the slice's keys into shared memory, word wi of score row h at
-    // keys_s[h * L + 32 wi + lane]; 0 marks a position outside C (no score
-    // has key 0: score_key maps every float, NaNs included, to a key of at
-    // least 0x007fffff).  The copies go out first, before the sequence's
-    // length is known: 16-byte chunks of 4 positions, asynchronous where the
-    // row is 16-byte aligned, in 4 groups (one score row each when there are
-    // 4).  Positions outside C are zeroed once the length is in, as each
-    // group lands.
-    constexpr int NG = 4;
-    static_assert(NH == 1 || NH == NG, "a copy group holds one score row, or part of the only one");
-    const int cpr = L / 4;  // chunks per score row of the slice; chunk c holds keys_s[4c .. 4c + 3]
-    const int nch = NH * cpr;
-    {
-        const bool vec = (Tcap & 3) == 0;
-        const int cend = min(s0 + L, Tcap);  // the row's positions in the slice
-#pragma unroll
-        for (int q = 0; q < NG; ++q) {
-            for (int c = q * nch / NG + tid; c < (q + 1) * nch / NG; c += kCThreads) {
-                const int h = c / cpr, p = s0 + 4 * (c % cpr);
-                uint32_t *dst = keys_s + 4 * c;
-                const uint32_t *src = gkeys + (krow0 + h) * Tcap + p;
-                if (vec && p + 4 <= cend) {
-                    cp_async16(smem_addr(dst), src, true);
-                } else if (p >= cend) {
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) dst[j] = p + j < cend ? __ldcg(src + j) : 0u;
-                }
-            }
-            cp_async_commit();
-        }
-    }
     const int T = clamp_ctx(ctx_len[b], Tcap, flags, tid == 0 && r == 0 && g == 0);
     const int lo = sink, hi = T - window;
     const int nC = hi > lo ? hi - lo : 0;
     const uint32_t mode = nC == 0 ? kModeEmpty : (nC <= budget ? kModeAll : kModeSelect);
     const int a = max(lo, s0), e = min(hi, s0 + L);  // this slice's part of C
+    const size_t krow0 = (size_t)b * Hq + (size_t)g * kGroup;  // first workspace key row of the group
 
-    // The value route (taken when every row's key range is finite and not a
-    // single value): the first pass bins keys linearly in the score between
-    // the row's smallest and largest key, which the scoring kernel leaves in
-    // words 0 and 1 of the row's histogram (the complement of the smallest,
-    // then the largest).  The B-th key's bin then holds few keys, which are
-    // gathered into every CTA and ranked there; if any row's bin holds more
-    // than kVCap, the key-bit radix passes run instead.  Every CTA of the
-    // cluster reads the same words, so all take the same route.
-    if (tid < NH) {
-        const uint32_t *rw = rng_words + (krow0 + tid) * kBins1;
-        const uint32_t kmn = ~__ldcg(rw), kmx = __ldcg(rw + 1);
-        const float fmn = key_value(kmn), fmx = key_value(kmx);
-        const float range = __fsub_rn(fmx, fmn);
-        const float scale = __fdiv_rn(2048.0f, range);
-        v_kmin[tid] = kmn;
-        v_kmax[tid] = kmx;
-        v_fmin[tid] = fmn;
-        v_scale[tid] = scale;
-        if (mode == kModeSelect && kmx > kmn && isfinite(fmn) && isfinite(fmx) && isfinite(range) &&
-            range > 0.0f && isfinite(scale) && scale > 0.0f)
-            atomicOr(&v_bits, 1u << tid);
-    }
-    __syncthreads();  // (also: the histograms are zeroed before any count)
-    bool vp = v_bits == (1u << NH) - 1u;
-
-    // each group as it lands: positions outside C zeroed, then counted into
-    // the first pass's histogram (bins linear in the score on the value
-    // route, key bits 31..21 otherwise)
-#pragma unroll 1
-    for (int q = 0; q < NG; ++q) {
-        cp_async_wait_upto(NG - 1 - q);
-        __syncthreads();
-        const int h = NH == 1 ? 0 : q;
-        const float fmn = v_fmin[h], sc = v_scale[h];
-        uint32_t *hist = histA + h * kHistWords;
-        uint4 *k4 = reinterpret_cast<uint4 *>(keys_s);
-        for (int c = q * nch / NG + tid; c < (q + 1) * nch / NG; c += kCThreads) {
-            const int p = s0 + 4 * (c % cpr);
-            uint4 v = k4[c];  // 4 keys at once: their bins are independent
-            if (p < a || p + 4 > e) {
-                v.x = p >= a && p < e ? v.x : 0u;
-                v.y = p + 1 >= a && p + 1 < e ? v.y : 0u;
-                v.z = p + 2 >= a && p + 2 < e ? v.z : 0u;
-                v.w = p + 3 >= a && p + 3 < e ? v.w : 0u;
-                k4[c] = v;
+    // ---- 1. the slice's keys into shared memory, word wi of score row h at
+    // keys_s[h * L + 32 wi + lane]; 0 marks a position outside C (no score
+    // has key 0: score_key maps every float, NaNs included, to a key of at
+    // least 0x007fffff)
+    {
+        // the thread's loads go out 8 at a time, each batch issued before
+        // its first key is used
+        constexpr int WPW = max_slice<SEL>() / 32 / kCWarps;  // words of a score row per warp, at most
+        constexpr int NLD = NH * WPW, BATCH = 8;
+        static_assert(NLD % BATCH == 0, "whole batches");
+#pragma unroll
+        for (int b0 = 0; b0 < NLD; b0 += BATCH) {
+            uint32_t kv[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                const int h = (b0 + i) / WPW, wi = warp + kCWarps * ((b0 + i) % WPW);
+                const int p = s0 + 32 * wi + lane;
+                kv[i] = (wi < LW && p >= a && p < e) ? __ldcg(gkeys + (krow0 + h) * Tcap + p) : 0u;
             }
-            if (mode == kModeSelect) {
-                const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
-                uint32_t bb[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) bb[j] = vp ? value_bin(kk[j], fmn, sc) : (kk[j] >> 21);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (kk[j] != 0u) atomicAdd(&hist[bb[j]], 1u);
+            for (int i = 0; i < BATCH; ++i) {
+                const int h = (b0 + i) / WPW, wi = warp + kCWarps * ((b0 + i) % WPW);
+                if (wi < LW) {  // warp-uniform
+                    const uint32_t k = kv[i];
+                    keys_s[h * L + 32 * wi + lane] = k;
+                    if (k != 0u) atomicAdd(&histA[h * kHistWords + (k >> 21)], 1u);
+                    if (wi == 0) edge_s[0][h][lane] = k;
+                    if (wi == LW - 1) edge_s[1][h][lane] = k;
+                }
             }
         }
-    }
-    __syncthreads();
-    for (int i = tid; i < NH * 64; i += kCThreads) {
-        const int h = i / 64, j = i % 64;
-        edge_s[j / 32][h][j % 32] = keys_s[h * L + (j < 32 ? j : 32 * (LW - 1) + j - 32)];
     }
     __syncthreads();
 
@@ -544,169 +252,6 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
         }
         group_sums<NH>(histA);
         cluster_sync();
-        if (vp) {
-            cluster_find_bin<NH>(histA, cs, gco, xbin, need, xtot, xcnt);
-            bool fits = true;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) fits = fits && xtot[h] <= (uint32_t)kVCap;
-            uint32_t *cand_g = histB;  // [NH][kVCap]: the cluster's keys in the crossing bin, CTA by CTA
-            if (fits) {
-                // the crossing bin's keys are those in [klo, khi)
-                if (warp < 2 * NH) {
-                    const int h = warp >> 1;
-                    const uint64_t k0 =
-                        first_key_of_bin(xbin[h] + (uint32_t)(warp & 1), v_kmin[h], v_kmax[h], v_fmin[h], v_scale[h], lane);
-                    if (lane == 0) {
-                        if (warp & 1)
-                            v_khi[h] = k0;
-                        else
-                            v_klo[h] = (uint32_t)k0;
-                    }
-                }
-                __syncthreads();
-                // Top bits of the keys above the bin, and the bin's keys as
-                // candidates: their positions kept here, the keys sent to
-                // every CTA of the cluster at the offset of this CTA's rank.
-                // A warp takes 4 words at a time (loads first).
-                uint32_t *cpos = histB + NH * kVCap;  // [NH][kVCap]: this CTA's candidates, as positions in the slice
-#pragma unroll 1
-                for (int h = 0; h < NH; ++h) {
-                    const uint32_t klo = v_klo[h];
-                    const unsigned long long khi = v_khi[h];
-                    const uint32_t *kh = keys_s + h * L;
-                    uint32_t my_top = 0u;
-                    int q = 0;  // this warp's words so far; lane j keeps the Top bits of word warp + kCWarps * j
-                    for (int w0 = warp; w0 < LW; w0 += 4 * kCWarps, q += 4) {
-                        uint32_t k[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int wi = w0 + u * kCWarps;
-                            k[u] = wi < LW ? kh[32 * wi + lane] : 0u;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            // (klo > 0: no position outside C passes)
-                            const bool cand = k[u] >= klo && (unsigned long long)k[u] < khi;
-                            const uint32_t tb = __ballot_sync(kFull, (unsigned long long)k[u] >= khi);
-                            const uint32_t cb = __ballot_sync(kFull, cand);
-                            my_top = lane == q + u ? tb : my_top;
-                            if (cb) {  // (few words)
-                                uint32_t slot = 0;
-                                if (lane == 0) slot = atomicAdd(&lcnt[h], (uint32_t)__popc(cb));
-                                slot = __shfl_sync(kFull, slot, 0) + (uint32_t)__popc(cb & lt);
-                                if (cand && slot < (uint32_t)kVCap)  // (always: the bin holds at most kVCap)
-                                    cpos[h * kVCap + slot] = (uint32_t)(32 * (w0 + u * kCWarps) + lane);
-                            }
-                        }
-                    }
-                    const int wi = warp + kCWarps * lane;
-                    if (lane < q && wi < LW) {
-                        top_s[h * LW + wi] = my_top;
-                        aux_s[h * LW + wi] = 0u;  // the tie bits, set below
-                    }
-                }
-                __syncthreads();
-                // the candidates' keys to every CTA of the cluster, one store
-                // per thread: item i is candidate i / cs (rows one after
-                // another) for CTA i % cs
-                {
-                    uint32_t n[NH], nall = 0;
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        n[h] = min(lcnt[h], xcnt[h][r]);
-                        nall += n[h];
-                    }
-                    for (int it = tid; it < (int)nall * cs; it += kCThreads) {
-                        const int v = it % cs;
-                        int j = it / cs, h = 0;
-#pragma unroll
-                        for (int u = 0; u + 1 < NH; ++u)
-                            if (h == u && j >= (int)n[u]) {
-                                j -= (int)n[u];
-                                h = u + 1;
-                            }
-                        uint32_t base = 0;
-                        for (int q = 0; q < (int)r; ++q) base += xcnt[h][q];
-                        st_dsmem(cand_g + h * kVCap + base + j, (uint32_t)v, keys_s[h * L + cpos[h * kVCap + j]]);
-                    }
-                }
-                cluster_sync();  // every CTA holds the cluster's lists (and is past its reads of histogram A)
-                // tau, the need[h]-th largest key of the row's list, and how
-                // many keys equal to it are taken: by counting, pairwise,
-                // when every list is short, by radix passes otherwise
-                bool shortl = true;
-#pragma unroll
-                for (int h = 0; h < NH; ++h) shortl = shortl && xtot[h] <= (uint32_t)kRankMax;
-                if (shortl) {
-                    for (int it = tid; it < NH * kRankMax; it += kCThreads) {
-                        const int h = it / kRankMax, i = it % kRankMax, n = (int)xtot[h];
-                        if (i < n) {
-                            const uint32_t *lst = cand_g + h * kVCap;
-                            const uint32_t x = lst[i];
-                            uint32_t gt = 0, eq = 0;
-                            for (int j = 0; j < n; ++j) {
-                                const uint32_t y = lst[j];
-                                gt += y > x ? 1u : 0u;
-                                eq += y == x ? 1u : 0u;
-                            }
-                            const uint32_t nd = need[h];
-                            if (gt < nd && nd <= gt + eq) {  // (every key equal to tau writes the same)
-                                v_tau[h] = x;
-                                v_take[h] = nd - gt;
-                            }
-                        }
-                    }
-                    __syncthreads();
-                    if (tid < NH) {
-                        prefix[tid] = v_tau[tid];
-                        need[tid] = v_take[tid];
-                    }
-                    __syncthreads();
-                } else {
-                    list_select<NH>(cand_g, xtot, histA, prefix, need);
-                }
-                // each CTA's keys equal to tau: its share of the ties (a warp per row and CTA)
-                for (int pr = warp; pr < NH * cs; pr += kCWarps) {
-                    const int h = pr / cs, q = pr % cs;
-                    uint32_t off = 0;
-                    for (int u = 0; u < q; ++u) off += xcnt[h][u];
-                    const uint32_t n = xcnt[h][q], tau = prefix[h];
-                    uint32_t c = 0;
-                    for (uint32_t j = lane; j < n; j += 32) c += cand_g[h * kVCap + off + j] == tau ? 1u : 0u;
-                    c = __reduce_add_sync(kFull, c);
-                    if (lane == 0) tieq[h][q] = c;
-                }
-                // this slice's candidates: above tau into Top, equal to it into the tie bits
-                for (int it = tid; it < NH * kVCap; it += kCThreads) {
-                    const int h = it / kVCap, j = it % kVCap;
-                    if (j < (int)min(lcnt[h], xcnt[h][r])) {
-                        const uint32_t pos = cpos[it];
-                        const uint32_t k = keys_s[h * L + pos], tau = prefix[h], bit = 1u << (pos & 31u);
-                        if (k > tau) atomicOr(&top_s[h * LW + (pos >> 5)], bit);
-                        if (k == tau) atomicOr(&aux_s[h * LW + (pos >> 5)], bit);
-                    }
-                }
-                __syncthreads();
-            } else {
-                // a crossing bin too full to gather: the key-bit passes from the start
-                vp = false;
-                cluster_sync();  // every CTA is past its reads of histogram A
-                for (int i = tid; i < NH * kHistWords; i += kCThreads) histA[i] = 0u;
-                if (tid < NH) need[tid] = (uint32_t)budget;
-                __syncthreads();
-#pragma unroll 1
-                for (int h = 0; h < NH; ++h)
-                    for (int i = tid; i < L; i += kCThreads) {
-                        const uint32_t k = keys_s[h * L + i];
-                        if (k != 0u) atomicAdd(&histA[h * kHistWords + (k >> 21)], 1u);
-                    }
-                __syncthreads();
-                group_sums<NH>(histA);
-                cluster_sync();
-            }
-        }
-    }
-    if (mode == kModeSelect && !vp) {
         cluster_find_digit<NH>(histA, 2048, 11, cs, gco, prefix, need);
         // key bits 20..10 of the keys whose bits 31..21 are prefix (few: counted with atomics)
 #pragma unroll 1
@@ -750,7 +295,7 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
     // (lane q keeps the ballots of the warp's q-th word and stores them after
     // the loop: one store per lane, no branch per word)
 #pragma unroll 1
-    for (int h = 0; h < (vp ? 0 : NH); ++h) {  // (the value route has made them)
+    for (int h = 0; h < NH; ++h) {
         const uint32_t tau = prefix[h];
         uint32_t my_top = 0u, my_tie = 0u;
         int q = 0;
@@ -782,9 +327,7 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
         if (warp < NH) {
             const int h = warp;
             const uint32_t tau = prefix[h], k = need[h];
-            const uint32_t t =
-                lane < cs ? (vp ? tieq[h][lane] : ld_dsmem(&histA[h * kHistWords + (tau & 0x3FFu)], (uint32_t)lane))
-                          : 0u;
+            const uint32_t t = lane < cs ? ld_dsmem(&histA[h * kHistWords + (tau & 0x3FFu)], (uint32_t)lane) : 0u;
             uint32_t incl = t;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -919,7 +462,6 @@ sel_cluster_kernel(const int32_t *__restrict__ ctx_len, int Hq, int Tcap, int W,
         }
     }
     cluster_arrive();  // this CTA reads no other CTA's shared memory from here on
-    if (r == 0 && tid < 2 * NH) rng_words[(krow0 + tid / 2) * kBins1 + (tid & 1)] = 0u;  // every CTA has read them
     __syncthreads();
     {
         uint32_t hstart = 0;  // this CTA's selected positions of the heads before h
@@ -1045,7 +587,7 @@ cudaError_t launch_cluster(const tb_dims &d, const Plan &p, const float *qp, int
     const int W = (d.ctx_cap + 31) / 32;
     return launch_pdl_cluster(sel_cluster_kernel<SEL>, dim3(p.cs, d.n_kv_heads, d.batch), dim3(kCThreads), p.cs,
                               p.smem, st, ctx_len, d.n_q_heads, d.ctx_cap, W, p.L, sink, window, budget, nbr, idx,
-                              idx_cap, count, sel_bits, (const uint32_t *)s.keys, s.hist, s.flags);
+                              idx_cap, count, sel_bits, (const uint32_t *)s.keys, s.flags);
 }
 
 template <int SEL>
