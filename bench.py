@@ -54,7 +54,8 @@ class Run:
     that rank owns under KV-head sharding, sliced from the same seeded data."""
 
     def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head",
-                 shard: tuple[int, int] | None = None, offload: bool = False, balance: bool = True):
+                 shard: tuple[int, int] | None = None, offload: bool = False, balance: bool = True,
+                 overlap_select: bool = True):
         self.w = w
         self.device = device
         self.steps = steps or w.steps
@@ -101,7 +102,7 @@ class Run:
         # the bench's streams run only libtb's kernels, the K/V append of the
         # e2e loop and copies, so every attention launch may prefetch its rows
         self.dec = cls(self.shape, list(self.K), list(self.V), self.Wk, self.mlp, self.ctx0, self.steps, device,
-                       selection=selection, prefetch_kv=True, balance=balance)
+                       selection=selection, prefetch_kv=True, balance=balance, overlap_select=overlap_select)
         self.out = torch.zeros(nL, w.batch, self.Hq, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):
@@ -668,7 +669,8 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
     each replayed as one CUDA graph; returns the figures the JSON line needs.
     With shard=(rank, world) this rank runs only its KV heads of the one
     workload (strong scaling: the job's tokens are the workload's tokens)."""
-    run = Run(w, device, steps=args.decode_steps, selection=selection, shard=shard, balance=not args.no_balance)
+    run = Run(w, device, steps=args.decode_steps, selection=selection, shard=shard, balance=not args.no_balance,
+              overlap_select=not args.no_overlap)
     copies = 1 if shard else world          # independent replicas count every rank's tokens
     run.dec.prefill()
     torch.cuda.synchronize()
@@ -699,8 +701,9 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
         ms_e2e = time_graph(g_e2e, warmup, steps, dist_on, device)
         clk_e2e = clocks.stop()
 
-    flags = L.workspace_check(run.dec.ws_attn) | L.workspace_check(run.dec.ws_sel) | \
-        L.workspace_check(run.dec.ws_proj) | (L.workspace_check(run.dec.ws_pred) if run.dec.ws_pred is not None else 0)
+    flags = 0
+    for ws in run.dec.workspaces():
+        flags |= L.workspace_check(ws)
 
     tokens_per_run = run.steps * w.batch
     per_step_sparse = ms_sparse / steps
@@ -768,7 +771,9 @@ def measure_offload(w, args, device, selection: str):
     ms = {k: time_graph(g, max(3, args.warmup), args.extra_steps, False, device) / args.extra_steps
           for k, g in graphs.items()}
     clk = clocks.stop()
-    flags = L.workspace_check(run.dec.ws_attn) | L.workspace_check(run.dec.ws_sel) | L.workspace_check(run.dec.ws_proj)
+    flags = 0
+    for ws in run.dec.workspaces():
+        flags |= L.workspace_check(ws)
     sparse_ms = (ms["pred"] + (P - 1) * ms["reuse"]) / P + ((ms["proj"] - ms["reuse"]) / N if "proj" in ms else 0.0)
     host_gb = sum(hb.nbytes for hb in run.dec.K_host + run.dec.V_host) / 1e9
     res = {"workload": w.name, "per_token_ms": round(sparse_ms, 3), "dense_per_token_ms": round(ms["dense"], 3),
@@ -822,6 +827,8 @@ def main():
                     help="skip the CPU-offloaded KV cache on long256k (per-token latency against dense), which the "
                          "default single-GPU run times after the headline workload")
     ap.add_argument("--offload-only", action="store_true", help="time only the CPU-offloaded workload")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="all of a prediction step's selections on one stream (no second selection stream)")
     ap.add_argument("--no-balance", action="store_true",
                     help="attention slices at equal shares of the length instead of the kept rows (no tb_attn_plan)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "kv_heads"],

@@ -273,7 +273,8 @@ class SparseDecoder:
     SELECTIONS = ("head", "group_max", "group_sum", "inclusive")
 
     def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda",
-                 selection: str = "head", prefetch_kv: bool = False, balance: bool = True):
+                 selection: str = "head", prefetch_kv: bool = False, balance: bool = True,
+                 overlap_select: bool = True):
         if selection not in self.SELECTIONS:
             raise ValueError(f"selection must be one of {self.SELECTIONS}")
         self.selection = selection
@@ -313,6 +314,17 @@ class SparseDecoder:
         self.ws_proj = L.workspace(L.project_keys_workspace_bytes(), device)
         self.ws_pred = (L.workspace(L.predict_queries_workspace_bytes(B, s.hidden, s.inter, s.n_out), device)
                         if s.hidden > 0 else None)
+        # overlap_select: a prediction step's selections alternate between the
+        # caller's stream and a second one (odd layers, with a selection and
+        # a plan workspace of their own), so that one layer's scoring runs on
+        # the SMs the other layer's cluster selection leaves free.  The layers'
+        # selections are independent; the attention launches wait for both.
+        self.overlap_select = overlap_select and s.n_layers > 1
+        self.side = torch.cuda.Stream(device=device) if self.overlap_select else None
+        self.ws_sel_side = (L.workspace(L.score_select_workspace_bytes(self.dims), device)
+                            if self.overlap_select else None)
+        self.ws_plan_side = (L.workspace(L.attn_workspace_bytes(self.dims), device)
+                             if self.overlap_select and balance else None)
         self.ctx = torch.tensor([[t + i + 1 for t in ctx0] for i in range(steps)], dtype=torch.int32,
                                 device=device)
         prefill, events = projection_schedule(self.ctx0, s.window, steps)
@@ -342,8 +354,15 @@ class SparseDecoder:
         W1, W2 = self.mlp[producer]
         L.predict_queries(h, W1, W2, self.qp[producer], self.ws_pred, stream)
 
-    def select(self, step: int, layer: int, qp_direct=None, stream=None):
+    def workspaces(self) -> list:
+        """Every workspace the decoder's launches use (for tb_workspace_check)."""
+        return [w for w in (self.ws_attn, self.ws_sel, self.ws_proj, self.ws_pred, self.ws_sel_side,
+                            self.ws_plan_side) if w is not None]
+
+    def select(self, step: int, layer: int, qp_direct=None, stream=None, ws_sel=None, ws_plan=None):
         s = self.shape
+        ws_sel = self.ws_sel if ws_sel is None else ws_sel
+        ws_plan = self.ws_attn if ws_plan is None else ws_plan
         if qp_direct is not None:
             qp, stride = qp_direct, s.n_q_heads * s.d_proj
         else:
@@ -354,17 +373,17 @@ class SparseDecoder:
             stride = s.stride * s.n_q_heads * s.d_proj
         if self.selection == "head":
             L.score_select(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window, s.budget,
-                           s.nbr, self.idx[layer], self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+                           s.nbr, self.idx[layer], self.cnt[layer], self.bits[layer], ws_sel, stream)
         elif self.selection == "inclusive":
             L.score_select_inclusive(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window,
                                      s.budget, s.nbr, self.idx[layer], self.cnt[layer], self.bits[layer],
-                                     self.ws_sel, stream)
+                                     ws_sel, stream)
         else:
             L.score_select_group(self.dims, qp, stride, self.Kp[layer], self.ctx[step], s.sink, s.window,
                                  s.budget, s.nbr, self.selection[len("group_"):], self.idx[layer],
-                                 self.cnt[layer], self.bits[layer], self.ws_sel, stream)
+                                 self.cnt[layer], self.bits[layer], ws_sel, stream)
         if self.balance:
-            L.attn_plan(self.dims, self.bits[layer], self.ctx[step], s.sink, s.window, self.plan[layer], self.ws_attn,
+            L.attn_plan(self.dims, self.bits[layer], self.ctx[step], s.sink, s.window, self.plan[layer], ws_plan,
                         stream)
 
     def attend(self, step: int, layer: int, Q, out, stream=None, prefetch: bool = False):
@@ -400,18 +419,37 @@ class SparseDecoder:
         attention launches; `marks(name)` is called between the two groups so
         a caller can bracket them with events.  `on_select(layer)`, if given,
         is called right after each layer's selection is issued (while the
-        selection workspace still holds that layer's scores)."""
+        selection workspace still holds that layer's scores); the selections
+        then all run on `stream`, without the second stream."""
         s = self.shape
         if step in self.proj_begin:
             for l in range(s.n_layers):
                 self.project(step, l, stream)
         if is_prediction_step(step, s.interval):
+            # the predictor calls first: every layer's queries are in place
+            # before any selection starts
             for l in range(s.n_layers):
                 if s.hidden > 0 and l in self.qp:
                     self.predict(l, h[self.producers.index(l)], stream)
-                self.select(step, l, None if qp_direct is None else qp_direct[l], stream)
+            two = self.overlap_select and on_select is None
+            if two:
+                main = (torch.cuda.current_stream(self.device) if stream is None else
+                        stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream)))
+                fork = torch.cuda.Event()
+                fork.record(main)
+                self.side.wait_event(fork)
+            for l in range(s.n_layers):
+                qd = None if qp_direct is None else qp_direct[l]
+                if two and l % 2 == 1:
+                    self.select(step, l, qd, self.side, self.ws_sel_side, self.ws_plan_side)
+                else:
+                    self.select(step, l, qd, stream)
                 if on_select:
                     on_select(l)
+            if two:
+                join = torch.cuda.Event()
+                join.record(self.side)
+                main.wait_event(join)
         if marks:
             marks("attn_begin")
         # the first launch after a prediction follows the last layer's

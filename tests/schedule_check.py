@@ -140,9 +140,8 @@ def check_schedule(run, layers, steps, seqs, heads, attn_steps, selection="head"
             before_step(i)
         dec.step(i, Q, run.out, h=h, qp_direct=qd, on_select=on_select)
         torch.cuda.synchronize()
-        for ws in (dec.ws_attn, dec.ws_sel, dec.ws_proj, dec.ws_pred):
-            if ws is not None:
-                assert tb.workspace_check(ws) == 0, f"device flag at step {i}"
+        for ws in dec.workspaces():
+            assert tb.workspace_check(ws) == 0, f"device flag at step {i}"
         now = [(dec.idx[l].clone(), dec.cnt[l].clone(), dec.bits[l].clone()) for l in layers]
         if is_prediction_step(i, w.interval):
             kept_sel = now

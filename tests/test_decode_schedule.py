@@ -43,9 +43,10 @@ def test_attention_prefetch_only_where_the_contract_holds():
                                             d_proj=16, hidden=0, inter=0, stride=1, sink=4, window=16, budget=8,
                                             nbr=1, interval=interval, ctx_cap=512)
             self.prefetch_kv = prefetch_kv
+            self.overlap_select = False  # (one stream: no GPU here)
             self.proj_begin, self.qp, self.calls = {}, {}, []
 
-        def select(self, step, layer, qp_direct=None, stream=None):
+        def select(self, step, layer, qp_direct=None, stream=None, ws_sel=None, ws_plan=None):
             self.calls.append(("select", step, layer))
 
         def attend(self, step, layer, Q, out, stream=None, prefetch=False):

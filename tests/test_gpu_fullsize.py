@@ -27,7 +27,7 @@ def test_full_size_sampled(name):
     Q, h, qd = run.step_inputs(0)
     dec.step(0, Q, run.out, h=h, qp_direct=qd)
     torch.cuda.synchronize()
-    for ws in (dec.ws_attn, dec.ws_sel, dec.ws_proj, dec.ws_pred):
+    for ws in dec.workspaces():
         assert tb.workspace_check(ws) == 0
 
     ctx0 = run.ctx0

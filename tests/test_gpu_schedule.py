@@ -10,7 +10,9 @@ decode loop (tests/schedule_check.py describes every check):
     producer layer and the layers its four query slots serve), across at
     least one whole prediction interval, on sampled sequences and KV heads;
     the 64K case runs to step 64, so the prediction there reads the key batch
-    projected at step 63.
+    projected at step 63;
+  * the decoder's second selection stream (odd layers' selections beside the
+    even layers') against all selections on one stream, bit for bit.
 """
 import pytest
 
@@ -65,3 +67,45 @@ def test_full_size_multi_step(name, steps, attn_steps, seqs, groups):
     n_pred = (steps + w.interval - 1) // w.interval
     assert st["selections"] == n_pred * 4 * len(seqs) * len(heads)
     assert st["outputs"] >= len(attn_steps) * 4 * len(seqs) * len(heads)
+
+
+@pytest.mark.parametrize("selection", ["head", "group_max"])
+def test_overlapped_selections_equal_one_stream(selection):
+    """The schedule checks above pass on_select, which keeps every selection
+    on one stream; here the default decoder alternates the layers' selections
+    between the caller's stream and its second one (with their own selection
+    and plan workspaces), eagerly and replayed from a CUDA graph, and must
+    leave every index list, count, bitmap and output of the one-stream run."""
+    import torch
+    w = _small()
+    runs = {ov: bench.Run(w, DEV, selection=selection, overlap_select=ov) for ov in (False, True)}
+    assert runs[True].dec.side is not None and runs[False].dec.side is None
+    for r in runs.values():
+        r.dec.prefill()
+    torch.cuda.synchronize()
+    for i in range(w.steps):
+        got = {}
+        for ov, r in runs.items():
+            Q, h, qd = r.step_inputs(i)
+            r.dec.step(i, Q, r.out, h=h, qp_direct=qd)
+            torch.cuda.synchronize()
+            got[ov] = [t.clone() for t in r.dec.idx + r.dec.cnt + r.dec.bits] + [r.out.clone()]
+        for a, b in zip(got[False], got[True]):
+            assert torch.equal(a, b), f"step {i}: the overlapped selections differ from one stream"
+    for r in runs.values():
+        for ws in r.dec.workspaces():
+            assert bench.L.workspace_check(ws) == 0
+    # the same steps captured in one graph (fork and join inside the capture)
+    r = runs[True]
+    ref = runs[False]
+    st = torch.cuda.Stream()
+    for i in range(w.steps):
+        Q, h, qd = r.step_inputs(i)
+        g = bench.capture(lambda s, i=i, Q=Q, h=h, qd=qd: r.dec.step(i, Q, r.out, h=h, qp_direct=qd, stream=s), st)
+        g.replay()
+        torch.cuda.synchronize()
+        Qr, hr, qdr = ref.step_inputs(i)
+        ref.dec.step(i, Qr, ref.out, h=hr, qp_direct=qdr)
+        torch.cuda.synchronize()
+        for a, b in zip(r.dec.idx + r.dec.cnt + r.dec.bits + [r.out], ref.dec.idx + ref.dec.cnt + ref.dec.bits + [ref.out]):
+            assert torch.equal(a, b), f"step {i}: the graph-replayed overlapped step differs"
