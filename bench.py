@@ -55,7 +55,7 @@ class Run:
 
     def __init__(self, w: tb_inputs.Workload, device: str, steps: int | None = None, selection: str = "head",
                  shard: tuple[int, int] | None = None, offload: bool = False, balance: bool = True,
-                 overlap_select: bool = True):
+                 overlap_select: bool = True, select_streams: int = 4):
         self.w = w
         self.device = device
         self.steps = steps or w.steps
@@ -102,7 +102,8 @@ class Run:
         # the bench's streams run only libtb's kernels, the K/V append of the
         # e2e loop and copies, so every attention launch may prefetch its rows
         self.dec = cls(self.shape, list(self.K), list(self.V), self.Wk, self.mlp, self.ctx0, self.steps, device,
-                       selection=selection, prefetch_kv=True, balance=balance, overlap_select=overlap_select)
+                       selection=selection, prefetch_kv=True, balance=balance, overlap_select=overlap_select,
+                       select_streams=select_streams)
         self.out = torch.zeros(nL, w.batch, self.Hq, w.head_dim, dtype=torch.float32, device=device)
 
     def step_inputs(self, i):
@@ -670,7 +671,7 @@ def measure(w, args, device, dist_on, world, with_e2e: bool, steps: int, warmup:
     With shard=(rank, world) this rank runs only its KV heads of the one
     workload (strong scaling: the job's tokens are the workload's tokens)."""
     run = Run(w, device, steps=args.decode_steps, selection=selection, shard=shard, balance=not args.no_balance,
-              overlap_select=not args.no_overlap)
+              overlap_select=not args.no_overlap, select_streams=args.select_streams)
     copies = 1 if shard else world          # independent replicas count every rank's tokens
     run.dec.prefill()
     torch.cuda.synchronize()
@@ -828,7 +829,9 @@ def main():
                          "default single-GPU run times after the headline workload")
     ap.add_argument("--offload-only", action="store_true", help="time only the CPU-offloaded workload")
     ap.add_argument("--no-overlap", action="store_true",
-                    help="all of a prediction step's selections on one stream (no second selection stream)")
+                    help="all of a prediction step's selections on one stream (no extra selection streams)")
+    ap.add_argument("--select-streams", type=int, default=4,
+                    help="streams a prediction step's selections go round-robin over (with the overlap on)")
     ap.add_argument("--no-balance", action="store_true",
                     help="attention slices at equal shares of the length instead of the kept rows (no tb_attn_plan)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "kv_heads"],

@@ -274,7 +274,7 @@ class SparseDecoder:
 
     def __init__(self, shape: DecodeShape, K, V, Wk, mlp, ctx0: list[int], steps: int, device="cuda",
                  selection: str = "head", prefetch_kv: bool = False, balance: bool = True,
-                 overlap_select: bool = True):
+                 overlap_select: bool = True, select_streams: int = 4):
         if selection not in self.SELECTIONS:
             raise ValueError(f"selection must be one of {self.SELECTIONS}")
         self.selection = selection
@@ -314,17 +314,19 @@ class SparseDecoder:
         self.ws_proj = L.workspace(L.project_keys_workspace_bytes(), device)
         self.ws_pred = (L.workspace(L.predict_queries_workspace_bytes(B, s.hidden, s.inter, s.n_out), device)
                         if s.hidden > 0 else None)
-        # overlap_select: a prediction step's selections alternate between the
-        # caller's stream and a second one (odd layers, with a selection and
-        # a plan workspace of their own), so that one layer's scoring runs on
-        # the SMs the other layer's cluster selection leaves free.  The layers'
-        # selections are independent; the attention launches wait for both.
-        self.overlap_select = overlap_select and s.n_layers > 1
-        self.side = torch.cuda.Stream(device=device) if self.overlap_select else None
-        self.ws_sel_side = (L.workspace(L.score_select_workspace_bytes(self.dims), device)
-                            if self.overlap_select else None)
-        self.ws_plan_side = (L.workspace(L.attn_workspace_bytes(self.dims), device)
-                             if self.overlap_select and balance else None)
+        # overlap_select: a prediction step's selections go round-robin over
+        # the caller's stream and select_streams - 1 more (layer l to stream
+        # l % select_streams, each extra stream with a selection and a plan
+        # workspace of its own), so that one layer's scoring runs on the SMs
+        # another layer's cluster selection leaves free.  The layers'
+        # selections are independent; the attention launches wait for all.
+        n_sel = max(1, int(select_streams)) if overlap_select and s.n_layers > 1 else 1
+        self.overlap_select = n_sel > 1
+        self.sel_lanes = [(torch.cuda.Stream(device=device),
+                           L.workspace(L.score_select_workspace_bytes(self.dims), device),
+                           L.workspace(L.attn_workspace_bytes(self.dims), device) if balance else None)
+                          for _ in range(n_sel - 1)]
+        self.side = self.sel_lanes[0][0] if self.sel_lanes else None
         self.ctx = torch.tensor([[t + i + 1 for t in ctx0] for i in range(steps)], dtype=torch.int32,
                                 device=device)
         prefill, events = projection_schedule(self.ctx0, s.window, steps)
@@ -356,8 +358,8 @@ class SparseDecoder:
 
     def workspaces(self) -> list:
         """Every workspace the decoder's launches use (for tb_workspace_check)."""
-        return [w for w in (self.ws_attn, self.ws_sel, self.ws_proj, self.ws_pred, self.ws_sel_side,
-                            self.ws_plan_side) if w is not None]
+        lanes = [w for _, ws, wp in self.sel_lanes for w in (ws, wp)]
+        return [w for w in [self.ws_attn, self.ws_sel, self.ws_proj, self.ws_pred] + lanes if w is not None]
 
     def select(self, step: int, layer: int, qp_direct=None, stream=None, ws_sel=None, ws_plan=None):
         s = self.shape
@@ -437,19 +439,23 @@ class SparseDecoder:
                         stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream)))
                 fork = torch.cuda.Event()
                 fork.record(main)
-                self.side.wait_event(fork)
+                for st, _, _ in self.sel_lanes:
+                    st.wait_event(fork)
+            n = 1 + len(self.sel_lanes) if two else 1
             for l in range(s.n_layers):
                 qd = None if qp_direct is None else qp_direct[l]
-                if two and l % 2 == 1:
-                    self.select(step, l, qd, self.side, self.ws_sel_side, self.ws_plan_side)
+                if l % n:
+                    st, ws_sel, ws_plan = self.sel_lanes[l % n - 1]
+                    self.select(step, l, qd, st, ws_sel, ws_plan)
                 else:
                     self.select(step, l, qd, stream)
                 if on_select:
                     on_select(l)
             if two:
-                join = torch.cuda.Event()
-                join.record(self.side)
-                main.wait_event(join)
+                for st, _, _ in self.sel_lanes:
+                    join = torch.cuda.Event()
+                    join.record(st)
+                    main.wait_event(join)
         if marks:
             marks("attn_begin")
         # the first launch after a prediction follows the last layer's

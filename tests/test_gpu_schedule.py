@@ -11,8 +11,9 @@ decode loop (tests/schedule_check.py describes every check):
     least one whole prediction interval, on sampled sequences and KV heads;
     the 64K case runs to step 64, so the prediction there reads the key batch
     projected at step 63;
-  * the decoder's second selection stream (odd layers' selections beside the
-    even layers') against all selections on one stream, bit for bit.
+  * the decoder's extra selection streams (the layers' selections round-robin
+    over two or four streams) against all selections on one stream, bit for
+    bit.
 """
 import pytest
 
@@ -69,17 +70,18 @@ def test_full_size_multi_step(name, steps, attn_steps, seqs, groups):
     assert st["outputs"] >= len(attn_steps) * 4 * len(seqs) * len(heads)
 
 
-@pytest.mark.parametrize("selection", ["head", "group_max"])
-def test_overlapped_selections_equal_one_stream(selection):
+@pytest.mark.parametrize("selection,streams", [("head", 2), ("head", 4), ("group_max", 4)])
+def test_overlapped_selections_equal_one_stream(selection, streams):
     """The schedule checks above pass on_select, which keeps every selection
-    on one stream; here the default decoder alternates the layers' selections
-    between the caller's stream and its second one (with their own selection
-    and plan workspaces), eagerly and replayed from a CUDA graph, and must
+    on one stream; here the decoder spreads the layers' selections over the
+    caller's stream and one or three more (each with its own selection and plan
+    workspaces), eagerly and replayed from a CUDA graph, and must
     leave every index list, count, bitmap and output of the one-stream run."""
     import torch
     w = _small()
-    runs = {ov: bench.Run(w, DEV, selection=selection, overlap_select=ov) for ov in (False, True)}
-    assert runs[True].dec.side is not None and runs[False].dec.side is None
+    runs = {ov: bench.Run(w, DEV, selection=selection, overlap_select=ov, select_streams=streams)
+            for ov in (False, True)}
+    assert len(runs[True].dec.sel_lanes) == streams - 1 and not runs[False].dec.sel_lanes
     for r in runs.values():
         r.dec.prefill()
     torch.cuda.synchronize()
