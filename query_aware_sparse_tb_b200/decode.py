@@ -28,6 +28,13 @@ import torch
 from . import _lib as L
 
 
+def main_stream_last_selected(n_layers: int, n_streams: int) -> int:
+    """The last layer whose selection the caller's stream issues when a
+    prediction step's selections go round-robin over n_streams streams (layer
+    l on stream l mod n_streams, the caller's stream first)."""
+    return (n_layers - 1) // n_streams * n_streams
+
+
 def is_prediction_step(step: int, interval: int) -> bool:
     return step % interval == 0
 
@@ -458,9 +465,12 @@ class SparseDecoder:
                     main.wait_event(join)
         if marks:
             marks("attn_begin")
-        # the first launch after a prediction follows the last layer's
-        # selection, which wrote that layer's selection words
-        after_own_select = is_prediction_step(step, s.interval) and s.n_layers == 1
+        # the first launch after a prediction follows the last selection the
+        # caller's stream issued; when that is layer 0's own, it wrote the
+        # selection words (and plan) this launch reads
+        n_streams = 1 + len(self.sel_lanes) if (self.overlap_select and on_select is None) else 1
+        after_own_select = (is_prediction_step(step, s.interval) and
+                            main_stream_last_selected(s.n_layers, n_streams) == 0)
         for l in range(s.n_layers):
             self.attend(step, l, Q[l], out[l], stream,
                         prefetch=self.prefetch_kv and not (l == 0 and after_own_select))

@@ -64,3 +64,12 @@ def test_attention_prefetch_only_where_the_contract_holds():
                     right_after_own_select = n_layers == 1 and step % interval == 0
                     assert pf == (prefetch_kv and not right_after_own_select), (n_layers, interval, step, layer)
     assert L.TB_ATTN_WAIT_ALL == 0 and L.TB_ATTN_PREFETCH_KV == 1
+
+
+def test_last_selection_on_the_callers_stream():
+    # with the selections round-robin over n streams, the caller's stream
+    # issues layers 0, n, 2n, ...; the first attention launch after them may
+    # prefetch only when the last of those is not layer 0
+    f = decode.main_stream_last_selected
+    assert [f(1, 1), f(3, 1), f(32, 1)] == [0, 2, 31]
+    assert [f(4, 4), f(5, 4), f(32, 4), f(4, 2), f(2, 4), f(32, 2)] == [0, 4, 28, 2, 0, 30]
