@@ -333,7 +333,6 @@ class SparseDecoder:
                            L.workspace(L.score_select_workspace_bytes(self.dims), device),
                            L.workspace(L.attn_workspace_bytes(self.dims), device) if balance else None)
                           for _ in range(n_sel - 1)]
-        self.side = self.sel_lanes[0][0] if self.sel_lanes else None
         self.ctx = torch.tensor([[t + i + 1 for t in ctx0] for i in range(steps)], dtype=torch.int32,
                                 device=device)
         prefill, events = projection_schedule(self.ctx0, s.window, steps)
@@ -429,7 +428,7 @@ class SparseDecoder:
         a caller can bracket them with events.  `on_select(layer)`, if given,
         is called right after each layer's selection is issued (while the
         selection workspace still holds that layer's scores); the selections
-        then all run on `stream`, without the second stream."""
+        then all run on `stream`, without the extra streams."""
         s = self.shape
         if step in self.proj_begin:
             for l in range(s.n_layers):
@@ -440,15 +439,15 @@ class SparseDecoder:
             for l in range(s.n_layers):
                 if s.hidden > 0 and l in self.qp:
                     self.predict(l, h[self.producers.index(l)], stream)
-            two = self.overlap_select and on_select is None
-            if two:
+            spread = self.overlap_select and on_select is None
+            if spread:
                 main = (torch.cuda.current_stream(self.device) if stream is None else
                         stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream)))
                 fork = torch.cuda.Event()
                 fork.record(main)
                 for st, _, _ in self.sel_lanes:
                     st.wait_event(fork)
-            n = 1 + len(self.sel_lanes) if two else 1
+            n = 1 + len(self.sel_lanes) if spread else 1
             for l in range(s.n_layers):
                 qd = None if qp_direct is None else qp_direct[l]
                 if l % n:
@@ -458,7 +457,7 @@ class SparseDecoder:
                     self.select(step, l, qd, stream)
                 if on_select:
                     on_select(l)
-            if two:
+            if spread:
                 for st, _, _ in self.sel_lanes:
                     join = torch.cuda.Event()
                     join.record(st)
