@@ -1,6 +1,8 @@
 """The decode driver's host-side schedule (query_aware_sparse_tb_b200.decode)
 against the oracle's independently written schedule (oracle.schedule), on CPU:
-projection batches, prediction steps, producer layers and query slots."""
+projection batches, prediction steps, producer layers and query slots; and the
+driver's own launch order: which attention launches may prefetch, and how a
+prediction step's selections are spread over streams (faked on the host)."""
 from oracle import schedule as oschedule
 from query_aware_sparse_tb_b200 import decode
 
@@ -73,3 +75,88 @@ def test_last_selection_on_the_callers_stream():
     f = decode.main_stream_last_selected
     assert [f(1, 1), f(3, 1), f(32, 1)] == [0, 2, 31]
     assert [f(4, 4), f(5, 4), f(32, 4), f(4, 2), f(2, 4), f(32, 2)] == [0, 4, 28, 2, 0, 30]
+
+
+def test_selection_streams_fork_route_and_join(monkeypatch):
+    # a prediction step with the selections spread over n streams, with the
+    # streams and events faked on the host: the predictors go first on the
+    # caller's stream, every extra stream waits for an event recorded after
+    # them, layer l's selection goes to stream l mod n with that stream's own
+    # workspaces, and the caller's stream waits for an event recorded on every
+    # extra stream after its last selection, before the first attention launch
+    import torch
+    log = []
+
+    class FakeStream:
+        def __init__(self, name):
+            self.name = name
+
+        def wait_event(self, ev):
+            log.append(("wait", self.name, ev.id))
+
+    class FakeEvent:
+        n = 0
+
+        def __init__(self):
+            FakeEvent.n += 1
+            self.id = FakeEvent.n
+
+        def record(self, stream):
+            log.append(("record", stream.name, self.id))
+
+    main = FakeStream("main")
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: main)
+
+    class Rec(decode.SparseDecoder):
+        def __init__(self, n_layers, n_streams):
+            self.shape = decode.DecodeShape(batch=1, n_layers=n_layers, n_q_heads=8, n_kv_heads=2, head_dim=64,
+                                            d_proj=16, hidden=16, inter=16, stride=4, sink=4, window=16, budget=8,
+                                            nbr=1, interval=4, ctx_cap=512)
+            self.device = "cuda"
+            self.prefetch_kv = True
+            self.overlap_select = n_streams > 1
+            self.sel_lanes = [(FakeStream(f"lane{k}"), f"ws_sel{k}", f"ws_plan{k}") for k in range(1, n_streams)]
+            self.producers = [l for l in range(n_layers) if l % 4 == 0]
+            self.proj_begin, self.qp = {}, {p: None for p in self.producers}
+
+        def predict(self, producer, h, stream=None):
+            log.append(("predict", producer))
+
+        def select(self, step, layer, qp_direct=None, stream=None, ws_sel=None, ws_plan=None):
+            log.append(("select", layer, getattr(stream, "name", "main"), ws_sel, ws_plan))
+
+        def attend(self, step, layer, Q, out, stream=None, prefetch=False):
+            log.append(("attend", layer, prefetch))
+
+    for n_layers, n_streams in ((8, 4), (6, 4), (4, 4), (5, 2), (3, 1)):
+        log.clear()
+        dec = Rec(n_layers, n_streams)
+        dec.step(0, [None] * n_layers, [None] * n_layers, h=[None] * len(dec.producers))
+        kinds = [e[0] for e in log]
+        first_select = kinds.index("select")
+        assert [e for e in log[:first_select] if e[0] == "predict"] == [("predict", p) for p in dec.producers]
+        sels = [e for e in log if e[0] == "select"]
+        assert [e[1] for e in sels] == list(range(n_layers))
+        for _, l, st, ws, wp in sels:
+            k = l % n_streams
+            assert st == ("main" if k == 0 else f"lane{k}")
+            assert (ws, wp) == ((None, None) if k == 0 else (f"ws_sel{k}", f"ws_plan{k}"))
+        if n_streams > 1:
+            fork = [e for e in log[:first_select] if e[0] == "record"]
+            assert len(fork) == 1 and fork[0][1] == "main"
+            waits = [e for e in log[:first_select] if e[0] == "wait"]
+            assert sorted(e[1] for e in waits) == [f"lane{k}" for k in range(1, n_streams)]
+            assert all(e[2] == fork[0][2] for e in waits)
+            first_attend = kinds.index("attend")
+            tail = log[max(i for i, e in enumerate(log) if e[0] == "select") + 1:first_attend]
+            joins = {e[1]: e[2] for e in tail if e[0] == "record"}
+            assert sorted(joins) == [f"lane{k}" for k in range(1, n_streams)]
+            assert sorted(e[2] for e in tail if e[0] == "wait" and e[1] == "main") == sorted(joins.values())
+        else:
+            assert "record" not in kinds and "wait" not in kinds
+        attends = [e for e in log if e[0] == "attend"]
+        assert [e[1] for e in attends] == list(range(n_layers))
+        # the first launch may prefetch unless the caller's stream selected layer 0 last
+        assert attends[0][2] == (decode.main_stream_last_selected(n_layers, n_streams) != 0)
+        assert all(e[2] for e in attends[1:])
