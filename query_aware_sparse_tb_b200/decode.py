@@ -333,6 +333,9 @@ class SparseDecoder:
                            L.workspace(L.score_select_workspace_bytes(self.dims), device),
                            L.workspace(L.attn_workspace_bytes(self.dims), device) if balance else None)
                           for _ in range(n_sel - 1)]
+        # with the selections spread, the producers' predictor calls run on a
+        # stream of their own; each selection waits only for its producer's
+        self.pred_stream = torch.cuda.Stream(device=device) if self.overlap_select and s.hidden > 0 else None
         self.ctx = torch.tensor([[t + i + 1 for t in ctx0] for i in range(steps)], dtype=torch.int32,
                                 device=device)
         prefill, events = projection_schedule(self.ctx0, s.window, steps)
@@ -434,30 +437,36 @@ class SparseDecoder:
             for l in range(s.n_layers):
                 self.project(step, l, stream)
         if is_prediction_step(step, s.interval):
-            # the predictor calls first: every layer's queries are in place
-            # before any selection starts
-            for l in range(s.n_layers):
-                if s.hidden > 0 and l in self.qp:
-                    self.predict(l, h[self.producers.index(l)], stream)
             spread = self.overlap_select and on_select is None
+            ready = {}
             if spread:
                 main = (torch.cuda.current_stream(self.device) if stream is None else
                         stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream)))
                 fork = torch.cuda.Event()
                 fork.record(main)
-                for st, _, _ in self.sel_lanes:
+                for st in [st for st, _, _ in self.sel_lanes] + ([self.pred_stream] if self.pred_stream else []):
                     st.wait_event(fork)
+            # the predictor calls first (on their own stream when spread, an
+            # event after each): a layer's queries are in place before its
+            # selection starts
+            for l in range(s.n_layers):
+                if s.hidden > 0 and l in self.qp:
+                    self.predict(l, h[self.producers.index(l)], self.pred_stream if spread else stream)
+                    if spread:
+                        ready[l] = torch.cuda.Event()
+                        ready[l].record(self.pred_stream)
             n = 1 + len(self.sel_lanes) if spread else 1
             for l in range(s.n_layers):
                 qd = None if qp_direct is None else qp_direct[l]
-                if l % n:
-                    st, ws_sel, ws_plan = self.sel_lanes[l % n - 1]
-                    self.select(step, l, qd, st, ws_sel, ws_plan)
-                else:
-                    self.select(step, l, qd, stream)
+                st, ws_sel, ws_plan = self.sel_lanes[l % n - 1] if l % n else (main if spread else stream, None, None)
+                if ready:
+                    st.wait_event(ready[producer_layer(l, s.stride)])
+                self.select(step, l, qd, st if l % n else stream, ws_sel, ws_plan)
                 if on_select:
                     on_select(l)
             if spread:
+                if ready:
+                    main.wait_event(ready[max(ready)])  # (the predictor stream's last call)
                 for st, _, _ in self.sel_lanes:
                     join = torch.cuda.Event()
                     join.record(st)

@@ -79,11 +79,14 @@ def test_last_selection_on_the_callers_stream():
 
 def test_selection_streams_fork_route_and_join(monkeypatch):
     # a prediction step with the selections spread over n streams, with the
-    # streams and events faked on the host: the predictors go first on the
-    # caller's stream, every extra stream waits for an event recorded after
-    # them, layer l's selection goes to stream l mod n with that stream's own
-    # workspaces, and the caller's stream waits for an event recorded on every
-    # extra stream after its last selection, before the first attention launch
+    # streams and events faked on the host: every extra stream (and the
+    # predictors' stream) waits for an event recorded on the caller's stream
+    # first; the producers' predictor calls run on their own stream with an
+    # event after each; layer l's selection goes to stream l mod n with that
+    # stream's own workspaces, after a wait for its producer's event; the
+    # caller's stream waits for the predictors' last event and for an event
+    # recorded on every extra stream after its last selection, before the
+    # first attention launch
     import torch
     log = []
 
@@ -117,11 +120,12 @@ def test_selection_streams_fork_route_and_join(monkeypatch):
             self.prefetch_kv = True
             self.overlap_select = n_streams > 1
             self.sel_lanes = [(FakeStream(f"lane{k}"), f"ws_sel{k}", f"ws_plan{k}") for k in range(1, n_streams)]
+            self.pred_stream = FakeStream("pred") if n_streams > 1 else None
             self.producers = [l for l in range(n_layers) if l % 4 == 0]
             self.proj_begin, self.qp = {}, {p: None for p in self.producers}
 
         def predict(self, producer, h, stream=None):
-            log.append(("predict", producer))
+            log.append(("predict", producer, getattr(stream, "name", "main")))
 
         def select(self, step, layer, qp_direct=None, stream=None, ws_sel=None, ws_plan=None):
             log.append(("select", layer, getattr(stream, "name", "main"), ws_sel, ws_plan))
@@ -133,28 +137,43 @@ def test_selection_streams_fork_route_and_join(monkeypatch):
         log.clear()
         dec = Rec(n_layers, n_streams)
         dec.step(0, [None] * n_layers, [None] * n_layers, h=[None] * len(dec.producers))
+        spread = n_streams > 1
         kinds = [e[0] for e in log]
         first_select = kinds.index("select")
-        assert [e for e in log[:first_select] if e[0] == "predict"] == [("predict", p) for p in dec.producers]
+        preds = [e for e in log[:first_select] if e[0] == "predict"]
+        assert [e[1] for e in preds] == dec.producers
+        assert all(e[2] == ("pred" if spread else "main") for e in preds)
         sels = [e for e in log if e[0] == "select"]
         assert [e[1] for e in sels] == list(range(n_layers))
         for _, l, st, ws, wp in sels:
             k = l % n_streams
             assert st == ("main" if k == 0 else f"lane{k}")
             assert (ws, wp) == ((None, None) if k == 0 else (f"ws_sel{k}", f"ws_plan{k}"))
-        if n_streams > 1:
-            fork = [e for e in log[:first_select] if e[0] == "record"]
-            assert len(fork) == 1 and fork[0][1] == "main"
-            waits = [e for e in log[:first_select] if e[0] == "wait"]
-            assert sorted(e[1] for e in waits) == [f"lane{k}" for k in range(1, n_streams)]
-            assert all(e[2] == fork[0][2] for e in waits)
+        if not spread:
+            assert "record" not in kinds and "wait" not in kinds
+        else:
+            # the fork: one event on the caller's stream, before anything else
+            assert log[0][:2] == ("record", "main")
+            fork = log[0][2]
+            forked = sorted(e[1] for e in log[:first_select] if e[0] == "wait" and e[2] == fork)
+            assert forked == sorted([f"lane{k}" for k in range(1, n_streams)] + ["pred"])
+            # an event on the predictors' stream after each predictor call
+            ready = {}
+            for i, e in enumerate(log):
+                if e[0] == "predict":
+                    assert log[i + 1][:2] == ("record", "pred")
+                    ready[e[1]] = log[i + 1][2]
+            # each selection right after its stream waits for its producer's event
+            for i, e in enumerate(log):
+                if e[0] == "select":
+                    assert log[i - 1] == ("wait", e[2], ready[decode.producer_layer(e[1], 4)])
+            # the join: the caller's stream waits for the predictors and every extra stream
             first_attend = kinds.index("attend")
             tail = log[max(i for i, e in enumerate(log) if e[0] == "select") + 1:first_attend]
             joins = {e[1]: e[2] for e in tail if e[0] == "record"}
             assert sorted(joins) == [f"lane{k}" for k in range(1, n_streams)]
-            assert sorted(e[2] for e in tail if e[0] == "wait" and e[1] == "main") == sorted(joins.values())
-        else:
-            assert "record" not in kinds and "wait" not in kinds
+            waited = sorted(e[2] for e in tail if e[0] == "wait" and e[1] == "main")
+            assert waited == sorted(list(joins.values()) + [ready[max(ready)]])
         attends = [e for e in log if e[0] == "attend"]
         assert [e[1] for e in attends] == list(range(n_layers))
         # the first launch may prefetch unless the caller's stream selected layer 0 last
